@@ -1,0 +1,530 @@
+"""Benchmark of the sparse decode step (one layer's append + decode per
+step; 48 layers per step for the 48-layer workload) on synthetic caches.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3] [--p P]
+    python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+
+Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) are independent
+replicas of the workload per rank (the step shards by sequence and KV head
+with no data exchange): value = steps of all ranks / max rank time.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from dynamic_top_sparse_b200 import ops, synth  # noqa: E402
+
+METRIC = "sparse decode attention steps/s and achieved HBM GB/s (% peak) at 64K-1M ctx"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_HBM = 6650.0
+
+
+# --------------------------------------------------------------------- utils
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM, "fallback"
+
+
+def csrc_hash():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "dynamic_top_sparse_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken
+    on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+    except Exception:
+        return None
+    for r in rec.get("records", []):
+        if r.get("kernel") == kernel and r.get("workload") == workload and r.get("csrc") == csrc_hash():
+            return r.get("bytes_per_launch")
+    return None
+
+
+class Clocks:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x2: "applications_clocks",
+               0x10: "sync_boost", 0x1: "gpu_idle"}
+
+    def __init__(self, dev: int):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                bus = torch.cuda.get_device_properties(dev).pci_bus_id
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(
+                    f"{torch.cuda.get_device_properties(dev).pci_domain_id:08x}:{bus:02x}:"
+                    f"{torch.cuda.get_device_properties(dev).pci_device_id:02x}.0")
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(dev)
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report nothing rather than guess
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h) if hasattr(
+            nv, "nvmlDeviceGetCurrentClocksEventReasons") else nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        for bit, name in self.REASONS.items():
+            if r & bit and name != "gpu_idle":
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def report(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "NVML unavailable"}
+        return {"sm_mhz": float(np.median(self.samples)) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ workload
+
+class Layer:
+    """Device tensors of one layer of the workload, plus the library state."""
+
+    def __init__(self, case: synth.Case):
+        self.case = case
+        self.q, self.q_rope = case.q.cuda(), (case.q_rope.cuda() if case.q_rope is not None else None)
+        self.k, self.v, self.kidx = case.k_cache, case.v_cache, case.kidx_cache
+        self.Wq, self.Wk = case.W_q_idx.cuda(), case.W_k_idx.cuda()
+        self.k_new = case.k_pre_new.cuda()
+        self.seq = case.seq_lens.cuda()
+        self.pos = (self.seq - 1).to(torch.int32)
+        self.hc = case.head_class
+        self.H_q = self.q.shape[1]
+        self.dims = ops.dims_for(self.k, self.kidx, self.H_q, self.seq)
+
+    def clone_caches(self):
+        other = object.__new__(Layer)
+        other.__dict__.update(self.__dict__)
+        other.k, other.v, other.kidx = self.k.clone(), self.v.clone(), self.kidx.clone()
+        other.dims = ops.dims_for(other.k, other.kidx, other.H_q, other.seq)
+        return other
+
+
+def build_workload(cfg: int, seed: int = 0):
+    spec = synth.spec_for(cfg)
+    layers = []
+    for l in range(spec.layers):
+        c = synth.make_case(spec, device="cuda", seed=seed, layer=l)
+        if c.k_pre_all is not None:
+            c.kidx_cache = c.kidx_cache.cuda()
+        layers.append(Layer(c))
+    return spec, layers
+
+
+def required_bytes(spec, layers, sel):
+    """Algorithmic bytes a step must read: index keys of retrieval heads,
+    the union of kept K/V rows per KV group, window+sink rows of local
+    heads, and the query projector of retrieval heads."""
+    total = 0
+    kv_el = 2 if spec.kv_dtype == "bf16" else 4
+    ix_el = 2 if spec.idx_dtype == "bf16" else 4
+    for li, L in enumerate(layers):
+        G = L.H_q // L.hc.shape[0]
+        lens = L.case.seq_lens.tolist()
+        for b in range(spec.B):
+            N = lens[b]
+            for g in range(L.hc.shape[0]):
+                if L.hc[g] == synth.HEAD_RETRIEVAL:
+                    total += N * spec.r * ix_el
+                    if spec.p >= 1.0 or sel is None:
+                        total += N * 2 * spec.d * kv_el
+                    else:
+                        idx, cnt = sel[li]
+                        u = set()
+                        for h in range(g * G, (g + 1) * G):
+                            u.update(idx[b, h, : int(cnt[b, h])].tolist())
+                        total += len(u) * 2 * spec.d * kv_el
+                else:
+                    rows = min(N, spec.n_sink) + (N - max(min(N, spec.n_sink), N - spec.window))
+                    total += rows * 2 * spec.d * kv_el
+        n_rq = sum(G for g in range(L.hc.shape[0]) if L.hc[g] == synth.HEAD_RETRIEVAL)
+        total += n_rq * spec.r * spec.d * 4
+    return total
+
+
+def index_bytes(spec, layers):
+    ix_el = 2 if spec.idx_dtype == "bf16" else 4
+    L = layers[0]
+    n_ret = int((L.hc == synth.HEAD_RETRIEVAL).sum())
+    return spec.B * n_ret * spec.N * spec.r * ix_el
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, rank, world, dev):
+    spec, layers0 = build_workload(args.config)
+    if args.p is not None:
+        spec.p = args.p
+    p = spec.p
+    one_step_bytes = None
+    out = torch.empty((spec.B, spec.H_q, spec.d), device=dev)
+    ws = ops.Workspace(layers0[0].dims)
+
+    def step(layers, prof=None, sel=None):
+        for li, L in enumerate(layers):
+            ops.append_index_keys(L.dims, L.k_new, L.Wk, L.pos, L.hc, L.kidx, ws)
+            opts = None
+            if prof is not None or sel is not None:
+                kw = {}
+                if sel is not None:
+                    kw = dict(sel_idx=sel[li][0], sel_count=sel[li][1])
+                opts = ops.make_opts(prof=prof, **kw)
+            ops.decode_step(L.dims, L.q, L.q_rope, L.k, L.v, L.kidx, L.Wq, L.hc, p, spec.window,
+                            spec.n_sink, out, ws, opts)
+
+    # kept sets of one step -> required bytes
+    sel = [(torch.full((spec.B, spec.H_q, L.k.shape[2]), -1, dtype=torch.int32, device=dev),
+            torch.zeros((spec.B, spec.H_q), dtype=torch.int32, device=dev)) for L in layers0]
+    step(layers0, sel=sel)
+    st = ws.check()
+    if st:
+        raise RuntimeError(f"device status {st}: {ops.error_string(st)}")
+    req = required_bytes(spec, layers0, [(a.cpu().numpy(), b.cpu().numpy()) for a, b in sel])
+    kept = [[int(x) for x in b.cpu().numpy().ravel() if x > 0] for _, b in sel]
+    del sel
+
+    # rotating replicas so that no step reads what the previous ones left in L2
+    n_rep = 1 if spec.layers > 1 else max(1, math.ceil(3 * L2_BYTES / max(req, 1)))
+    n_rep = min(n_rep, args.max_replicas)
+    reps = [layers0] + [[L.clone_caches() for L in layers0] for _ in range(n_rep - 1)]
+
+    # launches per step (all kernels)
+    pr_all = ops.Profiler(256)
+    step(reps[0], prof=pr_all)
+    torch.cuda.synchronize()
+    launches_per_step = pr_all.p.count
+    pr_all.close()
+
+    # CUDA graph per replica
+    graphs = []
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for R in reps:
+            step(R)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for R in reps:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(R)
+        graphs.append(g)
+    torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        graphs[i % n_rep].replay()
+    torch.cuda.synchronize()
+
+    clocks = Clocks(dev.index)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with clocks:
+        e0.record()
+        for i in range(args.steps):
+            graphs[i % n_rep].replay()
+        e1.record()
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1)
+    ms_max = allreduce_max(ms, world, dev)
+    ms_per_step = ms_max / args.steps
+    value = world * args.steps / (ms_max / 1e3)
+
+    # dominant kernel: the index scan (histogram pass); direct launches with
+    # events on the library's stream
+    n_prof = min(args.steps, args.prof_steps)
+    pr = ops.Profiler(n_prof * spec.layers + 8, filter="hist")
+    for i in range(n_prof):
+        step(reps[i % n_rep], prof=pr)
+    torch.cuda.synchronize()
+    hist_ms = [t for name, t in pr.times() if name == "hist"]
+    pr.close()
+    hist_avg_ms = float(np.mean(hist_ms)) if hist_ms else None
+    hbm_peak, peak_src = peaks()
+    idx_b = index_bytes(spec, layers0)
+    achieved = idx_b / (hist_avg_ms * 1e-3) / 1e9 if hist_avg_ms else None
+    workload = spec.name
+
+    # dense decode over the same caches
+    dgraphs = []
+    dense_out = torch.empty_like(out)
+
+    def dense_step(layers):
+        for L in layers:
+            ops.dense_decode(L.dims, L.q_rope if L.q_rope is not None else L.q, L.k, L.v, dense_out, ws)
+
+    with torch.cuda.stream(s):
+        for R in reps:
+            dense_step(R)
+    torch.cuda.synchronize()
+    for R in reps:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            dense_step(R)
+        dgraphs.append(g)
+    n_dense = max(3, min(args.steps, args.dense_steps))
+    for i in range(3):
+        dgraphs[i % n_rep].replay()
+    torch.cuda.synchronize()
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record()
+    for i in range(n_dense):
+        dgraphs[i % n_rep].replay()
+    d1.record()
+    torch.cuda.synchronize()
+    dense_ms = d0.elapsed_time(d1) / n_dense
+
+    # end to end: pinned host inputs -> device, graph, result -> host
+    e2e = None
+    if not args.no_e2e:
+        hq = [torch.empty(L.q.shape, dtype=L.q.dtype, pin_memory=True) for L in reps[0]]
+        hqr = [torch.empty(L.q.shape, dtype=L.q.dtype, pin_memory=True) for L in reps[0]]
+        hk = [torch.empty(L.k_new.shape, dtype=L.k_new.dtype, pin_memory=True) for L in reps[0]]
+        for i, L in enumerate(reps[0]):
+            hq[i].copy_(L.q)
+            hqr[i].copy_(L.q_rope if L.q_rope is not None else L.q)
+            hk[i].copy_(L.k_new)
+        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        n_e2e = max(3, min(args.steps, args.e2e_steps))
+        h2d = sum(t.numel() * t.element_size() for t in hq + hk) + (
+            sum(t.numel() * t.element_size() for t in hqr) if reps[0][0].q_rope is not None else 0)
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step(i):
+            R = reps[i % n_rep]
+            for j, L in enumerate(R):
+                L.q.copy_(hq[j], non_blocking=True)
+                if L.q_rope is not None:
+                    L.q_rope.copy_(hqr[j], non_blocking=True)
+                L.k_new.copy_(hk[j], non_blocking=True)
+            graphs[i % n_rep].replay()
+            hout.copy_(out, non_blocking=True)
+            torch.cuda.current_stream().synchronize()
+
+        for i in range(3):
+            e2e_step(i)
+        barrier(world)
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record()
+        for i in range(n_e2e):
+            e2e_step(i)
+        x1.record()
+        torch.cuda.synchronize()
+        e2e_ms = allreduce_max(x0.elapsed_time(x1), world, dev)
+        e2e = {"value": world * n_e2e / (e2e_ms / 1e3), "unit": "steps/s", "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": int(d2h), "steps": n_e2e,
+               "note": "pinned host q/q_rope/k_new -> device, CUDA-graph step, out -> host, sync each step"}
+
+    step_gbs = req / (ms_per_step * 1e-3) / 1e9
+    res = {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": workload, "cfg": args.config, "B": spec.B, "ctx": spec.N, "H_q": spec.H_q,
+                   "H_kv": spec.H_kv, "d": spec.d, "r": spec.r, "layers": spec.layers, "p": p,
+                   "window": spec.window, "n_sink": spec.n_sink, "cache_dtype": spec.kv_dtype,
+                   "index_dtype": spec.idx_dtype, "accumulate": "f32",
+                   "l2": f"rotating {n_rep} cache replicas per rank ({n_rep} x {req / 1e6:.1f} MB >= 3 x L2)"
+                   if n_rep > 1 else f"{spec.layers} distinct layers per step ({req / 1e6:.0f} MB > L2)",
+                   "timing": "CUDA graph replays, CUDA events, max over ranks",
+                   "parallelism": f"replicas x{world} (independent sequences per rank)"},
+        "required_bytes_per_step": int(req),
+        "achieved_gbs": step_gbs,
+        "pct_peak": step_gbs / hbm_peak,
+        "pct_of_8tbs": step_gbs / 8000.0,
+        "kept_rows_per_retrieval_head": {"min": min(min(k) for k in kept if k) if any(kept) else 0,
+                                         "max": max(max(k) for k in kept if k) if any(kept) else 0,
+                                         "mean": float(np.mean([x for k in kept for x in k])) if any(kept) else 0},
+        "roofline": {"bound": "hbm", "kernel": "hist (index-key scan + mass histogram)",
+                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": (achieved / hbm_peak) if achieved else None,
+                     "traffic": traffic_for("hist", workload),
+                     "bytes_per_launch": idx_b, "avg_launch_ms": hist_avg_ms,
+                     "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+                     else "fallback 6650 GB/s"},
+        "dense": {"ms_per_step": dense_ms, "speedup_sparse_vs_dense": dense_ms / ms_per_step,
+                  "bytes_per_step": int(sum(2 * L.k.numel() * L.k.element_size() for L in reps[0]))},
+        "gpu_launches": int(launches_per_step * args.steps),
+        "launches_per_step": launches_per_step,
+        "clocks": clocks.report(),
+        "e2e": e2e,
+        "pages_context": {"decode_speedup_1M_H20": 2.01, "prefill_speedup_1M_H20": 9.36},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu:
+        res["cpu_baseline"] = cpu_baseline(args.config, spec, args.cpu_seconds)
+    return res
+
+
+# ------------------------------------------------------------------ oracle arm
+
+def cpu_baseline(cfg, spec=None, budget_s=15.0):
+    """The oracle, as it stands, on host cores over a bounded sample of the
+    workload (whole layers of one replica); steps/s scaled to full steps."""
+    import oracle
+    try:
+        from threadpoolctl import threadpool_limits
+        lim = threadpool_limits(limits=1)
+    except Exception:
+        lim = None
+    spec = spec or synth.spec_for(cfg)
+    layers_done, t_tot = 0, 0.0
+    seqs = list(range(spec.B))
+    for l in range(spec.layers):
+        c = synth.make_case(spec, device="cuda" if torch.cuda.is_available() else "cpu", layer=l)
+        q = c.q.cpu().numpy()
+        qr = None if c.q_rope is None else c.q_rope.cpu().numpy()
+        K, V = c.k_cache.float().cpu().numpy(), c.v_cache.float().cpu().numpy()
+        if c.k_pre_all is not None:
+            kidx = oracle.append_index_keys(np.zeros(tuple(c.kidx_cache.shape)), c.k_pre_all.float().cpu().numpy(),
+                                            c.W_k_idx.cpu().numpy(), np.zeros(spec.B, np.int64), spec.idx_dtype)
+        else:
+            kidx = c.kidx_cache.float().cpu().numpy()
+        heads = [(b, h) for b in seqs for h in range(spec.H_q)]
+        t0 = time.perf_counter()
+        kidx = oracle.append_index_keys(kidx, c.k_pre_new.float().cpu().numpy(), c.W_k_idx.cpu().numpy(),
+                                        c.seq_lens.numpy() - 1, spec.idx_dtype, head_class=c.head_class)
+        oracle.decode_step(q, qr, K, V, kidx, c.W_q_idx.cpu().numpy(), c.head_class, c.seq_lens.numpy(),
+                           spec.p, spec.window, spec.n_sink, heads=heads)
+        t_tot += time.perf_counter() - t0
+        layers_done += 1
+        del K, V, kidx
+        if t_tot >= budget_s:
+            break
+    if lim is not None:
+        lim.unregister() if hasattr(lim, "unregister") else None
+    per_layer = t_tot / layers_done
+    step_s = per_layer * spec.layers
+    return {"value": 1.0 / step_s, "unit": "steps/s", "cores": 1, "kind": "oracle",
+            "sample": f"{layers_done} of {spec.layers} layer(s), all {spec.B} sequence(s) x {spec.H_q} heads, "
+                      f"{t_tot:.1f} s of single-threaded numpy fp64; steps/s = 1 / (per-layer time x layers)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    spec = synth.spec_for(args.config)
+    if args.p is not None:
+        spec.p = args.p
+    cb = cpu_baseline(args.config, spec, args.cpu_seconds)
+    v = cb["value"]
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": spec.name, "cfg": args.config, "B": spec.B, "ctx": spec.N, "p": spec.p},
+            "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "note": "the CPU oracle (numpy fp64), timed on host cores over a bounded sample"}
+
+
+# -------------------------------------------------------------- distributed
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def allreduce_max(x, world, dev):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--p", type=float, default=None)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--prof-steps", type=int, default=200)
+    ap.add_argument("--dense-steps", type=int, default=200)
+    ap.add_argument("--e2e-steps", type=int, default=2000)
+    ap.add_argument("--max-replicas", type=int, default=16)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res))
+        return
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    try:
+        res = run_ours(args, rank, world, dev)
+        if rank == 0:
+            print(json.dumps(res))
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

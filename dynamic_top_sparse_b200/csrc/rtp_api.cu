@@ -1,0 +1,523 @@
+// C ABI of librtp.so: argument checks, workspace layout and kernel launches
+// for the RTPurbo sparse decode step.  Contract: include/rtp.h.
+#include <algorithm>
+#include <cmath>
+#include <cstdlib>
+#include <cstdio>
+#include <cstring>
+
+#include "rtp.h"
+#include "rtp_common.cuh"
+#include "rtp_select.cuh"
+#include "rtp_attend.cuh"
+#include "rtp_append.cuh"
+
+using namespace rtp;
+
+namespace {
+
+constexpr int RANGE_SPLIT_MAX = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace regions, in the order ops need them (each op needs a prefix).
+struct Layout {
+    size_t status, arrive_hist, arrive_range, arrive_list, list_cnt, cand_cnt, hist;
+    size_t ctrl_end;
+    size_t res, qidx, counts, mass;
+    size_t end_scores;      // append / index_scores need up to here
+    size_t part_range;
+    size_t end_range;       // local / dense
+    size_t part_list;
+    size_t end_list;        // sparse decode
+    size_t tilebin, lists, cands;
+    size_t total;           // topp_select / decode_step
+};
+
+Layout make_layout(const rtp_dims *d) {
+    Layout L{};
+    const size_t BHq = (size_t)d->B * d->H_q, BHkv = (size_t)d->B * d->H_kv;
+    const size_t ntile = (size_t)((d->N_max + TILE - 1) / TILE);
+    size_t o = 0;
+    L.status = o; o += 256;
+    L.arrive_hist = o; o = align_up(o + BHkv * 4, 256);
+    L.arrive_range = o; o = align_up(o + BHkv * 4, 256);
+    L.arrive_list = o; o = align_up(o + BHq * 4, 256);
+    L.list_cnt = o; o = align_up(o + BHq * 4, 256);
+    L.cand_cnt = o; o = align_up(o + BHq * 4, 256);
+    L.hist = o; o = align_up(o + BHq * NBIN * 8, 256);
+    L.ctrl_end = o;
+    L.res = o; o = align_up(o + BHq * sizeof(Resolve), 256);
+    L.qidx = o; o = align_up(o + BHq * R * 4, 256);
+    L.counts = o; o = align_up(o + BHq * 4, 256);
+    L.mass = o; o = align_up(o + BHq * 4, 256);
+    L.end_scores = o;
+    L.part_range = o; o = align_up(o + BHkv * RANGE_SPLIT_MAX * GMAX * PSTRIDE * 4, 256);
+    L.end_range = o;
+    L.part_list = o; o = align_up(o + BHq * LIST_MAX_SPLIT * PSTRIDE * 4, 256);
+    L.end_list = o;
+    L.tilebin = o; o = align_up(o + BHq * ntile * 2, 256);
+    L.lists = o; o = align_up(o + BHq * (size_t)d->N_max * 4, 256);
+    L.cands = o; o = align_up(o + BHq * (size_t)d->N_max * 8, 256);
+    L.total = o;
+    return L;
+}
+
+size_t op_bytes(const Layout &L, int op) {
+    switch (op) {
+        case RTP_OP_APPEND_INDEX_KEYS: return L.ctrl_end;
+        case RTP_OP_INDEX_SCORES: return L.end_scores;
+        case RTP_OP_LOCAL_DECODE:
+        case RTP_OP_DENSE_DECODE: return L.end_range;
+        case RTP_OP_SPARSE_DECODE: return L.end_list;
+        case RTP_OP_TOPP_SELECT:
+        case RTP_OP_DECODE_STEP: return L.total;
+        default: return 0;
+    }
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+int check_dims(const rtp_dims *d) {
+    if (!d) return RTP_ERR_INVALID_ARG;
+    if (d->B < 1 || d->H_q < 1 || d->H_kv < 1 || d->N_max < 1 || !d->seq_lens)
+        return RTP_ERR_INVALID_ARG;
+    if (d->N_max > 0x7fffffffLL - 64) return RTP_ERR_INVALID_ARG;
+    if (d->H_q % d->H_kv != 0) return RTP_ERR_INVALID_ARG;
+    if (d->d != D || d->r != R) return RTP_ERR_UNSUPPORTED;
+    if (d->H_q / d->H_kv > GMAX) return RTP_ERR_UNSUPPORTED;
+    if (d->H_kv > MAX_GROUPS) return RTP_ERR_UNSUPPORTED;
+    if ((d->kv_dtype != RTP_F32 && d->kv_dtype != RTP_BF16) ||
+        (d->idx_dtype != RTP_F32 && d->idx_dtype != RTP_BF16))
+        return RTP_ERR_UNSUPPORTED;
+    if ((size_t)d->B * d->H_q > MAX_LIST_HEADS) return RTP_ERR_UNSUPPORTED;
+    if (d->B > 65535 / MAX_GROUPS) return RTP_ERR_UNSUPPORTED;   // grid.y = B * groups
+    return RTP_OK;
+}
+
+int check_ws(const rtp_dims *d, void *ws, size_t ws_bytes, int op) {
+    if (!ws || ((uintptr_t)ws & 255u)) return RTP_ERR_WORKSPACE;
+    if (ws_bytes < op_bytes(make_layout(d), op)) return RTP_ERR_WORKSPACE;
+    return RTP_OK;
+}
+
+int check_head_class(const rtp_dims *d, const uint8_t *hc) {
+    if (!hc) return RTP_ERR_INVALID_ARG;
+    for (int g = 0; g < d->H_kv; ++g)
+        if (hc[g] != RTP_HEAD_LOCAL && hc[g] != RTP_HEAD_RETRIEVAL) return RTP_ERR_INVALID_ARG;
+    return RTP_OK;
+}
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 0 || dev >= 64) return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+// Launch helper: records profiling events around a launch when asked.
+struct Launcher {
+    cudaStream_t st;
+    rtp_prof *prof;
+    template <typename K, typename... Args>
+    int run(const char *name, K kernel, dim3 grid, dim3 block, Args... args) {
+        if (grid.x == 0 || grid.y == 0 || grid.z == 0) return RTP_OK;
+        int slot = -1;
+        if (prof && prof->count < prof->capacity && (!prof->filter || std::strstr(name, prof->filter))) {
+            slot = prof->count++;
+            prof->name[slot] = name;
+            if (cudaEventRecord((cudaEvent_t)prof->ev_start[slot], st) != cudaSuccess) return RTP_ERR_CUDA;
+        }
+        kernel<<<grid, block, 0, st>>>(args...);
+        if (cudaGetLastError() != cudaSuccess) return RTP_ERR_CUDA;
+        if (slot >= 0 && cudaEventRecord((cudaEvent_t)prof->ev_stop[slot], st) != cudaSuccess)
+            return RTP_ERR_CUDA;
+        return RTP_OK;
+    }
+};
+
+#define RTP_TRY(x)                      \
+    do {                                \
+        int _e = (x);                   \
+        if (_e != RTP_OK) return _e;    \
+    } while (0)
+
+float scale_or_default(float s) { return s > 0.0f ? s : 1.0f / std::sqrt((float)D); }
+
+// ----------------------------------------------------------------- selection
+struct SelPlan {
+    SelArgs a;
+    SelWs w;
+};
+
+SelPlan make_sel(const rtp_dims *d, const uint8_t *hc, char *ws, const Layout &L) {
+    SelPlan s{};
+    SelArgs &a = s.a;
+    a.B = d->B; a.H_q = d->H_q; a.H_kv = d->H_kv; a.G = d->H_q / d->H_kv;
+    a.N_max = d->N_max;
+    a.ntile = (int)((d->N_max + TILE - 1) / TILE);
+    a.seq_lens = d->seq_lens;
+    a.n_ret = 0;
+    for (int g = 0; g < d->H_kv; ++g)
+        if (hc[g] == RTP_HEAD_RETRIEVAL) a.ret_g[a.n_ret++] = g;
+    SelWs &w = s.w;
+    w.status = reinterpret_cast<uint32_t *>(ws + L.status);
+    w.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_hist);
+    w.list_cnt = reinterpret_cast<uint32_t *>(ws + L.list_cnt);
+    w.cand_cnt = reinterpret_cast<uint32_t *>(ws + L.cand_cnt);
+    w.hist = reinterpret_cast<double *>(ws + L.hist);
+    w.res = reinterpret_cast<Resolve *>(ws + L.res);
+    w.tilebin = reinterpret_cast<uint16_t *>(ws + L.tilebin);
+    w.cands = reinterpret_cast<unsigned long long *>(ws + L.cands);
+    w.qidx = reinterpret_cast<float *>(ws + L.qidx);
+    return s;
+}
+
+unsigned long long ret_mask(const rtp_dims *d, const uint8_t *hc) {
+    unsigned long long m = 0;
+    for (int g = 0; g < d->H_kv; ++g)
+        if (hc[g] == RTP_HEAD_RETRIEVAL) m |= 1ull << g;
+    return m;
+}
+
+int launch_qidx(Launcher &ln, const rtp_dims *d, const float *q, const float *W,
+                const uint8_t *hc, const SelPlan &s, float idx_scale) {
+    return ln.run("qidx", qidx_kernel, dim3(d->B * d->H_q), dim3(512), q, W, s.w.qidx, d->H_q,
+                  d->H_q / d->H_kv, ret_mask(d, hc), idx_scale);
+}
+
+// histogram + collect + finalize over the logit source
+template <typename Src, typename IT>
+int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s) {
+    const unsigned nchunk = (unsigned)((d->N_max + SEL_CHUNK - 1) / SEL_CHUNK);
+    const dim3 grid(nchunk, (unsigned)(d->B * s.a.n_ret));
+    RTP_TRY(ln.run("hist", hist_kernel<Src, IT>, grid, dim3(SEL_THREADS), s.a, s.w));
+    RTP_TRY(ln.run("collect", collect_kernel<Src, IT>, grid, dim3(SEL_THREADS), s.a, s.w));
+    RTP_TRY(ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)),
+                   dim3(SEL_THREADS), s.a, s.w));
+    return RTP_OK;
+}
+
+// ----------------------------------------------------------------- attention
+int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
+                 const uint8_t *hc, int want_class, bool dense, int window, int n_sink, float *out,
+                 char *ws, const Layout &L, float attn_scale) {
+    RangeArgs a{};
+    a.B = d->B; a.H_q = d->H_q; a.H_kv = d->H_kv; a.G = d->H_q / d->H_kv;
+    a.N_max = d->N_max; a.seq_lens = d->seq_lens;
+    a.n_grp = 0;
+    for (int g = 0; g < d->H_kv; ++g)
+        if (want_class < 0 || hc[g] == want_class) a.grp[a.n_grp++] = g;
+    if (a.n_grp == 0) return RTP_OK;
+    a.dense = dense ? 1 : 0;
+    a.window = window; a.n_sink = n_sink;
+    const long long Lmax = dense ? d->N_max : std::min<long long>(d->N_max, (long long)window + n_sink);
+    const long long chunks = (Lmax + RCH - 1) / RCH;
+    long long want = (2LL * num_sms() + (long long)d->B * a.n_grp - 1) / ((long long)d->B * a.n_grp);
+    a.n_split = (int)std::max(1LL, std::min(want, std::min(chunks, (long long)RANGE_SPLIT_MAX)));
+    a.scale_log2 = attn_scale * 1.4426950408889634f;
+    a.q = q; a.k = k; a.v = v; a.out = out;
+    a.part = reinterpret_cast<float *>(ws + L.part_range);
+    a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_range);
+    a.status = reinterpret_cast<uint32_t *>(ws + L.status);
+    const dim3 grid((unsigned)a.n_split, (unsigned)(d->B * a.n_grp));
+    const char *name = dense ? "dense_attn" : "local_attn";
+    if (d->kv_dtype == RTP_BF16)
+        return ln.run(name, range_attn_kernel<__nv_bfloat16>, grid, dim3(ATT_THREADS), a);
+    return ln.run(name, range_attn_kernel<float>, grid, dim3(ATT_THREADS), a);
+}
+
+int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
+                const int32_t *lists, const int32_t *counts, const uint8_t *hc, float *out,
+                char *ws, const Layout &L, float attn_scale) {
+    ListArgs a{};
+    a.B = d->B; a.H_q = d->H_q; a.H_kv = d->H_kv; a.G = d->H_q / d->H_kv;
+    a.N_max = d->N_max; a.seq_lens = d->seq_lens;
+    a.n_rq = 0;
+    for (int h = 0; h < d->H_q; ++h)
+        if (hc[h / a.G] == RTP_HEAD_RETRIEVAL) a.ret_h[a.n_rq++] = h;
+    if (a.n_rq == 0) return RTP_OK;
+    a.scale_log2 = attn_scale * 1.4426950408889634f;
+    a.q = q; a.k = k; a.v = v; a.lists = lists; a.counts = counts; a.out = out;
+    a.part = reinterpret_cast<float *>(ws + L.part_list);
+    a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_list);
+    a.status = reinterpret_cast<uint32_t *>(ws + L.status);
+    const long long max_items = (long long)d->B * a.n_rq *
+        std::min<long long>(LIST_MAX_SPLIT, (d->N_max + LCH - 1) / LCH);
+    const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(max_items, 4LL * num_sms()));
+    if (d->kv_dtype == RTP_BF16)
+        return ln.run("sparse_attn", list_attn_kernel<__nv_bfloat16>, dim3(grid), dim3(ATT_THREADS), a);
+    return ln.run("sparse_attn", list_attn_kernel<float>, dim3(grid), dim3(ATT_THREADS), a);
+}
+
+template <typename IT>
+int select_from_index(Launcher &ln, const rtp_dims *d, const SelPlan &s) {
+    return launch_select<FromIndex<IT>, IT>(ln, d, s);
+}
+
+}  // namespace
+
+// =========================================================================
+// public entry points
+// =========================================================================
+extern "C" {
+
+int rtp_version(void) { return 100; }
+
+const char *rtp_error_string(int code) {
+    switch (code) {
+        case RTP_OK: return "ok";
+        case RTP_ERR_INVALID_ARG: return "invalid argument";
+        case RTP_ERR_UNSUPPORTED: return "unsupported shape or dtype (d=128, r=16, G<=8, f32/bf16)";
+        case RTP_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case RTP_ERR_CUDA: return "CUDA error";
+        case RTP_ERR_TIMEOUT: return "device-side wait timed out";
+        case RTP_ERR_DEVICE_ARG: return "device-resident argument out of range";
+        case RTP_ERR_RANGE: return "index logit not finite or |z| >= 1024";
+        default: return "unknown error";
+    }
+}
+
+size_t rtp_workspace_size(const rtp_dims *dims, int op) {
+    if (check_dims(dims) != RTP_OK) return 0;
+    return op_bytes(make_layout(dims), op);
+}
+
+int rtp_workspace_init(void *ws, size_t ws_bytes, rtp_stream_t stream) {
+    // The control region is a prefix whose size depends on the shapes; the
+    // caller's buffer is at least that large, so zero min(ws_bytes, 64 MiB)
+    // conservatively covers it for every shape this library accepts.
+    if (!ws || ((uintptr_t)ws & 255u) || ws_bytes == 0) return RTP_ERR_WORKSPACE;
+    const size_t n = ws_bytes < ((size_t)64 << 20) ? ws_bytes : ((size_t)64 << 20);
+    if (cudaMemsetAsync(ws, 0, n, (cudaStream_t)stream) != cudaSuccess) return RTP_ERR_CUDA;
+    return RTP_OK;
+}
+
+int rtp_check(void *ws, rtp_stream_t stream) {
+    if (!ws) return RTP_ERR_WORKSPACE;
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return RTP_ERR_CUDA;
+    uint32_t st = 0;
+    if (cudaMemcpy(&st, ws, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return RTP_ERR_CUDA;
+    if (st != 0) {
+        if (cudaMemset(ws, 0, 4) != cudaSuccess) return RTP_ERR_CUDA;
+    }
+    return (int)st;
+}
+
+int rtp_append_index_keys(const rtp_dims *dims, const void *k_pre, int32_t T, const float *W_k_idx,
+                          const int32_t *pos, const uint8_t *head_class, void *kidx_cache,
+                          void *ws, size_t ws_bytes, rtp_stream_t stream) {
+    RTP_TRY(check_dims(dims));
+    if (!k_pre || !W_k_idx || !pos || !kidx_cache || T < 1) return RTP_ERR_INVALID_ARG;
+    if (T > dims->N_max) return RTP_ERR_INVALID_ARG;
+    if (!aligned16(k_pre) || !aligned16(W_k_idx) || !aligned16(kidx_cache)) return RTP_ERR_INVALID_ARG;
+    if (head_class) RTP_TRY(check_head_class(dims, head_class));
+    RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_APPEND_INDEX_KEYS));
+    const Layout L = make_layout(dims);
+    uint32_t *status = reinterpret_cast<uint32_t *>((char *)ws + L.status);
+    unsigned long long mask = head_class ? ret_mask(dims, head_class)
+                                         : (dims->H_kv >= 64 ? ~0ull : ((1ull << dims->H_kv) - 1));
+    Launcher ln{(cudaStream_t)stream, nullptr};
+    const dim3 grid((unsigned)((T + APP_WARPS - 1) / APP_WARPS), (unsigned)(dims->B * dims->H_kv));
+    const dim3 block(APP_WARPS * 32);
+    const bool kb = dims->kv_dtype == RTP_BF16, ib = dims->idx_dtype == RTP_BF16;
+    if (kb && ib)
+        return ln.run("append", append_kernel<__nv_bfloat16, __nv_bfloat16>, grid, block,
+                      (const __nv_bfloat16 *)k_pre, W_k_idx, pos, (__nv_bfloat16 *)kidx_cache,
+                      dims->H_kv, (int)T, (long long)dims->N_max, mask, status);
+    if (kb && !ib)
+        return ln.run("append", append_kernel<__nv_bfloat16, float>, grid, block,
+                      (const __nv_bfloat16 *)k_pre, W_k_idx, pos, (float *)kidx_cache, dims->H_kv,
+                      (int)T, (long long)dims->N_max, mask, status);
+    if (!kb && ib)
+        return ln.run("append", append_kernel<float, __nv_bfloat16>, grid, block,
+                      (const float *)k_pre, W_k_idx, pos, (__nv_bfloat16 *)kidx_cache, dims->H_kv,
+                      (int)T, (long long)dims->N_max, mask, status);
+    return ln.run("append", append_kernel<float, float>, grid, block, (const float *)k_pre, W_k_idx,
+                  pos, (float *)kidx_cache, dims->H_kv, (int)T, (long long)dims->N_max, mask, status);
+}
+
+int rtp_index_scores(const rtp_dims *dims, const rtp_opts *opts, const float *q,
+                     const float *W_q_idx, const void *kidx_cache, const uint8_t *head_class,
+                     float *z_out, void *ws, size_t ws_bytes, rtp_stream_t stream) {
+    RTP_TRY(check_dims(dims));
+    if (!q || !W_q_idx || !kidx_cache || !z_out) return RTP_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(W_q_idx) || !aligned16(kidx_cache) || !aligned16(z_out))
+        return RTP_ERR_INVALID_ARG;
+    RTP_TRY(check_head_class(dims, head_class));
+    RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_INDEX_SCORES));
+    const Layout L = make_layout(dims);
+    char *w = (char *)ws;
+    SelPlan s = make_sel(dims, head_class, w, L);
+    if (s.a.n_ret == 0) return RTP_OK;
+    s.a.kidx = kidx_cache;
+    Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
+    RTP_TRY(launch_qidx(ln, dims, q, W_q_idx, head_class, s, scale_or_default(opts ? opts->idx_scale : 0.f)));
+    const unsigned nchunk = (unsigned)((dims->N_max + SEL_CHUNK - 1) / SEL_CHUNK);
+    const dim3 grid(nchunk, (unsigned)(dims->B * s.a.n_ret));
+    if (dims->idx_dtype == RTP_BF16)
+        return ln.run("scores", scores_kernel<__nv_bfloat16>, grid, dim3(SEL_THREADS), s.a, s.w, z_out);
+    return ln.run("scores", scores_kernel<float>, grid, dim3(SEL_THREADS), s.a, s.w, z_out);
+}
+
+int rtp_topp_select(const rtp_dims *dims, const float *z, const uint8_t *head_class, float p,
+                    int32_t *idx_out, int32_t *count_out, float *mass_out, void *ws, size_t ws_bytes,
+                    rtp_stream_t stream) {
+    RTP_TRY(check_dims(dims));
+    if (!z || !idx_out || !count_out) return RTP_ERR_INVALID_ARG;
+    if (std::isnan(p)) return RTP_ERR_INVALID_ARG;
+    if (!aligned16(z)) return RTP_ERR_INVALID_ARG;
+    RTP_TRY(check_head_class(dims, head_class));
+    RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_TOPP_SELECT));
+    const Layout L = make_layout(dims);
+    SelPlan s = make_sel(dims, head_class, (char *)ws, L);
+    if (s.a.n_ret == 0) return RTP_OK;
+    s.a.z = z;
+    s.a.p = p;
+    s.a.lists = idx_out;
+    s.a.count_out = count_out;
+    s.a.mass_out = mass_out;
+    Launcher ln{(cudaStream_t)stream, nullptr};
+    return launch_select<FromBuffer, float>(ln, dims, s);
+}
+
+int rtp_sparse_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
+                      const void *k_cache, const void *v_cache, const int32_t *idx,
+                      const int32_t *count, const uint8_t *head_class, float *out, void *ws,
+                      size_t ws_bytes, rtp_stream_t stream) {
+    RTP_TRY(check_dims(dims));
+    if (!q_rope || !k_cache || !v_cache || !idx || !count || !out) return RTP_ERR_INVALID_ARG;
+    if (!aligned16(q_rope) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return RTP_ERR_INVALID_ARG;
+    RTP_TRY(check_head_class(dims, head_class));
+    RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_SPARSE_DECODE));
+    const Layout L = make_layout(dims);
+    Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
+    return launch_list(ln, dims, q_rope, k_cache, v_cache, idx, count, head_class, out, (char *)ws, L,
+                       scale_or_default(opts ? opts->attn_scale : 0.f));
+}
+
+int rtp_local_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
+                     const void *k_cache, const void *v_cache, const uint8_t *head_class,
+                     int32_t window, int32_t n_sink, float *out, void *ws, size_t ws_bytes,
+                     rtp_stream_t stream) {
+    RTP_TRY(check_dims(dims));
+    if (!q_rope || !k_cache || !v_cache || !out) return RTP_ERR_INVALID_ARG;
+    if (window < 1 || n_sink < 0) return RTP_ERR_INVALID_ARG;
+    if (!aligned16(q_rope) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return RTP_ERR_INVALID_ARG;
+    RTP_TRY(check_head_class(dims, head_class));
+    RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_LOCAL_DECODE));
+    const Layout L = make_layout(dims);
+    Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
+    return launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
+                        n_sink, out, (char *)ws, L, scale_or_default(opts ? opts->attn_scale : 0.f));
+}
+
+int rtp_dense_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
+                     const void *k_cache, const void *v_cache, float *out, void *ws, size_t ws_bytes,
+                     rtp_stream_t stream) {
+    RTP_TRY(check_dims(dims));
+    if (!q_rope || !k_cache || !v_cache || !out) return RTP_ERR_INVALID_ARG;
+    if (!aligned16(q_rope) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return RTP_ERR_INVALID_ARG;
+    RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_DENSE_DECODE));
+    const Layout L = make_layout(dims);
+    Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
+    return launch_range(ln, dims, q_rope, k_cache, v_cache, nullptr, -1, true, 1, 0, out, (char *)ws, L,
+                        scale_or_default(opts ? opts->attn_scale : 0.f));
+}
+
+int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, const float *q_rope,
+                    const void *k_cache, const void *v_cache, const void *kidx_cache,
+                    const float *W_q_idx, const uint8_t *head_class, float p, int32_t window,
+                    int32_t n_sink, float *out, void *ws, size_t ws_bytes, rtp_stream_t stream) {
+    RTP_TRY(check_dims(dims));
+    if (!q || !k_cache || !v_cache || !kidx_cache || !W_q_idx || !out) return RTP_ERR_INVALID_ARG;
+    if (std::isnan(p) || window < 1 || n_sink < 0) return RTP_ERR_INVALID_ARG;
+    if (!q_rope) q_rope = q;
+    if (!aligned16(q) || !aligned16(q_rope) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        !aligned16(kidx_cache) || !aligned16(W_q_idx) || !aligned16(out))
+        return RTP_ERR_INVALID_ARG;
+    RTP_TRY(check_head_class(dims, head_class));
+    RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_DECODE_STEP));
+    const Layout L = make_layout(dims);
+    char *w = (char *)ws;
+    Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
+    const float asc = scale_or_default(opts ? opts->attn_scale : 0.f);
+    const float isc = scale_or_default(opts ? opts->idx_scale : 0.f);
+
+    // local heads: window + sinks
+    RTP_TRY(launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
+                         n_sink, out, w, L, asc));
+    SelPlan s = make_sel(dims, head_class, w, L);
+    if (s.a.n_ret == 0) return RTP_OK;
+    if (p >= 1.0f) {
+        // every token is kept: the retrieval heads' attention is dense
+        return launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_RETRIEVAL, true, 1,
+                            0, out, w, L, asc);
+    }
+    s.a.kidx = kidx_cache;
+    s.a.p = p;
+    s.a.lists = opts && opts->sel_idx ? opts->sel_idx : reinterpret_cast<int32_t *>(w + L.lists);
+    s.a.count_out = opts && opts->sel_count ? opts->sel_count : reinterpret_cast<int32_t *>(w + L.counts);
+    s.a.mass_out = opts ? opts->sel_mass : nullptr;
+    RTP_TRY(launch_qidx(ln, dims, q, W_q_idx, head_class, s, isc));
+    if (dims->idx_dtype == RTP_BF16) {
+        RTP_TRY(select_from_index<__nv_bfloat16>(ln, dims, s));
+    } else {
+        RTP_TRY(select_from_index<float>(ln, dims, s));
+    }
+    return launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out, w,
+                       L, asc);
+}
+
+int rtp_prof_init(rtp_prof *prof, int32_t capacity) {
+    if (!prof || capacity < 1) return RTP_ERR_INVALID_ARG;
+    prof->capacity = 0;
+    prof->count = 0;
+    prof->filter = nullptr;
+    prof->ev_start = (void **)std::calloc((size_t)capacity, sizeof(void *));
+    prof->ev_stop = (void **)std::calloc((size_t)capacity, sizeof(void *));
+    prof->name = (const char **)std::calloc((size_t)capacity, sizeof(char *));
+    if (!prof->ev_start || !prof->ev_stop || !prof->name) return RTP_ERR_INVALID_ARG;
+    for (int i = 0; i < capacity; ++i) {
+        cudaEvent_t a, b;
+        if (cudaEventCreate(&a) != cudaSuccess || cudaEventCreate(&b) != cudaSuccess) return RTP_ERR_CUDA;
+        prof->ev_start[i] = a;
+        prof->ev_stop[i] = b;
+        prof->capacity = i + 1;
+    }
+    return RTP_OK;
+}
+
+int rtp_prof_elapsed(const rtp_prof *prof, int32_t slot, float *ms) {
+    if (!prof || !ms || slot < 0 || slot >= prof->count) return RTP_ERR_INVALID_ARG;
+    if (cudaEventElapsedTime(ms, (cudaEvent_t)prof->ev_start[slot], (cudaEvent_t)prof->ev_stop[slot]) !=
+        cudaSuccess)
+        return RTP_ERR_CUDA;
+    return RTP_OK;
+}
+
+int rtp_prof_destroy(rtp_prof *prof) {
+    if (!prof) return RTP_ERR_INVALID_ARG;
+    for (int i = 0; i < prof->capacity; ++i) {
+        if (prof->ev_start && prof->ev_start[i]) cudaEventDestroy((cudaEvent_t)prof->ev_start[i]);
+        if (prof->ev_stop && prof->ev_stop[i]) cudaEventDestroy((cudaEvent_t)prof->ev_stop[i]);
+    }
+    std::free(prof->ev_start);
+    std::free(prof->ev_stop);
+    std::free((void *)prof->name);
+    prof->ev_start = prof->ev_stop = nullptr;
+    prof->name = nullptr;
+    prof->capacity = prof->count = 0;
+    return RTP_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,410 @@
+// Decode attention kernels (sm_100a): exact softmax attention of one new
+// query per head over a set of cached rows, fp32 accumulation.
+//
+//   range_attn_kernel  all G query heads of a KV head over a row range
+//                      set: the sink rows plus the sliding window of a
+//                      local head ("Full Attention Strikes Back",
+//                      gist.science technical summary, Method section 1),
+//                      or every row (dense comparison kernel).  Each K/V row
+//                      is read once for the whole GQA group.
+//   list_attn_kernel   one retrieval head over its kept rows (same summary,
+//                      Method section 5: sparse decode gathers only the
+//                      selected K/V rows).  Persistent CTAs walk a work list
+//                      of (head, row slice) items built on the device from
+//                      the kept-set sizes.
+// Both split the rows over CTAs and merge the flash-decoding partials
+// (running max m, sum l, unnormalised o, in log2 units) in the last CTA to
+// finish, found with an arrival counter.
+#pragma once
+
+#include "rtp_common.cuh"
+
+namespace rtp {
+
+constexpr int ATT_THREADS = 256;
+constexpr int RCH = 256;               // rows per range sub-chunk (one per thread)
+constexpr int PSTRIDE = D + 2;         // partial record: m, l, o[D]
+constexpr int LCH = 256;               // rows per list item (target)
+constexpr int LIST_MAX_SPLIT = 64;     // items per head at most
+constexpr int MAX_GROUPS = 64;
+constexpr int MAX_RET_Q = 512;
+constexpr int MAX_LIST_HEADS = 4096;
+
+struct RangeArgs {
+    int B, H_q, H_kv, G;
+    long long N_max;
+    const int32_t *seq_lens;
+    int n_grp;
+    int grp[MAX_GROUPS];
+    int dense;
+    int window, n_sink;
+    int n_split;
+    float scale_log2;
+    const float *q;
+    const void *k;
+    const void *v;
+    float *out;
+    float *part;        // [B*H_kv][n_split][GMAX][PSTRIDE]
+    uint32_t *arrive;   // [B*H_kv]
+    uint32_t *status;
+};
+
+template <typename KT>
+__global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
+    __shared__ __align__(16) float qs[GMAX][D];
+    __shared__ float S[GMAX][RCH];
+    __shared__ float s_m[GMAX], s_l[GMAX], s_alpha[GMAX];
+    __shared__ float O[GMAX][D];
+    __shared__ int s_last;
+    const int b = blockIdx.y / a.n_grp;
+    const int g = a.grp[blockIdx.y % a.n_grp];
+    const int G = a.G;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t bg = (size_t)b * a.H_kv + g;
+    const size_t bh0 = (size_t)b * a.H_q + (size_t)g * G;
+
+    int N = a.seq_lens[b];
+    if (N < 1 || (long long)N > a.N_max) {
+        if (blockIdx.x == 0) {
+            if (tid == 0) set_status(a.status, RTP_ERR_DEVICE_ARG);
+            for (int i = tid; i < G * D; i += blockDim.x) a.out[bh0 * D + i] = 0.0f;
+        }
+        return;
+    }
+    const int s1 = a.dense ? N : min(a.n_sink, N);
+    const int w0 = a.dense ? N : max(s1, N - a.window);
+    const long long L = (long long)s1 + (N - w0);
+    const long long seg = (L + a.n_split - 1) / a.n_split;
+    const int n_active = (int)((L + seg - 1) / seg);
+    if ((int)blockIdx.x >= n_active) return;
+    const long long lo = (long long)blockIdx.x * seg;
+    const long long hi = min(L, lo + seg);
+
+    for (int i = tid; i < G * D; i += blockDim.x)
+        (&qs[0][0])[i] = a.q[bh0 * D + i] * a.scale_log2;
+    for (int i = tid; i < GMAX * D; i += blockDim.x) (&O[0][0])[i] = 0.0f;
+    if (tid < GMAX) { s_m[tid] = -INFINITY; s_l[tid] = 0.0f; }
+    __syncthreads();
+
+    const KT *kb = reinterpret_cast<const KT *>(a.k) + bg * a.N_max * D;
+    const KT *vb = reinterpret_cast<const KT *>(a.v) + bg * a.N_max * D;
+    float acc[GMAX][4];
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[h][i] = 0.0f;
+
+    for (long long c = lo; c < hi; c += RCH) {
+        // phase 1: one row per thread, logits for every head of the group
+        {
+            const long long j = c + tid;
+            float s[GMAX];
+#pragma unroll
+            for (int h = 0; h < GMAX; ++h) s[h] = 0.0f;
+            if (j < hi) {
+                const long long row = j < s1 ? j : w0 + (j - s1);
+                const KT *kr = kb + row * D;
+#pragma unroll 4
+                for (int piece = 0; piece < D / 8; ++piece) {
+                    float kx[8];
+                    Row<KT>::load8(kr + piece * 8, kx);
+#pragma unroll
+                    for (int h = 0; h < GMAX; ++h) {
+                        if (h < G) {
+                            const float4 q0 = *reinterpret_cast<const float4 *>(&qs[h][piece * 8]);
+                            const float4 q1 = *reinterpret_cast<const float4 *>(&qs[h][piece * 8 + 4]);
+                            float t = s[h];
+                            t = fmaf(q0.x, kx[0], t); t = fmaf(q0.y, kx[1], t);
+                            t = fmaf(q0.z, kx[2], t); t = fmaf(q0.w, kx[3], t);
+                            t = fmaf(q1.x, kx[4], t); t = fmaf(q1.y, kx[5], t);
+                            t = fmaf(q1.z, kx[6], t); t = fmaf(q1.w, kx[7], t);
+                            s[h] = t;
+                        }
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int h = 0; h < GMAX; ++h) s[h] = -INFINITY;
+            }
+#pragma unroll
+            for (int h = 0; h < GMAX; ++h)
+                if (h < G) S[h][tid] = s[h];
+        }
+        __syncthreads();
+        // phase 2: per-head running max and weights (warp h <-> head h)
+        if (warp < G) {
+            float mc = -INFINITY;
+            for (int i = lane; i < RCH; i += 32) mc = fmaxf(mc, S[warp][i]);
+            mc = warp_max(mc);
+            const float mold = s_m[warp];
+            const float mnew = fmaxf(mold, mc);
+            float lc = 0.0f;
+            if (mnew != -INFINITY) {
+                for (int i = lane; i < RCH; i += 32) {
+                    float e = exp2f(S[warp][i] - mnew);
+                    S[warp][i] = e;
+                    lc += e;
+                }
+            }
+            lc = warp_sum(lc);
+            if (lane == 0) {
+                const float al = (mnew == -INFINITY) ? 1.0f : exp2f(mold - mnew);
+                s_alpha[warp] = al;
+                s_l[warp] = s_l[warp] * al + lc;
+                s_m[warp] = mnew;
+            }
+        }
+        __syncthreads();
+        // phase 3: P.V, warp w owns rows w*32 .. w*32+31 of the sub-chunk
+        {
+#pragma unroll
+            for (int h = 0; h < GMAX; ++h) {
+                const float al = h < G ? s_alpha[h] : 0.0f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[h][i] *= al;
+            }
+            const long long rbase = c + warp * 32;
+            const int nr = (int)max(0LL, min(32LL, hi - rbase));
+#pragma unroll 8
+            for (int i = 0; i < nr; ++i) {
+                const long long j = rbase + i;
+                const long long row = j < s1 ? j : w0 + (j - s1);
+                float vx[4];
+                Row<KT>::load4(vb + row * D + lane * 4, vx);
+#pragma unroll
+                for (int h = 0; h < GMAX; ++h) {
+                    if (h < G) {
+                        const float pw = S[h][warp * 32 + i];
+                        acc[h][0] = fmaf(pw, vx[0], acc[h][0]);
+                        acc[h][1] = fmaf(pw, vx[1], acc[h][1]);
+                        acc[h][2] = fmaf(pw, vx[2], acc[h][2]);
+                        acc[h][3] = fmaf(pw, vx[3], acc[h][3]);
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+    // reduce the warps' accumulators and publish this CTA's partial
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h)
+        if (h < G)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) atomicAdd(&O[h][lane * 4 + i], acc[h][i]);
+    __syncthreads();
+    float *pp = a.part + (bg * a.n_split + blockIdx.x) * GMAX * PSTRIDE;
+    for (int i = tid; i < G * PSTRIDE; i += blockDim.x) {
+        const int h = i / PSTRIDE, e = i % PSTRIDE;
+        pp[i] = e == 0 ? s_m[h] : (e == 1 ? s_l[h] : O[h][e - 2]);
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&a.arrive[bg], 1u) == (unsigned)(n_active - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    const float *pb = a.part + bg * a.n_split * GMAX * PSTRIDE;
+    for (int i = tid; i < G * D; i += blockDim.x) {
+        const int h = i / D, d = i % D;
+        float M = -INFINITY;
+        for (int sp = 0; sp < n_active; ++sp) M = fmaxf(M, pb[(sp * GMAX + h) * PSTRIDE]);
+        float l = 0.0f, o = 0.0f;
+        for (int sp = 0; sp < n_active; ++sp) {
+            const float *r = pb + (sp * GMAX + h) * PSTRIDE;
+            const float wgt = exp2f(r[0] - M);
+            l = fmaf(r[1], wgt, l);
+            o = fmaf(r[2 + d], wgt, o);
+        }
+        a.out[(bh0 + h) * D + d] = o / l;
+    }
+    if (tid == 0) a.arrive[bg] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// list attention
+// ---------------------------------------------------------------------------
+struct ListArgs {
+    int B, H_q, H_kv, G;
+    long long N_max;
+    const int32_t *seq_lens;
+    int n_rq;                    // retrieval query heads per sequence
+    int ret_h[MAX_RET_Q];
+    float scale_log2;
+    const float *q;
+    const void *k;
+    const void *v;
+    const int32_t *lists;        // [B*H_q*N_max]
+    const int32_t *counts;       // [B*H_q]
+    float *out;
+    float *part;                 // [B*H_q][LIST_MAX_SPLIT][PSTRIDE] (indexed by item)
+    uint32_t *arrive;            // [B*H_q]
+    uint32_t *status;
+};
+
+__device__ __forceinline__ int list_items(int count) {
+    if (count <= 0) return 0;
+    return min(LIST_MAX_SPLIT, (count + LCH - 1) / LCH);
+}
+
+template <typename KT>
+__global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
+    __shared__ int pre[MAX_LIST_HEADS + 1];
+    __shared__ int s_scan[ATT_THREADS];
+    __shared__ float wm[ATT_THREADS / 32], wl[ATT_THREADS / 32];
+    __shared__ float wo[ATT_THREADS / 32][D];
+    __shared__ int s_last;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nh = a.B * a.n_rq;
+
+    // items per head -> exclusive prefix (each CTA builds its own copy)
+    {
+        const int per = (nh + ATT_THREADS - 1) / ATT_THREADS;
+        int loc = 0;
+        for (int i = 0; i < per; ++i) {
+            const int hi = tid * per + i;
+            int it = 0;
+            if (hi < nh) {
+                const int b = hi / a.n_rq, h = a.ret_h[hi % a.n_rq];
+                const int cnt = a.counts[(size_t)b * a.H_q + h];
+                const int N = a.seq_lens[b];
+                if (cnt >= 1 && N >= 1 && (long long)N <= a.N_max && cnt <= N) it = list_items(cnt);
+                pre[hi] = it;
+            }
+            loc += it;
+        }
+        s_scan[tid] = loc;
+        __syncthreads();
+        for (int o = 1; o < ATT_THREADS; o <<= 1) {
+            int v = tid >= o ? s_scan[tid - o] : 0;
+            __syncthreads();
+            s_scan[tid] += v;
+            __syncthreads();
+        }
+        int run = s_scan[tid] - loc;
+        for (int i = 0; i < per; ++i) {
+            const int hi = tid * per + i;
+            if (hi < nh) { const int it = pre[hi]; pre[hi] = run; run += it; }
+        }
+        if (tid == ATT_THREADS - 1) pre[nh] = s_scan[tid];
+        __syncthreads();
+    }
+    const int total = pre[nh];
+    // heads with nothing to attend over get zeros (and a status if invalid)
+    if (blockIdx.x == 0) {
+        for (int hi = warp; hi < nh; hi += ATT_THREADS / 32) {
+            if (pre[hi + 1] != pre[hi]) continue;
+            const int b = hi / a.n_rq, h = a.ret_h[hi % a.n_rq];
+            a.out[((size_t)b * a.H_q + h) * D + lane * 4 + 0] = 0.0f;
+            a.out[((size_t)b * a.H_q + h) * D + lane * 4 + 1] = 0.0f;
+            a.out[((size_t)b * a.H_q + h) * D + lane * 4 + 2] = 0.0f;
+            a.out[((size_t)b * a.H_q + h) * D + lane * 4 + 3] = 0.0f;
+            if (lane == 0) set_status(a.status, RTP_ERR_DEVICE_ARG);
+        }
+    }
+
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        // find the head of this item (upper bound in pre[0..nh])
+        int lo_h = 0, hi_h = nh;
+        while (hi_h - lo_h > 1) {
+            const int mid = (lo_h + hi_h) >> 1;
+            if (pre[mid] <= item) lo_h = mid; else hi_h = mid;
+        }
+        const int hix = lo_h;
+        const int b = hix / a.n_rq, h = a.ret_h[hix % a.n_rq];
+        const int g = h / a.G;
+        const size_t bh = (size_t)b * a.H_q + h;
+        const int cnt = a.counts[bh];
+        const int N = a.seq_lens[b];
+        const int nit = pre[hix + 1] - pre[hix];
+        const int sub = item - pre[hix];
+        const int per_item = (cnt + nit - 1) / nit;
+        const int r0 = sub * per_item, r1 = min(cnt, r0 + per_item);
+
+        const float4 q4 = *reinterpret_cast<const float4 *>(a.q + bh * D + lane * 4);
+        const float qx[4] = {q4.x * a.scale_log2, q4.y * a.scale_log2, q4.z * a.scale_log2,
+                             q4.w * a.scale_log2};
+        const KT *kb = reinterpret_cast<const KT *>(a.k) + ((size_t)b * a.H_kv + g) * a.N_max * D;
+        const KT *vb = reinterpret_cast<const KT *>(a.v) + ((size_t)b * a.H_kv + g) * a.N_max * D;
+        const int32_t *lst = a.lists + bh * a.N_max;
+        float m = -INFINITY, l = 0.0f, o[4] = {0.f, 0.f, 0.f, 0.f};
+        constexpr int U = 4;
+        for (int rr = r0 + warp * U; rr < r1; rr += (ATT_THREADS / 32) * U) {
+            float kx[U][4], vx[U][4];
+            bool ok[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int r = rr + u;
+                int t = r < r1 ? __ldg(lst + r) : -1;
+                ok[u] = r < r1 && t >= 0 && t < N;
+                if (r < r1 && !ok[u] && lane == 0) set_status(a.status, RTP_ERR_DEVICE_ARG);
+                if (ok[u]) {
+                    Row<KT>::load4(kb + (size_t)t * D + lane * 4, kx[u]);
+                    Row<KT>::load4(vb + (size_t)t * D + lane * 4, vx[u]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) kx[u][i] = vx[u][i] = 0.0f;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                float s = qx[0] * kx[u][0];
+                s = fmaf(qx[1], kx[u][1], s);
+                s = fmaf(qx[2], kx[u][2], s);
+                s = fmaf(qx[3], kx[u][3], s);
+                s = warp_sum(s);
+                if (!ok[u]) continue;
+                const float mn = fmaxf(m, s);
+                const float al = exp2f(m - mn);
+                const float pw = exp2f(s - mn);
+                l = l * al + pw;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o[i] = fmaf(pw, vx[u][i], o[i] * al);
+                m = mn;
+            }
+        }
+        // merge warps
+        if (lane == 0) { wm[warp] = m; wl[warp] = l; }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) wo[warp][lane * 4 + i] = o[i];
+        __syncthreads();
+        float *pp = a.part + ((size_t)item) * PSTRIDE;
+        if (tid < D) {
+            float M = -INFINITY;
+            for (int w = 0; w < ATT_THREADS / 32; ++w) M = fmaxf(M, wm[w]);
+            float ls = 0.0f, os = 0.0f;
+            if (M != -INFINITY) {
+                for (int w = 0; w < ATT_THREADS / 32; ++w) {
+                    const float wg = wm[w] == -INFINITY ? 0.0f : exp2f(wm[w] - M);
+                    ls = fmaf(wl[w], wg, ls);
+                    os = fmaf(wo[w][tid], wg, os);
+                }
+            }
+            pp[2 + tid] = os;
+            if (tid == 0) { pp[0] = M; pp[1] = ls; }
+        }
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) s_last = atomicAdd(&a.arrive[bh], 1u) == (unsigned)(nit - 1);
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            const float *pb = a.part + (size_t)pre[hix] * PSTRIDE;
+            if (tid < D) {
+                float M = -INFINITY;
+                for (int i = 0; i < nit; ++i) M = fmaxf(M, pb[i * PSTRIDE]);
+                float ls = 0.0f, os = 0.0f;
+                for (int i = 0; i < nit; ++i) {
+                    const float *r = pb + i * PSTRIDE;
+                    const float wg = r[0] == -INFINITY ? 0.0f : exp2f(r[0] - M);
+                    ls = fmaf(r[1], wg, ls);
+                    os = fmaf(r[2 + tid], wg, os);
+                }
+                a.out[bh * D + tid] = ls > 0.0f ? os / ls : 0.0f;
+            }
+            if (tid == 0) a.arrive[bh] = 0;
+        }
+        __syncthreads();
+    }
+}
+
+}  // namespace rtp

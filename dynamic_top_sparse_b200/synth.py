@@ -284,9 +284,10 @@ def make_case(spec: Spec | int, device="cpu", seed: int = 0, layer: int = 0) -> 
             kidx[b, g].index_add_(0, pd, add_idx.to(torch.float32).to(dev))
             k_cache[b, g].index_add_(0, pd, add_k.to(torch.float32).to(dev))
             needles[(b, h)] = np.sort(pos.numpy())
-    return Case(spec, layer, q.to(dev), None if q_rope is None else q_rope.to(dev),
-                k_cache.to(kvdt), v_cache, kidx.to(idt), W_q_idx.to(dev), W_k_idx.to(dev),
-                k_pre_new.to(dev), head_class, seq_lens.to(dev), spec.p, spec.window,
+    c = lambda t: t.contiguous()
+    return Case(spec, layer, c(q.to(dev)), None if q_rope is None else c(q_rope.to(dev)),
+                c(k_cache.to(kvdt)), c(v_cache), c(kidx.to(idt)), c(W_q_idx.to(dev)), c(W_k_idx.to(dev)),
+                c(k_pre_new.to(dev)), head_class, seq_lens.to(dev), spec.p, spec.window,
                 spec.n_sink, needles)
 
 

@@ -1,0 +1,276 @@
+/*
+ * rtp.h -- C ABI of librtp.so: the per-head sparse decode step of RTPurbo
+ * ("Full Attention Strikes Back: Transferring Full Attention into Sparse
+ * within Hundred Training Steps", arXiv 2605.16928) on NVIDIA B200 (sm_100a).
+ *
+ * What the step computes, per sequence b and query head h of one layer
+ * (query head h reads KV head g = h / G, G = H_q / H_kv):
+ *
+ *   - local KV heads (gist.science technical summary, Method section 1):
+ *     exact softmax attention over the attention-sink rows [0, n_sink) and
+ *     the sliding window [N - window, N), as one set;
+ *   - retrieval KV heads (same summary, Method sections 2, 3 and 5; arXiv
+ *     abstract): score every cached token with the 16-dim indexer,
+ *     z_t = idx_scale * (W_q_idx[h] . q_h) . kidx[b, g, t], with q_h the
+ *     pre-RoPE query and kidx the pre-RoPE index keys; turn the scores into
+ *     softmax mass pi_t; keep the smallest set of tokens, taken by
+ *     descending z (equal z: lower index first), whose mass reaches p; then
+ *     run exact full-dimension softmax attention of the post-RoPE query over
+ *     only the kept K/V rows (softmax renormalised over the kept set).
+ *
+ * The threshold is found without sorting, by a mass histogram over the
+ * order-preserving bits of z followed by an exact radix select inside the
+ * boundary bin (same summary, Method section 5: sort-free histogram
+ * threshold and bandwidth-optimised sparse decode).
+ *
+ * Conventions shared by every call
+ *   - Tensor pointers are DEVICE pointers owned by the caller, dense
+ *     row-major in the layouts given below, 16-byte aligned.  The library
+ *     never allocates or frees device memory and keeps no pointer after a
+ *     call returns.
+ *   - `head_class` is a HOST array of H_kv bytes (RTP_HEAD_LOCAL or
+ *     RTP_HEAD_RETRIEVAL), read during the call only: the split of heads is
+ *     fixed offline per layer (Method section 1), so launch shapes are built
+ *     from it on the host.
+ *   - `dims->seq_lens` is a DEVICE array of B int32 valid lengths N_b
+ *     (1 <= N_b <= N_max; the current token is row N_b - 1 and is already in
+ *     the caches).  A length out of range is reported by rtp_check() as
+ *     RTP_ERR_DEVICE_ARG and that sequence's outputs are written as zeros.
+ *   - Scratch memory comes from a caller workspace `ws` of at least
+ *     rtp_workspace_size(dims, op) bytes, 256-byte aligned, zeroed once by
+ *     rtp_workspace_init() before first use.  Calls that share a workspace
+ *     must be ordered on one stream.  The library keeps the workspace's
+ *     control words consistent between calls itself.
+ *   - Every call is asynchronous on `stream` (NULL = legacy default stream)
+ *     and never synchronises it; calls can be captured in a CUDA graph.
+ *   - Argument errors are detected on the host, before any launch, and
+ *     returned; nothing is launched then.  Errors found on the device are
+ *     recorded in the workspace status word and returned by rtp_check().
+ */
+#ifndef RTP_H_
+#define RTP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Every entry point below is exported from librtp.so (built with hidden
+ * default visibility). */
+#if defined(__GNUC__)
+#define RTP_API __attribute__((visibility("default")))
+#else
+#define RTP_API
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *rtp_stream_t;
+
+/* Return codes. */
+enum {
+    RTP_OK = 0,
+    RTP_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment, NaN p, ...   */
+    RTP_ERR_UNSUPPORTED = 2, /* d != 128, r != 16, G > 8, dtype not f32/bf16 */
+    RTP_ERR_WORKSPACE = 3,   /* ws NULL, misaligned or smaller than needed  */
+    RTP_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed        */
+    RTP_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out          */
+    RTP_ERR_DEVICE_ARG = 6,  /* device-resident argument out of range       */
+    RTP_ERR_RANGE = 7        /* an index logit was not finite or |z| >= 1024 */
+};
+
+/* Element types of the caches. */
+enum { RTP_F32 = 0, RTP_BF16 = 1 };
+
+/* Head classes (per KV head). */
+enum { RTP_HEAD_LOCAL = 0, RTP_HEAD_RETRIEVAL = 1 };
+
+/* Operation ids for rtp_workspace_size(). */
+enum {
+    RTP_OP_APPEND_INDEX_KEYS = 0,
+    RTP_OP_INDEX_SCORES = 1,
+    RTP_OP_TOPP_SELECT = 2,
+    RTP_OP_SPARSE_DECODE = 3,
+    RTP_OP_LOCAL_DECODE = 4,
+    RTP_OP_DENSE_DECODE = 5,
+    RTP_OP_DECODE_STEP = 6 /* covers every other op */
+};
+
+/* Shapes of one layer.  d must be 128 and r must be 16 on this path. */
+typedef struct rtp_dims {
+    int32_t B;                /* sequences                                  */
+    int32_t H_q;              /* query heads                                */
+    int32_t H_kv;             /* KV heads; H_q % H_kv == 0, H_q/H_kv <= 8   */
+    int32_t d;                /* head dim (128)                             */
+    int32_t r;                /* indexer dim (16)                           */
+    int32_t kv_dtype;         /* RTP_F32 or RTP_BF16: k/v caches, k_pre     */
+    int32_t idx_dtype;        /* RTP_F32 or RTP_BF16: index-key cache       */
+    int32_t reserved;
+    int64_t N_max;            /* cache capacity in rows (row stride)        */
+    const int32_t *seq_lens;  /* device [B]: valid rows N_b per sequence    */
+} rtp_dims;
+
+/* Optional launch accounting: when rtp_opts.prof is set, every kernel a
+ * call launches whose name contains `filter` (NULL: all) is bracketed by a
+ * pair of CUDA events recorded on the call's stream.  Slots are used from
+ * `count` upwards and `count` is advanced; recording stops at `capacity`.
+ * Create the events with rtp_prof_init(), read them with rtp_prof_elapsed()
+ * once the stream has reached them, release with rtp_prof_destroy(). */
+typedef struct rtp_prof {
+    int32_t capacity;
+    int32_t count;
+    void **ev_start;          /* cudaEvent_t[capacity]                     */
+    void **ev_stop;           /* cudaEvent_t[capacity]                     */
+    const char **name;        /* kernel name per slot (static strings)     */
+    const char *filter;
+} rtp_prof;
+
+/* Options; pass NULL for all defaults. */
+typedef struct rtp_opts {
+    float idx_scale;          /* index logit scale; 0 -> 1/sqrt(d)          */
+    float attn_scale;         /* attention scale;   0 -> 1/sqrt(d)          */
+    /* rtp_decode_step only, optional device outputs describing the kept
+     * sets (NULL: not written): */
+    int32_t *sel_idx;         /* [B, H_q, N_max]: kept token ids of each
+                                 retrieval head, first sel_count entries,
+                                 order unspecified                          */
+    int32_t *sel_count;       /* [B, H_q]: |S_h| (retrieval heads only)      */
+    float *sel_mass;          /* [B, H_q]: index-softmax mass of S_h         */
+    rtp_prof *prof;           /* optional launch accounting                 */
+} rtp_opts;
+
+/* Workspace bytes `op` needs for these shapes (0 on invalid dims).  The
+ * size for RTP_OP_DECODE_STEP is at least the size of every other op. */
+RTP_API size_t rtp_workspace_size(const rtp_dims *dims, int op);
+
+/* Zero the workspace's control region (status word, counters, histograms)
+ * on `stream`.  Call once after allocating a workspace. */
+RTP_API int rtp_workspace_init(void *ws, size_t ws_bytes, rtp_stream_t stream);
+
+/* Synchronise `stream`, then return (and clear) the first device-side error
+ * recorded in `ws` since the last check, or RTP_ERR_CUDA if the stream
+ * reports a CUDA error; RTP_OK otherwise. */
+RTP_API int rtp_check(void *ws, rtp_stream_t stream);
+
+/* Static description of a return code. */
+RTP_API const char *rtp_error_string(int code);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+RTP_API int rtp_version(void);
+
+/*
+ * a0 -- index keys of new tokens (Method section 2: the projector acts on
+ * the key before RoPE).  For every sequence b, retrieval KV head g and
+ * t < T:  kidx_cache[b, g, pos[b] + t, :] = W_k_idx[g] . k_pre[b, g, t, :],
+ * accumulated in fp32 and rounded to nearest-even into dims->idx_dtype.
+ * Rows of local KV heads are not written (they keep no index keys).
+ *   k_pre      [B, H_kv, T, d]   dims->kv_dtype (pre-RoPE keys)
+ *   W_k_idx    [H_kv, r, d]      fp32
+ *   pos        device [B] int32: first row to write; 0 <= pos, pos + T <=
+ *              N_max, else RTP_ERR_DEVICE_ARG (that sequence is skipped)
+ *   head_class host [H_kv] (NULL: every head is written)
+ *   kidx_cache [B, H_kv, N_max, r] dims->idx_dtype (written)
+ */
+RTP_API int rtp_append_index_keys(const rtp_dims *dims, const void *k_pre, int32_t T,
+                          const float *W_k_idx, const int32_t *pos,
+                          const uint8_t *head_class, void *kidx_cache,
+                          void *ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * a1 + a2 -- index logits (Method sections 2 and 3).  For retrieval heads:
+ * z_out[b, h, t] = idx_scale * (W_q_idx[h] . q[b, h]) . kidx[b, g, t] for
+ * t < N_b (fp32 accumulation).  Rows t >= N_b and local heads' rows are not
+ * written.
+ *   q          [B, H_q, d]       fp32 pre-RoPE queries
+ *   W_q_idx    [H_q, r, d]       fp32
+ *   kidx_cache [B, H_kv, N_max, r] dims->idx_dtype
+ *   z_out      [B, H_q, N_max]   fp32
+ */
+RTP_API int rtp_index_scores(const rtp_dims *dims, const rtp_opts *opts, const float *q,
+                     const float *W_q_idx, const void *kidx_cache,
+                     const uint8_t *head_class, float *z_out,
+                     void *ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * a3 + a4 + a5 -- dynamic top-p selection (Method section 3) from given
+ * logits z [B, H_q, N_max] fp32 (rows t < N_b of retrieval heads are read).
+ * Writes, for each retrieval head, the smallest set S of tokens taken by
+ * descending z (equal z: lower index first) whose softmax mass reaches p:
+ *   idx_out   [B, H_q, N_max] int32: S in the first count entries (any order)
+ *   count_out [B, H_q] int32:   |S| (>= 1)
+ *   mass_out  [B, H_q] fp32:    mass of S (optional, NULL: not written)
+ * p >= 1 keeps all N_b tokens; p <= 0 keeps the top token; p NaN is
+ * RTP_ERR_INVALID_ARG.  |z| must be finite and below 1024 (RTP_ERR_RANGE).
+ */
+RTP_API int rtp_topp_select(const rtp_dims *dims, const float *z, const uint8_t *head_class,
+                    float p, int32_t *idx_out, int32_t *count_out, float *mass_out,
+                    void *ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * a6 -- sparse decode (Method section 5): exact softmax attention of each
+ * retrieval head over only its listed rows,
+ * out[b, h] = sum_{t in S} softmax_S(attn_scale * q_rope[b,h] . k[b,g,t]) v[b,g,t].
+ *   q_rope     [B, H_q, d]       fp32 (post-RoPE queries)
+ *   k_cache, v_cache [B, H_kv, N_max, d] dims->kv_dtype
+ *   idx        [B, H_q, N_max] int32 row ids, first count[b, h] valid
+ *   count      [B, H_q] int32, 1 <= count <= N_b
+ *   out        [B, H_q, d] fp32: retrieval heads written, others untouched
+ * Ids outside [0, N_b) or counts out of range: RTP_ERR_DEVICE_ARG; the
+ * offending rows are skipped.
+ */
+RTP_API int rtp_sparse_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
+                      const void *k_cache, const void *v_cache, const int32_t *idx,
+                      const int32_t *count, const uint8_t *head_class, float *out,
+                      void *ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * a7 -- local heads (Method section 1): exact softmax attention over the
+ * sink rows [0, min(n_sink, N)) and the window rows [max(0, N - window), N)
+ * as one set.  window >= 1, n_sink >= 0.  Writes out[b, h] for the query
+ * heads of local KV heads only.
+ */
+RTP_API int rtp_local_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
+                     const void *k_cache, const void *v_cache, const uint8_t *head_class,
+                     int32_t window, int32_t n_sink, float *out,
+                     void *ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * Comparison kernel: dense decode attention of every query head over all
+ * N_b rows (what the sparse step is measured against).
+ */
+RTP_API int rtp_dense_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
+                     const void *k_cache, const void *v_cache, float *out,
+                     void *ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * The fused decode step (a1-a8): local heads as rtp_local_decode, retrieval
+ * heads as rtp_index_scores -> rtp_topp_select -> rtp_sparse_decode, without
+ * writing the logits to memory: the index keys are streamed once to build
+ * the mass histogram, re-read (skipping tiles that cannot hold a kept
+ * token) to compact the kept set, and the kept K/V rows are gathered once.
+ *   q          [B, H_q, d] fp32 pre-RoPE queries (indexer input)
+ *   q_rope     [B, H_q, d] fp32 post-RoPE queries (attention); NULL: q
+ *   k_cache, v_cache [B, H_kv, N_max, d] dims->kv_dtype
+ *   kidx_cache [B, H_kv, N_max, r] dims->idx_dtype
+ *   W_q_idx    [H_q, r, d] fp32
+ *   p, window, n_sink as above
+ *   out        [B, H_q, d] fp32 (every head written)
+ * With p >= 1 retrieval heads attend densely over all N_b rows.
+ */
+RTP_API int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q,
+                    const float *q_rope, const void *k_cache, const void *v_cache,
+                    const void *kidx_cache, const float *W_q_idx,
+                    const uint8_t *head_class, float p, int32_t window, int32_t n_sink,
+                    float *out, void *ws, size_t ws_bytes, rtp_stream_t stream);
+
+/* Launch accounting helpers (see rtp_prof). */
+RTP_API int rtp_prof_init(rtp_prof *prof, int32_t capacity);
+RTP_API int rtp_prof_elapsed(const rtp_prof *prof, int32_t slot, float *ms);
+RTP_API int rtp_prof_destroy(rtp_prof *prof);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTP_H_ */

@@ -216,8 +216,8 @@ def attend(q: np.ndarray, K: np.ndarray, V: np.ndarray, rows, scale: float) -> n
     rows = np.asarray(rows, dtype=np.int64)
     if rows.size == 0:
         raise ValueError("empty row set")
-    Kr = np.asarray(K, np.float64)[rows]
-    Vr = np.asarray(V, np.float64)[rows]
+    Kr = np.asarray(K)[rows].astype(np.float64)
+    Vr = np.asarray(V)[rows].astype(np.float64)
     s = scale * (Kr @ np.asarray(q, np.float64))
     w = np.exp(s - s.max())
     w /= w.sum()

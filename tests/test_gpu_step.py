@@ -1,0 +1,148 @@
+"""GPU parity of the fused decode step (rtp_decode_step) against the CPU
+oracle: small ragged cases, then the five workloads at full size (the
+oracle checks every retrieval head of sampled sequences/layers)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dynamic_top_sparse_b200 import ops, synth
+from tests.helpers import (OUT_TOL, OUT_TOL_SAME_SET, GpuCase, check_selection, gpu_set,
+                           np32, np64, oracle_kidx, within)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    ops.lib()
+
+
+def _compare(gc: GpuCase, out, sel_idx, sel_cnt, sel_mass, p, heads=None, with_current=True):
+    """Check every (or the listed) head of a case against the oracle."""
+    c = gc.c
+    kdt = c.spec.idx_dtype
+    kidx = oracle_kidx(gc, kdt, with_current)
+    q = np64(c.q)
+    qr = q if c.q_rope is None else np64(c.q_rope)
+    K, V, Wq = np32(c.k_cache), np32(c.v_cache), np64(c.W_q_idx)
+    tau = 1 / math.sqrt(128)
+    G = gc.H_q // gc.H_kv
+    o = out.cpu().numpy()
+    todo = heads if heads is not None else [(b, h) for b in range(gc.B) for h in range(gc.H_q)]
+    stats = []
+    for b, h in todo:
+        N = int(c.seq_lens[b])
+        g = h // G
+        if c.head_class[g] == oracle.HEAD_RETRIEVAL:
+            z = oracle.index_logits(oracle.query_index(q[b, h], Wq[h]), kidx[b, g, :N], tau)
+            sel = oracle.topp_select(z, p)
+            if p < 1.0:
+                ids = gpu_set(sel_idx, sel_cnt, b, h)
+                nd, mass = check_selection(ids, sel, p, f"b={b} h={h}")
+                assert abs(float(sel_mass[b, h]) - mass) < 1e-5
+                same = oracle.attend(qr[b, h], K[b, g, :N], V[b, g, :N], ids, tau)
+                within(o[b, h], same, OUT_TOL_SAME_SET, f"b={b} h={h} (same set)")
+                stats.append((len(ids), nd))
+            rows = sel.kept
+        else:
+            rows = oracle.local_rows(N, c.window, c.n_sink)
+        ref = oracle.attend(qr[b, h], K[b, g, :N], V[b, g, :N], rows, tau)
+        within(o[b, h], ref, OUT_TOL, f"b={b} h={h}")
+    return stats
+
+
+SMALL = [
+    dict(B=2, H_q=8, H_kv=2, N=1000, head_class=(1, 0), p=0.9),
+    dict(B=3, H_q=16, H_kv=2, N=5000, head_class=(1, 1), p=0.5, seq_lens=[5000, 17, 4097]),
+    dict(B=1, H_q=32, H_kv=4, N=9000, head_class=(0, 1, 1, 0), p=0.95, window=256, n_sink=0),
+    dict(B=2, H_q=4, H_kv=4, N=3000, head_class=(1, 0, 1, 0), p=0.7, kv_dtype="f32", idx_dtype="f32"),
+    dict(B=1, H_q=8, H_kv=1, N=1, head_class=(1,), p=0.9),
+    dict(B=2, H_q=8, H_kv=1, N=40, head_class=(1,), p=1e-9, seq_lens=[40, 2]),
+    dict(B=1, H_q=6, H_kv=2, N=2049, head_class=(1, 0), p=0.99, needles="none"),
+    dict(B=1, H_q=8, H_kv=1, N=4096, head_class=(1,), p=0.9, needle_scale=4.0, needles_per_head=40),
+]
+
+
+@pytest.mark.parametrize("k", range(len(SMALL)))
+def test_step_small(k):
+    kw = dict(SMALL[k])
+    p = kw.pop("p")
+    spec = synth.small_spec(**kw, name=f"small{k}")
+    gc = GpuCase(synth.make_case(spec))
+    gc.append_current()
+    out, si, sc, sm = gc.step(p)
+    _compare(gc, out, si, sc, sm, p)
+
+
+def test_step_p_one_equals_dense():
+    spec = synth.small_spec(B=2, H_q=16, H_kv=2, N=7000, head_class=(1, 1), seq_lens=[7000, 3000])
+    gc = GpuCase(synth.make_case(spec))
+    out, _, _, _ = gc.step(1.0, want_sel=False)
+    dense = torch.zeros_like(out)
+    ops.dense_decode(gc.dims, gc.q_rope, gc.k, gc.v, dense, gc.ws)
+    assert gc.ws.check() == 0
+    within(out.cpu().numpy(), dense.cpu().numpy(), 1e-5, "p=1 vs dense")
+    _compare(gc, out, None, None, None, 1.0, with_current=False)
+
+
+def test_step_repeatable_on_one_workspace():
+    spec = synth.small_spec(B=2, H_q=16, H_kv=2, N=6000, head_class=(1, 0))
+    gc = GpuCase(synth.make_case(spec))
+    a = gc.step(0.9)
+    b = gc.step(0.9)
+    for x, y in ((a[2], b[2]),):
+        assert torch.equal(x, y)
+    within(a[0].cpu().numpy(), b[0].cpu().numpy(), 1e-6, "repeat")
+
+
+# --------------------------------------------------------------- workloads
+
+def _workload(cfg, ps, sample_heads=None, layer=0):
+    c = synth.make_case(cfg, device="cuda", layer=layer)
+    gc = GpuCase(c)
+    gc.append_current()
+    res = {}
+    for p in ps:
+        out, si, sc, sm = gc.step(p, want_sel=p < 1.0)
+        heads = sample_heads(p) if sample_heads else None
+        res[p] = _compare(gc, out, si, sc, sm, p, heads=heads)
+    return res
+
+
+def test_cfg1_4096_fp32():
+    _workload(1, [0.9])
+
+
+@pytest.mark.slow
+def test_cfg2_64k():
+    _workload(2, [0.9])
+
+
+@pytest.mark.slow
+def test_cfg3_512k():
+    _workload(3, [0.9])
+
+
+@pytest.mark.slow
+def test_cfg5_1m_p_sweep():
+    # p = 0.9: every head; the other p: four heads per KV group (peaked to
+    # broad) plus the dense p = 1.0 case on a sample.
+    def sample(p):
+        if p == 0.9:
+            return None
+        return [(0, h) for h in (0, 5, 9, 14, 18, 22, 27, 31)]
+    _workload(5, [0.8, 0.9, 0.95, 1.0], sample_heads=sample)
+
+
+@pytest.mark.slow
+def test_cfg4_128k_b8_sampled_layers():
+    # config 4 runs 48 layers x 8 sequences; the oracle checks two layers
+    # fully (all 8 sequences, all heads) and the launch shape is the same
+    # for every layer.
+    for layer in (0, 29):
+        _workload(4, [0.9], layer=layer)

@@ -1,0 +1,69 @@
+"""The multi-GPU host logic (sharding, barrier, max-over-ranks timing) on
+world_size-2 gloo ranks on CPU."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from dynamic_top_sparse_b200 import dist as rdist
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rdist.barrier(world)
+        t = rdist.allreduce_max(1.5 + rank, world)
+        s = rdist.allreduce_sum(10.0, world)
+        mine = rdist.shard_units(8, 4, world, rank)
+        gathered = [None] * world
+        dist.all_gather_object(gathered, mine)
+        q.put((rank, t, s, gathered))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, t, s, gathered in res:
+        assert t == 2.5          # slowest rank
+        assert s == 20.0
+        flat = [u for part in gathered for u in part]
+        assert sorted(flat) == [(b, g) for b in range(8) for g in range(4)]   # a partition
+        assert len(set(flat)) == len(flat)
+
+
+@pytest.mark.parametrize("B,H_kv,world", [(8, 4, 8), (1, 4, 4), (3, 4, 2), (1, 4, 8), (2, 1, 4)])
+def test_shard_units_partition(B, H_kv, world):
+    parts = [rdist.shard_units(B, H_kv, world, r) for r in range(world)]
+    flat = [u for p in parts for u in p]
+    assert sorted(flat) == [(b, g) for b in range(B) for g in range(H_kv)]
+    sizes = [len(p) for p in parts]
+    assert max(sizes) - min(sizes) <= max(1, H_kv)
+
+
+def test_shard_units_rejects_bad_rank():
+    with pytest.raises(ValueError):
+        rdist.shard_units(2, 2, 2, 2)
