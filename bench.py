@@ -128,6 +128,15 @@ class Clocks:
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+def ctypes_elapsed(prof, slot):
+    import ctypes
+    ms = ctypes.c_float()
+    rc = ops.lib().rtp_prof_elapsed(ctypes.byref(prof.p), slot, ctypes.byref(ms))
+    if rc != 0:
+        raise ops.RtpError(rc, "rtp_prof_elapsed")
+    return ms.value
+
+
 # ------------------------------------------------------------------ workload
 
 class Layer:
@@ -284,15 +293,35 @@ def run_ours(args, rank, world, dev):
     ms_per_step = ms_max / args.steps
     value = world * args.steps / (ms_max / 1e3)
 
-    # dominant kernel: the index scan (histogram pass); direct launches with
-    # events on the library's stream
-    n_prof = min(args.steps, args.prof_steps)
-    pr = ops.Profiler(n_prof * spec.layers + 8, filter="hist")
-    for i in range(n_prof):
-        step(reps[i % n_rep], prof=pr)
+    # per-kernel device times: the step captured with event-record nodes
+    # around every kernel (one graph per replica, distinct event slots),
+    # replayed with a sync after each replay to read the slots
+    per_step_slots = launches_per_step + 4
+    pr = ops.Profiler(per_step_slots * n_rep)
+    pgraphs = []
+    for R in reps:
+        g = torch.cuda.CUDAGraph()
+        first = pr.p.count
+        with torch.cuda.graph(g):
+            step(R, prof=pr)
+        pgraphs.append((g, first, pr.p.count))
     torch.cuda.synchronize()
-    hist_ms = [t for name, t in pr.times() if name == "hist"]
+    n_prof = max(1, min(args.steps, args.prof_steps))
+    breakdown = {}
+    for i in range(n_prof + n_rep):
+        g, lo, hi = pgraphs[i % n_rep]
+        g.replay()
+        torch.cuda.synchronize()
+        if i < n_rep:
+            continue          # first pass over each graph: warm-up
+        for slot in range(lo, hi):
+            name = pr.p.name[slot].decode()
+            ms_ = ctypes_elapsed(pr, slot)
+            breakdown.setdefault(name, []).append(ms_)
     pr.close()
+    hist_ms = breakdown.get("hist", [])
+    breakdown = {k: {"avg_ms": float(np.mean(v)), "launches_per_step": len(v) / n_prof}
+                 for k, v in breakdown.items()}
     hist_avg_ms = float(np.mean(hist_ms)) if hist_ms else None
     hbm_peak, peak_src = peaks()
     idx_b = index_bytes(spec, layers0)
@@ -398,6 +427,7 @@ def run_ours(args, rank, world, dev):
                      else "fallback 6650 GB/s"},
         "dense": {"ms_per_step": dense_ms, "speedup_sparse_vs_dense": dense_ms / ms_per_step,
                   "bytes_per_step": int(sum(2 * L.k.numel() * L.k.element_size() for L in reps[0]))},
+        "kernels": breakdown,
         "gpu_launches": int(launches_per_step * args.steps),
         "launches_per_step": launches_per_step,
         "clocks": clocks.report(),

@@ -11,6 +11,7 @@
 #include "rtp_select.cuh"
 #include "rtp_attend.cuh"
 #include "rtp_append.cuh"
+#include "rtp_gqa_mma.cuh"
 
 using namespace rtp;
 
@@ -22,9 +23,9 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace regions, in the order ops need them (each op needs a prefix).
 struct Layout {
-    size_t status, arrive_hist, arrive_range, arrive_list, list_cnt, cand_cnt, hist;
+    size_t status, arrive_scan, arrive_range, arrive_list, cand_cnt, list_cnt, fin_arrive, hist;
     size_t ctrl_end;
-    size_t res, qidx, counts, mass;
+    size_t res, qidx, counts, item_pre;
     size_t end_scores;      // append / index_scores need up to here
     size_t part_range;
     size_t end_range;       // local / dense
@@ -34,23 +35,26 @@ struct Layout {
     size_t total;           // topp_select / decode_step
 };
 
+constexpr int SCAN_CTAS_MAX = 1024;
+
 Layout make_layout(const rtp_dims *d) {
     Layout L{};
     const size_t BHq = (size_t)d->B * d->H_q, BHkv = (size_t)d->B * d->H_kv;
     const size_t ntile = (size_t)((d->N_max + TILE - 1) / TILE);
     size_t o = 0;
     L.status = o; o += 256;
-    L.arrive_hist = o; o = align_up(o + BHkv * 4, 256);
+    L.arrive_scan = o; o = align_up(o + BHkv * 4, 256);
     L.arrive_range = o; o = align_up(o + BHkv * 4, 256);
     L.arrive_list = o; o = align_up(o + BHq * 4, 256);
-    L.list_cnt = o; o = align_up(o + BHq * 4, 256);
     L.cand_cnt = o; o = align_up(o + BHq * 4, 256);
+    L.list_cnt = o; o = align_up(o + BHq * 4, 256);
+    L.fin_arrive = o; o = align_up(o + 4, 256);
     L.hist = o; o = align_up(o + BHq * NBIN * 8, 256);
     L.ctrl_end = o;
     L.res = o; o = align_up(o + BHq * sizeof(Resolve), 256);
     L.qidx = o; o = align_up(o + BHq * R * 4, 256);
     L.counts = o; o = align_up(o + BHq * 4, 256);
-    L.mass = o; o = align_up(o + BHq * 4, 256);
+    L.item_pre = o; o = align_up(o + (BHq + 1) * 4, 256);
     L.end_scores = o;
     L.part_range = o; o = align_up(o + BHkv * RANGE_SPLIT_MAX * GMAX * PSTRIDE * 4, 256);
     L.end_range = o;
@@ -125,19 +129,32 @@ int num_sms() {
 struct Launcher {
     cudaStream_t st;
     rtp_prof *prof;
+    // Inside stream capture an event becomes a timestamp node of the graph
+    // only when recorded as external.
+    cudaError_t record(void *ev, bool capturing) {
+        return capturing ? cudaEventRecordWithFlags((cudaEvent_t)ev, st, cudaEventRecordExternal)
+                         : cudaEventRecord((cudaEvent_t)ev, st);
+    }
     template <typename K, typename... Args>
     int run(const char *name, K kernel, dim3 grid, dim3 block, Args... args) {
+        return run_smem(name, kernel, grid, block, 0, args...);
+    }
+    template <typename K, typename... Args>
+    int run_smem(const char *name, K kernel, dim3 grid, dim3 block, size_t smem, Args... args) {
         if (grid.x == 0 || grid.y == 0 || grid.z == 0) return RTP_OK;
         int slot = -1;
+        bool capturing = false;
         if (prof && prof->count < prof->capacity && (!prof->filter || std::strstr(name, prof->filter))) {
             slot = prof->count++;
             prof->name[slot] = name;
-            if (cudaEventRecord((cudaEvent_t)prof->ev_start[slot], st) != cudaSuccess) return RTP_ERR_CUDA;
+            cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+            if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return RTP_ERR_CUDA;
+            capturing = cs == cudaStreamCaptureStatusActive;
+            if (record(prof->ev_start[slot], capturing) != cudaSuccess) return RTP_ERR_CUDA;
         }
-        kernel<<<grid, block, 0, st>>>(args...);
+        kernel<<<grid, block, smem, st>>>(args...);
         if (cudaGetLastError() != cudaSuccess) return RTP_ERR_CUDA;
-        if (slot >= 0 && cudaEventRecord((cudaEvent_t)prof->ev_stop[slot], st) != cudaSuccess)
-            return RTP_ERR_CUDA;
+        if (slot >= 0 && record(prof->ev_stop[slot], capturing) != cudaSuccess) return RTP_ERR_CUDA;
         return RTP_OK;
     }
 };
@@ -156,6 +173,19 @@ struct SelPlan {
     SelWs w;
 };
 
+// CTAs per (b, g) for the scan: two 512-thread CTAs per SM over the whole
+// GPU (one wave), each on a contiguous, tile-aligned token range.
+void plan_chunks(SelArgs &a, long long N_max) {
+    const long long groups = (long long)a.B * std::max(a.n_ret, 1);
+    long long ctas = (2LL * num_sms() + groups - 1) / groups;
+    const long long tiles = (N_max + TILE - 1) / TILE;
+    ctas = std::max(1LL, std::min({ctas, tiles, (long long)SCAN_CTAS_MAX}));
+    long long chunk = (tiles + ctas - 1) / ctas * TILE;
+    ctas = (N_max + chunk - 1) / chunk;
+    a.ctas = (int)ctas;
+    a.chunk = chunk;
+}
+
 SelPlan make_sel(const rtp_dims *d, const uint8_t *hc, char *ws, const Layout &L) {
     SelPlan s{};
     SelArgs &a = s.a;
@@ -166,17 +196,55 @@ SelPlan make_sel(const rtp_dims *d, const uint8_t *hc, char *ws, const Layout &L
     a.n_ret = 0;
     for (int g = 0; g < d->H_kv; ++g)
         if (hc[g] == RTP_HEAD_RETRIEVAL) a.ret_g[a.n_ret++] = g;
+    plan_chunks(a, d->N_max);
     SelWs &w = s.w;
     w.status = reinterpret_cast<uint32_t *>(ws + L.status);
-    w.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_hist);
-    w.list_cnt = reinterpret_cast<uint32_t *>(ws + L.list_cnt);
+    w.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_scan);
     w.cand_cnt = reinterpret_cast<uint32_t *>(ws + L.cand_cnt);
+    w.list_cnt = reinterpret_cast<uint32_t *>(ws + L.list_cnt);
     w.hist = reinterpret_cast<double *>(ws + L.hist);
     w.res = reinterpret_cast<Resolve *>(ws + L.res);
     w.tilebin = reinterpret_cast<uint16_t *>(ws + L.tilebin);
     w.cands = reinterpret_cast<unsigned long long *>(ws + L.cands);
     w.qidx = reinterpret_cast<float *>(ws + L.qidx);
+    w.fin_arrive = reinterpret_cast<uint32_t *>(ws + L.fin_arrive);
     return s;
+}
+
+// scan + collect + finalize over a logit source
+template <typename Src>
+int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s) {
+    const dim3 grid((unsigned)s.a.ctas, (unsigned)(d->B * s.a.n_ret));
+    RTP_TRY(ln.run("hist", scan_kernel<Src>, grid, dim3(SCAN_THREADS), s.a, s.w));
+    RTP_TRY(ln.run("collect", collect_kernel<Src>, grid, dim3(COL_THREADS), s.a, s.w));
+    RTP_TRY(ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)),
+                   dim3(FIN_THREADS), s.a, s.w));
+    return RTP_OK;
+}
+
+int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s) {
+    if (d->idx_dtype != RTP_BF16) return launch_select<SrcSimt<float>>(ln, d, s);
+    // bf16 index keys: the TMA-ring scan, one CTA per SM over all groups
+    static int attr_set[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(scan_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM) !=
+            cudaSuccess)
+            return RTP_ERR_CUDA;
+        attr_set[dev] = 1;
+    }
+    const long long groups = (long long)d->B * s.a.n_ret;
+    const long long tiles = (d->N_max + TILE - 1) / TILE;
+    long long ctas = std::max(1LL, std::min((long long)num_sms() / std::max(groups, 1LL), tiles));
+    s.a.chunk = (tiles + ctas - 1) / ctas * TILE;
+    s.a.ctas = (int)((d->N_max + s.a.chunk - 1) / s.a.chunk);
+    const dim3 grid((unsigned)s.a.ctas, (unsigned)groups);
+    RTP_TRY(ln.run_smem("hist", scan_tma_kernel, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w));
+    RTP_TRY(ln.run("collect", collect_kernel<SrcMma>, grid, dim3(COL_THREADS), s.a, s.w));
+    RTP_TRY(ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)), dim3(FIN_THREADS),
+                   s.a, s.w));
+    return RTP_OK;
 }
 
 unsigned long long ret_mask(const rtp_dims *d, const uint8_t *hc) {
@@ -186,21 +254,24 @@ unsigned long long ret_mask(const rtp_dims *d, const uint8_t *hc) {
     return m;
 }
 
-int launch_qidx(Launcher &ln, const rtp_dims *d, const float *q, const float *W,
-                const uint8_t *hc, const SelPlan &s, float idx_scale) {
-    return ln.run("qidx", qidx_kernel, dim3(d->B * d->H_q), dim3(512), q, W, s.w.qidx, d->H_q,
-                  d->H_q / d->H_kv, ret_mask(d, hc), idx_scale);
-}
+// Side stream per device and host thread, for work that overlaps the
+// retrieval pipeline (local heads).  Created on first use.
+struct Side {
+    cudaStream_t st = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
 
-// histogram + collect + finalize over the logit source
-template <typename Src, typename IT>
-int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s) {
-    const unsigned nchunk = (unsigned)((d->N_max + SEL_CHUNK - 1) / SEL_CHUNK);
-    const dim3 grid(nchunk, (unsigned)(d->B * s.a.n_ret));
-    RTP_TRY(ln.run("hist", hist_kernel<Src, IT>, grid, dim3(SEL_THREADS), s.a, s.w));
-    RTP_TRY(ln.run("collect", collect_kernel<Src, IT>, grid, dim3(SEL_THREADS), s.a, s.w));
-    RTP_TRY(ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)),
-                   dim3(SEL_THREADS), s.a, s.w));
+int side_stream(Side *&out) {
+    static thread_local Side sides[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
+    Side &sd = sides[dev];
+    if (!sd.st) {
+        if (cudaStreamCreateWithFlags(&sd.st, cudaStreamNonBlocking) != cudaSuccess) return RTP_ERR_CUDA;
+        if (cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming) != cudaSuccess) return RTP_ERR_CUDA;
+        if (cudaEventCreateWithFlags(&sd.join, cudaEventDisableTiming) != cudaSuccess) return RTP_ERR_CUDA;
+    }
+    out = &sd;
     return RTP_OK;
 }
 
@@ -218,8 +289,10 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
     a.dense = dense ? 1 : 0;
     a.window = window; a.n_sink = n_sink;
     const long long Lmax = dense ? d->N_max : std::min<long long>(d->N_max, (long long)window + n_sink);
-    const long long chunks = (Lmax + RCH - 1) / RCH;
-    long long want = (2LL * num_sms() + (long long)d->B * a.n_grp - 1) / ((long long)d->B * a.n_grp);
+    const int rows_min = 256;
+    const int per_sm = 2;
+    const long long chunks = (Lmax + rows_min - 1) / rows_min;
+    long long want = ((long long)per_sm * num_sms() + (long long)d->B * a.n_grp - 1) / ((long long)d->B * a.n_grp);
     a.n_split = (int)std::max(1LL, std::min(want, std::min(chunks, (long long)RANGE_SPLIT_MAX)));
     a.scale_log2 = attn_scale * 1.4426950408889634f;
     a.q = q; a.k = k; a.v = v; a.out = out;
@@ -229,13 +302,13 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
     const dim3 grid((unsigned)a.n_split, (unsigned)(d->B * a.n_grp));
     const char *name = dense ? "dense_attn" : "local_attn";
     if (d->kv_dtype == RTP_BF16)
-        return ln.run(name, range_attn_kernel<__nv_bfloat16>, grid, dim3(ATT_THREADS), a);
+        return ln.run(name, gqa_mma_attn_kernel, grid, dim3(GQ_THREADS), a);
     return ln.run(name, range_attn_kernel<float>, grid, dim3(ATT_THREADS), a);
 }
 
 int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
                 const int32_t *lists, const int32_t *counts, const uint8_t *hc, float *out,
-                char *ws, const Layout &L, float attn_scale) {
+                char *ws, const Layout &L, float attn_scale, const int32_t *item_pre = nullptr) {
     ListArgs a{};
     a.B = d->B; a.H_q = d->H_q; a.H_kv = d->H_kv; a.G = d->H_q / d->H_kv;
     a.N_max = d->N_max; a.seq_lens = d->seq_lens;
@@ -245,20 +318,16 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
     if (a.n_rq == 0) return RTP_OK;
     a.scale_log2 = attn_scale * 1.4426950408889634f;
     a.q = q; a.k = k; a.v = v; a.lists = lists; a.counts = counts; a.out = out;
+    a.item_pre = item_pre;
     a.part = reinterpret_cast<float *>(ws + L.part_list);
     a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_list);
     a.status = reinterpret_cast<uint32_t *>(ws + L.status);
     const long long max_items = (long long)d->B * a.n_rq *
         std::min<long long>(LIST_MAX_SPLIT, (d->N_max + LCH - 1) / LCH);
-    const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(max_items, 4LL * num_sms()));
+    const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(max_items, 2LL * num_sms()));
     if (d->kv_dtype == RTP_BF16)
         return ln.run("sparse_attn", list_attn_kernel<__nv_bfloat16>, dim3(grid), dim3(ATT_THREADS), a);
     return ln.run("sparse_attn", list_attn_kernel<float>, dim3(grid), dim3(ATT_THREADS), a);
-}
-
-template <typename IT>
-int select_from_index(Launcher &ln, const rtp_dims *d, const SelPlan &s) {
-    return launch_select<FromIndex<IT>, IT>(ln, d, s);
 }
 
 }  // namespace
@@ -279,7 +348,7 @@ const char *rtp_error_string(int code) {
         case RTP_ERR_CUDA: return "CUDA error";
         case RTP_ERR_TIMEOUT: return "device-side wait timed out";
         case RTP_ERR_DEVICE_ARG: return "device-resident argument out of range";
-        case RTP_ERR_RANGE: return "index logit not finite or |z| >= 1024";
+        case RTP_ERR_RANGE: return "index logit not finite";
         default: return "unknown error";
     }
 }
@@ -357,13 +426,14 @@ int rtp_index_scores(const rtp_dims *dims, const rtp_opts *opts, const float *q,
     SelPlan s = make_sel(dims, head_class, w, L);
     if (s.a.n_ret == 0) return RTP_OK;
     s.a.kidx = kidx_cache;
+    s.a.q = q;
+    s.a.Wq = W_q_idx;
+    s.a.idx_scale = scale_or_default(opts ? opts->idx_scale : 0.f);
     Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
-    RTP_TRY(launch_qidx(ln, dims, q, W_q_idx, head_class, s, scale_or_default(opts ? opts->idx_scale : 0.f)));
-    const unsigned nchunk = (unsigned)((dims->N_max + SEL_CHUNK - 1) / SEL_CHUNK);
-    const dim3 grid(nchunk, (unsigned)(dims->B * s.a.n_ret));
+    const dim3 grid((unsigned)s.a.ctas, (unsigned)(dims->B * s.a.n_ret));
     if (dims->idx_dtype == RTP_BF16)
-        return ln.run("scores", scores_kernel<__nv_bfloat16>, grid, dim3(SEL_THREADS), s.a, s.w, z_out);
-    return ln.run("scores", scores_kernel<float>, grid, dim3(SEL_THREADS), s.a, s.w, z_out);
+        return ln.run("scores", scores_kernel<SrcMma>, grid, dim3(SC_THREADS), s.a, s.w, z_out);
+    return ln.run("scores", scores_kernel<SrcSimt<float>>, grid, dim3(SC_THREADS), s.a, s.w, z_out);
 }
 
 int rtp_topp_select(const rtp_dims *dims, const float *z, const uint8_t *head_class, float p,
@@ -384,7 +454,7 @@ int rtp_topp_select(const rtp_dims *dims, const float *z, const uint8_t *head_cl
     s.a.count_out = count_out;
     s.a.mass_out = mass_out;
     Launcher ln{(cudaStream_t)stream, nullptr};
-    return launch_select<FromBuffer, float>(ln, dims, s);
+    return launch_select<SrcBuffer>(ln, dims, s);
 }
 
 int rtp_sparse_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
@@ -453,29 +523,47 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
     const float asc = scale_or_default(opts ? opts->attn_scale : 0.f);
     const float isc = scale_or_default(opts ? opts->idx_scale : 0.f);
 
-    // local heads: window + sinks
-    RTP_TRY(launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
-                         n_sink, out, w, L, asc));
     SelPlan s = make_sel(dims, head_class, w, L);
-    if (s.a.n_ret == 0) return RTP_OK;
-    if (p >= 1.0f) {
-        // every token is kept: the retrieval heads' attention is dense
-        return launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_RETRIEVAL, true, 1,
-                            0, out, w, L, asc);
+    const bool any_local = s.a.n_ret < dims->H_kv;
+    const cudaStream_t main = (cudaStream_t)stream;
+    Side *side = nullptr;
+    if (any_local && s.a.n_ret > 0) {
+        // local heads run on a side stream, overlapping the retrieval pipeline
+        RTP_TRY(side_stream(side));
+        if (cudaEventRecord(side->fork, main) != cudaSuccess) return RTP_ERR_CUDA;
+        if (cudaStreamWaitEvent(side->st, side->fork, 0) != cudaSuccess) return RTP_ERR_CUDA;
+        Launcher lside{side->st, ln.prof};
+        RTP_TRY(launch_range(lside, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
+                             n_sink, out, w, L, asc));
+        if (cudaEventRecord(side->join, side->st) != cudaSuccess) return RTP_ERR_CUDA;
+    } else if (any_local) {
+        RTP_TRY(launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
+                             n_sink, out, w, L, asc));
     }
-    s.a.kidx = kidx_cache;
-    s.a.p = p;
-    s.a.lists = opts && opts->sel_idx ? opts->sel_idx : reinterpret_cast<int32_t *>(w + L.lists);
-    s.a.count_out = opts && opts->sel_count ? opts->sel_count : reinterpret_cast<int32_t *>(w + L.counts);
-    s.a.mass_out = opts ? opts->sel_mass : nullptr;
-    RTP_TRY(launch_qidx(ln, dims, q, W_q_idx, head_class, s, isc));
-    if (dims->idx_dtype == RTP_BF16) {
-        RTP_TRY(select_from_index<__nv_bfloat16>(ln, dims, s));
-    } else {
-        RTP_TRY(select_from_index<float>(ln, dims, s));
+    int rc = RTP_OK;
+    if (s.a.n_ret > 0) {
+        if (p >= 1.0f) {
+            // every token is kept: the retrieval heads' attention is dense
+            rc = launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_RETRIEVAL, true, 1, 0,
+                              out, w, L, asc);
+        } else {
+            s.a.kidx = kidx_cache;
+            s.a.q = q;
+            s.a.Wq = W_q_idx;
+            s.a.idx_scale = isc;
+            s.a.p = p;
+            s.a.lists = opts && opts->sel_idx ? opts->sel_idx : reinterpret_cast<int32_t *>(w + L.lists);
+            s.a.count_out = opts && opts->sel_count ? opts->sel_count : reinterpret_cast<int32_t *>(w + L.counts);
+            s.a.mass_out = opts ? opts->sel_mass : nullptr;
+            s.a.item_pre = reinterpret_cast<int32_t *>(w + L.item_pre);
+            rc = select_from_index(ln, dims, s);
+            if (rc == RTP_OK)
+                rc = launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out,
+                                 w, L, asc, s.a.item_pre);
+        }
     }
-    return launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out, w,
-                       L, asc);
+    if (side && cudaStreamWaitEvent(main, side->join, 0) != cudaSuccess && rc == RTP_OK) rc = RTP_ERR_CUDA;
+    return rc;
 }
 
 int rtp_prof_init(rtp_prof *prof, int32_t capacity) {

@@ -23,12 +23,59 @@ namespace rtp {
 
 constexpr int ATT_THREADS = 256;
 constexpr int RCH = 256;               // rows per range sub-chunk (one per thread)
-constexpr int PSTRIDE = D + 2;         // partial record: m, l, o[D]
-constexpr int LCH = 256;               // rows per list item (target)
-constexpr int LIST_MAX_SPLIT = 64;     // items per head at most
+constexpr int PSTRIDE = D + 4;         // partial record: m, l, (2 unused), o[D]
+constexpr int POFF = 4;                // offset of o[] in a record (16-byte aligned)
+static_assert(PSTRIDE % 4 == 0 && POFF % 4 == 0, "partial records must keep o[] 16-byte aligned");
 constexpr int MAX_GROUPS = 64;
 constexpr int MAX_RET_Q = 512;
 constexpr int MAX_LIST_HEADS = 4096;
+
+// Merge n flash-decoding partial records (stride `rec` floats between
+// records; record h of a group at + h * PSTRIDE) for heads [0, nh) into
+// out[h * D + d].  Every thread owns 4 dims of one head and merges in one
+// pass with a running max, keeping 8 records' loads in flight.
+__device__ __forceinline__ void merge_partials(const float *__restrict__ pb, int n, int rec, int nh,
+                                               float *__restrict__ out) {
+    constexpr int U = 8;
+    for (int i = threadIdx.x; i < nh * (D / 4); i += blockDim.x) {
+        const int h = i / (D / 4), d4 = i % (D / 4);
+        const float *base = pb + h * PSTRIDE;
+        float M = -INFINITY, l = 0.0f;
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int sp = 0; sp < n; sp += U) {
+            float mm[U], ll[U];
+            float4 oo[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (sp + u < n) {
+                    const float *r = base + (size_t)(sp + u) * rec;
+                    mm[u] = __ldcg(r);
+                    ll[u] = __ldcg(r + 1);
+                    oo[u] = __ldcg(reinterpret_cast<const float4 *>(r + POFF) + d4);
+                } else {
+                    mm[u] = -INFINITY; ll[u] = 0.0f; oo[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            float Mb = M;
+#pragma unroll
+            for (int u = 0; u < U; ++u) Mb = fmaxf(Mb, mm[u]);
+            if (Mb == -INFINITY) continue;
+            const float sc = M == -INFINITY ? 0.0f : exp2f(M - Mb);
+            l *= sc;
+            o.x *= sc; o.y *= sc; o.z *= sc; o.w *= sc;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const float wg = mm[u] == -INFINITY ? 0.0f : exp2f(mm[u] - Mb);
+                l = fmaf(ll[u], wg, l);
+                o.x = fmaf(oo[u].x, wg, o.x); o.y = fmaf(oo[u].y, wg, o.y);
+                o.z = fmaf(oo[u].z, wg, o.z); o.w = fmaf(oo[u].w, wg, o.w);
+            }
+            M = Mb;
+        }
+        const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+        reinterpret_cast<float4 *>(out + h * D)[d4] = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+    }
+}
 
 struct RangeArgs {
     int B, H_q, H_kv, G;
@@ -195,7 +242,7 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
     float *pp = a.part + (bg * a.n_split + blockIdx.x) * GMAX * PSTRIDE;
     for (int i = tid; i < G * PSTRIDE; i += blockDim.x) {
         const int h = i / PSTRIDE, e = i % PSTRIDE;
-        pp[i] = e == 0 ? s_m[h] : (e == 1 ? s_l[h] : O[h][e - 2]);
+        pp[i] = e == 0 ? s_m[h] : (e == 1 ? s_l[h] : (e < POFF ? 0.0f : O[h][e - POFF]));
     }
     __threadfence();
     __syncthreads();
@@ -203,20 +250,7 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const float *pb = a.part + bg * a.n_split * GMAX * PSTRIDE;
-    for (int i = tid; i < G * D; i += blockDim.x) {
-        const int h = i / D, d = i % D;
-        float M = -INFINITY;
-        for (int sp = 0; sp < n_active; ++sp) M = fmaxf(M, pb[(sp * GMAX + h) * PSTRIDE]);
-        float l = 0.0f, o = 0.0f;
-        for (int sp = 0; sp < n_active; ++sp) {
-            const float *r = pb + (sp * GMAX + h) * PSTRIDE;
-            const float wgt = exp2f(r[0] - M);
-            l = fmaf(r[1], wgt, l);
-            o = fmaf(r[2 + d], wgt, o);
-        }
-        a.out[(bh0 + h) * D + d] = o / l;
-    }
+    merge_partials(a.part + bg * a.n_split * GMAX * PSTRIDE, n_active, GMAX * PSTRIDE, G, a.out + bh0 * D);
     if (tid == 0) a.arrive[bg] = 0;
 }
 
@@ -235,17 +269,16 @@ struct ListArgs {
     const void *v;
     const int32_t *lists;        // [B*H_q*N_max]
     const int32_t *counts;       // [B*H_q]
+    const int32_t *item_pre;     // [nh + 1] precomputed item prefix, or null
     float *out;
-    float *part;                 // [B*H_q][LIST_MAX_SPLIT][PSTRIDE] (indexed by item)
+    float *part;                 // [B*H_q*LIST_MAX_SPLIT][PSTRIDE] (indexed by item)
     uint32_t *arrive;            // [B*H_q]
     uint32_t *status;
 };
 
-__device__ __forceinline__ int list_items(int count) {
-    if (count <= 0) return 0;
-    return min(LIST_MAX_SPLIT, (count + LCH - 1) / LCH);
-}
-
+// One item = a slice of one head's kept rows.  Warp w takes rows
+// r0 + 8w .. r0 + 8w + 7, then every 64th: all 8 rows' K and V loads are
+// issued before the first dot product.
 template <typename KT>
 __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
     __shared__ int pre[MAX_LIST_HEADS + 1];
@@ -256,8 +289,12 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nh = a.B * a.n_rq;
 
-    // items per head -> exclusive prefix (each CTA builds its own copy)
-    {
+    // items per head -> exclusive prefix: precomputed by the selection
+    // stage, or built here by every CTA
+    if (a.item_pre) {
+        for (int i = tid; i <= nh; i += blockDim.x) pre[i] = __ldcg(a.item_pre + i);
+        __syncthreads();
+    } else {
         const int per = (nh + ATT_THREADS - 1) / ATT_THREADS;
         int loc = 0;
         for (int i = 0; i < per; ++i) {
@@ -289,21 +326,18 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
         __syncthreads();
     }
     const int total = pre[nh];
-    // heads with nothing to attend over get zeros (and a status if invalid)
+    // heads with nothing to attend over get zeros (and a status: invalid input)
     if (blockIdx.x == 0) {
         for (int hi = warp; hi < nh; hi += ATT_THREADS / 32) {
             if (pre[hi + 1] != pre[hi]) continue;
             const int b = hi / a.n_rq, h = a.ret_h[hi % a.n_rq];
-            a.out[((size_t)b * a.H_q + h) * D + lane * 4 + 0] = 0.0f;
-            a.out[((size_t)b * a.H_q + h) * D + lane * 4 + 1] = 0.0f;
-            a.out[((size_t)b * a.H_q + h) * D + lane * 4 + 2] = 0.0f;
-            a.out[((size_t)b * a.H_q + h) * D + lane * 4 + 3] = 0.0f;
+            float *o = a.out + ((size_t)b * a.H_q + h) * D + lane * 4;
+            o[0] = o[1] = o[2] = o[3] = 0.0f;
             if (lane == 0) set_status(a.status, RTP_ERR_DEVICE_ARG);
         }
     }
 
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
-        // find the head of this item (upper bound in pre[0..nh])
         int lo_h = 0, hi_h = nh;
         while (hi_h - lo_h > 1) {
             const int mid = (lo_h + hi_h) >> 1;
@@ -327,16 +361,16 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
         const KT *vb = reinterpret_cast<const KT *>(a.v) + ((size_t)b * a.H_kv + g) * a.N_max * D;
         const int32_t *lst = a.lists + bh * a.N_max;
         float m = -INFINITY, l = 0.0f, o[4] = {0.f, 0.f, 0.f, 0.f};
-        constexpr int U = 4;
-        for (int rr = r0 + warp * U; rr < r1; rr += (ATT_THREADS / 32) * U) {
+        constexpr int U = 8;
+        for (int rb = r0 + warp * U; rb < r1; rb += (ATT_THREADS / 32) * U) {
+            int myid = -1;
+            if (lane < U && rb + lane < r1) myid = __ldg(lst + rb + lane);
             float kx[U][4], vx[U][4];
             bool ok[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int r = rr + u;
-                int t = r < r1 ? __ldg(lst + r) : -1;
-                ok[u] = r < r1 && t >= 0 && t < N;
-                if (r < r1 && !ok[u] && lane == 0) set_status(a.status, RTP_ERR_DEVICE_ARG);
+                const int t = __shfl_sync(0xffffffffu, myid, u);
+                ok[u] = rb + u < r1 && t >= 0 && t < N;
                 if (ok[u]) {
                     Row<KT>::load4(kb + (size_t)t * D + lane * 4, kx[u]);
                     Row<KT>::load4(vb + (size_t)t * D + lane * 4, vx[u]);
@@ -344,7 +378,10 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) kx[u][i] = vx[u][i] = 0.0f;
                 }
+                if (rb + u < r1 && !ok[u] && lane == 0) set_status(a.status, RTP_ERR_DEVICE_ARG);
             }
+            float sc[U];
+            float mb = -INFINITY;
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 float s = qx[0] * kx[u][0];
@@ -352,15 +389,23 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
                 s = fmaf(qx[2], kx[u][2], s);
                 s = fmaf(qx[3], kx[u][3], s);
                 s = warp_sum(s);
-                if (!ok[u]) continue;
-                const float mn = fmaxf(m, s);
-                const float al = exp2f(m - mn);
-                const float pw = exp2f(s - mn);
-                l = l * al + pw;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) o[i] = fmaf(pw, vx[u][i], o[i] * al);
-                m = mn;
+                sc[u] = ok[u] ? s : -INFINITY;
+                mb = fmaxf(mb, sc[u]);
             }
+            const float mn = fmaxf(m, mb);
+            if (mn == -INFINITY) continue;
+            const float al = exp2f(m - mn);
+            l *= al;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) o[i] *= al;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const float pw = exp2f(sc[u] - mn);
+                l += pw;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) o[i] = fmaf(pw, vx[u][i], o[i]);
+            }
+            m = mn;
         }
         // merge warps
         if (lane == 0) { wm[warp] = m; wl[warp] = l; }
@@ -379,7 +424,7 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
                     os = fmaf(wo[w][tid], wg, os);
                 }
             }
-            pp[2 + tid] = os;
+            pp[POFF + tid] = os;
             if (tid == 0) { pp[0] = M; pp[1] = ls; }
         }
         __threadfence();
@@ -388,19 +433,7 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
         __syncthreads();
         if (s_last) {
             __threadfence();
-            const float *pb = a.part + (size_t)pre[hix] * PSTRIDE;
-            if (tid < D) {
-                float M = -INFINITY;
-                for (int i = 0; i < nit; ++i) M = fmaxf(M, pb[i * PSTRIDE]);
-                float ls = 0.0f, os = 0.0f;
-                for (int i = 0; i < nit; ++i) {
-                    const float *r = pb + i * PSTRIDE;
-                    const float wg = r[0] == -INFINITY ? 0.0f : exp2f(r[0] - M);
-                    ls = fmaf(r[1], wg, ls);
-                    os = fmaf(r[2 + tid], wg, os);
-                }
-                a.out[bh * D + tid] = ls > 0.0f ? os / ls : 0.0f;
-            }
+            merge_partials(a.part + (size_t)pre[hix] * PSTRIDE, nit, PSTRIDE, 1, a.out + bh * D);
             if (tid == 0) a.arrive[bh] = 0;
         }
         __syncthreads();

@@ -76,40 +76,58 @@ __device__ __forceinline__ float key_logit(uint32_t k) {
 }
 
 // ---------------------------------------------------------------------------
-// Level-1 mass histogram bins.  |z| in [2^E_LO, 2^E_HI) is binned by its
-// exponent and the top MB mantissa bits (relative width 2^-MB), one set of
-// bins per sign; |z| < 2^E_LO shares one central bin.  Bin order follows z.
-// Each bin stores the sum of exp(z - U) over its tokens, U = the bin's upper
-// edge, so no maximum is needed while scanning and every term is in (0, 1]
-// (bin widths are at most 32 nats below 2^E_HI).
+// mbarrier + bulk async copy (TMA, 1-D) helpers.  Every wait is bounded in
+// time: after the limit the caller gets `false` and reports RTP_ERR_TIMEOUT.
 // ---------------------------------------------------------------------------
-constexpr int MB = 4;
-constexpr int E_LO = -6;
-constexpr int E_HI = 10;
-constexpr int NPOS = (E_HI - E_LO) << MB;     // 256 bins per sign
-constexpr int NBIN = 2 * NPOS + 1;            // 513
-constexpr int ZERO_BIN = NPOS;
-constexpr float Z_LIMIT = 1024.0f;            // 2^E_HI
-constexpr uint32_t BIN_BASE = (uint32_t)(127 + E_LO) << MB;
-
-__device__ __forceinline__ int logit_bin(float z) {
-    uint32_t a = __float_as_uint(z) & 0x7fffffffu;
-    int k = (int)(a >> (23 - MB)) - (int)BIN_BASE;
-    if (k < 0) return ZERO_BIN;
-    return z > 0.0f ? ZERO_BIN + 1 + k : ZERO_BIN - 1 - k;
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
 }
-
-// Upper edge of a bin (an fp32 value; every z in the bin is <= it).
-__host__ __device__ __forceinline__ float bin_upper(int bin) {
-    if (bin == ZERO_BIN) {
-        union { uint32_t u; float f; } c; c.u = BIN_BASE << (23 - MB); return c.f;
-    }
-    if (bin > ZERO_BIN) {
-        uint32_t k = (uint32_t)(bin - ZERO_BIN - 1);
-        union { uint32_t u; float f; } c; c.u = (k + 1 + BIN_BASE) << (23 - MB); return c.f;
-    }
-    uint32_t k = (uint32_t)(ZERO_BIN - 1 - bin);
-    union { uint32_t u; float f; } c; c.u = (k + BIN_BASE) << (23 - MB); return -c.f;
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0u;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+constexpr uint64_t WAIT_LIMIT_NS = 200000000ull;   // 0.2 s: far beyond any healthy wait
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(bar, parity))
+        if (global_ns() - t0 > WAIT_LIMIT_NS) return false;
+    return true;
+}
+// global -> shared bulk copy completing on `bar` (16-byte aligned, size a
+// multiple of 16)
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -129,6 +147,15 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
+}
+
+// List attention splits a head's kept rows into items of about LCH rows,
+// at most LIST_MAX_SPLIT per head.
+constexpr int LCH = 128;
+constexpr int LIST_MAX_SPLIT = 64;
+__device__ __forceinline__ int list_items(int count) {
+    if (count <= 0) return 0;
+    return min(LIST_MAX_SPLIT, (count + LCH - 1) / LCH);
 }
 
 // Flash-decoding partial of one head over a set of rows.

@@ -6,20 +6,29 @@
 // smallest descending-score prefix whose mass reaches p; the kernels find
 // that threshold with histograms instead of a sort.
 //
-// Stages (per sequence b and retrieval KV head g, all G query heads of the
-// group at once so each index-key row is read once per pass):
-//   hist     stream the logits (from the index keys, or from a logit
-//            buffer), accumulate a per-head level-1 mass histogram over the
-//            order-preserving bits of z (rtp_common.cuh), record the
-//            largest bin of every 32-token tile; the last CTA of the group
-//            resolves the boundary bin b* of each head.
-//   collect  re-derive the logits of tiles whose largest bin reaches b*,
-//            append tokens above b* to the head's kept list and tokens in
-//            b* to its candidate list (64-bit composite key: logit key,
-//            then inverted token id, so the order is total).
-//   finalize exact radix select by mass over the candidates (8-bit digits
-//            of the composite key, most significant first) to the unique
-//            boundary token, then append the candidates at or above it.
+// Stages (per sequence b and retrieval KV head g; all G <= 8 query heads of
+// the group are scored from one read of each index-key row):
+//   scan      q_idx = W_q_idx . q (in-kernel), logits z for every token, and
+//             a level-1 mass histogram per head over the order-preserving
+//             bits of z: sign, exponent and 4 mantissa bits for |z| in
+//             [2^-6, 2^10) (512 bins, relative width 1/16; |z| < 2^-6 shares
+//             the innermost bin of its sign).  Each bin sums exp(z - U_b),
+//             U_b its upper edge, so every term is in (e^-32, 1], no maximum
+//             is needed while streaming, and CTAs' bins add directly.  The
+//             largest bin of every 32-token tile is recorded.  The last CTA
+//             of the group resolves each head: R = U(top bin), bin masses
+//             S_b exp(U_b - R), and the boundary bin b* where the mass
+//             accumulated from the top first reaches p Z.
+//   collect   re-derive the logits of tiles whose largest bin reaches b*;
+//             tokens above b* are kept, tokens in b* become candidates
+//             (64-bit key: order-preserving logit bits, then the inverted
+//             token id, so the order is total and equal logits go to the
+//             lower id first).
+//   finalize  exact radix select by mass over the candidates: 8-bit digits
+//             of the key from the first bit where candidates differ, digit
+//             masses summed in fixed point (order-independent), down to the
+//             unique boundary token; candidates at or above it are kept.
+//
 #pragma once
 
 #include <type_traits>
@@ -28,51 +37,114 @@
 
 namespace rtp {
 
-constexpr int SEL_THREADS = 256;
-constexpr int SEL_CHUNK = 4096;            // tokens per CTA in hist/collect
+constexpr int SC_THREADS = 256;
+constexpr int SC_WARPS = SC_THREADS / 32;
 constexpr int TILE = 32;                   // tokens per warp tile
 constexpr int MAX_RET_GROUPS = 64;
+constexpr float L2E = 1.4426950408889634f;
 
 enum ResolveMode : int32_t { MODE_NORMAL = 0, MODE_KEEP_ALL = 1, MODE_EMPTY = 2 };
 
+// Level-1 bins over the fp32 logit bits: k = (exponent, top MB mantissa bits)
+// of |z| relative to 2^E_LO, clamped to [0, 255]; bin = 256 + k for z > 0
+// and 255 - k for z <= 0, so bin order follows z.
+constexpr int MB = 4;
+constexpr int E_LO = -6;
+constexpr int NBIN = 512;
+constexpr uint32_t BIN_BASE = (uint32_t)(127 + E_LO) << MB;   // k = (bits >> 19) - BIN_BASE
+constexpr float Z_LIMIT = 256.0f;   // logits beyond are reported (bins up to 16 nats wide stay resolvable)
+
+// 2^x with the SFU (ex2.approx.ftz: relative error ~2^-22 on the range used
+// here, |x| <= 47).
+__device__ __forceinline__ float ex2_sfu(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Per-CTA bin sums are kept in fixed point: FX_ONE units per unit of mass
+// (every term is in (e^-32, 1], so terms below 2^-20 of a bin's upper edge
+// -- only possible for |z| >= 232 -- round to zero), as a 64-bit value split
+// over two 32-bit shared counters; the thread whose add wraps the low word
+// (seen in the value atomicAdd returns) carries into the high word, so the
+// sums are exact and independent of the order of the adds.
+constexpr float FX_ONE = 1048576.0f;   // 2^20
+
+// Bin of z (z already folded so that -0 is +0) and exp(z - U_bin) in fixed point.
+__device__ __forceinline__ int bin_and_fx(float z, uint32_t &fx) {
+    const uint32_t u = __float_as_uint(z);
+    const int s = (int)u >> 31;                                // 0 or -1
+    int k = (int)((u << 1) >> (24 - MB)) - (int)BIN_BASE;
+    k = min(max(k, 0), 255);
+    const uint32_t eb = (uint32_t)(k + (int)BIN_BASE + 1 + s) << (23 - MB);
+    const float U = __uint_as_float(eb | ((uint32_t)s & 0x80000000u));
+    fx = __float2uint_rn(ex2_sfu((z - U) * 1.4426950408889634f) * FX_ONE);
+    return 256 + (k ^ s);
+}
+
+// Bin only (same arithmetic as bin_and_fx).
+__device__ __forceinline__ int logit_bin(float z) {
+    const uint32_t u = __float_as_uint(z);
+    const int s = (int)u >> 31;
+    int k = (int)((u << 1) >> (24 - MB)) - (int)BIN_BASE;
+    k = min(max(k, 0), 255);
+    return 256 + (k ^ s);
+}
+
+// Upper edge of a bin, as used by bin_and_fx.
+__host__ __device__ __forceinline__ float bin_upper(int bin) {
+    union { uint32_t u; float f; } c;
+    if (bin >= 256) {
+        c.u = (uint32_t)(bin - 256 + (int)BIN_BASE + 1) << (23 - MB);
+        return c.f;
+    }
+    c.u = (uint32_t)(255 - bin + (int)BIN_BASE) << (23 - MB);
+    return -c.f;
+}
+
 struct Resolve {
-    double Z;          // sum of masses, relative to exp(R)
-    double above;      // mass of bins above b*, same units
-    double target;     // mass still needed inside b*, same units
+    double Z;          // total mass, relative to exp(R)
+    double above;      // mass of the bins above b*, same units
+    double target;     // mass still needed inside b*, same units (inf: keep all of b*)
     float R;           // reference logit: upper edge of the top bin
     int32_t bstar;     // boundary bin
     int32_t mode;      // ResolveMode
     int32_t N;         // valid tokens
-    int32_t pad[2];
 };
-static_assert(sizeof(Resolve) == 48, "Resolve layout");
+static_assert(sizeof(Resolve) == 40, "Resolve layout");
 
-// Pointers into the workspace used by the selection stages.
 struct SelWs {
     uint32_t *status;
-    uint32_t *arrive;      // [B*H_kv] hist arrivals
-    uint32_t *list_cnt;    // [B*H_q]
-    uint32_t *cand_cnt;    // [B*H_q]
-    double *hist;          // [B*H_q*NBIN]
-    Resolve *res;          // [B*H_q]
-    uint16_t *tilebin;     // [B*H_q*ntile]: 1 + largest bin of the tile (0: empty)
-    unsigned long long *cands;  // [B*H_q*N_max]
-    float *qidx;           // [B*H_q*R] scaled query projections
+    uint32_t *arrive;            // [B*H_kv] scan arrivals
+    uint32_t *cand_cnt;          // [B*H_q]
+    uint32_t *list_cnt;          // [B*H_q]
+    double *hist;                // [B*H_q][NBIN]
+    Resolve *res;                // [B*H_q]
+    uint16_t *tilebin;           // [B*H_q][ntile]: 1 + largest bin of the tile (0: none)
+    unsigned long long *cands;   // [B*H_q][N_max]
+    float *qidx;                 // [B*H_q][R]
+    uint32_t *fin_arrive;        // finalize arrivals (one counter)
 };
 
 struct SelArgs {
     int B, H_q, H_kv, G;
     long long N_max;
-    int ntile;             // ceil(N_max / TILE)
+    int ntile;
+    int ctas;                    // scan/collect CTAs per (b, g)
+    long long chunk;             // tokens per CTA, multiple of TILE
     const int32_t *seq_lens;
-    int n_ret;             // retrieval KV heads
+    int n_ret;
     int ret_g[MAX_RET_GROUPS];
     float p;
-    const void *kidx;      // [B, H_kv, N_max, R] (FromIndex)
-    const float *z;        // [B, H_q, N_max] (FromBuffer)
-    int32_t *lists;        // [B*H_q*N_max] kept ids
-    int32_t *count_out;    // [B*H_q]
-    float *mass_out;       // [B*H_q] or null
+    float idx_scale;
+    const float *q;              // [B, H_q, D] pre-RoPE queries
+    const float *Wq;             // [H_q, R, D]
+    const void *kidx;            // [B, H_kv, N_max, R]
+    const float *z;              // [B, H_q, N_max] (given logits)
+    int32_t *lists;              // [B*H_q][N_max] kept ids
+    int32_t *count_out;          // [B*H_q]
+    float *mass_out;             // [B*H_q] or null
+    int32_t *item_pre;           // [B*n_ret*G + 1] list-attention work prefix, or null
 };
 
 __device__ __forceinline__ int valid_len(const int32_t *seq_lens, int b, long long N_max,
@@ -85,104 +157,202 @@ __device__ __forceinline__ int valid_len(const int32_t *seq_lens, int b, long lo
     return N;
 }
 
-// ---------------------------------------------------------------------------
-// q_idx[b, h, :] = scale * W_q_idx[h] . q[b, h]   (one CTA per (b, h))
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(512) qidx_kernel(const float *__restrict__ q,
-                                                   const float *__restrict__ W,
-                                                   float *__restrict__ qidx, int H_q,
-                                                   int G, unsigned long long ret_mask,
-                                                   float scale) {
-    const int bh = blockIdx.x;
-    const int h = bh % H_q;
-    if (!((ret_mask >> (h / G)) & 1ull)) return;
-    const int j = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const float4 qv = __ldg(reinterpret_cast<const float4 *>(q + (size_t)bh * D) + lane);
-    const float4 wv = __ldg(reinterpret_cast<const float4 *>(W + ((size_t)h * R + j) * D) + lane);
-    float acc = qv.x * wv.x;
-    acc = fmaf(qv.y, wv.y, acc);
-    acc = fmaf(qv.z, wv.z, acc);
-    acc = fmaf(qv.w, wv.w, acc);
-    acc = warp_sum(acc);
-    if (lane == 0) qidx[(size_t)bh * R + j] = acc * scale;
-}
-
-// ---------------------------------------------------------------------------
-// logit sources.  Both passes derive z through the same code, so the
-// histogram pass and the collect pass see bit-identical logits.
-// ---------------------------------------------------------------------------
-template <typename IT>
-struct FromIndex {
-    const IT *rows;   // kidx of (b, g): [N_max, R]
-    const float *qs;  // shared [G][R]
-    int G;
-    __device__ __forceinline__ void logits(long long t, float (&z)[GMAX]) const {
-        float k[R];
-        float lo[8], hi[8];
-        Row<IT>::load8(rows + t * R, lo);
-        Row<IT>::load8(rows + t * R + 8, hi);
+// q_idx of the group's heads into shared memory: warp h computes head h's
+// 16 outputs (fixed lane partition and reduction order, so every CTA and
+// every kernel gets bit-identical values).
+__device__ __forceinline__ void project_query(const float *__restrict__ q_bh0,
+                                              const float *__restrict__ W_h0, float scale,
+                                              float *qs, int G) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp >= G) return;
+    const float4 qv = __ldg(reinterpret_cast<const float4 *>(q_bh0 + warp * D) + lane);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) { k[j] = lo[j]; k[8 + j] = hi[j]; }
+    for (int half = 0; half < 2; ++half) {
+        float4 wv[8];
 #pragma unroll
-        for (int h = 0; h < GMAX; ++h) {
-            if (h < G) {
-                const float4 *qh = reinterpret_cast<const float4 *>(qs + h * R);
-                float acc = 0.0f;
+        for (int j = 0; j < 8; ++j)
+            wv[j] = __ldg(reinterpret_cast<const float4 *>(W_h0 + (warp * R + half * 8 + j) * D) + lane);
 #pragma unroll
-                for (int j4 = 0; j4 < 4; ++j4) {
-                    float4 w = qh[j4];
-                    acc = __fmaf_rn(w.x, k[4 * j4 + 0], acc);
-                    acc = __fmaf_rn(w.y, k[4 * j4 + 1], acc);
-                    acc = __fmaf_rn(w.z, k[4 * j4 + 2], acc);
-                    acc = __fmaf_rn(w.w, k[4 * j4 + 3], acc);
-                }
-                z[h] = acc;
-            }
+        for (int j = 0; j < 8; ++j) {
+            float acc = qv.x * wv[j].x;
+            acc = fmaf(qv.y, wv[j].y, acc);
+            acc = fmaf(qv.z, wv[j].z, acc);
+            acc = fmaf(qv.w, wv[j].w, acc);
+            acc = warp_sum(acc);
+            if (lane == 0) qs[warp * R + half * 8 + j] = acc * scale;
         }
     }
-};
-
-struct FromBuffer {
-    const float *zb;  // z of head (b, g*G): [G][N_max]
-    long long N_max;
-    int G;
-    __device__ __forceinline__ void logits(long long t, float (&z)[GMAX]) const {
-#pragma unroll
-        for (int h = 0; h < GMAX; ++h)
-            if (h < G) z[h] = __ldg(zb + h * N_max + t);
-    }
-};
-
-// ---------------------------------------------------------------------------
-// rtp_index_scores: write z for every retrieval head
-// ---------------------------------------------------------------------------
-template <typename IT>
-__global__ void __launch_bounds__(SEL_THREADS) scores_kernel(SelArgs a, SelWs w, float *z_out) {
-    __shared__ __align__(16) float qs[GMAX * R];
-    const int b = blockIdx.y / a.n_ret;
-    const int g = a.ret_g[blockIdx.y % a.n_ret];
-    const int G = a.G;
-    for (int i = threadIdx.x; i < G * R; i += blockDim.x)
-        qs[i] = w.qidx[((size_t)b * a.H_q + g * G) * R + i];
-    __syncthreads();
-    const int N = valid_len(a.seq_lens, b, a.N_max, w.status);
-    const FromIndex<IT> src{reinterpret_cast<const IT *>(a.kidx) + ((size_t)b * a.H_kv + g) * a.N_max * R, qs, G};
-    float *zb = z_out + ((size_t)b * a.H_q + g * G) * a.N_max;
-    const long long t0 = (long long)blockIdx.x * SEL_CHUNK;
-    for (long long t = t0 + threadIdx.x; t < t0 + SEL_CHUNK && t < N; t += blockDim.x) {
-        float z[GMAX];
-        src.logits(t, z);
-#pragma unroll
-        for (int h = 0; h < GMAX; ++h)
-            if (h < G) zb[h * a.N_max + t] = z[h];
-    }
 }
 
 // ---------------------------------------------------------------------------
-// resolve: one warp per head, after the group's histogram is complete.
-// Bin masses M_b = S_b * exp(U_b - R) (fp64), R = U(top bin).  The boundary
-// bin is the first one, walking down from the top, whose inclusive
-// cumulative mass reaches p * Z.
+// logit sources.  A warp tile is 32 consecutive tokens; each lane gets NV
+// values (token offset tok(v), head slot slot(v)); slot s of a lane is head
+// head(s).  XOR_LO is the first lane-xor offset over which lanes share slots.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat16 l = __float2bfloat16_rn(lo), h = __float2bfloat16_rn(hi);
+    return (uint32_t)__bfloat16_as_ushort(l) | ((uint32_t)__bfloat16_as_ushort(h) << 16);
+}
+
+// bf16 index keys on the tensor cores.  m16n8k16: rows = 16 tokens, k = the
+// 16 index dims, n = the 8 heads of the group.  The k order is permuted so
+// that lane (gid, tig) reads dims 4*tig .. 4*tig+3 of a row with one 8-byte
+// load: k slots (2tig, 2tig+1) <- dims (4tig, 4tig+1) and k slots
+// (2tig+8, 2tig+9) <- dims (4tig+2, 4tig+3), in A and B alike.
+struct SrcMma {
+    static constexpr int NV = 8;        // 2 mma tiles x 2 rows x 2 heads
+    static constexpr int NSLOT = 2;
+    static constexpr int XOR_LO = 4;
+    struct Frag { uint2 a[2][2]; };
+    const __nv_bfloat16 *rows;          // [N_max][R] of (b, g)
+    long long N_max;
+    uint32_t bq[3][2];                  // q_idx split hi / mid / lo
+    int gid, tig;
+
+    __device__ __forceinline__ void init(const __nv_bfloat16 *r, long long nmax, const float *qs, int G) {
+        rows = r; N_max = nmax;
+        const int lane = threadIdx.x & 31;
+        gid = lane >> 2; tig = lane & 3;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (gid < G) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) x[i] = qs[gid * R + 4 * tig + i];
+        }
+        float hi[4], mid[4], lo[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            hi[i] = __bfloat162float(__float2bfloat16_rn(x[i]));
+            const float r1 = x[i] - hi[i];
+            mid[i] = __bfloat162float(__float2bfloat16_rn(r1));
+            lo[i] = r1 - mid[i];
+        }
+        bq[0][0] = pack_bf16(hi[0], hi[1]); bq[0][1] = pack_bf16(hi[2], hi[3]);
+        bq[1][0] = pack_bf16(mid[0], mid[1]); bq[1][1] = pack_bf16(mid[2], mid[3]);
+        bq[2][0] = pack_bf16(lo[0], lo[1]); bq[2][1] = pack_bf16(lo[2], lo[3]);
+    }
+    __device__ __forceinline__ void load(int tb, Frag &f) const {
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                int t = tb + 16 * i + gid + 8 * r;
+                t = t < N_max ? t : (int)N_max - 1;
+                f.a[i][r] = __ldg(reinterpret_cast<const uint2 *>(rows + (size_t)t * R + 4 * tig));
+            }
+    }
+    __device__ __forceinline__ void eval(const Frag &f, float (&z)[NV]) const {
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int term = 2; term >= 0; --term)
+                mma_bf16_16816(d, f.a[i][0].x, f.a[i][1].x, f.a[i][0].y, f.a[i][1].y, bq[term][0],
+                               bq[term][1]);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) z[4 * i + j] = d[j];
+        }
+    }
+    __device__ __forceinline__ int tok(int v) const { return 16 * (v >> 2) + gid + 8 * ((v >> 1) & 1); }
+    __device__ __forceinline__ int slot(int v) const { return v & 1; }
+    __device__ __forceinline__ int head(int s) const { return 2 * tig + s; }
+};
+
+// fp32 index keys (or bf16 without tensor cores): one token per lane.
+template <typename IT>
+struct SrcSimt {
+    static constexpr int NV = GMAX;
+    static constexpr int NSLOT = GMAX;
+    static constexpr int XOR_LO = 1;
+    struct Frag { float k[R]; };
+    const IT *rows;
+    long long N_max;
+    const float *qs;                    // shared [G][R]
+    int G, lane;
+    __device__ __forceinline__ void init(const IT *r, long long nmax, const float *q, int g) {
+        rows = r; N_max = nmax; qs = q; G = g; lane = threadIdx.x & 31;
+    }
+    __device__ __forceinline__ void load(int tb, Frag &f) const {
+        int t = tb + lane;
+        t = t < N_max ? t : (int)N_max - 1;
+        float a[8], b[8];
+        Row<IT>::load8(rows + (size_t)t * R, a);
+        Row<IT>::load8(rows + (size_t)t * R + 8, b);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) { f.k[j] = a[j]; f.k[8 + j] = b[j]; }
+    }
+    __device__ __forceinline__ void eval(const Frag &f, float (&z)[NV]) const {
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) {
+            float acc = 0.0f;
+            if (h < G) {
+#pragma unroll
+                for (int j = 0; j < R; ++j) acc = __fmaf_rn(qs[h * R + j], f.k[j], acc);
+            }
+            z[h] = acc;
+        }
+    }
+    __device__ __forceinline__ int tok(int) const { return lane; }
+    __device__ __forceinline__ int slot(int v) const { return v; }
+    __device__ __forceinline__ int head(int s) const { return s; }
+};
+
+// Given logits [G][N_max] of the group's heads.
+struct SrcBuffer {
+    static constexpr int NV = GMAX;
+    static constexpr int NSLOT = GMAX;
+    static constexpr int XOR_LO = 1;
+    struct Frag { float z[GMAX]; };
+    const float *zb;
+    long long N_max;
+    int G, lane;
+    __device__ __forceinline__ void init(const float *z, long long nmax, int g) {
+        zb = z; N_max = nmax; G = g; lane = threadIdx.x & 31;
+    }
+    __device__ __forceinline__ void load(int tb, Frag &f) const {
+        int t = tb + lane;
+        t = t < N_max ? t : (int)N_max - 1;
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) f.z[h] = h < G ? __ldg(zb + h * N_max + t) : 0.0f;
+    }
+    __device__ __forceinline__ void eval(const Frag &f, float (&z)[NV]) const {
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) z[h] = f.z[h];
+    }
+    __device__ __forceinline__ int tok(int) const { return lane; }
+    __device__ __forceinline__ int slot(int v) const { return v; }
+    __device__ __forceinline__ int head(int s) const { return s; }
+};
+
+// Set up a source for group (b, g); qs holds the scaled q_idx (if used).
+template <typename Src>
+__device__ __forceinline__ void init_src(Src &src, const SelArgs &a, int b, int g, const float *qs) {
+    const size_t bg = (size_t)b * a.H_kv + g;
+    if constexpr (std::is_same<Src, SrcMma>::value) {
+        src.init(reinterpret_cast<const __nv_bfloat16 *>(a.kidx) + bg * a.N_max * R, a.N_max, qs, a.G);
+    } else if constexpr (std::is_same<Src, SrcBuffer>::value) {
+        src.init(a.z + ((size_t)b * a.H_q + (size_t)g * a.G) * a.N_max, a.N_max, a.G);
+    } else {
+        using IT = typename std::remove_cv<typename std::remove_pointer<decltype(src.rows)>::type>::type;
+        src.init(reinterpret_cast<const IT *>(a.kidx) + bg * a.N_max * R, a.N_max, qs, a.G);
+    }
+}
+
+template <typename Src> struct NeedsQ : std::true_type {};
+template <> struct NeedsQ<SrcBuffer> : std::false_type {};
+
+// ---------------------------------------------------------------------------
+// resolve one head's histogram (one warp): R = U(top bin), bin masses
+// S_b exp(U_b - R) in fp64, the boundary bin where the mass accumulated
+// from the top first reaches p Z.  Zeroes the histogram for the next call.
 // ---------------------------------------------------------------------------
 __device__ void resolve_head(double *gh, Resolve *out, float p, int N) {
     const int lane = threadIdx.x & 31;
@@ -192,7 +362,6 @@ __device__ void resolve_head(double *gh, Resolve *out, float p, int N) {
     top = __reduce_max_sync(0xffffffffu, top);
     Resolve r;
     r.N = N;
-    r.pad[0] = r.pad[1] = 0;
     if (top < 0 || N == 0) {
         r.Z = 0; r.above = 0; r.target = 0; r.R = 0.f; r.bstar = -1; r.mode = MODE_EMPTY;
         if (lane == 0) *out = r;
@@ -201,19 +370,19 @@ __device__ void resolve_head(double *gh, Resolve *out, float p, int N) {
         return;
     }
     const float R = bin_upper(top);
-    constexpr int SEG = (NBIN + 31) / 32;
+    constexpr int SEG = NBIN / 32;
     // lane l covers bins top - l*SEG - i, i = 0..SEG-1 (descending)
     double seg = 0.0;
     for (int i = 0; i < SEG; ++i) {
-        int bin = top - lane * SEG - i;
+        const int bin = top - lane * SEG - i;
         if (bin < 0) break;
-        double s = gh[bin];
-        if (s > 0.0) seg += s * exp((double)bin_upper(bin) - (double)R);
+        const double sb = gh[bin];
+        if (sb > 0.0) seg += sb * exp((double)bin_upper(bin) - (double)R);
     }
     double incl = seg;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        double v = __shfl_up_sync(0xffffffffu, incl, o);
+        const double v = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += v;
     }
     const double Z = __shfl_sync(0xffffffffu, incl, 31);
@@ -224,26 +393,23 @@ __device__ void resolve_head(double *gh, Resolve *out, float p, int N) {
         r.mode = MODE_KEEP_ALL; r.bstar = -1; r.above = 0; r.target = 0;
     } else {
         const double target = p <= 0.0f ? 0.0 : (double)p * Z;
-        unsigned hit = __ballot_sync(0xffffffffu, seg > 0.0 && excl + seg >= target);
-        int L;
-        double cum;
+        const unsigned hit = __ballot_sync(0xffffffffu, seg > 0.0 && excl + seg >= target);
         int bstar = -1;
-        double above = 0.0, tin = 0.0;
+        double above = 0.0, tin = INFINITY;
         if (hit) {
-            L = __ffs(hit) - 1;
-            cum = __shfl_sync(0xffffffffu, excl, L);
+            const int L = __ffs(hit) - 1;
             if (lane == L) {
+                double cum = excl;
                 for (int i = 0; i < SEG; ++i) {
-                    int bin = top - lane * SEG - i;
+                    const int bin = top - lane * SEG - i;
                     if (bin < 0) break;
-                    double s = gh[bin];
-                    if (s <= 0.0) continue;
-                    double m = s * exp((double)bin_upper(bin) - (double)R);
-                    // if rounding never crosses, the last nonempty bin is kept whole
-                    bstar = bin;
+                    const double sb = gh[bin];
+                    if (sb <= 0.0) continue;
+                    const double mb = sb * exp((double)bin_upper(bin) - (double)R);
+                    bstar = bin;       // if rounding never crosses, the last bin is kept whole
                     above = cum;
-                    if (cum + m >= target) { tin = target - cum; break; }
-                    cum += m;
+                    if (cum + mb >= target) { tin = target - cum; break; }
+                    cum += mb;
                     tin = INFINITY;
                 }
             }
@@ -251,15 +417,13 @@ __device__ void resolve_head(double *gh, Resolve *out, float p, int N) {
             above = __shfl_sync(0xffffffffu, above, L);
             tin = __shfl_sync(0xffffffffu, tin, L);
         } else {
-            // rounding kept p * Z out of reach: keep everything down to the
-            // lowest nonempty bin
+            // rounding kept p Z out of reach: keep everything down to the lowest bin
             int low = NBIN;
             for (int bin = lane; bin < NBIN; bin += 32)
                 if (gh[bin] > 0.0) low = min(low, bin);
             low = __reduce_min_sync(0xffffffffu, low);
             bstar = low;
-            double m = gh[low] * exp((double)bin_upper(low) - (double)R);
-            above = Z - m;
+            above = Z - gh[low] * exp((double)bin_upper(low) - (double)R);
             tin = INFINITY;
         }
         r.mode = MODE_NORMAL;
@@ -273,159 +437,449 @@ __device__ void resolve_head(double *gh, Resolve *out, float p, int N) {
 }
 
 // ---------------------------------------------------------------------------
-// hist: level-1 histogram + tile maxima; last CTA per (b, g) resolves.
-// grid = (ceil(N_max / SEL_CHUNK), B * n_ret)
+// scan: level-1 histograms + tile maxima; the last CTA of a group resolves.
+// grid = (ctas, B * n_ret), SCAN_THREADS threads
 // ---------------------------------------------------------------------------
-template <typename Src, typename IT>
-__global__ void __launch_bounds__(SEL_THREADS) hist_kernel(SelArgs a, SelWs w) {
+constexpr int SCAN_THREADS = 512;
+constexpr int SCAN_WARPS = SCAN_THREADS / 32;
+
+template <typename Src>
+__global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(SelArgs a, SelWs w) {
     __shared__ __align__(16) float qs[GMAX * R];
-    __shared__ float sh[GMAX][NBIN];
-    __shared__ int s_last;
-    __shared__ int s_err;
+    __shared__ uint32_t shl[2 * GMAX * NBIN];   // fixed-point bin sums: low words, then high words
+    uint32_t *const shh = shl + GMAX * NBIN;
+    __shared__ int s_last, s_err;
     const int b = blockIdx.y / a.n_ret;
     const int g = a.ret_g[blockIdx.y % a.n_ret];
     const int G = a.G;
-    const size_t bh0 = (size_t)b * a.H_q + g * G;
-    for (int i = threadIdx.x; i < GMAX * NBIN; i += blockDim.x) (&sh[0][0])[i] = 0.0f;
+    const size_t bg = (size_t)b * a.H_kv + g;
+    const size_t bh0 = (size_t)b * a.H_q + (size_t)g * G;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) s_err = 0;
-    if constexpr (!std::is_same<Src, FromBuffer>::value)
-        for (int i = threadIdx.x; i < G * R; i += blockDim.x) qs[i] = w.qidx[bh0 * R + i];
+    for (int i = threadIdx.x; i < 2 * GMAX * NBIN; i += blockDim.x) shl[i] = 0u;
+    if constexpr (NeedsQ<Src>::value) {
+        project_query(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, a.idx_scale, qs, G);
+    }
     __syncthreads();
+    if constexpr (NeedsQ<Src>::value) {
+        if (blockIdx.x == 0)
+            for (int i = threadIdx.x; i < G * R; i += blockDim.x) w.qidx[bh0 * R + i] = qs[i];
+    }
     const int N = valid_len(a.seq_lens, b, a.N_max, w.status);
     Src src;
-    if constexpr (std::is_same<Src, FromBuffer>::value) {
-        src = FromBuffer{a.z + bh0 * a.N_max, a.N_max, G};
-    } else {
-        src = Src{reinterpret_cast<const IT *>(a.kidx) + ((size_t)b * a.H_kv + g) * a.N_max * R, qs, G};
-    }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long c0 = (long long)blockIdx.x * SEL_CHUNK;
+    init_src(src, a, b, g, qs);
+    const int t_lo = (int)((long long)blockIdx.x * a.chunk);
+    const int t_hi = (int)min((long long)N, (long long)t_lo + a.chunk);
+    uint16_t *tbin = w.tilebin + bh0 * a.ntile;
+
     int err = 0;
-    for (long long tb = c0 + warp * TILE; tb < c0 + SEL_CHUNK && tb < N; tb += (SEL_THREADS / 32) * TILE) {
-        const long long t = tb + lane;
-        const bool valid = t < N;
-        float z[GMAX];
-        if (valid) src.logits(t, z);
+    typename Src::Frag cur, nxt;
+    int tb = t_lo + warp * TILE;
+    if (tb < t_hi) src.load(tb, cur);
+    for (; tb < t_hi; tb += SCAN_WARPS * TILE) {
+        const int tn = tb + SCAN_WARPS * TILE;
+        if (tn < t_hi) src.load(tn, nxt);
+        float z[Src::NV];
+        src.eval(cur, z);
+        const int nvalid = t_hi - tb;
+        int tmax[Src::NSLOT];
 #pragma unroll
-        for (int h = 0; h < GMAX; ++h) {
-            if (h >= G) break;
-            int bin = -1;
-            if (valid) {
-                float zz = z[h];
-                if (!(fabsf(zz) < Z_LIMIT)) {
-                    err = 1;
-                } else {
-                    bin = logit_bin(zz);
-                    atomicAdd(&sh[h][bin], __expf(zz - bin_upper(bin)));
-                }
+        for (int i = 0; i < Src::NSLOT; ++i) tmax[i] = -1;
+        if (nvalid >= TILE && G == GMAX) {
+            // full tile, full group: no per-value validity tests
+#pragma unroll
+            for (int v = 0; v < Src::NV; ++v) {
+                const int sl = src.slot(v);
+                const float zz = z[v] + 0.0f;      // folds -0 onto +0
+                err |= !(fabsf(zz) < Z_LIMIT);
+                uint32_t fx;
+                const int bin = bin_and_fx(zz, fx);
+                uint32_t *cell = &shl[src.head(sl) * NBIN + bin];
+                const uint32_t old = atomicAdd(cell, fx);
+                if (old + fx < old) atomicAdd(cell + GMAX * NBIN, 1u);
+                tmax[sl] = max(tmax[sl], bin);
             }
-            int mx = __reduce_max_sync(0xffffffffu, bin);
-            if (lane == h) w.tilebin[(bh0 + h) * a.ntile + (tb / TILE)] = (uint16_t)(mx + 1);
+        } else {
+#pragma unroll
+            for (int v = 0; v < Src::NV; ++v) {
+                const int sl = src.slot(v);
+                const int h = src.head(sl);
+                if (h >= G || src.tok(v) >= nvalid) continue;
+                const float zz = z[v] + 0.0f;
+                if (!(fabsf(zz) < Z_LIMIT)) { err = 1; continue; }
+                uint32_t fx;
+                const int bin = bin_and_fx(zz, fx);
+                uint32_t *cell = &shl[h * NBIN + bin];
+                const uint32_t old = atomicAdd(cell, fx);
+                if (old + fx < old) atomicAdd(cell + GMAX * NBIN, 1u);
+                tmax[sl] = max(tmax[sl], bin);
+            }
         }
+#pragma unroll
+        for (int i = 0; i < Src::NSLOT; ++i)
+#pragma unroll
+            for (int o = Src::XOR_LO; o < 32; o <<= 1) tmax[i] = max(tmax[i], __shfl_xor_sync(0xffffffffu, tmax[i], o));
+        if (lane < Src::XOR_LO) {
+#pragma unroll
+            for (int i = 0; i < Src::NSLOT; ++i) {
+                const int h = src.head(i);
+                if (h < G) tbin[(size_t)h * a.ntile + tb / TILE] = (uint16_t)(tmax[i] + 1);
+            }
+        }
+        cur = nxt;
     }
     if (err) s_err = 1;
     __syncthreads();
     if (s_err && threadIdx.x == 0) set_status(w.status, RTP_ERR_RANGE);
     for (int i = threadIdx.x; i < G * NBIN; i += blockDim.x) {
-        float v = (&sh[0][0])[i];
-        if (v != 0.0f) atomicAdd(&w.hist[bh0 * NBIN + i], (double)v);
+        const uint32_t lo = shl[i], hi = shh[i];
+        if (lo | hi)
+            atomicAdd(&w.hist[bh0 * NBIN + i], ((double)hi * 4294967296.0 + (double)lo) * (1.0 / FX_ONE));
     }
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) {
-        unsigned old = atomicAdd(&w.arrive[(size_t)b * a.H_kv + g], 1u);
-        s_last = (old == gridDim.x - 1);
-    }
+    if (threadIdx.x == 0) s_last = atomicAdd(&w.arrive[bg], 1u) == (unsigned)(gridDim.x - 1);
     __syncthreads();
     if (!s_last) return;
     __threadfence();
     if (warp < G) {
         const size_t bh = bh0 + warp;
         resolve_head(w.hist + bh * NBIN, w.res + bh, a.p, N);
-        if (lane == 0) { w.list_cnt[bh] = 0; w.cand_cnt[bh] = 0; }
+        if (lane == 0) { w.cand_cnt[bh] = 0; w.list_cnt[bh] = 0; }
     }
-    if (threadIdx.x == 0) w.arrive[(size_t)b * a.H_kv + g] = 0;
+    if (threadIdx.x == 0) w.arrive[bg] = 0;
 }
 
 // ---------------------------------------------------------------------------
-// collect: kept ids and boundary-bin candidates.  grid as hist_kernel.
+// scan for bf16 index keys: TMA bulk-copy ring.  One producer warp streams
+// the CTA's contiguous index-key range into NSTAGE shared-memory stages
+// (cp.async.bulk, completion on mbarriers); TC_WARPS consumer warps take
+// one 32-token tile each per stage, compute the logits on the tensor cores
+// (fragments read from shared memory), and add their level-1 masses to
+// 32-bit fixed-point bin counters (2^18 units per unit of mass).  Every
+// SPILL_STAGES stages (<= 7680 tokens, so a counter cannot wrap) the
+// counters are moved into 64-bit accumulators.  All waits are bounded.
+// grid = (ctas, B * n_ret), TC_THREADS threads, TC_SMEM dynamic smem.
 // ---------------------------------------------------------------------------
-template <typename Src, typename IT>
-__global__ void __launch_bounds__(SEL_THREADS) collect_kernel(SelArgs a, SelWs w) {
+constexpr int TC_WARPS = 24;                             // consumer warps
+constexpr int TC_THREADS = (TC_WARPS + 1) * 32;          // + one producer warp
+constexpr int ST_TOK = TC_WARPS * TILE;                  // tokens per stage
+constexpr int ST_BYTES = ST_TOK * R * 2;                 // bf16 index keys
+constexpr int NSTAGE = 4;
+constexpr int SPILL_STAGES = 10;                         // 7680 tokens
+constexpr float FX18 = 262144.0f;                        // 2^18
+constexpr int TC_SMEM = NSTAGE * ST_BYTES + GMAX * NBIN * 4 + GMAX * NBIN * 8 + 2 * NSTAGE * 8;
+static_assert((long long)SPILL_STAGES * ST_TOK * 262144LL < 4294967296LL, "bin counters would wrap");
+
+__device__ __forceinline__ int bin_and_fx18(float z, uint32_t &fx) {
+    const uint32_t u = __float_as_uint(z);
+    const int s = (int)u >> 31;
+    int k = (int)((u << 1) >> (24 - MB)) - (int)BIN_BASE;
+    k = min(max(k, 0), 255);
+    const uint32_t eb = (uint32_t)(k + (int)BIN_BASE + 1 + s) << (23 - MB);
+    const float U = __uint_as_float(eb | ((uint32_t)s & 0x80000000u));
+    fx = __float2uint_rn(ex2_sfu(fmaf(z - U, 1.4426950408889634f, 18.0f)));
+    return 256 + (k ^ s);
+}
+
+__global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelWs w) {
+    extern __shared__ __align__(128) uint8_t dsm[];
+    uint8_t *ring = dsm;
+    uint32_t *h32 = reinterpret_cast<uint32_t *>(dsm + NSTAGE * ST_BYTES);
+    unsigned long long *h64 = reinterpret_cast<unsigned long long *>(dsm + NSTAGE * ST_BYTES + GMAX * NBIN * 4);
+    uint64_t *full = reinterpret_cast<uint64_t *>(dsm + NSTAGE * ST_BYTES + GMAX * NBIN * 12);
+    uint64_t *empty = full + NSTAGE;
     __shared__ __align__(16) float qs[GMAX * R];
-    __shared__ int s_bstar[GMAX];
-    __shared__ int s_mode[GMAX];
+    __shared__ int s_last, s_err, s_abort;
     const int b = blockIdx.y / a.n_ret;
     const int g = a.ret_g[blockIdx.y % a.n_ret];
     const int G = a.G;
-    const size_t bh0 = (size_t)b * a.H_q + g * G;
-    if (threadIdx.x < G) {
-        const Resolve &r = w.res[bh0 + threadIdx.x];
-        s_bstar[threadIdx.x] = r.bstar;
-        s_mode[threadIdx.x] = r.mode;
+    const size_t bg = (size_t)b * a.H_kv + g;
+    const size_t bh0 = (size_t)b * a.H_q + (size_t)g * G;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        s_err = 0;
+        s_abort = 0;
+        for (int i = 0; i < NSTAGE; ++i) { mbar_init(&full[i], 1u); mbar_init(&empty[i], (uint32_t)TC_WARPS); }
+        fence_mbar_init();
     }
-    if constexpr (!std::is_same<Src, FromBuffer>::value)
+    for (int i = threadIdx.x; i < GMAX * NBIN; i += blockDim.x) { h32[i] = 0u; h64[i] = 0ull; }
+    project_query(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, a.idx_scale, qs, G);
+    __syncthreads();
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < G * R; i += blockDim.x) w.qidx[bh0 * R + i] = qs[i];
+    const int N = valid_len(a.seq_lens, b, a.N_max, w.status);
+    const int t_lo = (int)((long long)blockIdx.x * a.chunk);
+    const int t_hi = (int)min((long long)N, (long long)t_lo + a.chunk);
+    const int n_st = t_hi > t_lo ? (t_hi - t_lo + ST_TOK - 1) / ST_TOK : 0;
+    const __nv_bfloat16 *rows = reinterpret_cast<const __nv_bfloat16 *>(a.kidx) + bg * a.N_max * R;
+
+    if (warp == TC_WARPS) {
+        // producer
+        if (lane == 0) {
+            int issued = 0;
+            for (int it = 0; it < n_st; ++it) {
+                const int st = it % NSTAGE;
+                if (it >= NSTAGE && !mbar_wait(&empty[st], (uint32_t)((it / NSTAGE - 1) & 1))) {
+                    set_status(w.status, RTP_ERR_TIMEOUT);
+                    s_abort = 1;
+                    break;
+                }
+                if (*(volatile int *)&s_abort) break;
+                fence_proxy_async();
+                const int tok0 = t_lo + it * ST_TOK;
+                const uint32_t bytes = (uint32_t)min(ST_TOK, t_hi - tok0) * (uint32_t)(R * 2);
+                mbar_expect_tx(&full[st], bytes);
+                bulk_g2s(ring + st * ST_BYTES, rows + (size_t)tok0 * R, bytes, &full[st]);
+                issued = it + 1;
+            }
+            // no copy may still be landing in shared memory when the CTA exits
+            for (int it = max(0, issued - NSTAGE); it < issued; ++it)
+                mbar_wait(&full[it % NSTAGE], (uint32_t)((it / NSTAGE) & 1));
+        }
+    } else {
+        // consumers
+        SrcMma src;
+        src.init(rows, a.N_max, qs, G);
+        const int gid = lane >> 2, tig = lane & 3;
+        uint32_t *hrow[2] = {h32 + (2 * tig) * NBIN, h32 + (2 * tig + 1) * NBIN};
+        const bool full_group = G == GMAX;
+        int err = 0;
+        uint16_t *tbin = w.tilebin + bh0 * a.ntile;
+        // After a timeout every consumer warp keeps iterating without
+        // waiting or working, so the named barrier below stays balanced.
+        bool dead = false;
+        for (int it = 0; it < n_st; ++it) {
+            const int st = it % NSTAGE;
+            if (!dead) dead = *(volatile int *)&s_abort != 0;
+            if (!dead && !mbar_wait(&full[st], (uint32_t)((it / NSTAGE) & 1))) {
+                set_status(w.status, RTP_ERR_TIMEOUT);
+                s_abort = 1;
+                dead = true;
+            }
+            const int tb = t_lo + it * ST_TOK + warp * TILE;
+            const int nvalid = dead ? 0 : t_hi - tb;
+            if (nvalid > 0) {
+                const uint8_t *tile = ring + st * ST_BYTES + warp * (TILE * R * 2);
+                SrcMma::Frag f;
+#pragma unroll
+                for (int i = 0; i < 2; ++i)
+#pragma unroll
+                    for (int r = 0; r < 2; ++r)
+                        f.a[i][r] = *reinterpret_cast<const uint2 *>(tile + (16 * i + gid + 8 * r) * (R * 2) + 8 * tig);
+                float z[SrcMma::NV];
+                src.eval(f, z);
+                int tmax[2] = {-1, -1};
+                if (nvalid >= TILE && full_group) {
+#pragma unroll
+                    for (int v = 0; v < SrcMma::NV; ++v) {
+                        const int sl = v & 1;
+                        const float zz = z[v] + 0.0f;       // folds -0 onto +0
+                        err |= !(fabsf(zz) < Z_LIMIT);
+                        uint32_t fx;
+                        const int bin = bin_and_fx18(zz, fx);
+                        atomicAdd(hrow[sl] + bin, fx);
+                        tmax[sl] = max(tmax[sl], bin);
+                    }
+                } else {
+#pragma unroll
+                    for (int v = 0; v < SrcMma::NV; ++v) {
+                        const int sl = v & 1;
+                        if (2 * tig + sl >= G || src.tok(v) >= nvalid) continue;
+                        const float zz = z[v] + 0.0f;
+                        if (!(fabsf(zz) < Z_LIMIT)) { err = 1; continue; }
+                        uint32_t fx;
+                        const int bin = bin_and_fx18(zz, fx);
+                        atomicAdd(hrow[sl] + bin, fx);
+                        tmax[sl] = max(tmax[sl], bin);
+                    }
+                }
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    tmax[i] = max(tmax[i], __shfl_xor_sync(0xffffffffu, tmax[i], 4));
+                    tmax[i] = max(tmax[i], __shfl_xor_sync(0xffffffffu, tmax[i], 8));
+                    tmax[i] = max(tmax[i], __shfl_xor_sync(0xffffffffu, tmax[i], 16));
+                }
+                if (lane < 4) {
+#pragma unroll
+                    for (int i = 0; i < 2; ++i)
+                        if (2 * lane + i < G) tbin[(size_t)(2 * lane + i) * a.ntile + tb / TILE] = (uint16_t)(tmax[i] + 1);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);
+            if ((it + 1) % SPILL_STAGES == 0 && it + 1 < n_st) {
+                asm volatile("bar.sync 1, %0;" ::"r"(TC_WARPS * 32) : "memory");
+                for (int i = threadIdx.x; i < GMAX * NBIN; i += TC_WARPS * 32) {
+                    h64[i] += h32[i];
+                    h32[i] = 0u;
+                }
+                asm volatile("bar.sync 1, %0;" ::"r"(TC_WARPS * 32) : "memory");
+            }
+        }
+        if (err) s_err = 1;
+    }
+    __syncthreads();
+    if (s_err && threadIdx.x == 0) set_status(w.status, RTP_ERR_RANGE);
+    for (int i = threadIdx.x; i < G * NBIN; i += blockDim.x) {
+        const unsigned long long v = h64[i] + h32[i];
+        if (v) atomicAdd(&w.hist[bh0 * NBIN + i], (double)v * (1.0 / FX18));
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = atomicAdd(&w.arrive[bg], 1u) == (unsigned)(gridDim.x - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (warp < G) {
+        const size_t bh = bh0 + warp;
+        resolve_head(w.hist + bh * NBIN, w.res + bh, a.p, N);
+        if (lane == 0) { w.cand_cnt[bh] = 0; w.list_cnt[bh] = 0; }
+    }
+    if (threadIdx.x == 0) w.arrive[bg] = 0;
+}
+
+// ---------------------------------------------------------------------------
+// collect: kept ids above b*, candidates in b*.  grid as scan.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void warp_append(bool c, int h, unsigned lane_lt, uint32_t *cnt_base,
+                                            unsigned &pos) {
+    const unsigned act = __ballot_sync(0xffffffffu, c);
+    if (!act) return;
+    if (c) {
+        const unsigned grp = __match_any_sync(act, h);
+        const int leader = __ffs(grp) - 1;
+        unsigned base = 0;
+        if ((threadIdx.x & 31) == leader) base = atomicAdd(&cnt_base[h], (unsigned)__popc(grp));
+        base = __shfl_sync(grp, base, leader);
+        pos = base + __popc(grp & lane_lt);
+    }
+}
+
+constexpr int COL_THREADS = 512;
+constexpr int COL_WARPS = COL_THREADS / 32;
+
+constexpr int KCAP = 256;     // kept ids staged per head per CTA
+constexpr int CCAP = 128;     // candidates staged per head per CTA
+
+template <typename Src>
+__global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w) {
+    __shared__ __align__(16) float qs[GMAX * R];
+    __shared__ int s_bstar[GMAX];
+    __shared__ int s_mode[GMAX];
+    __shared__ unsigned s_kc[GMAX], s_cc[GMAX];
+    __shared__ int32_t s_kbuf[GMAX * KCAP];
+    __shared__ unsigned long long s_cbuf[GMAX * CCAP];
+    const int b = blockIdx.y / a.n_ret;
+    const int g = a.ret_g[blockIdx.y % a.n_ret];
+    const int G = a.G;
+    const size_t bh0 = (size_t)b * a.H_q + (size_t)g * G;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x < GMAX) {
+        int mode = MODE_EMPTY, bs = NBIN;
+        if (threadIdx.x < G) {
+            const Resolve r = w.res[bh0 + threadIdx.x];
+            mode = r.mode;
+            bs = r.bstar;
+        }
+        s_mode[threadIdx.x] = mode;
+        // keep-all heads need no collect pass: finalize lists every token
+        s_bstar[threadIdx.x] = mode == MODE_NORMAL ? bs : NBIN;
+        s_kc[threadIdx.x] = 0u;
+        s_cc[threadIdx.x] = 0u;
+    }
+    if constexpr (NeedsQ<Src>::value)
         for (int i = threadIdx.x; i < G * R; i += blockDim.x) qs[i] = w.qidx[bh0 * R + i];
     __syncthreads();
     const int N = w.res[bh0].N;
     Src src;
-    if constexpr (std::is_same<Src, FromBuffer>::value) {
-        src = FromBuffer{a.z + bh0 * a.N_max, a.N_max, G};
-    } else {
-        src = Src{reinterpret_cast<const IT *>(a.kidx) + ((size_t)b * a.H_kv + g) * a.N_max * R, qs, G};
-    }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const unsigned lt_mask = (1u << lane) - 1u;
-    const long long c0 = (long long)blockIdx.x * SEL_CHUNK;
-    for (long long tb = c0 + warp * TILE; tb < c0 + SEL_CHUNK && tb < N; tb += (SEL_THREADS / 32) * TILE) {
-        // skip tiles whose largest bin is below every head's boundary bin
-        bool need = false;
-        for (int h = 0; h < G; ++h) {
-            int mode = s_mode[h];
-            if (mode == MODE_KEEP_ALL) { need = true; break; }
-            if (mode == MODE_NORMAL &&
-                (int)w.tilebin[(bh0 + h) * a.ntile + tb / TILE] - 1 >= s_bstar[h]) { need = true; break; }
-        }
-        if (!need) continue;
-        const long long t = tb + lane;
-        const bool valid = t < N;
-        float z[GMAX];
-        if (valid) src.logits(t, z);
+    init_src(src, a, b, g, qs);
+    const int t_lo = (int)((long long)blockIdx.x * a.chunk);
+    const int t_hi = (int)min((long long)N, (long long)t_lo + a.chunk);
+    const unsigned lt = (1u << lane) - 1u;
+    const uint16_t *tbin = w.tilebin + bh0 * a.ntile;
+    int bst[GMAX];
 #pragma unroll
-        for (int h = 0; h < GMAX; ++h) {
-            if (h >= G) break;
-            const int mode = s_mode[h];
-            if (mode == MODE_EMPTY) continue;
-            bool keep = false, cand = false;
-            uint32_t key = 0;
-            if (valid) {
-                if (mode == MODE_KEEP_ALL) {
-                    keep = true;
-                } else if (fabsf(z[h]) < Z_LIMIT) {
-                    const int bin = logit_bin(z[h]);
-                    keep = bin > s_bstar[h];
-                    cand = bin == s_bstar[h];
-                    key = logit_key(z[h]);
+    for (int h = 0; h < GMAX; ++h) bst[h] = s_bstar[h];
+
+    // Warp w owns tiles w, w + COL_WARPS, ...; windows of 32 of them are
+    // screened at once (lane i: the i-th tile of the window, all heads),
+    // then the needed ones are processed with the next one's load in flight.
+    for (int wbase = 0;; wbase += 32) {
+        const int tb_l = t_lo + (warp + (wbase + lane) * COL_WARPS) * TILE;
+        unsigned hm = 0u;                        // heads that need lane's tile
+        if (tb_l < t_hi) {
+            const int ti = tb_l / TILE;
+#pragma unroll
+            for (int h = 0; h < GMAX; ++h)
+                if (h < G && (int)tbin[(size_t)h * a.ntile + ti] - 1 >= bst[h]) hm |= 1u << h;
+        }
+        const unsigned any_valid = __ballot_sync(0xffffffffu, tb_l < t_hi);
+        if (!any_valid) break;
+        unsigned todo = __ballot_sync(0xffffffffu, hm != 0u);
+        if (!todo) continue;
+        int i = __ffs(todo) - 1;
+        typename Src::Frag cur, nxt;
+        src.load(__shfl_sync(0xffffffffu, tb_l, i), cur);
+        while (true) {
+            const int tb = __shfl_sync(0xffffffffu, tb_l, i);
+            const unsigned hmask = __shfl_sync(0xffffffffu, hm, i);
+            todo &= todo - 1u;
+            const int inext = todo ? __ffs(todo) - 1 : -1;
+            if (inext >= 0) src.load(__shfl_sync(0xffffffffu, tb_l, inext), nxt);
+            float z[Src::NV];
+            src.eval(cur, z);
+#pragma unroll
+            for (int v = 0; v < Src::NV; ++v) {
+                const int h = src.head(src.slot(v));
+                const int t = tb + src.tok(v);
+                if (h < G && t < t_hi && ((hmask >> h) & 1u)) {
+                    const float zz = z[v] + 0.0f;
+                    if (fabsf(zz) < Z_LIMIT) {
+                        const int bin = logit_bin(zz);
+                        const int bs = s_bstar[h];
+                        if (bin > bs) {
+                            const unsigned p = atomicAdd(&s_kc[h], 1u);
+                            if (p < (unsigned)KCAP) {
+                                s_kbuf[h * KCAP + p] = t;
+                            } else {
+                                const unsigned q = atomicAdd(&w.list_cnt[bh0 + h], 1u);
+                                a.lists[(bh0 + h) * a.N_max + q] = t;
+                            }
+                        } else if (bin == bs) {
+                            const unsigned long long key =
+                                ((unsigned long long)logit_key(zz) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)t);
+                            const unsigned p = atomicAdd(&s_cc[h], 1u);
+                            if (p < (unsigned)CCAP) {
+                                s_cbuf[h * CCAP + p] = key;
+                            } else {
+                                const unsigned q = atomicAdd(&w.cand_cnt[bh0 + h], 1u);
+                                w.cands[(bh0 + h) * a.N_max + q] = key;
+                            }
+                        }
+                    }
                 }
             }
-            const size_t bh = bh0 + h;
-            unsigned bk = __ballot_sync(0xffffffffu, keep);
-            if (bk) {
-                unsigned base = 0;
-                if (lane == 0) base = atomicAdd(&w.list_cnt[bh], (unsigned)__popc(bk));
-                base = __shfl_sync(0xffffffffu, base, 0);
-                if (keep) a.lists[bh * a.N_max + base + __popc(bk & lt_mask)] = (int32_t)t;
-            }
-            unsigned bc = __ballot_sync(0xffffffffu, cand);
-            if (bc) {
-                unsigned base = 0;
-                if (lane == 0) base = atomicAdd(&w.cand_cnt[bh], (unsigned)__popc(bc));
-                base = __shfl_sync(0xffffffffu, base, 0);
-                if (cand)
-                    w.cands[bh * a.N_max + base + __popc(bc & lt_mask)] =
-                        ((unsigned long long)key << 32) | (unsigned long long)(0xffffffffu - (uint32_t)t);
-            }
+            if (inext < 0) break;
+            i = inext;
+            cur = nxt;
         }
+    }
+    // flush the staged ids: one global reservation per head and kind
+    __syncthreads();
+    if (warp < G) {
+        const size_t bh = bh0 + warp;
+        const unsigned nk = min(s_kc[warp], (unsigned)KCAP);
+        const unsigned ncd = min(s_cc[warp], (unsigned)CCAP);
+        unsigned kb = 0u, cb = 0u;
+        if (lane == 0) {
+            if (nk) kb = atomicAdd(&w.list_cnt[bh], nk);
+            if (ncd) cb = atomicAdd(&w.cand_cnt[bh], ncd);
+        }
+        kb = __shfl_sync(0xffffffffu, kb, 0);
+        cb = __shfl_sync(0xffffffffu, cb, 0);
+        for (unsigned j = lane; j < nk; j += 32) a.lists[bh * a.N_max + kb + j] = s_kbuf[warp * KCAP + j];
+        for (unsigned j = lane; j < ncd; j += 32) w.cands[bh * a.N_max + cb + j] = s_cbuf[warp * CCAP + j];
     }
 }
 
@@ -433,135 +887,248 @@ __global__ void __launch_bounds__(SEL_THREADS) collect_kernel(SelArgs a, SelWs w
 // finalize: exact selection inside the boundary bin.  One CTA per head.
 // grid = (B * n_ret * G)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ double cand_mass(unsigned long long c, float R) {
-    return exp((double)key_logit((uint32_t)(c >> 32)) - (double)R);
-}
+__device__ __forceinline__ float cand_logit(unsigned long long c) { return key_logit((uint32_t)(c >> 32)); }
 
-__global__ void __launch_bounds__(SEL_THREADS) finalize_kernel(SelArgs a, SelWs w) {
-    __shared__ double smass[256];
-    __shared__ unsigned scnt[256];
-    __shared__ int s_digit;
+constexpr int FIN_THREADS = 256;
+constexpr int FIN_WARPS = FIN_THREADS / 32;
+constexpr int FIN_CAP = 2048;             // candidates staged in shared memory
+// Exact selection inside the boundary bin.  One CTA per retrieval head;
+// grid = (B * n_ret * G).  Candidate masses relative to the boundary bin's
+// upper edge U* are each in (e^-32, 1]; they are summed in fixed point with
+// S = 2^62 / nc units per unit of mass, so sums stay below 2^62 and do not
+// depend on the order of the adds.  The last CTA to finish writes the
+// exclusive prefix of list-attention items per head (item_pre).
+__global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs w) {
+    __shared__ unsigned long long hfx[256];
+    __shared__ unsigned hcnt[256];
+    __shared__ unsigned long long cbuf[FIN_CAP];
+    __shared__ unsigned long long fbuf[FIN_CAP];
+    __shared__ unsigned long long s_min, s_max, s_theta, s_excl, s_kept;
+    __shared__ unsigned s_base;
+    __shared__ int s_digit, s_last;
     __shared__ unsigned s_dcnt;
-    __shared__ double s_excl;
-    __shared__ unsigned long long s_theta;
-    __shared__ double s_red[SEL_THREADS / 32];
     const int G = a.G;
-    const int hb = blockIdx.x;                  // (b, ret group, head in group)
+    const int hb = blockIdx.x;
     const int b = hb / (a.n_ret * G);
     const int gi = (hb / G) % a.n_ret;
     const int h = a.ret_g[gi] * G + hb % G;
     const size_t bh = (size_t)b * a.H_q + h;
     const Resolve r = w.res[bh];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (r.mode != MODE_NORMAL) {
-        if (tid == 0) {
-            a.count_out[bh] = r.mode == MODE_KEEP_ALL ? (int32_t)w.list_cnt[bh] : 0;
-            if (a.mass_out) a.mass_out[bh] = r.mode == MODE_KEEP_ALL ? 1.0f : 0.0f;
-        }
-        return;
-    }
-    const unsigned nc = w.cand_cnt[bh];
-    const unsigned long long *cs = w.cands + bh * a.N_max;
-    double t = r.target;
-    unsigned long long prefix = 0;
-    unsigned long long theta = 0;
-    bool found = false;
-    for (int level = 0; level < 8 && !found; ++level) {
-        const int shift = 56 - 8 * level;
-        for (int i = tid; i < 256; i += blockDim.x) { smass[i] = 0.0; scnt[i] = 0; }
+    const unsigned nc = r.mode == MODE_NORMAL ? w.cand_cnt[bh] : 0u;
+    const unsigned long long *cg = w.cands + bh * a.N_max;
+    int32_t *lst = a.lists + bh * a.N_max;
+    int count = 0;
+    float mass = 0.0f;
+
+    if (r.mode == MODE_KEEP_ALL) {
+        for (int t = tid; t < r.N; t += blockDim.x) lst[t] = t;
+        count = r.N;
+        mass = 1.0f;
+    } else if (r.mode != MODE_NORMAL || nc == 0u) {
+        count = r.mode == MODE_EMPTY ? 0 : (int)w.list_cnt[bh];
+        mass = r.mode == MODE_EMPTY ? 0.0f : (float)(r.above / r.Z);
+    } else {
+        const float Ub = bin_upper(r.bstar);
+        const double S = ldexp(1.0, 62) / (double)nc;
+        const bool staged = nc <= (unsigned)FIN_CAP;
+        auto fx_of = [&](unsigned long long v) -> unsigned long long {
+            const float m = ex2_sfu((cand_logit(v) - Ub) * 1.4426950408889634f);
+            return (unsigned long long)((double)m * S);
+        };
+        if (tid == 0) { s_min = ~0ull; s_max = 0ull; s_kept = 0ull; s_base = 0u; }
         __syncthreads();
-        for (unsigned c = tid; c < nc; c += blockDim.x) {
-            unsigned long long v = cs[c];
-            if (level > 0 && (v >> (shift + 8)) != prefix) continue;
-            int dg = (int)((v >> shift) & 255ull);
-            atomicAdd(&smass[dg], cand_mass(v, r.R));
-            atomicAdd(&scnt[dg], 1u);
-        }
-        __syncthreads();
-        if (warp == 0) {
-            // lane covers digits 255 - 8*lane - i, i = 0..7 (descending)
-            double seg = 0.0;
-            for (int i = 0; i < 8; ++i) seg += smass[255 - 8 * lane - i];
-            unsigned segc = 0;
-            for (int i = 0; i < 8; ++i) segc += scnt[255 - 8 * lane - i];
-            double incl = seg;
-            for (int o = 1; o < 32; o <<= 1) {
-                double v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
+        {
+            unsigned long long lo = ~0ull, hi = 0ull;
+            for (unsigned c = tid; c < nc; c += blockDim.x) {
+                const unsigned long long v = cg[c];
+                if (staged) { cbuf[c] = v; fbuf[c] = fx_of(v); }
+                lo = v < lo ? v : lo;
+                hi = v > hi ? v : hi;
             }
-            const double excl = incl - seg;
-            unsigned hit = __ballot_sync(0xffffffffu, segc > 0 && excl + seg >= t);
-            int L;
-            if (hit) {
-                L = __ffs(hit) - 1;
-            } else {
-                unsigned ne = __ballot_sync(0xffffffffu, segc > 0);
-                L = 31 - __clz(ne);   // lowest nonempty segment: keep everything above
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const unsigned long long l2 = __shfl_xor_sync(0xffffffffu, lo, o);
+                const unsigned long long h2 = __shfl_xor_sync(0xffffffffu, hi, o);
+                lo = l2 < lo ? l2 : lo;
+                hi = h2 > hi ? h2 : hi;
             }
-            if (lane == L) {
-                double cum = excl;
-                int dsel = -1;
-                for (int i = 0; i < 8; ++i) {
-                    int dg = 255 - 8 * lane - i;
-                    if (scnt[dg] == 0) continue;
-                    dsel = dg;
-                    if (hit && cum + smass[dg] >= t) break;
-                    if (!hit) { /* keep scanning to the last nonempty digit */ }
-                    cum += smass[dg];
-                }
-                if (!hit) {
-                    // every candidate under this prefix is kept: cum counts all but dsel
-                    cum = excl;
-                    for (int i = 0; i < 8; ++i) {
-                        int dg = 255 - 8 * lane - i;
-                        if (dg == dsel) break;
-                        cum += smass[dg];
-                    }
-                }
-                s_digit = dsel;
-                s_dcnt = scnt[dsel];
-                s_excl = cum;
+            if (lane == 0) {
+                atomicMin(&s_min, lo);
+                atomicMax(&s_max, hi);
             }
         }
         __syncthreads();
-        const int dsel = s_digit;
-        t -= s_excl;
-        prefix = (prefix << 8) | (unsigned long long)dsel;
-        if (s_dcnt == 1u || level == 7) {
-            if (level == 7) {
-                theta = prefix;
-            } else {
-                if (tid == 0) s_theta = 0;
+        const double tS = r.target * exp((double)r.R - (double)Ub) * S;
+        unsigned long long T = !(tS < 9.0e18) ? ~0ull : (unsigned long long)llrint(tS);
+        const unsigned long long diff = s_min ^ s_max;
+        unsigned long long theta = s_min;          // one candidate (or all equal): keep all
+        if (diff != 0ull) {
+            int shift = 63 - __clzll((long long)diff);
+            shift = shift >= 7 ? shift - 7 : 0;
+            unsigned long long pmask = shift + 8 >= 64 ? 0ull : ~((1ull << (shift + 8)) - 1ull);
+            unsigned long long prefix = s_min & pmask;
+            for (int level = 0; level < 16; ++level) {
+                for (int i = tid; i < 256; i += blockDim.x) { hfx[i] = 0ull; hcnt[i] = 0u; }
                 __syncthreads();
                 for (unsigned c = tid; c < nc; c += blockDim.x) {
-                    unsigned long long v = cs[c];
-                    if ((v >> shift) == prefix) s_theta = v;
+                    const unsigned long long v = staged ? cbuf[c] : cg[c];
+                    if ((v & pmask) != prefix) continue;
+                    const int dg = (int)((v >> shift) & 255ull);
+                    atomicAdd(&hfx[dg], staged ? fbuf[c] : fx_of(v));
+                    atomicAdd(&hcnt[dg], 1u);
                 }
                 __syncthreads();
-                theta = s_theta;
+                if (warp == 0) {
+                    // lane covers digits 255 - 8 lane - i (descending)
+                    unsigned long long seg = 0ull;
+                    unsigned segc = 0u;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) { seg += hfx[255 - 8 * lane - i]; segc += hcnt[255 - 8 * lane - i]; }
+                    unsigned long long incl = seg;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += v;
+                    }
+                    const unsigned long long excl = incl - seg;
+                    const unsigned hit = __ballot_sync(0xffffffffu, segc > 0u && incl >= T);
+                    const unsigned ne = __ballot_sync(0xffffffffu, segc > 0u);
+                    const int L = hit ? __ffs(hit) - 1 : 31 - __clz(ne);
+                    if (lane == L) {
+                        unsigned long long cum = excl, before = excl;
+                        int dsel = -1;
+                        for (int i = 0; i < 8; ++i) {
+                            const int dg = 255 - 8 * lane - i;
+                            if (hcnt[dg] == 0u) continue;
+                            dsel = dg;
+                            before = cum;
+                            if (hit && cum + hfx[dg] >= T) break;
+                            cum += hfx[dg];
+                        }
+                        s_digit = dsel;
+                        s_dcnt = hcnt[dsel];
+                        s_excl = before;
+                    }
+                }
+                __syncthreads();
+                const int dsel = s_digit;
+                T = T >= s_excl ? T - s_excl : 0ull;
+                prefix |= (unsigned long long)dsel << shift;
+                pmask |= 255ull << shift;
+                if (s_dcnt == 1u) {
+                    for (unsigned c = tid; c < nc; c += blockDim.x) {
+                        const unsigned long long v = staged ? cbuf[c] : cg[c];
+                        if ((v & pmask) == prefix) s_theta = v;
+                    }
+                    __syncthreads();
+                    theta = s_theta;
+                    break;
+                }
+                if (shift == 0) { theta = prefix; break; }    // every bit fixed
+                shift = shift >= 8 ? shift - 8 : 0;
+                __syncthreads();
             }
-            found = true;
         }
+        // kept = candidates at or above theta, appended after the ids the
+        // collect pass wrote (block-wide ranks, no global atomics)
+        const unsigned base0 = w.list_cnt[bh];
+        unsigned long long kept = 0ull;
+        const unsigned lt = (1u << lane) - 1u;
+        for (unsigned c0 = 0; c0 < nc; c0 += blockDim.x) {
+            const unsigned c = c0 + tid;
+            unsigned long long v = 0ull;
+            bool k = false;
+            if (c < nc) {
+                v = staged ? cbuf[c] : cg[c];
+                k = v >= theta;
+            }
+            const unsigned bal = __ballot_sync(0xffffffffu, k);
+            unsigned wbase = 0u;
+            if (lane == 0 && bal) wbase = atomicAdd(&s_base, (unsigned)__popc(bal));
+            wbase = __shfl_sync(0xffffffffu, wbase, 0);
+            if (k) {
+                lst[base0 + wbase + __popc(bal & lt)] = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
+                kept += staged ? fbuf[c] : fx_of(v);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
+        if (lane == 0) atomicAdd(&s_kept, kept);
         __syncthreads();
+        count = (int)(base0 + s_base);
+        const double kept_mass = (double)s_kept / S * exp((double)Ub - (double)r.R);
+        mass = (float)((r.above + kept_mass) / r.Z);
     }
-    // append candidates at or above theta
-    double kept = 0.0;
-    for (unsigned c = tid; c < nc; c += blockDim.x) {
-        unsigned long long v = cs[c];
-        if (v >= theta) {
-            unsigned pos = atomicAdd(&w.list_cnt[bh], 1u);
-            a.lists[bh * a.N_max + pos] = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
-            kept += cand_mass(v, r.R);
+    if (tid == 0) {
+        a.count_out[bh] = count;
+        if (a.mass_out) a.mass_out[bh] = mass;
+    }
+    // the last CTA builds the list-attention work prefix over all heads
+    if (!a.item_pre) return;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(w.fin_arrive, 1u) == gridDim.x - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    if (warp == 0) {
+        const int nh = gridDim.x;
+        int run = 0;
+        for (int base = 0; base < nh; base += 32) {
+            const int hi = base + lane;
+            int it = 0;
+            if (hi < nh) {
+                const int bb = hi / (a.n_ret * G);
+                const int hh = a.ret_g[(hi / G) % a.n_ret] * G + hi % G;
+                it = list_items(__ldcg(a.count_out + (size_t)bb * a.H_q + hh));
+            }
+            int incl = it;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (hi < nh) a.item_pre[hi] = run + incl - it;
+            run += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) {
+            a.item_pre[nh] = run;
+            *w.fin_arrive = 0u;
         }
     }
-    kept = warp_sum_d(kept);
-    if (lane == 0) s_red[warp] = kept;
+}
+
+// ---------------------------------------------------------------------------
+// rtp_index_scores: write z for every retrieval head (same logit sources)
+// ---------------------------------------------------------------------------
+template <typename Src>
+__global__ void __launch_bounds__(SC_THREADS) scores_kernel(SelArgs a, SelWs w, float *z_out) {
+    __shared__ __align__(16) float qs[GMAX * R];
+    const int b = blockIdx.y / a.n_ret;
+    const int g = a.ret_g[blockIdx.y % a.n_ret];
+    const int G = a.G;
+    const size_t bh0 = (size_t)b * a.H_q + (size_t)g * G;
+    project_query(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, a.idx_scale, qs, G);
     __syncthreads();
-    if (tid == 0) {
-        double tot = 0.0;
-        for (int i = 0; i < SEL_THREADS / 32; ++i) tot += s_red[i];
-        a.count_out[bh] = (int32_t)w.list_cnt[bh];
-        if (a.mass_out) a.mass_out[bh] = (float)((r.above + tot) / r.Z);
+    const int N = valid_len(a.seq_lens, b, a.N_max, w.status);
+    Src src;
+    init_src(src, a, b, g, qs);
+    const int warp = threadIdx.x >> 5;
+    const int t_lo = (int)((long long)blockIdx.x * a.chunk);
+    const int t_hi = (int)min((long long)N, (long long)t_lo + a.chunk);
+    float *zb = z_out + bh0 * a.N_max;
+    for (int tb = t_lo + warp * TILE; tb < t_hi; tb += SC_WARPS * TILE) {
+        typename Src::Frag f;
+        src.load(tb, f);
+        float z[Src::NV];
+        src.eval(f, z);
+#pragma unroll
+        for (int v = 0; v < Src::NV; ++v) {
+            const int h = src.head(src.slot(v));
+            const int t = tb + src.tok(v);
+            if (h < G && t < t_hi) zb[h * a.N_max + t] = z[v];
+        }
     }
 }
 

@@ -18,10 +18,14 @@
  *     run exact full-dimension softmax attention of the post-RoPE query over
  *     only the kept K/V rows (softmax renormalised over the kept set).
  *
- * The threshold is found without sorting, by a mass histogram over the
- * order-preserving bits of z followed by an exact radix select inside the
- * boundary bin (same summary, Method section 5: sort-free histogram
- * threshold and bandwidth-optimised sparse decode).
+ * The threshold is found without sorting (same summary, Method section 5:
+ * sort-free histogram threshold and bandwidth-optimised sparse decode): one
+ * streaming pass over the index keys gives each head's softmax statistics
+ * (max m, sum Z); tokens with z < m + ln(Z (1 - p) / N) - 1 carry less than
+ * (1 - p) / N of the mass each and can never be kept; the remaining
+ * candidates are ranked by an exact radix select on the order-preserving
+ * bits of z (then the token id), with per-digit mass histograms, down to
+ * the boundary token.
  *
  * Conventions shared by every call
  *   - Tensor pointers are DEVICE pointers owned by the caller, dense
@@ -77,7 +81,7 @@ enum {
     RTP_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed        */
     RTP_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out          */
     RTP_ERR_DEVICE_ARG = 6,  /* device-resident argument out of range       */
-    RTP_ERR_RANGE = 7        /* an index logit was not finite or |z| >= 1024 */
+    RTP_ERR_RANGE = 7        /* an index logit was not finite               */
 };
 
 /* Element types of the caches. */
@@ -201,7 +205,8 @@ RTP_API int rtp_index_scores(const rtp_dims *dims, const rtp_opts *opts, const f
  *   count_out [B, H_q] int32:   |S| (>= 1)
  *   mass_out  [B, H_q] fp32:    mass of S (optional, NULL: not written)
  * p >= 1 keeps all N_b tokens; p <= 0 keeps the top token; p NaN is
- * RTP_ERR_INVALID_ARG.  |z| must be finite and below 1024 (RTP_ERR_RANGE).
+ * RTP_ERR_INVALID_ARG.  A logit that is not finite is skipped and reported
+ * as RTP_ERR_RANGE.
  */
 RTP_API int rtp_topp_select(const rtp_dims *dims, const float *z, const uint8_t *head_class,
                     float p, int32_t *idx_out, int32_t *count_out, float *mass_out,

@@ -95,9 +95,15 @@ def test_step_repeatable_on_one_workspace():
     gc = GpuCase(synth.make_case(spec))
     a = gc.step(0.9)
     b = gc.step(0.9)
-    for x, y in ((a[2], b[2]),):
-        assert torch.equal(x, y)
-    within(a[0].cpu().numpy(), b[0].cpu().numpy(), 1e-6, "repeat")
+    # the kept sets and their sizes are identical; the attention output may
+    # differ in the last bits because the kept ids are listed in the order
+    # CTAs append them, which sets the fp32 summation order
+    assert torch.equal(a[2], b[2])
+    for bb in range(2):
+        for h in range(8):
+            n = int(a[2][bb, h])
+            assert set(a[1][bb, h, :n].tolist()) == set(b[1][bb, h, :n].tolist())
+    within(a[0].cpu().numpy(), b[0].cpu().numpy(), 1e-5, "repeat")
 
 
 # --------------------------------------------------------------- workloads
