@@ -277,8 +277,9 @@ struct ListArgs {
 };
 
 // One item = a slice of one head's kept rows.  Warp w takes rows
-// r0 + 8w .. r0 + 8w + 7, then every 64th: all 8 rows' K and V loads are
-// issued before the first dot product.
+// r0 + 16w .. r0 + 16w + 15, then every 128th: the 16 row ids come in one
+// load and all 16 rows' K and V loads are issued before the first dot
+// product.
 template <typename KT>
 __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
     __shared__ int pre[MAX_LIST_HEADS + 1];
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
         const KT *vb = reinterpret_cast<const KT *>(a.v) + ((size_t)b * a.H_kv + g) * a.N_max * D;
         const int32_t *lst = a.lists + bh * a.N_max;
         float m = -INFINITY, l = 0.0f, o[4] = {0.f, 0.f, 0.f, 0.f};
-        constexpr int U = 8;
+        constexpr int U = 16;      // rows per warp per pass: all their K/V loads in flight
         for (int rb = r0 + warp * U; rb < r1; rb += (ATT_THREADS / 32) * U) {
             int myid = -1;
             if (lane < U && rb + lane < r1) myid = __ldg(lst + rb + lane);

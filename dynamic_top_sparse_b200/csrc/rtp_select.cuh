@@ -91,6 +91,33 @@ __device__ __forceinline__ int logit_bin(float z) {
     return 256 + (k ^ s);
 }
 
+// Largest and smallest float of a bin (the bins partition the floats, with
+// -0 counted as +0): z is in a bin above b  <=>  z > bin_hi_incl(b), and z is
+// in b  <=>  bin_lo_incl(b) <= z <= bin_hi_incl(b).
+__host__ __device__ __forceinline__ float bits_f(uint32_t u) {
+    union { uint32_t u; float f; } c; c.u = u; return c.f;
+}
+__host__ __device__ __forceinline__ float bin_hi_incl(int bin) {
+    if (bin >= 256) {
+        const int k = bin - 256;
+        if (k == 255) return bits_f(0x7f800000u);                         // +inf
+        return bits_f(((uint32_t)(k + 1 + (int)BIN_BASE) << (23 - MB)) - 1u);
+    }
+    const int k = 255 - bin;
+    if (k == 0) return bits_f(0x80000001u);                               // -denorm_min
+    return bits_f(((uint32_t)(k + (int)BIN_BASE) << (23 - MB)) | 0x80000000u);
+}
+__host__ __device__ __forceinline__ float bin_lo_incl(int bin) {
+    if (bin >= 256) {
+        const int k = bin - 256;
+        if (k == 0) return 0.0f;
+        return bits_f((uint32_t)(k + (int)BIN_BASE) << (23 - MB));
+    }
+    const int k = 255 - bin;
+    if (k == 255) return bits_f(0xff800000u);                             // -inf
+    return bits_f((((uint32_t)(k + 1 + (int)BIN_BASE) << (23 - MB)) - 1u) | 0x80000000u);
+}
+
 // Upper edge of a bin, as used by bin_and_fx.
 __host__ __device__ __forceinline__ float bin_upper(int bin) {
     union { uint32_t u; float f; } c;
@@ -377,7 +404,7 @@ __device__ void resolve_head(double *gh, Resolve *out, float p, int N) {
         const int bin = top - lane * SEG - i;
         if (bin < 0) break;
         const double sb = gh[bin];
-        if (sb > 0.0) seg += sb * exp((double)bin_upper(bin) - (double)R);
+        if (sb > 0.0) seg += sb * (double)ex2_sfu((bin_upper(bin) - R) * 1.4426950408889634f);
     }
     double incl = seg;
 #pragma unroll
@@ -405,7 +432,7 @@ __device__ void resolve_head(double *gh, Resolve *out, float p, int N) {
                     if (bin < 0) break;
                     const double sb = gh[bin];
                     if (sb <= 0.0) continue;
-                    const double mb = sb * exp((double)bin_upper(bin) - (double)R);
+                    const double mb = sb * (double)ex2_sfu((bin_upper(bin) - R) * 1.4426950408889634f);
                     bstar = bin;       // if rounding never crosses, the last bin is kept whole
                     above = cum;
                     if (cum + mb >= target) { tin = target - cum; break; }
@@ -423,7 +450,7 @@ __device__ void resolve_head(double *gh, Resolve *out, float p, int N) {
                 if (gh[bin] > 0.0) low = min(low, bin);
             low = __reduce_min_sync(0xffffffffu, low);
             bstar = low;
-            above = Z - gh[low] * exp((double)bin_upper(low) - (double)R);
+            above = Z - gh[low] * (double)ex2_sfu((bin_upper(low) - R) * 1.4426950408889634f);
             tin = INFINITY;
         }
         r.mode = MODE_NORMAL;
@@ -571,15 +598,22 @@ constexpr float FX18 = 262144.0f;                        // 2^18
 constexpr int TC_SMEM = NSTAGE * ST_BYTES + GMAX * NBIN * 4 + GMAX * NBIN * 8 + 2 * NSTAGE * 8;
 static_assert((long long)SPILL_STAGES * ST_TOK * 262144LL < 4294967296LL, "bin counters would wrap");
 
-__device__ __forceinline__ int bin_and_fx18(float z, uint32_t &fx) {
+// Hot path of the scan for one value z (already folded so that -0 is +0):
+// adds exp(z - U_bin) in 2^18 fixed point to the head's bin counter at
+// shared address `row` (32-bit, bins of 4 bytes) and returns the raw
+// (unclamped) k, whose maximum the caller checks once (k > KMAX_OK: z out
+// of range or not finite).  The clamped bin index is returned in `bin`.
+constexpr int KMAX_OK = (int)((127 + 7) << MB) + 15 - (int)BIN_BASE;   // |z| < 256
+__device__ __forceinline__ int scan_value(float z, uint32_t row, int &bin) {
     const uint32_t u = __float_as_uint(z);
-    const int s = (int)u >> 31;
-    int k = (int)((u << 1) >> (24 - MB)) - (int)BIN_BASE;
-    k = min(max(k, 0), 255);
-    const uint32_t eb = (uint32_t)(k + (int)BIN_BASE + 1 + s) << (23 - MB);
-    const float U = __uint_as_float(eb | ((uint32_t)s & 0x80000000u));
-    fx = __float2uint_rn(ex2_sfu(fmaf(z - U, 1.4426950408889634f, 18.0f)));
-    return 256 + (k ^ s);
+    const int s = (int)u >> 31;                                          // 0 or -1
+    const int kr = (int)((u << 1) >> (24 - MB)) - (int)BIN_BASE;
+    const int k = max(kr, 0) & 255;
+    const uint32_t eb = ((uint32_t)(k + (int)BIN_BASE + 1 + s) << (23 - MB)) | (u & 0x80000000u);
+    const uint32_t fx = __float2uint_rn(ex2_sfu(fmaf(z - __uint_as_float(eb), 1.4426950408889634f, 18.0f)));
+    bin = 256 + (k ^ s);
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row + 4u * (uint32_t)bin), "r"(fx) : "memory");
+    return kr;
 }
 
 __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelWs w) {
@@ -604,10 +638,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
         fence_mbar_init();
     }
     for (int i = threadIdx.x; i < GMAX * NBIN; i += blockDim.x) { h32[i] = 0u; h64[i] = 0ull; }
-    project_query(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, a.idx_scale, qs, G);
     __syncthreads();
-    if (blockIdx.x == 0)
-        for (int i = threadIdx.x; i < G * R; i += blockDim.x) w.qidx[bh0 * R + i] = qs[i];
     const int N = valid_len(a.seq_lens, b, a.N_max, w.status);
     const int t_lo = (int)((long long)blockIdx.x * a.chunk);
     const int t_hi = (int)min((long long)N, (long long)t_lo + a.chunk);
@@ -639,12 +670,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
         }
     } else {
         // consumers
+        // q_idx of the group (consumer warps only; the producer is already streaming)
+        project_query(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, a.idx_scale, qs, G);
+        asm volatile("bar.sync 1, %0;" ::"r"(TC_WARPS * 32) : "memory");
+        if (blockIdx.x == 0)
+            for (int i = threadIdx.x; i < G * R; i += TC_WARPS * 32) w.qidx[bh0 * R + i] = qs[i];
         SrcMma src;
         src.init(rows, a.N_max, qs, G);
         const int gid = lane >> 2, tig = lane & 3;
-        uint32_t *hrow[2] = {h32 + (2 * tig) * NBIN, h32 + (2 * tig + 1) * NBIN};
+        const uint32_t hrow0 = smem_u32(h32 + (2 * tig) * NBIN), hrow1 = smem_u32(h32 + (2 * tig + 1) * NBIN);
         const bool full_group = G == GMAX;
-        int err = 0;
+        int kmax = 0;
         uint16_t *tbin = w.tilebin + bh0 * a.ntile;
         // After a timeout every consumer warp keeps iterating without
         // waiting or working, so the named barrier below stays balanced.
@@ -674,11 +710,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
 #pragma unroll
                     for (int v = 0; v < SrcMma::NV; ++v) {
                         const int sl = v & 1;
-                        const float zz = z[v] + 0.0f;       // folds -0 onto +0
-                        err |= !(fabsf(zz) < Z_LIMIT);
-                        uint32_t fx;
-                        const int bin = bin_and_fx18(zz, fx);
-                        atomicAdd(hrow[sl] + bin, fx);
+                        int bin;
+                        kmax = max(kmax, scan_value(z[v] + 0.0f, sl ? hrow1 : hrow0, bin));
                         tmax[sl] = max(tmax[sl], bin);
                     }
                 } else {
@@ -686,11 +719,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
                     for (int v = 0; v < SrcMma::NV; ++v) {
                         const int sl = v & 1;
                         if (2 * tig + sl >= G || src.tok(v) >= nvalid) continue;
-                        const float zz = z[v] + 0.0f;
-                        if (!(fabsf(zz) < Z_LIMIT)) { err = 1; continue; }
-                        uint32_t fx;
-                        const int bin = bin_and_fx18(zz, fx);
-                        atomicAdd(hrow[sl] + bin, fx);
+                        int bin;
+                        kmax = max(kmax, scan_value(z[v] + 0.0f, sl ? hrow1 : hrow0, bin));
                         tmax[sl] = max(tmax[sl], bin);
                     }
                 }
@@ -717,7 +747,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
                 asm volatile("bar.sync 1, %0;" ::"r"(TC_WARPS * 32) : "memory");
             }
         }
-        if (err) s_err = 1;
+        if (kmax > KMAX_OK) s_err = 1;
     }
     __syncthreads();
     if (s_err && threadIdx.x == 0) set_status(w.status, RTP_ERR_RANGE);
@@ -768,6 +798,7 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
     __shared__ int s_bstar[GMAX];
     __shared__ int s_mode[GMAX];
     __shared__ unsigned s_kc[GMAX], s_cc[GMAX];
+    __shared__ float s_khi[GMAX], s_clo[GMAX];      // keep: z > s_khi; candidate: s_clo <= z <= s_khi
     __shared__ int32_t s_kbuf[GMAX * KCAP];
     __shared__ unsigned long long s_cbuf[GMAX * CCAP];
     const int b = blockIdx.y / a.n_ret;
@@ -785,6 +816,8 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
         s_mode[threadIdx.x] = mode;
         // keep-all heads need no collect pass: finalize lists every token
         s_bstar[threadIdx.x] = mode == MODE_NORMAL ? bs : NBIN;
+        s_khi[threadIdx.x] = mode == MODE_NORMAL ? bin_hi_incl(bs) : INFINITY;
+        s_clo[threadIdx.x] = mode == MODE_NORMAL ? bin_lo_incl(bs) : INFINITY;
         s_kc[threadIdx.x] = 0u;
         s_cc[threadIdx.x] = 0u;
     }
@@ -836,9 +869,8 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
                 if (h < G && t < t_hi && ((hmask >> h) & 1u)) {
                     const float zz = z[v] + 0.0f;
                     if (fabsf(zz) < Z_LIMIT) {
-                        const int bin = logit_bin(zz);
-                        const int bs = s_bstar[h];
-                        if (bin > bs) {
+                        const float khi = s_khi[h];
+                        if (zz > khi) {
                             const unsigned p = atomicAdd(&s_kc[h], 1u);
                             if (p < (unsigned)KCAP) {
                                 s_kbuf[h * KCAP + p] = t;
@@ -846,7 +878,7 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
                                 const unsigned q = atomicAdd(&w.list_cnt[bh0 + h], 1u);
                                 a.lists[(bh0 + h) * a.N_max + q] = t;
                             }
-                        } else if (bin == bs) {
+                        } else if (zz >= s_clo[h]) {
                             const unsigned long long key =
                                 ((unsigned long long)logit_key(zz) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)t);
                             const unsigned p = atomicAdd(&s_cc[h], 1u);
@@ -889,9 +921,9 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float cand_logit(unsigned long long c) { return key_logit((uint32_t)(c >> 32)); }
 
-constexpr int FIN_THREADS = 256;
+constexpr int FIN_THREADS = 512;
 constexpr int FIN_WARPS = FIN_THREADS / 32;
-constexpr int FIN_CAP = 2048;             // candidates staged in shared memory
+constexpr int FIN_CAP = 3072;             // candidates staged in shared memory
 // Exact selection inside the boundary bin.  One CTA per retrieval head;
 // grid = (B * n_ret * G).  Candidate masses relative to the boundary bin's
 // upper edge U* are each in (e^-32, 1]; they are summed in fixed point with
@@ -900,9 +932,10 @@ constexpr int FIN_CAP = 2048;             // candidates staged in shared memory
 // exclusive prefix of list-attention items per head (item_pre).
 __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs w) {
     __shared__ unsigned long long hfx[256];
+    __shared__ uint32_t hfx32[256];
     __shared__ unsigned hcnt[256];
     __shared__ unsigned long long cbuf[FIN_CAP];
-    __shared__ unsigned long long fbuf[FIN_CAP];
+    __shared__ uint32_t fbuf[FIN_CAP];
     __shared__ unsigned long long s_min, s_max, s_theta, s_excl, s_kept;
     __shared__ unsigned s_base;
     __shared__ int s_digit, s_last;
@@ -930,8 +963,11 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         mass = r.mode == MODE_EMPTY ? 0.0f : (float)(r.above / r.Z);
     } else {
         const float Ub = bin_upper(r.bstar);
-        const double S = ldexp(1.0, 62) / (double)nc;
+        // Staged candidates: 32-bit fixed point, S = floor((2^31 - 1) / nc)
+        // units per unit of mass (sums cannot wrap; with nc <= FIN_CAP each
+        // mass keeps >= 19 bits).  Otherwise 64-bit, S = 2^62 / nc.
         const bool staged = nc <= (unsigned)FIN_CAP;
+        const double S = staged ? (double)(0x7fffffffu / nc) : ldexp(1.0, 62) / (double)nc;
         auto fx_of = [&](unsigned long long v) -> unsigned long long {
             const float m = ex2_sfu((cand_logit(v) - Ub) * 1.4426950408889634f);
             return (unsigned long long)((double)m * S);
@@ -942,7 +978,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             unsigned long long lo = ~0ull, hi = 0ull;
             for (unsigned c = tid; c < nc; c += blockDim.x) {
                 const unsigned long long v = cg[c];
-                if (staged) { cbuf[c] = v; fbuf[c] = fx_of(v); }
+                if (staged) { cbuf[c] = v; fbuf[c] = (uint32_t)fx_of(v); }
                 lo = v < lo ? v : lo;
                 hi = v > hi ? v : hi;
             }
@@ -959,7 +995,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             }
         }
         __syncthreads();
-        const double tS = r.target * exp((double)r.R - (double)Ub) * S;
+        const double tS = r.target / (double)ex2_sfu((Ub - r.R) * 1.4426950408889634f) * S;
         unsigned long long T = !(tS < 9.0e18) ? ~0ull : (unsigned long long)llrint(tS);
         const unsigned long long diff = s_min ^ s_max;
         unsigned long long theta = s_min;          // one candidate (or all equal): keep all
@@ -969,14 +1005,26 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             unsigned long long pmask = shift + 8 >= 64 ? 0ull : ~((1ull << (shift + 8)) - 1ull);
             unsigned long long prefix = s_min & pmask;
             for (int level = 0; level < 16; ++level) {
-                for (int i = tid; i < 256; i += blockDim.x) { hfx[i] = 0ull; hcnt[i] = 0u; }
+                for (int i = tid; i < 256; i += blockDim.x) { hfx[i] = 0ull; hfx32[i] = 0u; hcnt[i] = 0u; }
                 __syncthreads();
-                for (unsigned c = tid; c < nc; c += blockDim.x) {
-                    const unsigned long long v = staged ? cbuf[c] : cg[c];
-                    if ((v & pmask) != prefix) continue;
-                    const int dg = (int)((v >> shift) & 255ull);
-                    atomicAdd(&hfx[dg], staged ? fbuf[c] : fx_of(v));
-                    atomicAdd(&hcnt[dg], 1u);
+                if (staged) {
+                    for (unsigned c = tid; c < nc; c += blockDim.x) {
+                        const unsigned long long v = cbuf[c];
+                        if ((v & pmask) != prefix) continue;
+                        const int dg = (int)((v >> shift) & 255ull);
+                        atomicAdd(&hfx32[dg], fbuf[c]);
+                        atomicAdd(&hcnt[dg], 1u);
+                    }
+                    __syncthreads();
+                    for (int i = tid; i < 256; i += blockDim.x) hfx[i] = hfx32[i];
+                } else {
+                    for (unsigned c = tid; c < nc; c += blockDim.x) {
+                        const unsigned long long v = cg[c];
+                        if ((v & pmask) != prefix) continue;
+                        const int dg = (int)((v >> shift) & 255ull);
+                        atomicAdd(&hfx[dg], fx_of(v));
+                        atomicAdd(&hcnt[dg], 1u);
+                    }
                 }
                 __syncthreads();
                 if (warp == 0) {
@@ -1057,7 +1105,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         if (lane == 0) atomicAdd(&s_kept, kept);
         __syncthreads();
         count = (int)(base0 + s_base);
-        const double kept_mass = (double)s_kept / S * exp((double)Ub - (double)r.R);
+        const double kept_mass = (double)s_kept / S * (double)ex2_sfu((Ub - r.R) * 1.4426950408889634f);
         mass = (float)((r.above + kept_mass) / r.Z);
     }
     if (tid == 0) {
