@@ -466,8 +466,8 @@ def cpu_baseline(cfg, spec=None, budget_s=15.0):
         heads = [(b, h) for b in seqs for h in range(spec.H_q)]
         t0 = time.perf_counter()
         kidx = oracle.append_index_keys(kidx, c.k_pre_new.float().cpu().numpy(), c.W_k_idx.cpu().numpy(),
-                                        c.seq_lens.numpy() - 1, spec.idx_dtype, head_class=c.head_class)
-        oracle.decode_step(q, qr, K, V, kidx, c.W_q_idx.cpu().numpy(), c.head_class, c.seq_lens.numpy(),
+                                        c.seq_lens.cpu().numpy() - 1, spec.idx_dtype, head_class=c.head_class)
+        oracle.decode_step(q, qr, K, V, kidx, c.W_q_idx.cpu().numpy(), c.head_class, c.seq_lens.cpu().numpy(),
                            spec.p, spec.window, spec.n_sink, heads=heads)
         t_tot += time.perf_counter() - t0
         layers_done += 1
