@@ -332,6 +332,33 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
 
 }  // namespace
 
+// Scratch of rtp_dense_decode_noalloc: one fixed array per device, so
+// callers that cannot allocate still get the split-K partials, arrival
+// counters and status word the dense kernel needs.  Host code must not use
+// the symbol's host-side name as a device address: the device address comes
+// from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[RTP_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+
+constexpr size_t NOALLOC_ARRIVE_OFF = 256;                       // after the status word
+constexpr size_t NOALLOC_PART_OFF = 256 + RTP_NOALLOC_MAX_GROUPS * 4;
+
+int noalloc_scratch(char *&out) {
+    static void *ptrs[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RTP_ERR_CUDA;
+        ptrs[dev] = p;
+    }
+    out = static_cast<char *>(ptrs[dev]);
+    return RTP_OK;
+}
+
+}  // namespace
+
 // =========================================================================
 // public entry points
 // =========================================================================
@@ -502,6 +529,50 @@ int rtp_dense_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_
     Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
     return launch_range(ln, dims, q_rope, k_cache, v_cache, nullptr, -1, true, 1, 0, out, (char *)ws, L,
                         scale_or_default(opts ? opts->attn_scale : 0.f));
+}
+
+int rtp_dense_decode_noalloc(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
+                             const void *k_cache, const void *v_cache, float *out, int32_t *dev_status,
+                             rtp_stream_t stream) {
+    RTP_TRY(check_dims(dims));
+    if (!q_rope || !k_cache || !v_cache || !out) return RTP_ERR_INVALID_ARG;
+    if (!aligned16(q_rope) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
+        return RTP_ERR_INVALID_ARG;
+    const long long groups = (long long)dims->B * dims->H_kv;
+    if (groups > RTP_NOALLOC_MAX_GROUPS) return RTP_ERR_WORKSPACE;
+    char *scr = nullptr;
+    RTP_TRY(noalloc_scratch(scr));
+    const cudaStream_t st = (cudaStream_t)stream;
+    // status word and arrival counters must start at zero
+    if (cudaMemsetAsync(scr, 0, NOALLOC_PART_OFF, st) != cudaSuccess) return RTP_ERR_CUDA;
+    RangeArgs a{};
+    a.B = dims->B; a.H_q = dims->H_q; a.H_kv = dims->H_kv; a.G = dims->H_q / dims->H_kv;
+    a.N_max = dims->N_max; a.seq_lens = dims->seq_lens;
+    a.n_grp = dims->H_kv;
+    for (int g = 0; g < dims->H_kv; ++g) a.grp[g] = g;
+    a.dense = 1;
+    a.window = 1;
+    a.n_sink = 0;
+    const long long rec = (long long)GMAX * PSTRIDE * 4;            // bytes per split per group
+    const long long cap = ((long long)RTP_NOALLOC_SCRATCH_BYTES - (long long)NOALLOC_PART_OFF) / (groups * rec);
+    const long long chunks = (dims->N_max + 255) / 256;
+    const long long want = (2LL * num_sms() + groups - 1) / groups;
+    a.n_split = (int)std::max(1LL, std::min({want, chunks, cap, (long long)RANGE_SPLIT_MAX}));
+    a.scale_log2 = scale_or_default(opts ? opts->attn_scale : 0.f) * 1.4426950408889634f;
+    a.q = q_rope; a.k = k_cache; a.v = v_cache; a.out = out;
+    a.part = reinterpret_cast<float *>(scr + NOALLOC_PART_OFF);
+    a.arrive = reinterpret_cast<uint32_t *>(scr + NOALLOC_ARRIVE_OFF);
+    a.status = reinterpret_cast<uint32_t *>(scr);
+    Launcher ln{st, opts ? opts->prof : nullptr};
+    const dim3 grid((unsigned)a.n_split, (unsigned)groups);
+    if (dims->kv_dtype == RTP_BF16) {
+        RTP_TRY(ln.run("dense_attn", gqa_mma_attn_kernel, grid, dim3(GQ_THREADS), a));
+    } else {
+        RTP_TRY(ln.run("dense_attn", range_attn_kernel<float>, grid, dim3(ATT_THREADS), a));
+    }
+    if (dev_status && cudaMemcpyAsync(dev_status, scr, 4, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return RTP_ERR_CUDA;
+    return RTP_OK;
 }
 
 int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, const float *q_rope,

@@ -269,6 +269,38 @@ RTP_API int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const fl
                     const uint8_t *head_class, float p, int32_t window, int32_t n_sink,
                     float *out, void *ws, size_t ws_bytes, rtp_stream_t stream);
 
+/*
+ * Dense decode without a caller workspace.  (The paper has no counterpart:
+ * this is a deployment variant of rtp_dense_decode.)
+ *
+ * For callers that cannot allocate device memory -- for example a plug-in
+ * inside a host framework that owns every device allocation and hands the
+ * plug-in none, or a serving path where cudaMalloc is off limits because it
+ * can synchronise the device or fail under memory pressure.  The scratch
+ * this call needs (status word, arrival counters, split partials) lives in
+ * one fixed device array inside librtp.so, RTP_NOALLOC_SCRATCH_BYTES per
+ * device; every GPU that loads the library holds it until the process
+ * exits.  The call allocates nothing and frees nothing.
+ *
+ * Inputs and outputs are as for rtp_dense_decode; dev_status, if not NULL,
+ * is a device int32 that receives this call's device-side status (0: ok,
+ * else an RTP_ERR_* code such as RTP_ERR_DEVICE_ARG for a bad sequence
+ * length).  Returns RTP_ERR_WORKSPACE when B * H_kv exceeds
+ * RTP_NOALLOC_MAX_GROUPS (the partials would not fit), before any launch.
+ *
+ * The first call on a device, with that device current, looks up the
+ * array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  All calls share the one array and it keeps
+ * the last call's contents: each call clears the part that must start at
+ * zero, and calls whose executions overlap on the GPU (different streams,
+ * no ordering between them) race on it -- order them on one stream.
+ */
+#define RTP_NOALLOC_SCRATCH_BYTES (8u << 20)
+#define RTP_NOALLOC_MAX_GROUPS 1024
+RTP_API int rtp_dense_decode_noalloc(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
+                                     const void *k_cache, const void *v_cache, float *out,
+                                     int32_t *dev_status, rtp_stream_t stream);
+
 /* Launch accounting helpers (see rtp_prof). */
 RTP_API int rtp_prof_init(rtp_prof *prof, int32_t capacity);
 RTP_API int rtp_prof_elapsed(const rtp_prof *prof, int32_t slot, float *ms);
