@@ -5,6 +5,7 @@
 #include <cstdlib>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 
 #include "rtp.h"
 #include "rtp_common.cuh"
@@ -23,9 +24,9 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace regions, in the order ops need them (each op needs a prefix).
 struct Layout {
-    size_t status, arrive_scan, arrive_range, arrive_list, cand_cnt, list_cnt, fin_arrive, hist;
+    size_t status, arrive_range, arrive_list, cand_cnt, list_cnt, hist;
     size_t ctrl_end;
-    size_t res, qidx, counts, item_pre;
+    size_t res, qidx, counts;
     size_t end_scores;      // append / index_scores need up to here
     size_t part_range;
     size_t end_range;       // local / dense
@@ -43,18 +44,15 @@ Layout make_layout(const rtp_dims *d) {
     const size_t ntile = (size_t)((d->N_max + TILE - 1) / TILE);
     size_t o = 0;
     L.status = o; o += 256;
-    L.arrive_scan = o; o = align_up(o + BHkv * 4, 256);
     L.arrive_range = o; o = align_up(o + BHkv * 4, 256);
     L.arrive_list = o; o = align_up(o + BHq * 4, 256);
     L.cand_cnt = o; o = align_up(o + BHq * 4, 256);
     L.list_cnt = o; o = align_up(o + BHq * 4, 256);
-    L.fin_arrive = o; o = align_up(o + 4, 256);
     L.hist = o; o = align_up(o + BHq * NBIN * 8, 256);
     L.ctrl_end = o;
     L.res = o; o = align_up(o + BHq * sizeof(Resolve), 256);
     L.qidx = o; o = align_up(o + BHq * R * 4, 256);
     L.counts = o; o = align_up(o + BHq * 4, 256);
-    L.item_pre = o; o = align_up(o + (BHq + 1) * 4, 256);
     L.end_scores = o;
     L.part_range = o; o = align_up(o + BHkv * RANGE_SPLIT_MAX * GMAX * PSTRIDE * 4, 256);
     L.end_range = o;
@@ -129,6 +127,11 @@ int num_sms() {
 struct Launcher {
     cudaStream_t st;
     rtp_prof *prof;
+    // Launch the next kernels with programmatic stream serialization: they
+    // may start while the previous kernel of the stream drains, and wait for
+    // it on the device (pdl_wait).  Only for kernels that call pdl_wait
+    // before touching global memory.
+    bool pdl = false;
     // Inside stream capture an event becomes a timestamp node of the graph
     // only when recorded as external.
     cudaError_t record(void *ev, bool capturing) {
@@ -152,7 +155,21 @@ struct Launcher {
             capturing = cs == cudaStreamCaptureStatusActive;
             if (record(prof->ev_start[slot], capturing) != cudaSuccess) return RTP_ERR_CUDA;
         }
-        kernel<<<grid, block, smem, st>>>(args...);
+        if (pdl) {
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = grid;
+            cfg.blockDim = block;
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = st;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            at[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) return RTP_ERR_CUDA;
+        } else {
+            kernel<<<grid, block, smem, st>>>(args...);
+        }
         if (cudaGetLastError() != cudaSuccess) return RTP_ERR_CUDA;
         if (slot >= 0 && record(prof->ev_stop[slot], capturing) != cudaSuccess) return RTP_ERR_CUDA;
         return RTP_OK;
@@ -199,7 +216,6 @@ SelPlan make_sel(const rtp_dims *d, const uint8_t *hc, char *ws, const Layout &L
     plan_chunks(a, d->N_max);
     SelWs &w = s.w;
     w.status = reinterpret_cast<uint32_t *>(ws + L.status);
-    w.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_scan);
     w.cand_cnt = reinterpret_cast<uint32_t *>(ws + L.cand_cnt);
     w.list_cnt = reinterpret_cast<uint32_t *>(ws + L.list_cnt);
     w.hist = reinterpret_cast<double *>(ws + L.hist);
@@ -207,23 +223,28 @@ SelPlan make_sel(const rtp_dims *d, const uint8_t *hc, char *ws, const Layout &L
     w.tilebin = reinterpret_cast<uint16_t *>(ws + L.tilebin);
     w.cands = reinterpret_cast<unsigned long long *>(ws + L.cands);
     w.qidx = reinterpret_cast<float *>(ws + L.qidx);
-    w.fin_arrive = reinterpret_cast<uint32_t *>(ws + L.fin_arrive);
     return s;
 }
 
+// Work queued right after the scan kernel (the local heads of a decode
+// step, forked onto a side stream so that they overlap the latency-bound
+// collect / finalize / list kernels instead of holding SMs the scan needs).
+using AfterScan = std::function<int()>;
+
 // scan + collect + finalize over a logit source
 template <typename Src>
-int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s) {
+int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s, const AfterScan &after_scan = {}) {
     const dim3 grid((unsigned)s.a.ctas, (unsigned)(d->B * s.a.n_ret));
     RTP_TRY(ln.run("hist", scan_kernel<Src>, grid, dim3(SCAN_THREADS), s.a, s.w));
+    if (after_scan) RTP_TRY(after_scan());
     RTP_TRY(ln.run("collect", collect_kernel<Src>, grid, dim3(COL_THREADS), s.a, s.w));
     RTP_TRY(ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)),
                    dim3(FIN_THREADS), s.a, s.w));
     return RTP_OK;
 }
 
-int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s) {
-    if (d->idx_dtype != RTP_BF16) return launch_select<SrcSimt<float>>(ln, d, s);
+int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, const AfterScan &after_scan = {}) {
+    if (d->idx_dtype != RTP_BF16) return launch_select<SrcSimt<float>>(ln, d, s, after_scan);
     // bf16 index keys: the TMA-ring scan, one CTA per SM over all groups
     static int attr_set[64] = {0};
     int dev = 0;
@@ -240,11 +261,19 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s) {
     s.a.chunk = (tiles + ctas - 1) / ctas * TILE;
     s.a.ctas = (int)((d->N_max + s.a.chunk - 1) / s.a.chunk);
     const dim3 grid((unsigned)s.a.ctas, (unsigned)groups);
-    RTP_TRY(ln.run_smem("hist", scan_tma_kernel, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w));
-    RTP_TRY(ln.run("collect", collect_kernel<SrcMma>, grid, dim3(COL_THREADS), s.a, s.w));
-    RTP_TRY(ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)), dim3(FIN_THREADS),
-                   s.a, s.w));
-    return RTP_OK;
+    // scan, collect and finalize wait on the device for their predecessor
+    // (programmatic dependent launch), so each one's launch overlaps the
+    // previous kernel's tail
+    const bool pdl0 = ln.pdl;
+    ln.pdl = true;
+    int rc = ln.run_smem("hist", scan_tma_kernel, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w);
+    if (rc == RTP_OK && after_scan) rc = after_scan();
+    if (rc == RTP_OK) rc = ln.run("collect", collect_kernel<SrcMma>, grid, dim3(COL_THREADS), s.a, s.w);
+    if (rc == RTP_OK)
+        rc = ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)), dim3(FIN_THREADS),
+                    s.a, s.w);
+    ln.pdl = pdl0;
+    return rc;
 }
 
 unsigned long long ret_mask(const rtp_dims *d, const uint8_t *hc) {
@@ -289,8 +318,9 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
     a.dense = dense ? 1 : 0;
     a.window = window; a.n_sink = n_sink;
     const long long Lmax = dense ? d->N_max : std::min<long long>(d->N_max, (long long)window + n_sink);
-    const int rows_min = 256;
-    const int per_sm = 2;
+    // at least two 16-row tiles per warp; one CTA per SM
+    const int rows_min = 2 * GQ_WARPS * GQ_TILE;
+    const int per_sm = 1;
     const long long chunks = (Lmax + rows_min - 1) / rows_min;
     long long want = ((long long)per_sm * num_sms() + (long long)d->B * a.n_grp - 1) / ((long long)d->B * a.n_grp);
     a.n_split = (int)std::max(1LL, std::min(want, std::min(chunks, (long long)RANGE_SPLIT_MAX)));
@@ -308,7 +338,7 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
 
 int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
                 const int32_t *lists, const int32_t *counts, const uint8_t *hc, float *out,
-                char *ws, const Layout &L, float attn_scale, const int32_t *item_pre = nullptr) {
+                char *ws, const Layout &L, float attn_scale) {
     ListArgs a{};
     a.B = d->B; a.H_q = d->H_q; a.H_kv = d->H_kv; a.G = d->H_q / d->H_kv;
     a.N_max = d->N_max; a.seq_lens = d->seq_lens;
@@ -318,7 +348,6 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
     if (a.n_rq == 0) return RTP_OK;
     a.scale_log2 = attn_scale * 1.4426950408889634f;
     a.q = q; a.k = k; a.v = v; a.lists = lists; a.counts = counts; a.out = out;
-    a.item_pre = item_pre;
     a.part = reinterpret_cast<float *>(ws + L.part_list);
     a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_list);
     a.status = reinterpret_cast<uint32_t *>(ws + L.status);
@@ -598,8 +627,10 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
     const bool any_local = s.a.n_ret < dims->H_kv;
     const cudaStream_t main = (cudaStream_t)stream;
     Side *side = nullptr;
-    if (any_local && s.a.n_ret > 0) {
-        // local heads run on a side stream, overlapping the retrieval pipeline
+    // Local heads run on a side stream that forks from the main stream at
+    // the point where this is called (so they start once the work queued
+    // before it has finished) and joins it at the end of the step.
+    auto fork_local = [&]() -> int {
         RTP_TRY(side_stream(side));
         if (cudaEventRecord(side->fork, main) != cudaSuccess) return RTP_ERR_CUDA;
         if (cudaStreamWaitEvent(side->st, side->fork, 0) != cudaSuccess) return RTP_ERR_CUDA;
@@ -607,7 +638,12 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
         RTP_TRY(launch_range(lside, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
                              n_sink, out, w, L, asc));
         if (cudaEventRecord(side->join, side->st) != cudaSuccess) return RTP_ERR_CUDA;
-    } else if (any_local) {
+        return RTP_OK;
+    };
+    const bool selecting = s.a.n_ret > 0 && p < 1.0f;
+    if (any_local && s.a.n_ret > 0 && !selecting) {
+        RTP_TRY(fork_local());
+    } else if (any_local && s.a.n_ret == 0) {
         RTP_TRY(launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
                              n_sink, out, w, L, asc));
     }
@@ -626,11 +662,15 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
             s.a.lists = opts && opts->sel_idx ? opts->sel_idx : reinterpret_cast<int32_t *>(w + L.lists);
             s.a.count_out = opts && opts->sel_count ? opts->sel_count : reinterpret_cast<int32_t *>(w + L.counts);
             s.a.mass_out = opts ? opts->sel_mass : nullptr;
-            s.a.item_pre = reinterpret_cast<int32_t *>(w + L.item_pre);
-            rc = select_from_index(ln, dims, s);
-            if (rc == RTP_OK)
+            // the scan of the index keys gets the whole GPU; the local heads
+            // fork after it and overlap the rest of the selection
+            rc = select_from_index(ln, dims, s, any_local ? AfterScan(fork_local) : AfterScan());
+            if (rc == RTP_OK) {
+                ln.pdl = dims->idx_dtype == RTP_BF16;    // follows finalize_kernel
                 rc = launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out,
-                                 w, L, asc, s.a.item_pre);
+                                 w, L, asc);
+                ln.pdl = false;
+            }
         }
     }
     if (side && cudaStreamWaitEvent(main, side->join, 0) != cudaSuccess && rc == RTP_OK) rc = RTP_ERR_CUDA;

@@ -33,10 +33,10 @@ constexpr int MAX_LIST_HEADS = 4096;
 // Merge n flash-decoding partial records (stride `rec` floats between
 // records; record h of a group at + h * PSTRIDE) for heads [0, nh) into
 // out[h * D + d].  Every thread owns 4 dims of one head and merges in one
-// pass with a running max, keeping 8 records' loads in flight.
+// pass with a running max, keeping 16 records' loads in flight.
 __device__ __forceinline__ void merge_partials(const float *__restrict__ pb, int n, int rec, int nh,
                                                float *__restrict__ out) {
-    constexpr int U = 8;
+    constexpr int U = 16;
     for (int i = threadIdx.x; i < nh * (D / 4); i += blockDim.x) {
         const int h = i / (D / 4), d4 = i % (D / 4);
         const float *base = pb + h * PSTRIDE;
@@ -269,7 +269,6 @@ struct ListArgs {
     const void *v;
     const int32_t *lists;        // [B*H_q*N_max]
     const int32_t *counts;       // [B*H_q]
-    const int32_t *item_pre;     // [nh + 1] precomputed item prefix, or null
     float *out;
     float *part;                 // [B*H_q*LIST_MAX_SPLIT][PSTRIDE] (indexed by item)
     uint32_t *arrive;            // [B*H_q]
@@ -289,41 +288,52 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
     __shared__ int s_last;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nh = a.B * a.n_rq;
+    pdl_wait();
+    pdl_trigger();
 
-    // items per head -> exclusive prefix: precomputed by the selection
-    // stage, or built here by every CTA
-    if (a.item_pre) {
-        for (int i = tid; i <= nh; i += blockDim.x) pre[i] = __ldcg(a.item_pre + i);
-        __syncthreads();
-    } else {
+    // items per head -> exclusive prefix, built by every CTA
+    {
+        // thread t owns heads [t * per, t * per + per): item counts, then a
+        // block-wide exclusive scan (warp shuffles, one pass over warp totals)
         const int per = (nh + ATT_THREADS - 1) / ATT_THREADS;
         int loc = 0;
+#pragma unroll 4
         for (int i = 0; i < per; ++i) {
             const int hi = tid * per + i;
             int it = 0;
             if (hi < nh) {
                 const int b = hi / a.n_rq, h = a.ret_h[hi % a.n_rq];
-                const int cnt = a.counts[(size_t)b * a.H_q + h];
+                const int cnt = __ldcg(a.counts + (size_t)b * a.H_q + h);
                 const int N = a.seq_lens[b];
                 if (cnt >= 1 && N >= 1 && (long long)N <= a.N_max && cnt <= N) it = list_items(cnt);
                 pre[hi] = it;
             }
             loc += it;
         }
-        s_scan[tid] = loc;
-        __syncthreads();
-        for (int o = 1; o < ATT_THREADS; o <<= 1) {
-            int v = tid >= o ? s_scan[tid - o] : 0;
-            __syncthreads();
-            s_scan[tid] += v;
-            __syncthreads();
+        int incl = loc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
         }
-        int run = s_scan[tid] - loc;
+        if (lane == 31) s_scan[warp] = incl;
+        __syncthreads();
+        if (warp == 0) {
+            int t = lane < ATT_THREADS / 32 ? s_scan[lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, t, o);
+                if (lane >= o) t += v;
+            }
+            if (lane < ATT_THREADS / 32) s_scan[lane] = t;
+        }
+        __syncthreads();
+        int run = (warp > 0 ? s_scan[warp - 1] : 0) + incl - loc;
         for (int i = 0; i < per; ++i) {
             const int hi = tid * per + i;
             if (hi < nh) { const int it = pre[hi]; pre[hi] = run; run += it; }
         }
-        if (tid == ATT_THREADS - 1) pre[nh] = s_scan[tid];
+        if (tid == 0) pre[nh] = s_scan[ATT_THREADS / 32 - 1];
         __syncthreads();
     }
     const int total = pre[nh];
@@ -425,8 +435,17 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
                     os = fmaf(wo[w][tid], wg, os);
                 }
             }
-            pp[POFF + tid] = os;
-            if (tid == 0) { pp[0] = M; pp[1] = ls; }
+            if (nit == 1) {
+                // the head's only item: normalise and write the output directly
+                a.out[bh * D + tid] = os * (ls > 0.0f ? 1.0f / ls : 0.0f);
+            } else {
+                pp[POFF + tid] = os;
+                if (tid == 0) { pp[0] = M; pp[1] = ls; }
+            }
+        }
+        if (nit == 1) {
+            __syncthreads();
+            continue;
         }
         __threadfence();
         __syncthreads();

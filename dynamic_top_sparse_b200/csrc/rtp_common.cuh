@@ -131,6 +131,17 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel of the selection chain may be
+// launched while its predecessor in the stream is still running; it calls
+// pdl_wait() before its first global-memory access (read or write), which
+// returns once every earlier grid of the stream has completed and its writes
+// are visible (a no-op when the kernel was launched normally).
+// pdl_trigger() lets the next kernel's CTAs be scheduled from then on.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// ---------------------------------------------------------------------------
 // warp helpers
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ float warp_sum(float v) {

@@ -24,7 +24,7 @@
 
 namespace rtp {
 
-constexpr int GQ_WARPS = 4;
+constexpr int GQ_WARPS = 8;
 constexpr int GQ_THREADS = GQ_WARPS * 32;
 constexpr int GQ_TILE = 16;                 // rows per mma tile
 
@@ -56,7 +56,7 @@ __device__ __forceinline__ void split3(float x, float &hi, float &mid, float &lo
     lo = r - mid;
 }
 
-__global__ void __launch_bounds__(GQ_THREADS, 2) gqa_mma_attn_kernel(RangeArgs a) {
+__global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a) {
     __shared__ float s_m[GQ_WARPS][GMAX], s_l[GQ_WARPS][GMAX];
     __shared__ float s_o[GQ_WARPS][GMAX][D];
     __shared__ int s_last;

@@ -142,7 +142,6 @@ static_assert(sizeof(Resolve) == 40, "Resolve layout");
 
 struct SelWs {
     uint32_t *status;
-    uint32_t *arrive;            // [B*H_kv] scan arrivals
     uint32_t *cand_cnt;          // [B*H_q]
     uint32_t *list_cnt;          // [B*H_q]
     double *hist;                // [B*H_q][NBIN]
@@ -150,7 +149,6 @@ struct SelWs {
     uint16_t *tilebin;           // [B*H_q][ntile]: 1 + largest bin of the tile (0: none)
     unsigned long long *cands;   // [B*H_q][N_max]
     float *qidx;                 // [B*H_q][R]
-    uint32_t *fin_arrive;        // finalize arrivals (one counter)
 };
 
 struct SelArgs {
@@ -171,7 +169,6 @@ struct SelArgs {
     int32_t *lists;              // [B*H_q][N_max] kept ids
     int32_t *count_out;          // [B*H_q]
     float *mass_out;             // [B*H_q] or null
-    int32_t *item_pre;           // [B*n_ret*G + 1] list-attention work prefix, or null
 };
 
 __device__ __forceinline__ int valid_len(const int32_t *seq_lens, int b, long long N_max,
@@ -184,31 +181,54 @@ __device__ __forceinline__ int valid_len(const int32_t *seq_lens, int b, long lo
     return N;
 }
 
-// q_idx of the group's heads into shared memory: warp h computes head h's
-// 16 outputs (fixed lane partition and reduction order, so every CTA and
-// every kernel gets bit-identical values).
-__device__ __forceinline__ void project_query(const float *__restrict__ q_bh0,
-                                              const float *__restrict__ W_h0, float scale,
-                                              float *qs, int G) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (warp >= G) return;
-    const float4 qv = __ldg(reinterpret_cast<const float4 *>(q_bh0 + warp * D) + lane);
+// q_idx of the group's heads into shared memory.  Output o = h * R + j
+// (head h, index dim j) is one warp's dot product of q[h] with row o of
+// W_q_idx: lane l owns dims 4l .. 4l + 3, and the warp sums the lanes with
+// warp_sum, so the value does not depend on which warp computes it (every
+// CTA and every kernel gets bit-identical q_idx).  The nwarps warps of the
+// caller (warp index `warp`) take outputs warp, warp + nwarps, ..., all of
+// their loads in flight at once; PER_WARP >= ceil(G * R / nwarps).
+template <int PER_WARP>
+struct QProj {
+    float acc[PER_WARP];
+    // loads and per-lane partial dot products
+    __device__ __forceinline__ void load(const float *__restrict__ q_bh0, const float *__restrict__ W_h0, int G,
+                                         int warp, int nwarps) {
+        const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        float4 wv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            wv[j] = __ldg(reinterpret_cast<const float4 *>(W_h0 + (warp * R + half * 8 + j) * D) + lane);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            float acc = qv.x * wv[j].x;
-            acc = fmaf(qv.y, wv[j].y, acc);
-            acc = fmaf(qv.z, wv[j].z, acc);
-            acc = fmaf(qv.w, wv[j].w, acc);
-            acc = warp_sum(acc);
-            if (lane == 0) qs[warp * R + half * 8 + j] = acc * scale;
+        for (int k = 0; k < PER_WARP; ++k) {
+            const int o = warp + k * nwarps;
+            acc[k] = 0.0f;
+            if (o < G * R) {
+                const float4 qv = __ldg(reinterpret_cast<const float4 *>(q_bh0 + (o / R) * D) + lane);
+                const float4 wv = __ldg(reinterpret_cast<const float4 *>(W_h0 + (size_t)o * D) + lane);
+                float x = qv.x * wv.x;
+                x = fmaf(qv.y, wv.y, x);
+                x = fmaf(qv.z, wv.z, x);
+                x = fmaf(qv.w, wv.w, x);
+                acc[k] = x;
+            }
         }
     }
+    // warp sums -> qs[o]
+    __device__ __forceinline__ void store(float scale, float *qs, int G, int warp, int nwarps) {
+        const int lane = threadIdx.x & 31;
+#pragma unroll
+        for (int k = 0; k < PER_WARP; ++k) {
+            const int o = warp + k * nwarps;
+            const float v = warp_sum(acc[k]);
+            if (o < G * R && lane == 0) qs[o] = v * scale;
+        }
+    }
+};
+
+template <int PER_WARP>
+__device__ __forceinline__ void project_query(const float *__restrict__ q_bh0,
+                                              const float *__restrict__ W_h0, float scale,
+                                              float *qs, int G, int warp, int nwarps) {
+    QProj<PER_WARP> qp;
+    qp.load(q_bh0, W_h0, G, warp, nwarps);
+    qp.store(scale, qs, G, warp, nwarps);
 }
 
 // ---------------------------------------------------------------------------
@@ -381,86 +401,94 @@ template <> struct NeedsQ<SrcBuffer> : std::false_type {};
 // S_b exp(U_b - R) in fp64, the boundary bin where the mass accumulated
 // from the top first reaches p Z.  Zeroes the histogram for the next call.
 // ---------------------------------------------------------------------------
-__device__ void resolve_head(double *gh, Resolve *out, float p, int N) {
+// Resolve one head from its level-1 histogram `gh` (global memory, all of
+// the group's scan CTAs done).  One warp; lane l holds bins 16 l .. 16 l + 15
+// in registers (one round of loads).  Bin masses are taken relative to the
+// upper edge R of the top non-empty bin; in descending bin order the first
+// bin where the cumulative mass reaches p Z is b*, `above` is the mass of
+// the bins before it and `target` what b* must still supply (infinite: all
+// of b*).  Every lane returns the same record.
+__device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, float p, int N) {
+    constexpr int SEG = NBIN / 32;
     const int lane = threadIdx.x & 31;
-    int top = -1;
-    for (int bin = lane; bin < NBIN; bin += 32)
-        if (gh[bin] > 0.0) top = bin;
+    double v[SEG];
+#pragma unroll
+    for (int j = 0; j < SEG; j += 2) {
+        const double2 t = __ldcg(reinterpret_cast<const double2 *>(gh + lane * SEG + j));
+        v[j] = t.x;
+        v[j + 1] = t.y;
+    }
+    int top = -1, low = NBIN;
+#pragma unroll
+    for (int j = 0; j < SEG; ++j)
+        if (v[j] > 0.0) { top = lane * SEG + j; low = min(low, lane * SEG + j); }
     top = __reduce_max_sync(0xffffffffu, top);
+    low = __reduce_min_sync(0xffffffffu, low);
     Resolve r;
     r.N = N;
     if (top < 0 || N == 0) {
         r.Z = 0; r.above = 0; r.target = 0; r.R = 0.f; r.bstar = -1; r.mode = MODE_EMPTY;
-        if (lane == 0) *out = r;
-        __syncwarp();
-        for (int bin = lane; bin < NBIN; bin += 32) gh[bin] = 0.0;
-        return;
+        return r;
     }
     const float R = bin_upper(top);
-    constexpr int SEG = NBIN / 32;
-    // lane l covers bins top - l*SEG - i, i = 0..SEG-1 (descending)
     double seg = 0.0;
-    for (int i = 0; i < SEG; ++i) {
-        const int bin = top - lane * SEG - i;
-        if (bin < 0) break;
-        const double sb = gh[bin];
-        if (sb > 0.0) seg += sb * (double)ex2_sfu((bin_upper(bin) - R) * 1.4426950408889634f);
+#pragma unroll
+    for (int j = 0; j < SEG; ++j) {
+        v[j] = v[j] > 0.0 ? v[j] * (double)ex2_sfu((bin_upper(lane * SEG + j) - R) * 1.4426950408889634f) : 0.0;
+        seg += v[j];
     }
+    // inclusive suffix sums over lanes: mass of this lane's bins and all above
     double incl = seg;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        const double v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
+        const double t = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += t;
     }
-    const double Z = __shfl_sync(0xffffffffu, incl, 31);
+    const double Z = __shfl_sync(0xffffffffu, incl, 0);
     const double excl = incl - seg;
     r.Z = Z;
     r.R = R;
     if (p >= 1.0f) {
         r.mode = MODE_KEEP_ALL; r.bstar = -1; r.above = 0; r.target = 0;
-    } else {
-        const double target = p <= 0.0f ? 0.0 : (double)p * Z;
-        const unsigned hit = __ballot_sync(0xffffffffu, seg > 0.0 && excl + seg >= target);
-        int bstar = -1;
-        double above = 0.0, tin = INFINITY;
-        if (hit) {
-            const int L = __ffs(hit) - 1;
-            if (lane == L) {
-                double cum = excl;
-                for (int i = 0; i < SEG; ++i) {
-                    const int bin = top - lane * SEG - i;
-                    if (bin < 0) break;
-                    const double sb = gh[bin];
-                    if (sb <= 0.0) continue;
-                    const double mb = sb * (double)ex2_sfu((bin_upper(bin) - R) * 1.4426950408889634f);
-                    bstar = bin;       // if rounding never crosses, the last bin is kept whole
-                    above = cum;
-                    if (cum + mb >= target) { tin = target - cum; break; }
-                    cum += mb;
-                    tin = INFINITY;
-                }
-            }
-            bstar = __shfl_sync(0xffffffffu, bstar, L);
-            above = __shfl_sync(0xffffffffu, above, L);
-            tin = __shfl_sync(0xffffffffu, tin, L);
-        } else {
-            // rounding kept p Z out of reach: keep everything down to the lowest bin
-            int low = NBIN;
-            for (int bin = lane; bin < NBIN; bin += 32)
-                if (gh[bin] > 0.0) low = min(low, bin);
-            low = __reduce_min_sync(0xffffffffu, low);
-            bstar = low;
-            above = Z - gh[low] * (double)ex2_sfu((bin_upper(low) - R) * 1.4426950408889634f);
-            tin = INFINITY;
-        }
-        r.mode = MODE_NORMAL;
-        r.bstar = bstar;
-        r.above = above;
-        r.target = tin;
+        return r;
     }
-    if (lane == 0) *out = r;
-    __syncwarp();
-    for (int bin = lane; bin < NBIN; bin += 32) gh[bin] = 0.0;
+    const double target = p <= 0.0f ? 0.0 : (double)p * Z;
+    const unsigned hit = __ballot_sync(0xffffffffu, seg > 0.0 && incl >= target);
+    int bstar = -1;
+    double above = 0.0, tin = INFINITY;
+    if (hit) {
+        const int L = 31 - __clz(hit);            // highest bins first
+        if (lane == L) {
+            double cum = excl;
+            bool done = false;
+#pragma unroll
+            for (int j = SEG - 1; j >= 0; --j) {
+                if (done || !(v[j] > 0.0)) continue;
+                bstar = lane * SEG + j;           // if rounding never crosses, the last bin is kept whole
+                above = cum;
+                if (cum + v[j] >= target) { tin = target - cum; done = true; }
+                else { cum += v[j]; tin = INFINITY; }
+            }
+        }
+        bstar = __shfl_sync(0xffffffffu, bstar, L);
+        above = __shfl_sync(0xffffffffu, above, L);
+        tin = __shfl_sync(0xffffffffu, tin, L);
+    } else {
+        // rounding kept p Z out of reach: keep everything down to the lowest bin
+        double m_low = 0.0;
+#pragma unroll
+        for (int j = 0; j < SEG; ++j)
+            if (lane * SEG + j == low) m_low = v[j];
+        m_low = __shfl_sync(0xffffffffu, m_low, low / SEG);
+        bstar = low;
+        above = Z - m_low;
+        tin = INFINITY;
+    }
+    r.mode = MODE_NORMAL;
+    r.bstar = bstar;
+    r.above = above;
+    r.target = tin;
+    return r;
 }
 
 // ---------------------------------------------------------------------------
@@ -473,19 +501,21 @@ constexpr int SCAN_WARPS = SCAN_THREADS / 32;
 template <typename Src>
 __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(SelArgs a, SelWs w) {
     __shared__ __align__(16) float qs[GMAX * R];
-    __shared__ uint32_t shl[2 * GMAX * NBIN];   // fixed-point bin sums: low words, then high words
+    __shared__ __align__(16) uint32_t shl[2 * GMAX * NBIN];   // fixed-point bin sums: low words, then high words
     uint32_t *const shh = shl + GMAX * NBIN;
-    __shared__ int s_last, s_err;
+    __shared__ int s_err;
     const int b = blockIdx.y / a.n_ret;
     const int g = a.ret_g[blockIdx.y % a.n_ret];
     const int G = a.G;
-    const size_t bg = (size_t)b * a.H_kv + g;
     const size_t bh0 = (size_t)b * a.H_q + (size_t)g * G;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) s_err = 0;
+    // this call's collect pass appends from zero
+    if (blockIdx.x == 0 && threadIdx.x < G) { w.cand_cnt[bh0 + threadIdx.x] = 0u; w.list_cnt[bh0 + threadIdx.x] = 0u; }
     for (int i = threadIdx.x; i < 2 * GMAX * NBIN; i += blockDim.x) shl[i] = 0u;
     if constexpr (NeedsQ<Src>::value) {
-        project_query(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, a.idx_scale, qs, G);
+        project_query<(GMAX * R + SCAN_WARPS - 1) / SCAN_WARPS>(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D,
+                                                               a.idx_scale, qs, G, warp, SCAN_WARPS);
     }
     __syncthreads();
     if constexpr (NeedsQ<Src>::value) {
@@ -563,18 +593,6 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(SelArgs a, SelWs w) 
         if (lo | hi)
             atomicAdd(&w.hist[bh0 * NBIN + i], ((double)hi * 4294967296.0 + (double)lo) * (1.0 / FX_ONE));
     }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(&w.arrive[bg], 1u) == (unsigned)(gridDim.x - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    if (warp < G) {
-        const size_t bh = bh0 + warp;
-        resolve_head(w.hist + bh * NBIN, w.res + bh, a.p, N);
-        if (lane == 0) { w.cand_cnt[bh] = 0; w.list_cnt[bh] = 0; }
-    }
-    if (threadIdx.x == 0) w.arrive[bg] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -624,7 +642,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
     uint64_t *full = reinterpret_cast<uint64_t *>(dsm + NSTAGE * ST_BYTES + GMAX * NBIN * 12);
     uint64_t *empty = full + NSTAGE;
     __shared__ __align__(16) float qs[GMAX * R];
-    __shared__ int s_last, s_err, s_abort;
+    __shared__ int s_err, s_abort;
     const int b = blockIdx.y / a.n_ret;
     const int g = a.ret_g[blockIdx.y % a.n_ret];
     const int G = a.G;
@@ -638,6 +656,13 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
         fence_mbar_init();
     }
     for (int i = threadIdx.x; i < GMAX * NBIN; i += blockDim.x) { h32[i] = 0u; h64[i] = 0ull; }
+    pdl_wait();
+    pdl_trigger();
+    // this call's collect pass appends from zero
+    if (blockIdx.x == 0 && threadIdx.x < G) { w.cand_cnt[bh0 + threadIdx.x] = 0u; w.list_cnt[bh0 + threadIdx.x] = 0u; }
+    // the consumers' q_idx loads go out before the producer's first bulk copy
+    QProj<(GMAX * R + TC_WARPS - 1) / TC_WARPS> qp;
+    if (warp < TC_WARPS) qp.load(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, G, warp, TC_WARPS);
     __syncthreads();
     const int N = valid_len(a.seq_lens, b, a.N_max, w.status);
     const int t_lo = (int)((long long)blockIdx.x * a.chunk);
@@ -669,9 +694,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
                 mbar_wait(&full[it % NSTAGE], (uint32_t)((it / NSTAGE) & 1));
         }
     } else {
-        // consumers
-        // q_idx of the group (consumer warps only; the producer is already streaming)
-        project_query(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, a.idx_scale, qs, G);
+        // consumers: finish q_idx of the group (the producer is already streaming)
+        qp.store(a.idx_scale, qs, G, warp, TC_WARPS);
         asm volatile("bar.sync 1, %0;" ::"r"(TC_WARPS * 32) : "memory");
         if (blockIdx.x == 0)
             for (int i = threadIdx.x; i < G * R; i += TC_WARPS * 32) w.qidx[bh0 * R + i] = qs[i];
@@ -755,18 +779,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
         const unsigned long long v = h64[i] + h32[i];
         if (v) atomicAdd(&w.hist[bh0 * NBIN + i], (double)v * (1.0 / FX18));
     }
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) s_last = atomicAdd(&w.arrive[bg], 1u) == (unsigned)(gridDim.x - 1);
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    if (warp < G) {
-        const size_t bh = bh0 + warp;
-        resolve_head(w.hist + bh * NBIN, w.res + bh, a.p, N);
-        if (lane == 0) { w.cand_cnt[bh] = 0; w.list_cnt[bh] = 0; }
-    }
-    if (threadIdx.x == 0) w.arrive[bg] = 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -806,25 +818,32 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
     const int G = a.G;
     const size_t bh0 = (size_t)b * a.H_q + (size_t)g * G;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x < GMAX) {
+    pdl_wait();
+    pdl_trigger();
+    // Every CTA resolves the group's heads from the finished histograms
+    // (warp h: head h); the group's first CTA records them for finalize.
+    const int N = valid_len(a.seq_lens, b, a.N_max, w.status);
+    if (warp < GMAX) {
         int mode = MODE_EMPTY, bs = NBIN;
-        if (threadIdx.x < G) {
-            const Resolve r = w.res[bh0 + threadIdx.x];
+        if (warp < G) {
+            const Resolve r = resolve_head(w.hist + (bh0 + warp) * NBIN, a.p, N);
+            if (blockIdx.x == 0 && lane == 0) w.res[bh0 + warp] = r;
             mode = r.mode;
             bs = r.bstar;
         }
-        s_mode[threadIdx.x] = mode;
-        // keep-all heads need no collect pass: finalize lists every token
-        s_bstar[threadIdx.x] = mode == MODE_NORMAL ? bs : NBIN;
-        s_khi[threadIdx.x] = mode == MODE_NORMAL ? bin_hi_incl(bs) : INFINITY;
-        s_clo[threadIdx.x] = mode == MODE_NORMAL ? bin_lo_incl(bs) : INFINITY;
-        s_kc[threadIdx.x] = 0u;
-        s_cc[threadIdx.x] = 0u;
+        if (lane == 0) {
+            s_mode[warp] = mode;
+            // keep-all heads need no collect pass: finalize lists every token
+            s_bstar[warp] = mode == MODE_NORMAL ? bs : NBIN;
+            s_khi[warp] = mode == MODE_NORMAL ? bin_hi_incl(bs) : INFINITY;
+            s_clo[warp] = mode == MODE_NORMAL ? bin_lo_incl(bs) : INFINITY;
+            s_kc[warp] = 0u;
+            s_cc[warp] = 0u;
+        }
     }
     if constexpr (NeedsQ<Src>::value)
         for (int i = threadIdx.x; i < G * R; i += blockDim.x) qs[i] = w.qidx[bh0 * R + i];
     __syncthreads();
-    const int N = w.res[bh0].N;
     Src src;
     init_src(src, a, b, g, qs);
     const int t_lo = (int)((long long)blockIdx.x * a.chunk);
@@ -928,8 +947,8 @@ constexpr int FIN_CAP = 3072;             // candidates staged in shared memory
 // grid = (B * n_ret * G).  Candidate masses relative to the boundary bin's
 // upper edge U* are each in (e^-32, 1]; they are summed in fixed point with
 // S = 2^62 / nc units per unit of mass, so sums stay below 2^62 and do not
-// depend on the order of the adds.  The last CTA to finish writes the
-// exclusive prefix of list-attention items per head (item_pre).
+// depend on the order of the adds.  The head's level-1 histogram is cleared
+// here for the next call.
 __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs w) {
     __shared__ unsigned long long hfx[256];
     __shared__ uint32_t hfx32[256];
@@ -938,7 +957,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     __shared__ uint32_t fbuf[FIN_CAP];
     __shared__ unsigned long long s_min, s_max, s_theta, s_excl, s_kept;
     __shared__ unsigned s_base;
-    __shared__ int s_digit, s_last;
+    __shared__ int s_digit;
     __shared__ unsigned s_dcnt;
     const int G = a.G;
     const int hb = blockIdx.x;
@@ -946,9 +965,16 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     const int gi = (hb / G) % a.n_ret;
     const int h = a.ret_g[gi] * G + hb % G;
     const size_t bh = (size_t)b * a.H_q + h;
+    pdl_wait();
+    pdl_trigger();
+    // the collect pass is done with the histogram: clear it for the next call
+    for (int i = threadIdx.x; i < NBIN; i += blockDim.x) w.hist[bh * NBIN + i] = 0.0;
+    // the head's resolve record and both counters in one round of loads
     const Resolve r = w.res[bh];
+    const unsigned nc_all = w.cand_cnt[bh];
+    const unsigned base0 = w.list_cnt[bh];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const unsigned nc = r.mode == MODE_NORMAL ? w.cand_cnt[bh] : 0u;
+    const unsigned nc = r.mode == MODE_NORMAL ? nc_all : 0u;
     const unsigned long long *cg = w.cands + bh * a.N_max;
     int32_t *lst = a.lists + bh * a.N_max;
     int count = 0;
@@ -959,7 +985,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         count = r.N;
         mass = 1.0f;
     } else if (r.mode != MODE_NORMAL || nc == 0u) {
-        count = r.mode == MODE_EMPTY ? 0 : (int)w.list_cnt[bh];
+        count = r.mode == MODE_EMPTY ? 0 : (int)base0;
         mass = r.mode == MODE_EMPTY ? 0.0f : (float)(r.above / r.Z);
     } else {
         const float Ub = bin_upper(r.bstar);
@@ -1080,7 +1106,6 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         }
         // kept = candidates at or above theta, appended after the ids the
         // collect pass wrote (block-wide ranks, no global atomics)
-        const unsigned base0 = w.list_cnt[bh];
         unsigned long long kept = 0ull;
         const unsigned lt = (1u << lane) - 1u;
         for (unsigned c0 = 0; c0 < nc; c0 += blockDim.x) {
@@ -1112,39 +1137,6 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         a.count_out[bh] = count;
         if (a.mass_out) a.mass_out[bh] = mass;
     }
-    // the last CTA builds the list-attention work prefix over all heads
-    if (!a.item_pre) return;
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) s_last = atomicAdd(w.fin_arrive, 1u) == gridDim.x - 1;
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    if (warp == 0) {
-        const int nh = gridDim.x;
-        int run = 0;
-        for (int base = 0; base < nh; base += 32) {
-            const int hi = base + lane;
-            int it = 0;
-            if (hi < nh) {
-                const int bb = hi / (a.n_ret * G);
-                const int hh = a.ret_g[(hi / G) % a.n_ret] * G + hi % G;
-                it = list_items(__ldcg(a.count_out + (size_t)bb * a.H_q + hh));
-            }
-            int incl = it;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int v = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += v;
-            }
-            if (hi < nh) a.item_pre[hi] = run + incl - it;
-            run += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) {
-            a.item_pre[nh] = run;
-            *w.fin_arrive = 0u;
-        }
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1157,7 +1149,8 @@ __global__ void __launch_bounds__(SC_THREADS) scores_kernel(SelArgs a, SelWs w, 
     const int g = a.ret_g[blockIdx.y % a.n_ret];
     const int G = a.G;
     const size_t bh0 = (size_t)b * a.H_q + (size_t)g * G;
-    project_query(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, a.idx_scale, qs, G);
+    project_query<(GMAX * R + SC_WARPS - 1) / SC_WARPS>(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, a.idx_scale,
+                                                         qs, G, threadIdx.x >> 5, SC_WARPS);
     __syncthreads();
     const int N = valid_len(a.seq_lens, b, a.N_max, w.status);
     Src src;
