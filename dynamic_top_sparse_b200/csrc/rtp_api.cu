@@ -5,7 +5,6 @@
 #include <cstdlib>
 #include <cstdio>
 #include <cstring>
-#include <functional>
 
 #include "rtp.h"
 #include "rtp_common.cuh"
@@ -19,6 +18,8 @@ using namespace rtp;
 namespace {
 
 constexpr int RANGE_SPLIT_MAX = 256;
+// SMs given to the local heads while the selection runs beside them
+constexpr int LOCAL_SMS = 12;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -58,7 +59,7 @@ Layout make_layout(const rtp_dims *d) {
     L.end_range = o;
     L.part_list = o; o = align_up(o + BHq * LIST_MAX_SPLIT * PSTRIDE * 4, 256);
     L.end_list = o;
-    L.tilebin = o; o = align_up(o + BHq * ntile * 2, 256);
+    L.tilebin = o; o = align_up(o + BHkv * ntile * GMAX * 2, 256);
     L.lists = o; o = align_up(o + BHq * (size_t)d->N_max * 4, 256);
     L.cands = o; o = align_up(o + BHq * (size_t)d->N_max * 8, 256);
     L.total = o;
@@ -226,25 +227,21 @@ SelPlan make_sel(const rtp_dims *d, const uint8_t *hc, char *ws, const Layout &L
     return s;
 }
 
-// Work queued right after the scan kernel (the local heads of a decode
-// step, forked onto a side stream so that they overlap the latency-bound
-// collect / finalize / list kernels instead of holding SMs the scan needs).
-using AfterScan = std::function<int()>;
-
 // scan + collect + finalize over a logit source
 template <typename Src>
-int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s, const AfterScan &after_scan = {}) {
+int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s) {
     const dim3 grid((unsigned)s.a.ctas, (unsigned)(d->B * s.a.n_ret));
     RTP_TRY(ln.run("hist", scan_kernel<Src>, grid, dim3(SCAN_THREADS), s.a, s.w));
-    if (after_scan) RTP_TRY(after_scan());
     RTP_TRY(ln.run("collect", collect_kernel<Src>, grid, dim3(COL_THREADS), s.a, s.w));
     RTP_TRY(ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)),
                    dim3(FIN_THREADS), s.a, s.w));
     return RTP_OK;
 }
 
-int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, const AfterScan &after_scan = {}) {
-    if (d->idx_dtype != RTP_BF16) return launch_select<SrcSimt<float>>(ln, d, s, after_scan);
+// reserve_sms: SMs left free for work running beside the selection (the
+// local heads of a decode step), so that neither waits for the other.
+int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sms = 0) {
+    if (d->idx_dtype != RTP_BF16) return launch_select<SrcSimt<float>>(ln, d, s);
     // bf16 index keys: the TMA-ring scan, one CTA per SM over all groups
     static int attr_set[64] = {0};
     int dev = 0;
@@ -257,7 +254,8 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, const AfterSca
     }
     const long long groups = (long long)d->B * s.a.n_ret;
     const long long tiles = (d->N_max + TILE - 1) / TILE;
-    long long ctas = std::max(1LL, std::min((long long)num_sms() / std::max(groups, 1LL), tiles));
+    const long long sms = std::max(1LL, (long long)num_sms() - std::max(0, reserve_sms));
+    long long ctas = std::max(1LL, std::min(sms / std::max(groups, 1LL), tiles));
     s.a.chunk = (tiles + ctas - 1) / ctas * TILE;
     s.a.ctas = (int)((d->N_max + s.a.chunk - 1) / s.a.chunk);
     const dim3 grid((unsigned)s.a.ctas, (unsigned)groups);
@@ -267,8 +265,7 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, const AfterSca
     const bool pdl0 = ln.pdl;
     ln.pdl = true;
     int rc = ln.run_smem("hist", scan_tma_kernel, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w);
-    if (rc == RTP_OK && after_scan) rc = after_scan();
-    if (rc == RTP_OK) rc = ln.run("collect", collect_kernel<SrcMma>, grid, dim3(COL_THREADS), s.a, s.w);
+    if (rc == RTP_OK) rc = ln.run("collect", collect_mma_kernel, grid, dim3(CL_THREADS), s.a, s.w);
     if (rc == RTP_OK)
         rc = ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)), dim3(FIN_THREADS),
                     s.a, s.w);
@@ -307,7 +304,7 @@ int side_stream(Side *&out) {
 // ----------------------------------------------------------------- attention
 int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
                  const uint8_t *hc, int want_class, bool dense, int window, int n_sink, float *out,
-                 char *ws, const Layout &L, float attn_scale) {
+                 char *ws, const Layout &L, float attn_scale, int max_ctas = 0) {
     RangeArgs a{};
     a.B = d->B; a.H_q = d->H_q; a.H_kv = d->H_kv; a.G = d->H_q / d->H_kv;
     a.N_max = d->N_max; a.seq_lens = d->seq_lens;
@@ -323,6 +320,7 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
     const int per_sm = 1;
     const long long chunks = (Lmax + rows_min - 1) / rows_min;
     long long want = ((long long)per_sm * num_sms() + (long long)d->B * a.n_grp - 1) / ((long long)d->B * a.n_grp);
+    if (max_ctas > 0) want = std::max(1LL, (long long)max_ctas / ((long long)d->B * a.n_grp));
     a.n_split = (int)std::max(1LL, std::min(want, std::min(chunks, (long long)RANGE_SPLIT_MAX)));
     a.scale_log2 = attn_scale * 1.4426950408889634f;
     a.q = q; a.k = k; a.v = v; a.out = out;
@@ -627,23 +625,28 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
     const bool any_local = s.a.n_ret < dims->H_kv;
     const cudaStream_t main = (cudaStream_t)stream;
     Side *side = nullptr;
-    // Local heads run on a side stream that forks from the main stream at
-    // the point where this is called (so they start once the work queued
-    // before it has finished) and joins it at the end of the step.
-    auto fork_local = [&]() -> int {
+    // Local heads run on a side stream forked at the start of the step and
+    // joined at its end.  Beside the selection they get a few SMs of their
+    // own (the selection kernels take one CTA per SM on the rest), so that
+    // neither waits for the other's CTAs to drain.
+    const bool selecting = s.a.n_ret > 0 && p < 1.0f;
+    int local_ctas = 0;
+    if (any_local && s.a.n_ret > 0) {
+        int max_ctas = 0;
+        if (selecting) {
+            const int groups = dims->B * (dims->H_kv - s.a.n_ret);
+            local_ctas = groups * std::max(1, LOCAL_SMS / groups);
+            local_ctas = std::min(local_ctas, num_sms() / 2);
+            max_ctas = local_ctas;
+        }
         RTP_TRY(side_stream(side));
         if (cudaEventRecord(side->fork, main) != cudaSuccess) return RTP_ERR_CUDA;
         if (cudaStreamWaitEvent(side->st, side->fork, 0) != cudaSuccess) return RTP_ERR_CUDA;
         Launcher lside{side->st, ln.prof};
         RTP_TRY(launch_range(lside, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
-                             n_sink, out, w, L, asc));
+                             n_sink, out, w, L, asc, max_ctas));
         if (cudaEventRecord(side->join, side->st) != cudaSuccess) return RTP_ERR_CUDA;
-        return RTP_OK;
-    };
-    const bool selecting = s.a.n_ret > 0 && p < 1.0f;
-    if (any_local && s.a.n_ret > 0 && !selecting) {
-        RTP_TRY(fork_local());
-    } else if (any_local && s.a.n_ret == 0) {
+    } else if (any_local) {
         RTP_TRY(launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
                              n_sink, out, w, L, asc));
     }
@@ -662,9 +665,11 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
             s.a.lists = opts && opts->sel_idx ? opts->sel_idx : reinterpret_cast<int32_t *>(w + L.lists);
             s.a.count_out = opts && opts->sel_count ? opts->sel_count : reinterpret_cast<int32_t *>(w + L.counts);
             s.a.mass_out = opts ? opts->sel_mass : nullptr;
-            // the scan of the index keys gets the whole GPU; the local heads
-            // fork after it and overlap the rest of the selection
-            rc = select_from_index(ln, dims, s, any_local ? AfterScan(fork_local) : AfterScan());
+            // kept rows are prefetched into L2 for the sparse attention
+            s.a.k_rows = static_cast<const uint8_t *>(k_cache);
+            s.a.v_rows = static_cast<const uint8_t *>(v_cache);
+            s.a.kv_row_bytes = D * (dims->kv_dtype == RTP_BF16 ? 2 : 4);
+            rc = select_from_index(ln, dims, s, local_ctas);
             if (rc == RTP_OK) {
                 ln.pdl = dims->idx_dtype == RTP_BF16;    // follows finalize_kernel
                 rc = launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out,

@@ -279,9 +279,13 @@ struct ListArgs {
 // r0 + 16w .. r0 + 16w + 15, then every 128th: the 16 row ids come in one
 // load and all 16 rows' K and V loads are issued before the first dot
 // product.
+constexpr int MAX_LIST_B = 1024;        // sequences per call
+static_assert(65535 / MAX_GROUPS < MAX_LIST_B, "the argument checks must bound B below MAX_LIST_B");
 template <typename KT>
 __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
     __shared__ int pre[MAX_LIST_HEADS + 1];
+    __shared__ int s_cnt[MAX_LIST_HEADS];   // kept rows per head (0 when invalid)
+    __shared__ int s_len[MAX_LIST_B];       // sequence lengths
     __shared__ int s_scan[ATT_THREADS];
     __shared__ float wm[ATT_THREADS / 32], wl[ATT_THREADS / 32];
     __shared__ float wo[ATT_THREADS / 32][D];
@@ -305,8 +309,11 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
                 const int b = hi / a.n_rq, h = a.ret_h[hi % a.n_rq];
                 const int cnt = __ldcg(a.counts + (size_t)b * a.H_q + h);
                 const int N = a.seq_lens[b];
-                if (cnt >= 1 && N >= 1 && (long long)N <= a.N_max && cnt <= N) it = list_items(cnt);
+                const bool ok = cnt >= 1 && N >= 1 && (long long)N <= a.N_max && cnt <= N;
+                if (ok) it = list_items(cnt);
                 pre[hi] = it;
+                s_cnt[hi] = ok ? cnt : 0;
+                s_len[b] = N;
             }
             loc += it;
         }
@@ -358,8 +365,8 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
         const int b = hix / a.n_rq, h = a.ret_h[hix % a.n_rq];
         const int g = h / a.G;
         const size_t bh = (size_t)b * a.H_q + h;
-        const int cnt = a.counts[bh];
-        const int N = a.seq_lens[b];
+        const int cnt = s_cnt[hix];
+        const int N = s_len[b];
         const int nit = pre[hix + 1] - pre[hix];
         const int sub = item - pre[hix];
         const int per_item = (cnt + nit - 1) / nit;

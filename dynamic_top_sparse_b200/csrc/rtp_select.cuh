@@ -146,7 +146,7 @@ struct SelWs {
     uint32_t *list_cnt;          // [B*H_q]
     double *hist;                // [B*H_q][NBIN]
     Resolve *res;                // [B*H_q]
-    uint16_t *tilebin;           // [B*H_q][ntile]: 1 + largest bin of the tile (0: none)
+    uint16_t *tilebin;           // [B*H_kv][ntile][GMAX]: per tile, 1 + largest bin of each head (0: none)
     unsigned long long *cands;   // [B*H_q][N_max]
     float *qidx;                 // [B*H_q][R]
 };
@@ -169,7 +169,19 @@ struct SelArgs {
     int32_t *lists;              // [B*H_q][N_max] kept ids
     int32_t *count_out;          // [B*H_q]
     float *mass_out;             // [B*H_q] or null
+    // K/V caches ([B, H_kv, N_max, D] rows of kv_row_bytes) whose kept rows
+    // are prefetched into L2 as soon as they are known, or null
+    const uint8_t *k_rows, *v_rows;
+    int kv_row_bytes;
 };
+
+// Prefetch the K and V rows of token t of group (b, g) into L2.
+__device__ __forceinline__ void prefetch_kv(const SelArgs &a, size_t bg, int t) {
+    if (!a.k_rows) return;
+    const size_t off = (bg * (size_t)a.N_max + (size_t)t) * (size_t)a.kv_row_bytes;
+    prefetch_l2(a.k_rows + off, (uint32_t)a.kv_row_bytes);
+    prefetch_l2(a.v_rows + off, (uint32_t)a.kv_row_bytes);
+}
 
 __device__ __forceinline__ int valid_len(const int32_t *seq_lens, int b, long long N_max,
                                          uint32_t *status) {
@@ -411,17 +423,19 @@ template <> struct NeedsQ<SrcBuffer> : std::false_type {};
 __device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, float p, int N) {
     constexpr int SEG = NBIN / 32;
     const int lane = threadIdx.x & 31;
-    double v[SEG];
+    // bin sums, rounded to fp32 (relative error 2^-24 per bin; the cut and
+    // the masses downstream are accurate to far better than 1e-5 of Z)
+    float v[SEG];
 #pragma unroll
     for (int j = 0; j < SEG; j += 2) {
         const double2 t = __ldcg(reinterpret_cast<const double2 *>(gh + lane * SEG + j));
-        v[j] = t.x;
-        v[j + 1] = t.y;
+        v[j] = (float)t.x;
+        v[j + 1] = (float)t.y;
     }
     int top = -1, low = NBIN;
 #pragma unroll
     for (int j = 0; j < SEG; ++j)
-        if (v[j] > 0.0) { top = lane * SEG + j; low = min(low, lane * SEG + j); }
+        if (v[j] > 0.0f) { top = lane * SEG + j; low = min(low, lane * SEG + j); }
     top = __reduce_max_sync(0xffffffffu, top);
     low = __reduce_min_sync(0xffffffffu, low);
     Resolve r;
@@ -434,8 +448,8 @@ __device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, f
     double seg = 0.0;
 #pragma unroll
     for (int j = 0; j < SEG; ++j) {
-        v[j] = v[j] > 0.0 ? v[j] * (double)ex2_sfu((bin_upper(lane * SEG + j) - R) * 1.4426950408889634f) : 0.0;
-        seg += v[j];
+        v[j] = v[j] > 0.0f ? v[j] * ex2_sfu((bin_upper(lane * SEG + j) - R) * 1.4426950408889634f) : 0.0f;
+        seg += (double)v[j];
     }
     // inclusive suffix sums over lanes: mass of this lane's bins and all above
     double incl = seg;
@@ -463,11 +477,11 @@ __device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, f
             bool done = false;
 #pragma unroll
             for (int j = SEG - 1; j >= 0; --j) {
-                if (done || !(v[j] > 0.0)) continue;
+                if (done || !(v[j] > 0.0f)) continue;
                 bstar = lane * SEG + j;           // if rounding never crosses, the last bin is kept whole
                 above = cum;
-                if (cum + v[j] >= target) { tin = target - cum; done = true; }
-                else { cum += v[j]; tin = INFINITY; }
+                if (cum + (double)v[j] >= target) { tin = target - cum; done = true; }
+                else { cum += (double)v[j]; tin = INFINITY; }
             }
         }
         bstar = __shfl_sync(0xffffffffu, bstar, L);
@@ -478,7 +492,7 @@ __device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, f
         double m_low = 0.0;
 #pragma unroll
         for (int j = 0; j < SEG; ++j)
-            if (lane * SEG + j == low) m_low = v[j];
+            if (lane * SEG + j == low) m_low = (double)v[j];
         m_low = __shfl_sync(0xffffffffu, m_low, low / SEG);
         bstar = low;
         above = Z - m_low;
@@ -507,6 +521,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(SelArgs a, SelWs w) 
     const int b = blockIdx.y / a.n_ret;
     const int g = a.ret_g[blockIdx.y % a.n_ret];
     const int G = a.G;
+    const size_t bg = (size_t)b * a.H_kv + g;
     const size_t bh0 = (size_t)b * a.H_q + (size_t)g * G;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) s_err = 0;
@@ -527,7 +542,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(SelArgs a, SelWs w) 
     init_src(src, a, b, g, qs);
     const int t_lo = (int)((long long)blockIdx.x * a.chunk);
     const int t_hi = (int)min((long long)N, (long long)t_lo + a.chunk);
-    uint16_t *tbin = w.tilebin + bh0 * a.ntile;
+    uint16_t *tbin = w.tilebin + bg * a.ntile * GMAX;
 
     int err = 0;
     typename Src::Frag cur, nxt;
@@ -580,7 +595,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(SelArgs a, SelWs w) 
 #pragma unroll
             for (int i = 0; i < Src::NSLOT; ++i) {
                 const int h = src.head(i);
-                if (h < G) tbin[(size_t)h * a.ntile + tb / TILE] = (uint16_t)(tmax[i] + 1);
+                if (h < G) tbin[(size_t)(tb / TILE) * GMAX + h] = (uint16_t)(tmax[i] + 1);
             }
         }
         cur = nxt;
@@ -608,13 +623,16 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(SelArgs a, SelWs w) 
 // ---------------------------------------------------------------------------
 constexpr int TC_WARPS = 24;                             // consumer warps
 constexpr int TC_THREADS = (TC_WARPS + 1) * 32;          // + one producer warp
-constexpr int ST_TOK = TC_WARPS * TILE;                  // tokens per stage
+constexpr int TPW = 2;                                   // tiles per consumer warp per stage
+constexpr int ST_TOK = TC_WARPS * TPW * TILE;            // tokens per stage
 constexpr int ST_BYTES = ST_TOK * R * 2;                 // bf16 index keys
-constexpr int NSTAGE = 4;
-constexpr int SPILL_STAGES = 10;                         // 7680 tokens
+constexpr int NSTAGE = 3;
+constexpr int SPILL_STAGES = 10;                         // 15360 tokens
 constexpr float FX18 = 262144.0f;                        // 2^18
 constexpr int TC_SMEM = NSTAGE * ST_BYTES + GMAX * NBIN * 4 + GMAX * NBIN * 8 + 2 * NSTAGE * 8;
-static_assert((long long)SPILL_STAGES * ST_TOK * 262144LL < 4294967296LL, "bin counters would wrap");
+// largest single add: 2^18 e^(2^-6) < 266240 (values of the k = 0 bins may
+// sit slightly above the bin's upper edge)
+static_assert((long long)SPILL_STAGES * ST_TOK * 266240LL < 4294967296LL, "bin counters would wrap");
 
 // Hot path of the scan for one value z (already folded so that -0 is +0):
 // adds exp(z - U_bin) in 2^18 fixed point to the head's bin counter at
@@ -632,6 +650,35 @@ __device__ __forceinline__ int scan_value(float z, uint32_t row, int &bin) {
     bin = 256 + (k ^ s);
     asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row + 4u * (uint32_t)bin), "r"(fx) : "memory");
     return kr;
+}
+
+// Producer of a TMA ring (lane 0 of the producer warp): streams the index
+// keys of tokens [t_lo, t_hi) stage by stage into `ring` (ST_TOK tokens per
+// stage).  Waits are bounded: on a timeout it records RTP_ERR_TIMEOUT and
+// sets *abort.  Before returning it waits for its own copies still in flight.
+template <int NS>
+__device__ __forceinline__ void ring_produce(int t_lo, int t_hi, const __nv_bfloat16 *rows, uint8_t *ring,
+                                             uint64_t *full, uint64_t *empty, uint32_t *status, int *abort) {
+    const int n_st = t_hi > t_lo ? (t_hi - t_lo + ST_TOK - 1) / ST_TOK : 0;
+    int issued = 0;
+    for (int it = 0; it < n_st; ++it) {
+        const int st = it % NS;
+        if (it >= NS && !mbar_wait(&empty[st], (uint32_t)((it / NS - 1) & 1))) {
+            set_status(status, RTP_ERR_TIMEOUT);
+            *abort = 1;
+            break;
+        }
+        if (*(volatile int *)abort) break;
+        fence_proxy_async();
+        const int tok0 = t_lo + it * ST_TOK;
+        const uint32_t bytes = (uint32_t)min(ST_TOK, t_hi - tok0) * (uint32_t)(R * 2);
+        mbar_expect_tx(&full[st], bytes);
+        bulk_g2s(ring + st * ST_BYTES, rows + (size_t)tok0 * R, bytes, &full[st]);
+        issued = it + 1;
+    }
+    // no copy may still be landing in shared memory when the CTA exits
+    for (int it = max(0, issued - NS); it < issued; ++it)
+        mbar_wait(&full[it % NS], (uint32_t)((it / NS) & 1));
 }
 
 __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelWs w) {
@@ -671,28 +718,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
     const __nv_bfloat16 *rows = reinterpret_cast<const __nv_bfloat16 *>(a.kidx) + bg * a.N_max * R;
 
     if (warp == TC_WARPS) {
-        // producer
-        if (lane == 0) {
-            int issued = 0;
-            for (int it = 0; it < n_st; ++it) {
-                const int st = it % NSTAGE;
-                if (it >= NSTAGE && !mbar_wait(&empty[st], (uint32_t)((it / NSTAGE - 1) & 1))) {
-                    set_status(w.status, RTP_ERR_TIMEOUT);
-                    s_abort = 1;
-                    break;
-                }
-                if (*(volatile int *)&s_abort) break;
-                fence_proxy_async();
-                const int tok0 = t_lo + it * ST_TOK;
-                const uint32_t bytes = (uint32_t)min(ST_TOK, t_hi - tok0) * (uint32_t)(R * 2);
-                mbar_expect_tx(&full[st], bytes);
-                bulk_g2s(ring + st * ST_BYTES, rows + (size_t)tok0 * R, bytes, &full[st]);
-                issued = it + 1;
-            }
-            // no copy may still be landing in shared memory when the CTA exits
-            for (int it = max(0, issued - NSTAGE); it < issued; ++it)
-                mbar_wait(&full[it % NSTAGE], (uint32_t)((it / NSTAGE) & 1));
-        }
+        if (lane == 0)
+            ring_produce<NSTAGE>(t_lo, t_hi, rows, ring, full, empty, w.status, &s_abort);
     } else {
         // consumers: finish q_idx of the group (the producer is already streaming)
         qp.store(a.idx_scale, qs, G, warp, TC_WARPS);
@@ -705,64 +732,73 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
         const uint32_t hrow0 = smem_u32(h32 + (2 * tig) * NBIN), hrow1 = smem_u32(h32 + (2 * tig + 1) * NBIN);
         const bool full_group = G == GMAX;
         int kmax = 0;
-        uint16_t *tbin = w.tilebin + bh0 * a.ntile;
+        uint32_t *tbin = reinterpret_cast<uint32_t *>(w.tilebin + bg * a.ntile * GMAX);
+
+        // One 32-token tile: logits on the tensor cores, level-1 masses into
+        // the bin counters, the tile's largest bin per head into its record.
+        auto scan_tile = [&](const uint8_t *tile, int tb, int nvalid) {
+            SrcMma::Frag f;
+#pragma unroll
+            for (int i = 0; i < 2; ++i)
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+                    f.a[i][r] = *reinterpret_cast<const uint2 *>(tile + (16 * i + gid + 8 * r) * (R * 2) + 8 * tig);
+            float z[SrcMma::NV];
+            src.eval(f, z);
+            int tmax[2] = {-1, -1};
+            if (nvalid >= TILE && full_group) {
+#pragma unroll
+                for (int v = 0; v < SrcMma::NV; ++v) {
+                    const int sl = v & 1;
+                    int bin;
+                    kmax = max(kmax, scan_value(z[v] + 0.0f, sl ? hrow1 : hrow0, bin));
+                    tmax[sl] = max(tmax[sl], bin);
+                }
+            } else {
+#pragma unroll
+                for (int v = 0; v < SrcMma::NV; ++v) {
+                    const int sl = v & 1;
+                    if (2 * tig + sl >= G || src.tok(v) >= nvalid) continue;
+                    int bin;
+                    kmax = max(kmax, scan_value(z[v] + 0.0f, sl ? hrow1 : hrow0, bin));
+                    tmax[sl] = max(tmax[sl], bin);
+                }
+            }
+            // both head slots in one word: (1 + max bin) per 16-bit half
+            uint32_t pk = (uint32_t)(tmax[0] + 1) | ((uint32_t)(tmax[1] + 1) << 16);
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                const uint32_t other = __shfl_xor_sync(0xffffffffu, pk, o);
+                asm("max.u16x2 %0, %0, %1;" : "+r"(pk) : "r"(other));
+            }
+            // lane l < 4 writes heads 2l, 2l + 1 of the tile's record
+            if (lane < 4) tbin[(size_t)(tb / TILE) * (GMAX / 2) + lane] = pk;
+        };
         // After a timeout every consumer warp keeps iterating without
         // waiting or working, so the named barrier below stays balanced.
         bool dead = false;
+        int st = 0, phase = 0, spill_in = SPILL_STAGES;
         for (int it = 0; it < n_st; ++it) {
-            const int st = it % NSTAGE;
             if (!dead) dead = *(volatile int *)&s_abort != 0;
-            if (!dead && !mbar_wait(&full[st], (uint32_t)((it / NSTAGE) & 1))) {
+            if (!dead && !mbar_wait(&full[st], (uint32_t)phase)) {
                 set_status(w.status, RTP_ERR_TIMEOUT);
                 s_abort = 1;
                 dead = true;
             }
-            const int tb = t_lo + it * ST_TOK + warp * TILE;
-            const int nvalid = dead ? 0 : t_hi - tb;
-            if (nvalid > 0) {
-                const uint8_t *tile = ring + st * ST_BYTES + warp * (TILE * R * 2);
-                SrcMma::Frag f;
+            if (!dead) {
+                const int tb0 = t_lo + it * ST_TOK + warp * TILE;
+                const uint8_t *tiles = ring + st * ST_BYTES + warp * (TILE * R * 2);
 #pragma unroll
-                for (int i = 0; i < 2; ++i)
-#pragma unroll
-                    for (int r = 0; r < 2; ++r)
-                        f.a[i][r] = *reinterpret_cast<const uint2 *>(tile + (16 * i + gid + 8 * r) * (R * 2) + 8 * tig);
-                float z[SrcMma::NV];
-                src.eval(f, z);
-                int tmax[2] = {-1, -1};
-                if (nvalid >= TILE && full_group) {
-#pragma unroll
-                    for (int v = 0; v < SrcMma::NV; ++v) {
-                        const int sl = v & 1;
-                        int bin;
-                        kmax = max(kmax, scan_value(z[v] + 0.0f, sl ? hrow1 : hrow0, bin));
-                        tmax[sl] = max(tmax[sl], bin);
-                    }
-                } else {
-#pragma unroll
-                    for (int v = 0; v < SrcMma::NV; ++v) {
-                        const int sl = v & 1;
-                        if (2 * tig + sl >= G || src.tok(v) >= nvalid) continue;
-                        int bin;
-                        kmax = max(kmax, scan_value(z[v] + 0.0f, sl ? hrow1 : hrow0, bin));
-                        tmax[sl] = max(tmax[sl], bin);
-                    }
-                }
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    tmax[i] = max(tmax[i], __shfl_xor_sync(0xffffffffu, tmax[i], 4));
-                    tmax[i] = max(tmax[i], __shfl_xor_sync(0xffffffffu, tmax[i], 8));
-                    tmax[i] = max(tmax[i], __shfl_xor_sync(0xffffffffu, tmax[i], 16));
-                }
-                if (lane < 4) {
-#pragma unroll
-                    for (int i = 0; i < 2; ++i)
-                        if (2 * lane + i < G) tbin[(size_t)(2 * lane + i) * a.ntile + tb / TILE] = (uint16_t)(tmax[i] + 1);
+                for (int tt = 0; tt < TPW; ++tt) {
+                    const int tb = tb0 + tt * TC_WARPS * TILE;
+                    if (t_hi - tb > 0) scan_tile(tiles + tt * (TC_WARPS * TILE * R * 2), tb, t_hi - tb);
                 }
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);
-            if ((it + 1) % SPILL_STAGES == 0 && it + 1 < n_st) {
+            if (++st == NSTAGE) { st = 0; phase ^= 1; }
+            if (--spill_in == 0 && it + 1 < n_st) {
+                spill_in = SPILL_STAGES;
                 asm volatile("bar.sync 1, %0;" ::"r"(TC_WARPS * 32) : "memory");
                 for (int i = threadIdx.x; i < GMAX * NBIN; i += TC_WARPS * 32) {
                     h64[i] += h32[i];
@@ -849,7 +885,7 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
     const int t_lo = (int)((long long)blockIdx.x * a.chunk);
     const int t_hi = (int)min((long long)N, (long long)t_lo + a.chunk);
     const unsigned lt = (1u << lane) - 1u;
-    const uint16_t *tbin = w.tilebin + bh0 * a.ntile;
+    const uint16_t *tbin = w.tilebin + ((size_t)b * a.H_kv + g) * a.ntile * GMAX;
     int bst[GMAX];
 #pragma unroll
     for (int h = 0; h < GMAX; ++h) bst[h] = s_bstar[h];
@@ -864,7 +900,7 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
             const int ti = tb_l / TILE;
 #pragma unroll
             for (int h = 0; h < GMAX; ++h)
-                if (h < G && (int)tbin[(size_t)h * a.ntile + ti] - 1 >= bst[h]) hm |= 1u << h;
+                if (h < G && (int)tbin[(size_t)ti * GMAX + h] - 1 >= bst[h]) hm |= 1u << h;
         }
         const unsigned any_valid = __ballot_sync(0xffffffffu, tb_l < t_hi);
         if (!any_valid) break;
@@ -935,6 +971,185 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
 }
 
 // ---------------------------------------------------------------------------
+// collect for bf16 index keys.  Every CTA first resolves the group's heads
+// from the finished histograms (warp h: head h; the group's first CTA
+// records them for finalize) while its other warps load q_idx and every warp
+// loads the scan's tile records of its first window.  Warp w then owns
+// tiles w, w + CL_WARPS, ... of the CTA's range, screened 32 at a time by
+// their records (a tile is needed when some head's largest bin in it
+// reaches b*); the needed ones are loaded CL_BATCH at a time, all loads in
+// flight, their logits recomputed with the scan's tensor-core arithmetic,
+// and kept ids (z above b*) and b*'s candidates staged per head.
+// grid = the scan's, CL_THREADS threads.
+// ---------------------------------------------------------------------------
+constexpr int CL_WARPS = 16;
+constexpr int CL_THREADS = CL_WARPS * 32;
+constexpr int CL_BATCH = 4;
+
+__global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, SelWs w) {
+    __shared__ __align__(16) float qs[GMAX * R];
+    __shared__ int s_bstar[GMAX];
+    __shared__ unsigned s_kc[GMAX], s_cc[GMAX];
+    __shared__ float s_khi[GMAX], s_clo[GMAX];      // keep: z > s_khi; candidate: s_clo <= z <= s_khi
+    __shared__ int32_t s_kbuf[GMAX * KCAP];
+    __shared__ unsigned long long s_cbuf[GMAX * CCAP];
+    const int b = blockIdx.y / a.n_ret;
+    const int g = a.ret_g[blockIdx.y % a.n_ret];
+    const int G = a.G;
+    const size_t bg = (size_t)b * a.H_kv + g;
+    const size_t bh0 = (size_t)b * a.H_q + (size_t)g * G;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x < GMAX) { s_kc[threadIdx.x] = 0u; s_cc[threadIdx.x] = 0u; }
+    pdl_wait();
+    pdl_trigger();
+    const int N = valid_len(a.seq_lens, b, a.N_max, w.status);
+    const int t_lo = (int)((long long)blockIdx.x * a.chunk);
+    const int t_hi = (int)min((long long)N, (long long)t_lo + a.chunk);
+    const uint4 *recs = reinterpret_cast<const uint4 *>(w.tilebin + bg * a.ntile * GMAX);
+    // tile of lane `lane` in window `win` of this warp
+    auto tile_of = [&](int win) { return t_lo / TILE + warp + (win * 32 + lane) * CL_WARPS; };
+    const int ti_end = (t_hi + TILE - 1) / TILE;
+    uint4 rec = make_uint4(0u, 0u, 0u, 0u);
+    if (t_hi > t_lo && tile_of(0) < ti_end) rec = __ldcg(recs + tile_of(0));
+    if (warp < GMAX) {
+        int bs = NBIN, mode = MODE_EMPTY;
+        if (warp < G) {
+            const Resolve r = resolve_head(w.hist + (bh0 + warp) * NBIN, a.p, N);
+            if (blockIdx.x == 0 && lane == 0) w.res[bh0 + warp] = r;
+            mode = r.mode;
+            bs = r.bstar;
+        }
+        if (lane == 0) {
+            // keep-all heads need no collect pass: finalize lists every token
+            s_bstar[warp] = mode == MODE_NORMAL ? bs : NBIN;
+            s_khi[warp] = mode == MODE_NORMAL ? bin_hi_incl(bs) : INFINITY;
+            s_clo[warp] = mode == MODE_NORMAL ? bin_lo_incl(bs) : INFINITY;
+        }
+    } else {
+        for (int i = threadIdx.x - GMAX * 32; i < G * R; i += (CL_WARPS - GMAX) * 32) qs[i] = w.qidx[bh0 * R + i];
+    }
+    __syncthreads();
+    if (t_hi <= t_lo) return;
+    const __nv_bfloat16 *rows = reinterpret_cast<const __nv_bfloat16 *>(a.kidx) + bg * a.N_max * R;
+    SrcMma src;
+    src.init(rows, a.N_max, qs, G);
+    const int tig = lane & 3;
+    int bst[GMAX];
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) bst[h] = h < G ? s_bstar[h] : NBIN;
+    // thresholds of the lane's two head slots (heads 2 tig, 2 tig + 1):
+    // kept  khi < z < Z_LIMIT, candidate  clo <= z <= khi and z < Z_LIMIT,
+    // with khi and clo raised so that z > -Z_LIMIT too (|z| < Z_LIMIT is the
+    // binned range; -255.99998 is the smallest float above -Z_LIMIT)
+    float khi[2], clo[2];
+#pragma unroll
+    for (int sl = 0; sl < 2; ++sl) {
+        const int h = 2 * tig + sl;
+        khi[sl] = h < G ? fmaxf(s_khi[h], -Z_LIMIT) : INFINITY;
+        clo[sl] = h < G ? fmaxf(s_clo[h], -255.99998f) : INFINITY;
+    }
+
+    for (int win = 0; t_lo / TILE + warp + win * 32 * CL_WARPS < ti_end; ++win) {
+        if (win > 0) rec = tile_of(win) < ti_end ? __ldcg(recs + tile_of(win)) : make_uint4(0u, 0u, 0u, 0u);
+        // heads whose largest bin in lane's tile reaches their b*
+        const uint32_t rw[4] = {rec.x, rec.y, rec.z, rec.w};
+        unsigned hm = 0u;
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) {
+            const int tbmax = (int)((rw[h >> 1] >> (16 * (h & 1))) & 0xffffu) - 1;
+            if (tbmax >= bst[h]) hm |= 1u << h;
+        }
+        if (tile_of(win) >= ti_end) hm = 0u;
+        unsigned todo = __ballot_sync(0xffffffffu, hm != 0u);
+        while (todo) {
+            // up to CL_BATCH needed tiles, all loads in flight
+            int sel[CL_BATCH];
+            SrcMma::Frag f[CL_BATCH];
+#pragma unroll
+            for (int k = 0; k < CL_BATCH; ++k) {
+                sel[k] = todo ? __ffs(todo) - 1 : -1;
+                if (todo) todo &= todo - 1u;
+                if (sel[k] >= 0) src.load(__shfl_sync(0xffffffffu, tile_of(win), sel[k]) * TILE, f[k]);
+            }
+#pragma unroll
+            for (int k = 0; k < CL_BATCH; ++k) {
+                if (sel[k] < 0) break;
+                const int tb = __shfl_sync(0xffffffffu, tile_of(win), sel[k]) * TILE;
+                const unsigned hmask = __shfl_sync(0xffffffffu, hm, sel[k]);
+                float z[SrcMma::NV];
+                src.eval(f[k], z);
+                // fast pass: bit v of km / cm marks value v as kept / candidate
+                const float khi0 = (hmask >> (2 * tig)) & 1u ? khi[0] : INFINITY;
+                const float khi1 = (hmask >> (2 * tig + 1)) & 1u ? khi[1] : INFINITY;
+                const float clo0 = (hmask >> (2 * tig)) & 1u ? clo[0] : INFINITY;
+                const float clo1 = (hmask >> (2 * tig + 1)) & 1u ? clo[1] : INFINITY;
+                unsigned km = 0u, cm = 0u;
+#pragma unroll
+                for (int v = 0; v < SrcMma::NV; ++v) {
+                    const float zz = z[v];
+                    const float kh = (v & 1) ? khi1 : khi0, cl = (v & 1) ? clo1 : clo0;
+                    km |= (unsigned)(zz > kh && zz < Z_LIMIT) << v;
+                    cm |= (unsigned)(zz >= cl && zz <= kh && zz < Z_LIMIT) << v;
+                }
+                if (t_hi - tb < TILE) {
+#pragma unroll
+                    for (int v = 0; v < SrcMma::NV; ++v)
+                        if (tb + src.tok(v) >= t_hi) { km &= ~(1u << v); cm &= ~(1u << v); }
+                }
+                // rare pass: stage the marked values
+                while (km | cm) {
+                    const int v = __ffs(km | cm) - 1;
+                    const bool kept = (km >> v) & 1u;
+                    km &= ~(1u << v);
+                    cm &= ~(1u << v);
+                    const int h = src.head(src.slot(v));
+                    const int t = tb + src.tok(v);
+                    if (kept) {
+                        prefetch_kv(a, bg, t);
+                        const unsigned p = atomicAdd(&s_kc[h], 1u);
+                        if (p < (unsigned)KCAP) {
+                            s_kbuf[h * KCAP + p] = t;
+                        } else {
+                            const unsigned q = atomicAdd(&w.list_cnt[bh0 + h], 1u);
+                            a.lists[(bh0 + h) * a.N_max + q] = t;
+                        }
+                    } else {
+                        float zv = 0.0f;                  // z[v] without dynamic register indexing
+#pragma unroll
+                        for (int u = 0; u < SrcMma::NV; ++u) zv = u == v ? z[u] : zv;
+                        const unsigned long long key = ((unsigned long long)logit_key(zv + 0.0f) << 32) |
+                                                       (unsigned long long)(0xffffffffu - (uint32_t)t);
+                        const unsigned p = atomicAdd(&s_cc[h], 1u);
+                        if (p < (unsigned)CCAP) {
+                            s_cbuf[h * CCAP + p] = key;
+                        } else {
+                            const unsigned q = atomicAdd(&w.cand_cnt[bh0 + h], 1u);
+                            w.cands[(bh0 + h) * a.N_max + q] = key;
+                        }
+                    }
+                }
+            }
+        }
+    }
+    // flush the staged ids: one global reservation per head and kind
+    __syncthreads();
+    if (warp < G) {
+        const size_t bh = bh0 + warp;
+        const unsigned nk = min(s_kc[warp], (unsigned)KCAP);
+        const unsigned ncd = min(s_cc[warp], (unsigned)CCAP);
+        unsigned kb = 0u, cb = 0u;
+        if (lane == 0) {
+            if (nk) kb = atomicAdd(&w.list_cnt[bh], nk);
+            if (ncd) cb = atomicAdd(&w.cand_cnt[bh], ncd);
+        }
+        kb = __shfl_sync(0xffffffffu, kb, 0);
+        cb = __shfl_sync(0xffffffffu, cb, 0);
+        for (unsigned j = lane; j < nk; j += 32) a.lists[bh * a.N_max + kb + j] = s_kbuf[warp * KCAP + j];
+        for (unsigned j = lane; j < ncd; j += 32) w.cands[bh * a.N_max + cb + j] = s_cbuf[warp * CCAP + j];
+    }
+}
+
+// ---------------------------------------------------------------------------
 // finalize: exact selection inside the boundary bin.  One CTA per head.
 // grid = (B * n_ret * G)
 // ---------------------------------------------------------------------------
@@ -974,8 +1189,11 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     const unsigned nc_all = w.cand_cnt[bh];
     const unsigned base0 = w.list_cnt[bh];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const unsigned nc = r.mode == MODE_NORMAL ? nc_all : 0u;
     const unsigned long long *cg = w.cands + bh * a.N_max;
+    // first candidate of each thread, loaded before the count is known (the
+    // buffer holds N_max entries, so the read is in bounds)
+    const unsigned long long c_first = tid < a.N_max ? __ldcg(cg + tid) : 0ull;
+    const unsigned nc = r.mode == MODE_NORMAL ? nc_all : 0u;
     int32_t *lst = a.lists + bh * a.N_max;
     int count = 0;
     float mass = 0.0f;
@@ -1003,7 +1221,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         {
             unsigned long long lo = ~0ull, hi = 0ull;
             for (unsigned c = tid; c < nc; c += blockDim.x) {
-                const unsigned long long v = cg[c];
+                const unsigned long long v = c == (unsigned)tid ? c_first : __ldcg(cg + c);
                 if (staged) { cbuf[c] = v; fbuf[c] = (uint32_t)fx_of(v); }
                 lo = v < lo ? v : lo;
                 hi = v > hi ? v : hi;
@@ -1121,7 +1339,9 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             if (lane == 0 && bal) wbase = atomicAdd(&s_base, (unsigned)__popc(bal));
             wbase = __shfl_sync(0xffffffffu, wbase, 0);
             if (k) {
-                lst[base0 + wbase + __popc(bal & lt)] = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
+                const int t = (int)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
+                prefetch_kv(a, (size_t)b * a.H_kv + (size_t)(h / G), t);
+                lst[base0 + wbase + __popc(bal & lt)] = t;
                 kept += staged ? fbuf[c] : fx_of(v);
             }
         }
