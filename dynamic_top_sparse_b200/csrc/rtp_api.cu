@@ -5,6 +5,7 @@
 #include <cstdlib>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 
 #include "rtp.h"
 #include "rtp_common.cuh"
@@ -57,7 +58,7 @@ Layout make_layout(const rtp_dims *d) {
     L.end_scores = o;
     L.part_range = o; o = align_up(o + BHkv * RANGE_SPLIT_MAX * GMAX * PSTRIDE * 4, 256);
     L.end_range = o;
-    L.part_list = o; o = align_up(o + BHq * LIST_MAX_SPLIT * PSTRIDE * 4, 256);
+    L.part_list = o; o = align_up(o + BHq * LIST_SLOTS * PSTRIDE * 4, 256);
     L.end_list = o;
     L.tilebin = o; o = align_up(o + BHkv * ntile * GMAX * 2, 256);
     L.lists = o; o = align_up(o + BHq * (size_t)d->N_max * 4, 256);
@@ -227,12 +228,18 @@ SelPlan make_sel(const rtp_dims *d, const uint8_t *hc, char *ws, const Layout &L
     return s;
 }
 
+// Work queued right after the collect kernel (in a decode step: the
+// attention over the rows the collect pass kept, forked onto a side stream
+// so that it overlaps finalize).
+using AfterCollect = std::function<int()>;
+
 // scan + collect + finalize over a logit source
 template <typename Src>
-int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s) {
+int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s, const AfterCollect &after_collect = {}) {
     const dim3 grid((unsigned)s.a.ctas, (unsigned)(d->B * s.a.n_ret));
     RTP_TRY(ln.run("hist", scan_kernel<Src>, grid, dim3(SCAN_THREADS), s.a, s.w));
     RTP_TRY(ln.run("collect", collect_kernel<Src>, grid, dim3(COL_THREADS), s.a, s.w));
+    if (after_collect) RTP_TRY(after_collect());
     RTP_TRY(ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)),
                    dim3(FIN_THREADS), s.a, s.w));
     return RTP_OK;
@@ -240,8 +247,9 @@ int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s) {
 
 // reserve_sms: SMs left free for work running beside the selection (the
 // local heads of a decode step), so that neither waits for the other.
-int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sms = 0) {
-    if (d->idx_dtype != RTP_BF16) return launch_select<SrcSimt<float>>(ln, d, s);
+int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sms = 0,
+                      const AfterCollect &after_collect = {}) {
+    if (d->idx_dtype != RTP_BF16) return launch_select<SrcSimt<float>>(ln, d, s, after_collect);
     // bf16 index keys: the TMA-ring scan, one CTA per SM over all groups
     static int attr_set[64] = {0};
     int dev = 0;
@@ -266,6 +274,7 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sm
     ln.pdl = true;
     int rc = ln.run_smem("hist", scan_tma_kernel, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w);
     if (rc == RTP_OK) rc = ln.run("collect", collect_mma_kernel, grid, dim3(CL_THREADS), s.a, s.w);
+    if (rc == RTP_OK && after_collect) rc = after_collect();
     if (rc == RTP_OK)
         rc = ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)), dim3(FIN_THREADS),
                     s.a, s.w);
@@ -287,11 +296,11 @@ struct Side {
     cudaEvent_t fork = nullptr, join = nullptr;
 };
 
-int side_stream(Side *&out) {
-    static thread_local Side sides[64];
+int side_stream(Side *&out, int slot = 0) {
+    static thread_local Side sides[64][2];
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
-    Side &sd = sides[dev];
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64 || slot < 0 || slot > 1) return RTP_ERR_CUDA;
+    Side &sd = sides[dev][slot];
     if (!sd.st) {
         if (cudaStreamCreateWithFlags(&sd.st, cudaStreamNonBlocking) != cudaSuccess) return RTP_ERR_CUDA;
         if (cudaEventCreateWithFlags(&sd.fork, cudaEventDisableTiming) != cudaSuccess) return RTP_ERR_CUDA;
@@ -336,7 +345,20 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
 
 int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
                 const int32_t *lists, const int32_t *counts, const uint8_t *hc, float *out,
-                char *ws, const Layout &L, float attn_scale) {
+                char *ws, const Layout &L, float attn_scale, int phase = LIST_ALL,
+                const uint32_t *first = nullptr) {
+    static int attr_set[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
+    if (!attr_set[dev]) {
+        const int mx = (int)list_smem_bytes(MAX_LIST_HEADS, MAX_LIST_B);
+        if (cudaFuncSetAttribute(list_attn_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 mx) != cudaSuccess ||
+            cudaFuncSetAttribute(list_attn_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) !=
+                cudaSuccess)
+            return RTP_ERR_CUDA;
+        attr_set[dev] = 1;
+    }
     ListArgs a{};
     a.B = d->B; a.H_q = d->H_q; a.H_kv = d->H_kv; a.G = d->H_q / d->H_kv;
     a.N_max = d->N_max; a.seq_lens = d->seq_lens;
@@ -346,15 +368,19 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
     if (a.n_rq == 0) return RTP_OK;
     a.scale_log2 = attn_scale * 1.4426950408889634f;
     a.q = q; a.k = k; a.v = v; a.lists = lists; a.counts = counts; a.out = out;
+    a.first = first;
+    a.phase = phase;
     a.part = reinterpret_cast<float *>(ws + L.part_list);
     a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_list);
     a.status = reinterpret_cast<uint32_t *>(ws + L.status);
     const long long max_items = (long long)d->B * a.n_rq *
         std::min<long long>(LIST_MAX_SPLIT, (d->N_max + LCH - 1) / LCH);
     const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(max_items, 2LL * num_sms()));
+    const size_t smem = list_smem_bytes(d->B * a.n_rq, d->B);
+    const char *name = phase == LIST_FIRST ? "sparse_attn_first" : "sparse_attn";
     if (d->kv_dtype == RTP_BF16)
-        return ln.run("sparse_attn", list_attn_kernel<__nv_bfloat16>, dim3(grid), dim3(ATT_THREADS), a);
-    return ln.run("sparse_attn", list_attn_kernel<float>, dim3(grid), dim3(ATT_THREADS), a);
+        return ln.run_smem(name, list_attn_kernel<__nv_bfloat16>, dim3(grid), dim3(ATT_THREADS), smem, a);
+    return ln.run_smem(name, list_attn_kernel<float>, dim3(grid), dim3(ATT_THREADS), smem, a);
 }
 
 }  // namespace
@@ -665,17 +691,26 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
             s.a.lists = opts && opts->sel_idx ? opts->sel_idx : reinterpret_cast<int32_t *>(w + L.lists);
             s.a.count_out = opts && opts->sel_count ? opts->sel_count : reinterpret_cast<int32_t *>(w + L.counts);
             s.a.mass_out = opts ? opts->sel_mass : nullptr;
-            // kept rows are prefetched into L2 for the sparse attention
-            s.a.k_rows = static_cast<const uint8_t *>(k_cache);
-            s.a.v_rows = static_cast<const uint8_t *>(v_cache);
-            s.a.kv_row_bytes = D * (dims->kv_dtype == RTP_BF16 ? 2 : 4);
-            rc = select_from_index(ln, dims, s, local_ctas);
-            if (rc == RTP_OK) {
-                ln.pdl = dims->idx_dtype == RTP_BF16;    // follows finalize_kernel
+            // The rows the collect pass kept (clearly above the boundary bin)
+            // are attended on a side stream while finalize resolves the
+            // boundary bin; the rest and the merge follow finalize.
+            Side *side2 = nullptr;
+            const uint32_t *first = reinterpret_cast<const uint32_t *>(w + L.list_cnt);
+            auto first_pass = [&]() -> int {
+                RTP_TRY(side_stream(side2, 1));
+                if (cudaEventRecord(side2->fork, main) != cudaSuccess) return RTP_ERR_CUDA;
+                if (cudaStreamWaitEvent(side2->st, side2->fork, 0) != cudaSuccess) return RTP_ERR_CUDA;
+                Launcher l2{side2->st, ln.prof};
+                RTP_TRY(launch_list(l2, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out,
+                                    w, L, asc, LIST_FIRST, first));
+                if (cudaEventRecord(side2->join, side2->st) != cudaSuccess) return RTP_ERR_CUDA;
+                return RTP_OK;
+            };
+            rc = select_from_index(ln, dims, s, local_ctas, first_pass);
+            if (side2 && cudaStreamWaitEvent(main, side2->join, 0) != cudaSuccess && rc == RTP_OK) rc = RTP_ERR_CUDA;
+            if (rc == RTP_OK)
                 rc = launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out,
-                                 w, L, asc);
-                ln.pdl = false;
-            }
+                                 w, L, asc, LIST_REST, first);
         }
     }
     if (side && cudaStreamWaitEvent(main, side->join, 0) != cudaSuccess && rc == RTP_OK) rc = RTP_ERR_CUDA;

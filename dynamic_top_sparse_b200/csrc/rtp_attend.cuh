@@ -257,6 +257,15 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
 // ---------------------------------------------------------------------------
 // list attention
 // ---------------------------------------------------------------------------
+// The rows of a head may be attended in one pass (phase LIST_ALL) or in two
+// (the prefix of the list that the collect pass wrote -- rows clearly above
+// the boundary bin -- while the boundary is still being resolved, then the
+// rest): LIST_FIRST writes partials only; LIST_REST adds the remaining rows
+// and merges everything.  Partials live in per-head slots: the first pass
+// uses slots [0, it_first), the second [it_first, it_first + it_rest).
+enum ListPhase : int32_t { LIST_ALL = 0, LIST_FIRST = 1, LIST_REST = 2 };
+constexpr int LIST_SLOTS = 2 * LIST_MAX_SPLIT;   // partial slots per head
+
 struct ListArgs {
     int B, H_q, H_kv, G;
     long long N_max;
@@ -268,37 +277,47 @@ struct ListArgs {
     const void *k;
     const void *v;
     const int32_t *lists;        // [B*H_q*N_max]
-    const int32_t *counts;       // [B*H_q]
+    const int32_t *counts;       // [B*H_q] kept rows per head (read by LIST_ALL and LIST_REST)
+    const uint32_t *first;       // [B*H_q] rows of the collect pass (LIST_FIRST, LIST_REST), or null
+    int phase;
     float *out;
-    float *part;                 // [B*H_q*LIST_MAX_SPLIT][PSTRIDE] (indexed by item)
+    float *part;                 // [B*H_q][LIST_SLOTS][PSTRIDE]
     uint32_t *arrive;            // [B*H_q]
     uint32_t *status;
 };
 
-// One item = a slice of one head's kept rows.  Warp w takes rows
-// r0 + 16w .. r0 + 16w + 15, then every 128th: the 16 row ids come in one
-// load and all 16 rows' K and V loads are issued before the first dot
-// product.
+// Dynamic shared memory of list_attn_kernel: per head the item prefix, the
+// rows of this pass, the first row and the first partial slot; per sequence
+// its length.
+__host__ __device__ constexpr size_t list_smem_bytes(int nh, int B) {
+    return (size_t)(4 * nh + 1 + B) * sizeof(int);
+}
+
+// One item = a slice of one head's rows for this pass.  Warp w takes rows
+// r0 + 8w .. r0 + 8w + 7, then every 64th: the 8 row ids come in one load and
+// all 8 rows' K and V loads are issued before the first dot product.
 constexpr int MAX_LIST_B = 1024;        // sequences per call
 static_assert(65535 / MAX_GROUPS < MAX_LIST_B, "the argument checks must bound B below MAX_LIST_B");
 template <typename KT>
-__global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
-    __shared__ int pre[MAX_LIST_HEADS + 1];
-    __shared__ int s_cnt[MAX_LIST_HEADS];   // kept rows per head (0 when invalid)
-    __shared__ int s_len[MAX_LIST_B];       // sequence lengths
-    __shared__ int s_scan[ATT_THREADS];
+__global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
+    extern __shared__ int lsm[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nh = a.B * a.n_rq;
+    int *pre = lsm;                  // [nh + 1] item prefix
+    int *s_rows = pre + nh + 1;      // [nh] rows of this pass (0 when invalid)
+    int *s_row0 = s_rows + nh;       // [nh] first row of this pass in the head's list
+    int *s_slot0 = s_row0 + nh;      // [nh] first partial slot of this pass
+    int *s_len = s_slot0 + nh;       // [B] sequence lengths
+    __shared__ int s_scan[ATT_THREADS / 32];
     __shared__ float wm[ATT_THREADS / 32], wl[ATT_THREADS / 32];
     __shared__ float wo[ATT_THREADS / 32][D];
     __shared__ int s_last;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nh = a.B * a.n_rq;
     pdl_wait();
     pdl_trigger();
 
-    // items per head -> exclusive prefix, built by every CTA
+    // items per head -> exclusive prefix, built by every CTA: thread t owns
+    // heads [t * per, t * per + per), then a block-wide exclusive scan
     {
-        // thread t owns heads [t * per, t * per + per): item counts, then a
-        // block-wide exclusive scan (warp shuffles, one pass over warp totals)
         const int per = (nh + ATT_THREADS - 1) / ATT_THREADS;
         int loc = 0;
 #pragma unroll 4
@@ -307,12 +326,30 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
             int it = 0;
             if (hi < nh) {
                 const int b = hi / a.n_rq, h = a.ret_h[hi % a.n_rq];
-                const int cnt = __ldcg(a.counts + (size_t)b * a.H_q + h);
+                const size_t bh = (size_t)b * a.H_q + h;
                 const int N = a.seq_lens[b];
-                const bool ok = cnt >= 1 && N >= 1 && (long long)N <= a.N_max && cnt <= N;
-                if (ok) it = list_items(cnt);
+                const bool okN = N >= 1 && (long long)N <= a.N_max;
+                int rows = 0, row0 = 0, slot0 = 0;
+                if (a.phase == LIST_ALL) {
+                    const int cnt = __ldcg(a.counts + bh);
+                    if (okN && cnt >= 1 && cnt <= N) { rows = cnt; it = list_items(cnt); }
+                } else if (a.phase == LIST_FIRST) {
+                    const int nf = (int)__ldcg(a.first + bh);
+                    if (okN && nf >= 1 && nf <= N) { rows = nf; it = list_items(nf); }
+                } else {
+                    const int cnt = __ldcg(a.counts + bh);
+                    const int nf = (int)__ldcg(a.first + bh);
+                    if (okN && cnt >= 1 && cnt <= N && nf >= 0 && nf <= cnt) {
+                        row0 = nf;
+                        rows = cnt - nf;
+                        slot0 = list_items(nf);
+                        it = max(1, list_items(rows));       // at least one item: it merges the head
+                    }
+                }
                 pre[hi] = it;
-                s_cnt[hi] = ok ? cnt : 0;
+                s_rows[hi] = rows;
+                s_row0[hi] = row0;
+                s_slot0[hi] = slot0;
                 s_len[b] = N;
             }
             loc += it;
@@ -345,7 +382,7 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
     }
     const int total = pre[nh];
     // heads with nothing to attend over get zeros (and a status: invalid input)
-    if (blockIdx.x == 0) {
+    if (blockIdx.x == 0 && a.phase != LIST_FIRST) {
         for (int hi = warp; hi < nh; hi += ATT_THREADS / 32) {
             if (pre[hi + 1] != pre[hi]) continue;
             const int b = hi / a.n_rq, h = a.ret_h[hi % a.n_rq];
@@ -365,12 +402,15 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
         const int b = hix / a.n_rq, h = a.ret_h[hix % a.n_rq];
         const int g = h / a.G;
         const size_t bh = (size_t)b * a.H_q + h;
-        const int cnt = s_cnt[hix];
+        const int rows = s_rows[hix];
         const int N = s_len[b];
         const int nit = pre[hix + 1] - pre[hix];
         const int sub = item - pre[hix];
-        const int per_item = (cnt + nit - 1) / nit;
-        const int r0 = sub * per_item, r1 = min(cnt, r0 + per_item);
+        const int slot = s_slot0[hix] + sub;
+        const int nrec = s_slot0[hix] + nit;       // partials the merge of this head reads
+        const int per_item = (rows + nit - 1) / nit;
+        const int r0 = s_row0[hix] + sub * per_item;
+        const int r1 = s_row0[hix] + min(rows, sub * per_item + per_item);
 
         const float4 q4 = *reinterpret_cast<const float4 *>(a.q + bh * D + lane * 4);
         const float qx[4] = {q4.x * a.scale_log2, q4.y * a.scale_log2, q4.z * a.scale_log2,
@@ -379,10 +419,10 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
         const KT *vb = reinterpret_cast<const KT *>(a.v) + ((size_t)b * a.H_kv + g) * a.N_max * D;
         const int32_t *lst = a.lists + bh * a.N_max;
         float m = -INFINITY, l = 0.0f, o[4] = {0.f, 0.f, 0.f, 0.f};
-        constexpr int U = 16;      // rows per warp per pass: all their K/V loads in flight
+        constexpr int U = 8;       // rows per warp per pass: all their K/V loads in flight
         for (int rb = r0 + warp * U; rb < r1; rb += (ATT_THREADS / 32) * U) {
             int myid = -1;
-            if (lane < U && rb + lane < r1) myid = __ldg(lst + rb + lane);
+            if (lane < U && rb + lane < r1) myid = __ldcg(lst + rb + lane);
             float kx[U][4], vx[U][4];
             bool ok[U];
 #pragma unroll
@@ -430,7 +470,10 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) wo[warp][lane * 4 + i] = o[i];
         __syncthreads();
-        float *pp = a.part + ((size_t)item) * PSTRIDE;
+        float *hp = a.part + bh * (size_t)LIST_SLOTS * PSTRIDE;
+        float *pp = hp + (size_t)slot * PSTRIDE;
+        // a head attended by this one item only: normalise and write directly
+        const bool direct = a.phase != LIST_FIRST && nrec == 1;
         if (tid < D) {
             float M = -INFINITY;
             for (int w = 0; w < ATT_THREADS / 32; ++w) M = fmaxf(M, wm[w]);
@@ -442,15 +485,14 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
                     os = fmaf(wo[w][tid], wg, os);
                 }
             }
-            if (nit == 1) {
-                // the head's only item: normalise and write the output directly
+            if (direct) {
                 a.out[bh * D + tid] = os * (ls > 0.0f ? 1.0f / ls : 0.0f);
             } else {
                 pp[POFF + tid] = os;
                 if (tid == 0) { pp[0] = M; pp[1] = ls; }
             }
         }
-        if (nit == 1) {
+        if (direct || a.phase == LIST_FIRST) {
             __syncthreads();
             continue;
         }
@@ -460,7 +502,7 @@ __global__ void __launch_bounds__(ATT_THREADS) list_attn_kernel(ListArgs a) {
         __syncthreads();
         if (s_last) {
             __threadfence();
-            merge_partials(a.part + (size_t)pre[hix] * PSTRIDE, nit, PSTRIDE, 1, a.out + bh * D);
+            merge_partials(hp, nrec, PSTRIDE, 1, a.out + bh * D);
             if (tid == 0) a.arrive[bh] = 0;
         }
         __syncthreads();

@@ -28,19 +28,20 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 // 8 consecutive elements starting at element `i` of a row (16-byte aligned
-// for bf16, two 16-byte loads for fp32).
+// for bf16, two 16-byte loads for fp32).  Cache rows are read once per use:
+// loads are cached in L2 only.
 template <typename T> struct Row;
 
 template <> struct Row<__nv_bfloat16> {
     static __device__ __forceinline__ void load8(const __nv_bfloat16 *p, float (&x)[8]) {
-        uint4 u = __ldg(reinterpret_cast<const uint4 *>(p));
+        uint4 u = __ldcg(reinterpret_cast<const uint4 *>(p));
         x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x);
         x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
         x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z);
         x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
     }
     static __device__ __forceinline__ void load4(const __nv_bfloat16 *p, float (&x)[4]) {
-        uint2 u = __ldg(reinterpret_cast<const uint2 *>(p));
+        uint2 u = __ldcg(reinterpret_cast<const uint2 *>(p));
         x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x);
         x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
     }
@@ -49,13 +50,13 @@ template <> struct Row<__nv_bfloat16> {
 
 template <> struct Row<float> {
     static __device__ __forceinline__ void load8(const float *p, float (&x)[8]) {
-        float4 a = __ldg(reinterpret_cast<const float4 *>(p));
-        float4 b = __ldg(reinterpret_cast<const float4 *>(p) + 1);
+        float4 a = __ldcg(reinterpret_cast<const float4 *>(p));
+        float4 b = __ldcg(reinterpret_cast<const float4 *>(p) + 1);
         x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
         x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
     }
     static __device__ __forceinline__ void load4(const float *p, float (&x)[4]) {
-        float4 a = __ldg(reinterpret_cast<const float4 *>(p));
+        float4 a = __ldcg(reinterpret_cast<const float4 *>(p));
         x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
     }
     static __device__ __forceinline__ float from_float(float v) { return v; }
@@ -141,12 +142,6 @@ __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t by
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
-// Bring `bytes` (a multiple of 16, 16-byte aligned) at `p` into L2 without
-// waiting for it (warms the translation and the cache for a later gather).
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 // ---------------------------------------------------------------------------
 // warp helpers
 // ---------------------------------------------------------------------------
@@ -168,7 +163,7 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 
 // List attention splits a head's kept rows into items of about LCH rows,
 // at most LIST_MAX_SPLIT per head.
-constexpr int LCH = 128;
+constexpr int LCH = 64;
 constexpr int LIST_MAX_SPLIT = 64;
 __device__ __forceinline__ int list_items(int count) {
     if (count <= 0) return 0;

@@ -169,19 +169,7 @@ struct SelArgs {
     int32_t *lists;              // [B*H_q][N_max] kept ids
     int32_t *count_out;          // [B*H_q]
     float *mass_out;             // [B*H_q] or null
-    // K/V caches ([B, H_kv, N_max, D] rows of kv_row_bytes) whose kept rows
-    // are prefetched into L2 as soon as they are known, or null
-    const uint8_t *k_rows, *v_rows;
-    int kv_row_bytes;
 };
-
-// Prefetch the K and V rows of token t of group (b, g) into L2.
-__device__ __forceinline__ void prefetch_kv(const SelArgs &a, size_t bg, int t) {
-    if (!a.k_rows) return;
-    const size_t off = (bg * (size_t)a.N_max + (size_t)t) * (size_t)a.kv_row_bytes;
-    prefetch_l2(a.k_rows + off, (uint32_t)a.kv_row_bytes);
-    prefetch_l2(a.v_rows + off, (uint32_t)a.kv_row_bytes);
-}
 
 __device__ __forceinline__ int valid_len(const int32_t *seq_lens, int b, long long N_max,
                                          uint32_t *status) {
@@ -1105,7 +1093,6 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
                     const int h = src.head(src.slot(v));
                     const int t = tb + src.tok(v);
                     if (kept) {
-                        prefetch_kv(a, bg, t);
                         const unsigned p = atomicAdd(&s_kc[h], 1u);
                         if (p < (unsigned)KCAP) {
                             s_kbuf[h * KCAP + p] = t;
@@ -1339,9 +1326,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             if (lane == 0 && bal) wbase = atomicAdd(&s_base, (unsigned)__popc(bal));
             wbase = __shfl_sync(0xffffffffu, wbase, 0);
             if (k) {
-                const int t = (int)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
-                prefetch_kv(a, (size_t)b * a.H_kv + (size_t)(h / G), t);
-                lst[base0 + wbase + __popc(bal & lt)] = t;
+                lst[base0 + wbase + __popc(bal & lt)] = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
                 kept += staged ? fbuf[c] : fx_of(v);
             }
         }
