@@ -1,7 +1,7 @@
 """Benchmark of the sparse decode step (one layer's append + decode per
 step; 48 layers per step for the 48-layer workload) on synthetic caches.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config 3] [--p P]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ctx512k] [--p P]
     python bench.py --impl reference ...   # the CPU oracle, timed on host cores
 
 Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) are independent
@@ -163,8 +163,8 @@ class Layer:
         return other
 
 
-def build_workload(cfg: int, seed: int = 0):
-    spec = synth.spec_for(cfg)
+def build_workload(key: str, seed: int = 0):
+    spec = synth.spec_for(key)
     layers = []
     for l in range(spec.layers):
         c = synth.make_case(spec, device="cuda", seed=seed, layer=l)
@@ -215,7 +215,7 @@ def index_bytes(spec, layers):
 # ------------------------------------------------------------------ our arm
 
 def run_ours(args, rank, world, dev):
-    spec, layers0 = build_workload(args.config)
+    spec, layers0 = build_workload(args.workload)
     if args.p is not None:
         spec.p = args.p
     p = spec.p
@@ -415,7 +415,7 @@ def run_ours(args, rank, world, dev):
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": workload, "cfg": args.config, "B": spec.B, "ctx": spec.N, "H_q": spec.H_q,
+        "config": {"workload": workload, "key": args.workload, "B": spec.B, "ctx": spec.N, "H_q": spec.H_q,
                    "H_kv": spec.H_kv, "d": spec.d, "r": spec.r, "layers": spec.layers, "p": p,
                    "window": spec.window, "n_sink": spec.n_sink, "cache_dtype": spec.kv_dtype,
                    "index_dtype": spec.idx_dtype, "accumulate": "f32",
@@ -447,13 +447,13 @@ def run_ours(args, rank, world, dev):
         "pages_context": {"decode_speedup_1M_H20": 2.01, "prefill_speedup_1M_H20": 9.36},
     }
     if rank == 0 and world == 1 and not args.no_cpu:
-        res["cpu_baseline"] = cpu_baseline(args.config, spec, args.cpu_seconds)
+        res["cpu_baseline"] = cpu_baseline(args.workload, spec, args.cpu_seconds)
     return res
 
 
 # ------------------------------------------------------------------ oracle arm
 
-def cpu_baseline(cfg, spec=None, budget_s=15.0):
+def cpu_baseline(key, spec=None, budget_s=15.0):
     """The oracle, as it stands, on host cores over a bounded sample of the
     workload (whole layers of one replica); steps/s scaled to full steps."""
     import oracle
@@ -462,7 +462,7 @@ def cpu_baseline(cfg, spec=None, budget_s=15.0):
         lim = threadpool_limits(limits=1)
     except Exception:
         lim = None
-    spec = spec or synth.spec_for(cfg)
+    spec = spec or synth.spec_for(key)
     layers_done, t_tot = 0, 0.0
     seqs = list(range(spec.B))
     # layers are taken in turn (again from the first when the step has fewer
@@ -507,15 +507,15 @@ def cpu_baseline(cfg, spec=None, budget_s=15.0):
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    spec = synth.spec_for(args.config)
+    spec = synth.spec_for(args.workload)
     if args.p is not None:
         spec.p = args.p
-    cb = cpu_baseline(args.config, spec, args.cpu_seconds)
+    cb = cpu_baseline(args.workload, spec, args.cpu_seconds)
     v = cb["value"]
     return {"impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": spec.name, "cfg": args.config, "B": spec.B, "ctx": spec.N, "p": spec.p},
+            "config": {"workload": spec.name, "key": args.workload, "B": spec.B, "ctx": spec.N, "p": spec.p},
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "note": "the CPU oracle (numpy fp64), timed on host cores over a bounded sample"}
@@ -541,7 +541,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=50)
-    ap.add_argument("--config", type=int, default=3, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", default="ctx512k", choices=list(synth.WORKLOADS))
     ap.add_argument("--p", type=float, default=None)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")

@@ -68,7 +68,7 @@ class Spec:
     rope: bool = True
     # head_class per layer: list of lists of length H_kv
     head_class: list = field(default_factory=list)
-    # needle recipe: "cfg1", "uniform", "ranked" or "none"
+    # needle recipe: "direction", "uniform", "ranked" or "none"
     needles: str = "uniform"
     needles_per_head: int = 4
     needle_scale: float = 3.0
@@ -76,33 +76,38 @@ class Spec:
     N_max: int | None = None
 
 
-def spec_for(cfg: int) -> Spec:
-    if cfg == 1:
-        return Spec("cfg1: 4096 ctx, B1, 4q/1kv, fp32, all retrieval, p=0.9",
+# The workloads, by key: the shapes of the pages' 64K-1M decode settings plus
+# a small fp32 case that the oracle finishes in seconds.
+WORKLOADS = ("ctx4k-fp32", "ctx64k", "ctx512k", "ctx128k-b8-48layer", "ctx1m")
+
+
+def spec_for(key: str) -> Spec:
+    if key == "ctx4k-fp32":
+        return Spec("4K ctx, B1, 4q/1kv, fp32, all retrieval, 8 planted needles, p=0.9",
                     B=1, H_q=4, H_kv=1, N=4096, kv_dtype="f32", idx_dtype="f32",
-                    rope=False, head_class=[[1]], needles="cfg1", window=4096, n_sink=4)
-    if cfg == 2:
-        return Spec("cfg2: 64K ctx, B1, 32q/4kv, bf16, KV0 retrieval + 3 local (w4096+4 sinks), p=0.9",
+                    rope=False, head_class=[[1]], needles="direction", window=4096, n_sink=4)
+    if key == "ctx64k":
+        return Spec("64K ctx, B1, 32q/4kv, bf16, KV0 retrieval + 3 local (w4096+4 sinks), p=0.9",
                     B=1, H_q=32, H_kv=4, N=65536, head_class=[[1, 0, 0, 0]],
                     needles="uniform", needles_per_head=4, needle_scale=3.0)
-    if cfg == 3:
-        return Spec("cfg3: 512K ctx, B1, 32q/4kv, bf16, KV0+KV2 retrieval, ranked needles, p=0.9",
+    if key == "ctx512k":
+        return Spec("512K ctx, B1, 32q/4kv, bf16, KV0+KV2 retrieval, ranked needles, p=0.9",
                     B=1, H_q=32, H_kv=4, N=524288, head_class=[[1, 0, 1, 0]],
                     needles="ranked")
-    if cfg == 4:
-        return Spec("cfg4: 48 layers, B8, 128K ctx, 32q/4kv, bf16, 1 retrieval KV head/layer, p=0.9",
+    if key == "ctx128k-b8-48layer":
+        return Spec("48 layers, B8, 128K ctx, 32q/4kv, bf16, 1 retrieval KV head/layer, p=0.9",
                     B=8, H_q=32, H_kv=4, N=131072, layers=48, head_class=[],
                     needles="uniform", needles_per_head=4, needle_scale=3.0)
-    if cfg == 5:
-        return Spec("cfg5: 1M ctx, B1, 32q/4kv, bf16, all retrieval, ranked needles",
+    if key == "ctx1m":
+        return Spec("1M ctx, B1, 32q/4kv, bf16, all retrieval, ranked needles",
                     B=1, H_q=32, H_kv=4, N=1048576, head_class=[[1, 1, 1, 1]],
                     needles="ranked")
-    raise ValueError(cfg)
+    raise ValueError(f"unknown workload {key!r}; one of {WORKLOADS}")
 
 
 def layer_head_class(spec: Spec, layer: int, seed: int) -> np.ndarray:
-    """Head classes of one layer; config 4 picks its one retrieval KV head
-    per layer with a seeded uniform draw."""
+    """Head classes of one layer; the 48-layer workload picks its one
+    retrieval KV head per layer with a seeded uniform draw."""
     if spec.head_class:
         hc = spec.head_class[layer % len(spec.head_class)]
         return np.asarray(hc, dtype=np.uint8)
@@ -144,7 +149,7 @@ class Case:
     window: int
     n_sink: int
     needles: dict                # (b, h) -> np.ndarray of needle positions
-    k_pre_all: torch.Tensor | None = None  # cfg1: pre-RoPE keys of every row (index keys come from the append step)
+    k_pre_all: torch.Tensor | None = None  # ctx4k-fp32: pre-RoPE keys of every row (index keys come from the append step)
 
     @property
     def B(self):
@@ -192,11 +197,11 @@ def _needle_plan(spec: Spec, head_class: np.ndarray, N: int):
     return plan
 
 
-def make_case(spec: Spec | int, device="cpu", seed: int = 0, layer: int = 0) -> Case:
+def make_case(spec: Spec | str, device="cpu", seed: int = 0, layer: int = 0) -> Case:
     """Build one layer of synthetic decode-step inputs, seeded by
-    (seed, config name, layer).  Large cases should be built with
+    (seed, workload name, layer).  Large cases should be built with
     device='cuda' (torch's CUDA generator is deterministic for a seed)."""
-    if isinstance(spec, int):
+    if isinstance(spec, str):
         spec = spec_for(spec)
     dev = torch.device(device)
     B, H_q, H_kv, d, r, N = spec.B, spec.H_q, spec.H_kv, spec.d, spec.r, spec.N
@@ -218,7 +223,7 @@ def make_case(spec: Spec | int, device="cpu", seed: int = 0, layer: int = 0) -> 
     k_pre_new = _randn((B, H_kv, 1, d), cpu_gen, "cpu").to(kvdt)
     needles: dict = {}
 
-    if spec.needles == "cfg1":
+    if spec.needles == "direction":
         # q, k, v ~ N(0,1); one 16x128 query projector shared by the group's
         # heads; 8 needle keys k = 3*q_dir + N(0, 0.3^2), needle i for head i mod G.
         W1 = _randn((r, d), cpu_gen, "cpu", std=1.0 / math.sqrt(d))
@@ -243,7 +248,7 @@ def make_case(spec: Spec | int, device="cpu", seed: int = 0, layer: int = 0) -> 
                     k_pre_all=k_pre.to(kvdt).to(dev))
         return case
 
-    # --- configs 2-5 and generic cases: needles planted in index space -----
+    # --- the bf16 workloads and generic cases: needles planted in index space
     W_q_idx = _randn((H_q, r, d), cpu_gen, "cpu", std=1.0 / math.sqrt(d)).to(torch.float64)
     qi = torch.randn((B, H_q, r), generator=cpu_gen, dtype=torch.float64)
     noise = torch.randn((B, H_q, d), generator=cpu_gen, dtype=torch.float64)

@@ -127,7 +127,7 @@ def oracle_inputs(gc: GpuCase, kidx_override=None):
 
 
 def oracle_kidx(gc: GpuCase, idx_dtype: str, with_current: bool):
-    """The oracle's own index-key cache: cfg1 builds every row with its
+    """The oracle's own index-key cache: the 4K fp32 workload builds every row with its
     append; with_current appends the current token's key at N_b - 1."""
     c = gc.c
     if c.k_pre_all is not None:

@@ -108,8 +108,8 @@ def test_step_repeatable_on_one_workspace():
 
 # --------------------------------------------------------------- workloads
 
-def _workload(cfg, ps, sample_heads=None, layer=0):
-    c = synth.make_case(cfg, device="cuda", layer=layer)
+def _workload(key, ps, sample_heads=None, layer=0):
+    c = synth.make_case(key, device="cuda", layer=layer)
     gc = GpuCase(c)
     gc.append_current()
     res = {}
@@ -120,35 +120,35 @@ def _workload(cfg, ps, sample_heads=None, layer=0):
     return res
 
 
-def test_cfg1_4096_fp32():
-    _workload(1, [0.9])
+def test_ctx4k_fp32():
+    _workload("ctx4k-fp32", [0.9])
 
 
 @pytest.mark.slow
-def test_cfg2_64k():
-    _workload(2, [0.9])
+def test_ctx64k():
+    _workload("ctx64k", [0.9])
 
 
 @pytest.mark.slow
-def test_cfg3_512k():
-    _workload(3, [0.9])
+def test_ctx512k():
+    _workload("ctx512k", [0.9])
 
 
 @pytest.mark.slow
-def test_cfg5_1m_p_sweep():
+def test_ctx1m_p_sweep():
     # p = 0.9: every head; the other p: four heads per KV group (peaked to
     # broad) plus the dense p = 1.0 case on a sample.
     def sample(p):
         if p == 0.9:
             return None
         return [(0, h) for h in (0, 5, 9, 14, 18, 22, 27, 31)]
-    _workload(5, [0.8, 0.9, 0.95, 1.0], sample_heads=sample)
+    _workload("ctx1m", [0.8, 0.9, 0.95, 1.0], sample_heads=sample)
 
 
 @pytest.mark.slow
-def test_cfg4_128k_b8_sampled_layers():
-    # config 4 runs 48 layers x 8 sequences; the oracle checks two layers
+def test_ctx128k_b8_sampled_layers():
+    # the 48-layer workload runs 48 layers x 8 sequences; the oracle checks two layers
     # fully (all 8 sequences, all heads) and the launch shape is the same
     # for every layer.
     for layer in (0, 29):
-        _workload(4, [0.9], layer=layer)
+        _workload("ctx128k-b8-48layer", [0.9], layer=layer)
