@@ -34,11 +34,13 @@ struct Layout {
     size_t end_range;       // local / dense
     size_t part_list;
     size_t end_list;        // sparse decode
-    size_t tilebin, lists, cands;
+    size_t tilebin, lists, cands, part_sel, ovf, rest0;
     size_t total;           // topp_select / decode_step
 };
 
 constexpr int SCAN_CTAS_MAX = 1024;
+
+int num_sms();
 
 Layout make_layout(const rtp_dims *d) {
     Layout L{};
@@ -63,6 +65,12 @@ Layout make_layout(const rtp_dims *d) {
     L.tilebin = o; o = align_up(o + BHkv * ntile * GMAX * 2, 256);
     L.lists = o; o = align_up(o + BHq * (size_t)d->N_max * 4, 256);
     L.cands = o; o = align_up(o + BHq * (size_t)d->N_max * 8, 256);
+    // one record per collect CTA and head slot: the bf16 selection grid has
+    // max(1, SMs / groups) CTAs per (b, g), at most max(SMs, B * H_kv) in all,
+    // and the collect grid twice as many
+    L.part_sel = o; o = align_up(o + 2 * std::max((size_t)num_sms(), BHkv) * GMAX * PSTRIDE * 4, 256);
+    L.ovf = o; o = align_up(o + BHq * 4, 256);
+    L.rest0 = o; o = align_up(o + BHq * 4, 256);
     L.total = o;
     return L;
 }
@@ -256,7 +264,9 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sm
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
     if (!attr_set[dev]) {
         if (cudaFuncSetAttribute(scan_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM) !=
-            cudaSuccess)
+                cudaSuccess ||
+            cudaFuncSetAttribute(collect_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CL_SMEM) !=
+                cudaSuccess)
             return RTP_ERR_CUDA;
         attr_set[dev] = 1;
     }
@@ -266,14 +276,19 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sm
     long long ctas = std::max(1LL, std::min(sms / std::max(groups, 1LL), tiles));
     s.a.chunk = (tiles + ctas - 1) / ctas * TILE;
     s.a.ctas = (int)((d->N_max + s.a.chunk - 1) / s.a.chunk);
+    // collect: one CTA per SM, the scan's ranges
+    const long long cl = s.a.ctas;
+    s.a.cl_chunk = (tiles + cl - 1) / cl * TILE;
+    s.a.cl_ctas = (int)((d->N_max + s.a.cl_chunk - 1) / s.a.cl_chunk);
     const dim3 grid((unsigned)s.a.ctas, (unsigned)groups);
+    const dim3 cl_grid((unsigned)s.a.cl_ctas, (unsigned)groups);
     // scan, collect and finalize wait on the device for their predecessor
     // (programmatic dependent launch), so each one's launch overlaps the
     // previous kernel's tail
     const bool pdl0 = ln.pdl;
     ln.pdl = true;
     int rc = ln.run_smem("hist", scan_tma_kernel, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w);
-    if (rc == RTP_OK) rc = ln.run("collect", collect_mma_kernel, grid, dim3(CL_THREADS), s.a, s.w);
+    if (rc == RTP_OK) rc = ln.run_smem("collect", collect_mma_kernel, cl_grid, dim3(CL_THREADS), CL_SMEM, s.a, s.w);
     if (rc == RTP_OK && after_collect) rc = after_collect();
     if (rc == RTP_OK)
         rc = ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)), dim3(FIN_THREADS),
@@ -346,7 +361,7 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
 int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
                 const int32_t *lists, const int32_t *counts, const uint8_t *hc, float *out,
                 char *ws, const Layout &L, float attn_scale, int phase = LIST_ALL,
-                const uint32_t *first = nullptr) {
+                const int32_t *first = nullptr) {
     static int attr_set[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
@@ -691,11 +706,36 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
             s.a.lists = opts && opts->sel_idx ? opts->sel_idx : reinterpret_cast<int32_t *>(w + L.lists);
             s.a.count_out = opts && opts->sel_count ? opts->sel_count : reinterpret_cast<int32_t *>(w + L.counts);
             s.a.mass_out = opts ? opts->sel_mass : nullptr;
+            const bool fused = dims->kv_dtype == RTP_BF16 && dims->idx_dtype == RTP_BF16;
+            if (fused) {
+                // the sparse attention runs inside collect and finalize
+                s.a.q_rope = q_rope;
+                s.a.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
+                s.a.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
+                s.a.attn_scale_log2 = asc * 1.4426950408889634f;
+                s.a.out = out;
+                s.a.part_sel = reinterpret_cast<float *>(w + L.part_sel);
+                s.a.ovf = reinterpret_cast<uint32_t *>(w + L.ovf);
+                s.a.part_list = reinterpret_cast<float *>(w + L.part_list);
+                s.a.rest0 = reinterpret_cast<int32_t *>(w + L.rest0);
+                rc = select_from_index(ln, dims, s, local_ctas);
+                if (rc == RTP_OK) {
+                    // the kept rows the selection left (the boundary bin's), merged
+                    // with the selection's partial
+                    ln.pdl = true;                      // follows finalize_kernel
+                    rc = launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class,
+                                     out, w, L, asc, LIST_TAIL, s.a.rest0);
+                    ln.pdl = false;
+                }
+                if (side && cudaStreamWaitEvent(main, side->join, 0) != cudaSuccess && rc == RTP_OK)
+                    rc = RTP_ERR_CUDA;
+                return rc;
+            }
             // The rows the collect pass kept (clearly above the boundary bin)
             // are attended on a side stream while finalize resolves the
             // boundary bin; the rest and the merge follow finalize.
             Side *side2 = nullptr;
-            const uint32_t *first = reinterpret_cast<const uint32_t *>(w + L.list_cnt);
+            const int32_t *first = reinterpret_cast<const int32_t *>(w + L.list_cnt);
             auto first_pass = [&]() -> int {
                 RTP_TRY(side_stream(side2, 1));
                 if (cudaEventRecord(side2->fork, main) != cudaSuccess) return RTP_ERR_CUDA;

@@ -165,10 +165,17 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 // at most LIST_MAX_SPLIT per head.
 constexpr int LCH = 64;
 constexpr int LIST_MAX_SPLIT = 64;
+constexpr int LIST_SLOTS = 2 * LIST_MAX_SPLIT;   // partial record slots per head
 __device__ __forceinline__ int list_items(int count) {
     if (count <= 0) return 0;
     return min(LIST_MAX_SPLIT, (count + LCH - 1) / LCH);
 }
+
+// Flash-decoding partial record of one head over a set of rows (log2
+// units): m = running max, l = sum of 2^(s - m), o[D] = unnormalised output.
+constexpr int PSTRIDE = D + 4;         // partial record: m, l, (2 unused), o[D]
+constexpr int POFF = 4;                // offset of o[] in a record (16-byte aligned)
+static_assert(PSTRIDE % 4 == 0 && POFF % 4 == 0, "partial records must keep o[] 16-byte aligned");
 
 // Flash-decoding partial of one head over a set of rows.
 struct Partial {

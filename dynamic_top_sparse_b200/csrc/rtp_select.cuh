@@ -157,6 +157,8 @@ struct SelArgs {
     int ntile;
     int ctas;                    // scan/collect CTAs per (b, g)
     long long chunk;             // tokens per CTA, multiple of TILE
+    int cl_ctas;                 // collect_mma_kernel CTAs per (b, g)
+    long long cl_chunk;          // its tokens per CTA, multiple of TILE
     const int32_t *seq_lens;
     int n_ret;
     int ret_g[MAX_RET_GROUPS];
@@ -169,7 +171,105 @@ struct SelArgs {
     int32_t *lists;              // [B*H_q][N_max] kept ids
     int32_t *count_out;          // [B*H_q]
     float *mass_out;             // [B*H_q] or null
+    // Fused sparse attention of a decode step (bf16 caches); q_rope null = off.
+    // Every collect CTA attends the rows it kept and writes one partial per
+    // head of its group; finalize attends the boundary bin's kept rows and
+    // merges.  A head whose kept rows overflowed a CTA's staging is attended
+    // wholly by finalize (ovf flag).
+    const float *q_rope;                 // [B, H_q, D]
+    const __nv_bfloat16 *k_cache;        // [B, H_kv, N_max, D]
+    const __nv_bfloat16 *v_cache;
+    float attn_scale_log2;
+    float *out;                          // [B, H_q, D]
+    float *part_sel;                     // [collect CTAs][GMAX][PSTRIDE]
+    uint32_t *ovf;                       // [B*H_q]
+    float *part_list;                    // [B*H_q][LIST_SLOTS][PSTRIDE]: slot 0 = collect partials merged
+    int32_t *rest0;                      // [B*H_q] first list row left to the list pass
 };
+
+// ---------------------------------------------------------------------------
+// fused sparse attention helpers
+// ---------------------------------------------------------------------------
+// Running flash-decoding partial of one head held by one warp (log2 units);
+// lane l holds dims 4l .. 4l + 3 of o.
+struct WarpPart {
+    float m, l, o[4];
+    __device__ __forceinline__ void reset() {
+        m = -INFINITY; l = 0.0f;
+        o[0] = o[1] = o[2] = o[3] = 0.0f;
+    }
+    // fold in another partial (mx, lx, ox) of the same head
+    __device__ __forceinline__ void add(float mx, float lx, const float (&ox)[4]) {
+        if (mx == -INFINITY) return;
+        const float mn = fmaxf(m, mx);
+        const float a0 = m == -INFINITY ? 0.0f : exp2f(m - mn), a1 = exp2f(mx - mn);
+        l = l * a0 + lx * a1;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) o[i] = o[i] * a0 + ox[i] * a1;
+        m = mn;
+    }
+    // write as a record (m, l at [0], [1]; o at [POFF + 4 lane ..])
+    __device__ __forceinline__ void store(float *rec) const {
+        const int lane = threadIdx.x & 31;
+        if (lane == 0) { rec[0] = m; rec[1] = l; }
+        *reinterpret_cast<float4 *>(rec + POFF + 4 * lane) = make_float4(o[0], o[1], o[2], o[3]);
+    }
+    __device__ __forceinline__ void load_add(const float *rec) {
+        const int lane = threadIdx.x & 31;
+        const float mx = rec[0], lx = rec[1];
+        const float4 v = *reinterpret_cast<const float4 *>(rec + POFF + 4 * lane);
+        const float ox[4] = {v.x, v.y, v.z, v.w};
+        add(mx, lx, ox);
+    }
+};
+
+// The warp attends up to 8 rows of one head: lane u < 8 holds row id `id`
+// (-1: none), all 16 row loads in flight before the dot products.  qx: the
+// lane's 4 query dims times the softmax scale times log2(e).
+__device__ __forceinline__ void attend8(const __nv_bfloat16 *kb, const __nv_bfloat16 *vb, int id,
+                                        const float (&qx)[4], WarpPart &p) {
+    const int lane = threadIdx.x & 31;
+    float kx[8][4], vx[8][4];
+    bool ok[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int t = __shfl_sync(0xffffffffu, id, u);
+        ok[u] = t >= 0;
+        if (ok[u]) {
+            Row<__nv_bfloat16>::load4(kb + (size_t)t * D + lane * 4, kx[u]);
+            Row<__nv_bfloat16>::load4(vb + (size_t)t * D + lane * 4, vx[u]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) kx[u][i] = vx[u][i] = 0.0f;
+        }
+    }
+    float sc[8];
+    float mb = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        float sv = qx[0] * kx[u][0];
+        sv = fmaf(qx[1], kx[u][1], sv);
+        sv = fmaf(qx[2], kx[u][2], sv);
+        sv = fmaf(qx[3], kx[u][3], sv);
+        sv = warp_sum(sv);
+        sc[u] = ok[u] ? sv : -INFINITY;
+        mb = fmaxf(mb, sc[u]);
+    }
+    const float mn = fmaxf(p.m, mb);
+    if (mn == -INFINITY) return;
+    const float al = exp2f(p.m - mn);
+    p.l *= al;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) p.o[i] *= al;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const float pw = exp2f(sc[u] - mn);
+        p.l += pw;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) p.o[i] = fmaf(pw, vx[u][i], p.o[i]);
+    }
+    p.m = mn;
+}
 
 __device__ __forceinline__ int valid_len(const int32_t *seq_lens, int b, long long N_max,
                                          uint32_t *status) {
@@ -514,7 +614,11 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(SelArgs a, SelWs w) 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) s_err = 0;
     // this call's collect pass appends from zero
-    if (blockIdx.x == 0 && threadIdx.x < G) { w.cand_cnt[bh0 + threadIdx.x] = 0u; w.list_cnt[bh0 + threadIdx.x] = 0u; }
+    if (blockIdx.x == 0 && threadIdx.x < G) {
+        w.cand_cnt[bh0 + threadIdx.x] = 0u;
+        w.list_cnt[bh0 + threadIdx.x] = 0u;
+        if (a.ovf) a.ovf[bh0 + threadIdx.x] = 0u;
+    }
     for (int i = threadIdx.x; i < 2 * GMAX * NBIN; i += blockDim.x) shl[i] = 0u;
     if constexpr (NeedsQ<Src>::value) {
         project_query<(GMAX * R + SCAN_WARPS - 1) / SCAN_WARPS>(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D,
@@ -694,7 +798,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
     pdl_wait();
     pdl_trigger();
     // this call's collect pass appends from zero
-    if (blockIdx.x == 0 && threadIdx.x < G) { w.cand_cnt[bh0 + threadIdx.x] = 0u; w.list_cnt[bh0 + threadIdx.x] = 0u; }
+    if (blockIdx.x == 0 && threadIdx.x < G) {
+        w.cand_cnt[bh0 + threadIdx.x] = 0u;
+        w.list_cnt[bh0 + threadIdx.x] = 0u;
+        if (a.ovf) a.ovf[bh0 + threadIdx.x] = 0u;
+    }
     // the consumers' q_idx loads go out before the producer's first bulk copy
     QProj<(GMAX * R + TC_WARPS - 1) / TC_WARPS> qp;
     if (warp < TC_WARPS) qp.load(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, G, warp, TC_WARPS);
@@ -973,13 +1081,22 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
 constexpr int CL_WARPS = 16;
 constexpr int CL_THREADS = CL_WARPS * 32;
 constexpr int CL_BATCH = 4;
+constexpr int CL_KCAP = 1024;     // kept ids staged per head per CTA
+static_assert(GMAX * D % CL_THREADS == 0 && GMAX * R <= CL_THREADS && CL_WARPS >= GMAX,
+              "collect prologue: load split, one resolving warp per head slot");
+// dynamic shared memory: staged kept ids, scaled q_rope of the group, and one
+// partial record per (warp, head) for the fused attention
+constexpr int CL_SMEM = GMAX * CL_KCAP * 4 + GMAX * D * 4 + CL_WARPS * GMAX * PSTRIDE * 4;
 
 __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, SelWs w) {
+    extern __shared__ __align__(16) uint8_t csm[];
+    int32_t *s_kbuf = reinterpret_cast<int32_t *>(csm);                       // [GMAX][CL_KCAP]
+    float *s_qr = reinterpret_cast<float *>(csm + GMAX * CL_KCAP * 4);         // [GMAX][D]
+    float *s_slot = s_qr + GMAX * D;                                            // [CL_WARPS][GMAX][PSTRIDE]
     __shared__ __align__(16) float qs[GMAX * R];
     __shared__ int s_bstar[GMAX];
     __shared__ unsigned s_kc[GMAX], s_cc[GMAX];
     __shared__ float s_khi[GMAX], s_clo[GMAX];      // keep: z > s_khi; candidate: s_clo <= z <= s_khi
-    __shared__ int32_t s_kbuf[GMAX * KCAP];
     __shared__ unsigned long long s_cbuf[GMAX * CCAP];
     const int b = blockIdx.y / a.n_ret;
     const int g = a.ret_g[blockIdx.y % a.n_ret];
@@ -991,15 +1108,25 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
     pdl_wait();
     pdl_trigger();
     const int N = valid_len(a.seq_lens, b, a.N_max, w.status);
-    const int t_lo = (int)((long long)blockIdx.x * a.chunk);
-    const int t_hi = (int)min((long long)N, (long long)t_lo + a.chunk);
+    const int t_lo = (int)((long long)blockIdx.x * a.cl_chunk);
+    const int t_hi = (int)min((long long)N, (long long)t_lo + a.cl_chunk);
     const uint4 *recs = reinterpret_cast<const uint4 *>(w.tilebin + bg * a.ntile * GMAX);
     // tile of lane `lane` in window `win` of this warp
     auto tile_of = [&](int win) { return t_lo / TILE + warp + (win * 32 + lane) * CL_WARPS; };
     const int ti_end = (t_hi + TILE - 1) / TILE;
     uint4 rec = make_uint4(0u, 0u, 0u, 0u);
     if (t_hi > t_lo && tile_of(0) < ti_end) rec = __ldcg(recs + tile_of(0));
-    if (warp < GMAX) {
+    // q_idx and (fused attention) the scaled q_rope of the group: loads first,
+    // stored to shared memory after the resolve
+    constexpr int QR_PER = GMAX * D / CL_THREADS;
+    const float qv = threadIdx.x < G * R ? w.qidx[bh0 * R + threadIdx.x] : 0.0f;
+    float qrv[QR_PER];
+#pragma unroll
+    for (int k = 0; k < QR_PER; ++k) {
+        const int i = threadIdx.x + k * CL_THREADS;
+        qrv[k] = a.q_rope && i < G * D ? a.q_rope[bh0 * D + i] : 0.0f;
+    }
+    {
         int bs = NBIN, mode = MODE_EMPTY;
         if (warp < G) {
             const Resolve r = resolve_head(w.hist + (bh0 + warp) * NBIN, a.p, N);
@@ -1007,17 +1134,31 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
             mode = r.mode;
             bs = r.bstar;
         }
-        if (lane == 0) {
+        if (lane == 0 && warp < GMAX) {
             // keep-all heads need no collect pass: finalize lists every token
             s_bstar[warp] = mode == MODE_NORMAL ? bs : NBIN;
             s_khi[warp] = mode == MODE_NORMAL ? bin_hi_incl(bs) : INFINITY;
             s_clo[warp] = mode == MODE_NORMAL ? bin_lo_incl(bs) : INFINITY;
         }
-    } else {
-        for (int i = threadIdx.x - GMAX * 32; i < G * R; i += (CL_WARPS - GMAX) * 32) qs[i] = w.qidx[bh0 * R + i];
+    }
+    if (threadIdx.x < G * R) qs[threadIdx.x] = qv;
+#pragma unroll
+    for (int k = 0; k < QR_PER; ++k) {
+        const int i = threadIdx.x + k * CL_THREADS;
+        if (i < G * D) s_qr[i] = qrv[k] * a.attn_scale_log2;
     }
     __syncthreads();
-    if (t_hi <= t_lo) return;
+    if (t_hi <= t_lo) {
+        // an empty range: empty partials for the fused attention
+        if (a.q_rope) {
+            const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+            for (int i = threadIdx.x; i < G * PSTRIDE; i += blockDim.x) {
+                const int h = i / PSTRIDE, j = i % PSTRIDE;
+                a.part_sel[(cta * GMAX + h) * PSTRIDE + j] = j == 0 ? -INFINITY : 0.0f;
+            }
+        }
+        return;
+    }
     const __nv_bfloat16 *rows = reinterpret_cast<const __nv_bfloat16 *>(a.kidx) + bg * a.N_max * R;
     SrcMma src;
     src.init(rows, a.N_max, qs, G);
@@ -1094,8 +1235,8 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
                     const int t = tb + src.tok(v);
                     if (kept) {
                         const unsigned p = atomicAdd(&s_kc[h], 1u);
-                        if (p < (unsigned)KCAP) {
-                            s_kbuf[h * KCAP + p] = t;
+                        if (p < (unsigned)CL_KCAP) {
+                            s_kbuf[h * CL_KCAP + p] = t;
                         } else {
                             const unsigned q = atomicAdd(&w.list_cnt[bh0 + h], 1u);
                             a.lists[(bh0 + h) * a.N_max + q] = t;
@@ -1122,7 +1263,7 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
     __syncthreads();
     if (warp < G) {
         const size_t bh = bh0 + warp;
-        const unsigned nk = min(s_kc[warp], (unsigned)KCAP);
+        const unsigned nk = min(s_kc[warp], (unsigned)CL_KCAP);
         const unsigned ncd = min(s_cc[warp], (unsigned)CCAP);
         unsigned kb = 0u, cb = 0u;
         if (lane == 0) {
@@ -1131,8 +1272,76 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
         }
         kb = __shfl_sync(0xffffffffu, kb, 0);
         cb = __shfl_sync(0xffffffffu, cb, 0);
-        for (unsigned j = lane; j < nk; j += 32) a.lists[bh * a.N_max + kb + j] = s_kbuf[warp * KCAP + j];
+        for (unsigned j = lane; j < nk; j += 32) a.lists[bh * a.N_max + kb + j] = s_kbuf[warp * CL_KCAP + j];
         for (unsigned j = lane; j < ncd; j += 32) w.cands[bh * a.N_max + cb + j] = s_cbuf[warp * CCAP + j];
+    }
+    if (!a.q_rope) return;
+
+    // Fused attention over the rows staged here: chunks of 8 rows, head by
+    // head, dealt round-robin to the warps; each warp keeps one running
+    // partial and files it under (warp, head) when its head changes.  A head
+    // whose staging overflowed is left to finalize (ovf flag, empty partial).
+    int cpre[GMAX + 1];
+    cpre[0] = 0;
+#pragma unroll
+    for (int h = 0; h < GMAX; ++h) {
+        const int nkh = h < G && s_kc[h] <= (unsigned)CL_KCAP ? (int)s_kc[h] : 0;
+        cpre[h + 1] = cpre[h] + (nkh + 7) / 8;
+    }
+    if (threadIdx.x < G && s_kc[threadIdx.x] > (unsigned)CL_KCAP) a.ovf[bh0 + threadIdx.x] = 1u;
+    float *my = s_slot + warp * GMAX * PSTRIDE;
+    {
+        WarpPart e;
+        e.reset();
+#pragma unroll
+        for (int h = 0; h < GMAX; ++h) e.store(my + h * PSTRIDE);
+    }
+    __syncwarp();
+    const __nv_bfloat16 *kb = a.k_cache + bg * a.N_max * D;
+    const __nv_bfloat16 *vb = a.v_cache + bg * a.N_max * D;
+    WarpPart part;
+    part.reset();
+    int cur = -1;
+    float qx[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int k = warp; k < cpre[GMAX]; k += CL_WARPS) {
+        // head of chunk k and its first chunk (no dynamic register indexing)
+        int h = 0, c0 = 0;
+#pragma unroll
+        for (int j = 1; j <= GMAX; ++j)
+            if (cpre[j] <= k) { h = j; c0 = cpre[j]; }
+        if (h != cur) {
+            if (cur >= 0) part.store(my + cur * PSTRIDE);
+            part.reset();
+            cur = h;
+            const float4 q4 = *reinterpret_cast<const float4 *>(s_qr + h * D + 4 * lane);
+            qx[0] = q4.x; qx[1] = q4.y; qx[2] = q4.z; qx[3] = q4.w;
+        }
+        const int r = (k - c0) * 8 + lane;
+        const int id = lane < 8 && r < (int)s_kc[h] ? s_kbuf[h * CL_KCAP + r] : -1;
+        attend8(kb, vb, id, qx, part);
+    }
+    if (cur >= 0) part.store(my + cur * PSTRIDE);
+    __syncthreads();
+    // merge the warps' partials per head into this CTA's record of the head
+    const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+    for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+        const int h = i / D, d = i % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w2 = 0; w2 < CL_WARPS; ++w2) M = fmaxf(M, s_slot[(w2 * GMAX + h) * PSTRIDE]);
+        float L = 0.0f, O = 0.0f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w2 = 0; w2 < CL_WARPS; ++w2) {
+                const float *sl = s_slot + (w2 * GMAX + h) * PSTRIDE;
+                const float wg = sl[0] == -INFINITY ? 0.0f : exp2f(sl[0] - M);
+                L = fmaf(sl[1], wg, L);
+                O = fmaf(sl[POFF + d], wg, O);
+            }
+        }
+        float *rec = a.part_sel + (cta * GMAX + h) * PSTRIDE;
+        rec[POFF + d] = O;
+        if (d == 0) { rec[0] = M; rec[1] = L; }
     }
 }
 
@@ -1155,7 +1364,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     __shared__ unsigned long long hfx[256];
     __shared__ uint32_t hfx32[256];
     __shared__ unsigned hcnt[256];
-    __shared__ unsigned long long cbuf[FIN_CAP];
+    __shared__ __align__(16) unsigned long long cbuf[FIN_CAP];
     __shared__ uint32_t fbuf[FIN_CAP];
     __shared__ unsigned long long s_min, s_max, s_theta, s_excl, s_kept;
     __shared__ unsigned s_base;
@@ -1175,11 +1384,32 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     const Resolve r = w.res[bh];
     const unsigned nc_all = w.cand_cnt[bh];
     const unsigned base0 = w.list_cnt[bh];
+    const unsigned ovf = a.q_rope ? a.ovf[bh] : 0u;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned long long *cg = w.cands + bh * a.N_max;
     // first candidate of each thread, loaded before the count is known (the
     // buffer holds N_max entries, so the read is in bounds)
     const unsigned long long c_first = tid < a.N_max ? __ldcg(cg + tid) : 0ull;
+    // fused attention: fold the collect CTAs' partials of this head while the
+    // selection's own loads are in flight (discarded below after an overflow)
+    WarpPart part;
+    part.reset();
+    if (a.q_rope) {
+        const size_t y = (size_t)b * a.n_ret + gi;
+        const float *recs = a.part_sel + (size_t)(hb % G) * PSTRIDE;
+        for (int x = warp; x < a.cl_ctas; x += 2 * FIN_WARPS) {
+            // two records in flight per warp
+            const float *r0 = recs + (y * a.cl_ctas + x) * GMAX * PSTRIDE;
+            const bool has1 = x + FIN_WARPS < a.cl_ctas;
+            const float *r1 = recs + (y * a.cl_ctas + (has1 ? x + FIN_WARPS : x)) * GMAX * PSTRIDE;
+            const float m0 = __ldcg(r0), l0 = __ldcg(r0 + 1), m1 = __ldcg(r1), l1 = __ldcg(r1 + 1);
+            const float4 o0 = __ldcg(reinterpret_cast<const float4 *>(r0 + POFF) + lane);
+            const float4 o1 = __ldcg(reinterpret_cast<const float4 *>(r1 + POFF) + lane);
+            const float ox0[4] = {o0.x, o0.y, o0.z, o0.w}, ox1[4] = {o1.x, o1.y, o1.z, o1.w};
+            part.add(m0, l0, ox0);
+            if (has1) part.add(m1, l1, ox1);
+        }
+    }
     const unsigned nc = r.mode == MODE_NORMAL ? nc_all : 0u;
     int32_t *lst = a.lists + bh * a.N_max;
     int count = 0;
@@ -1341,6 +1571,49 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     if (tid == 0) {
         a.count_out[bh] = count;
         if (a.mass_out) a.mass_out[bh] = mass;
+    }
+    if (!a.q_rope) return;
+
+    // Fused attention: merge the collect CTAs' partials of this head into
+    // one record (slot 0 of the head's list partials); the rows the collect
+    // pass did not attend -- the boundary bin's, or all of them after a
+    // staging overflow -- are left to the list pass (rest0 = first of them).
+    // A head with no such rows gets its output here.
+    float *hrec = a.part_list + bh * (size_t)LIST_SLOTS * PSTRIDE;
+    const int rest0 = ovf ? 0 : (int)base0;
+    if (tid == 0) a.rest0[bh] = rest0;
+    if (count <= 0) {
+        // nothing kept (invalid input): zeros and a status
+        for (int d = tid; d < D; d += blockDim.x) a.out[bh * D + d] = 0.0f;
+        if (tid == 0) set_status(w.status, RTP_ERR_DEVICE_ARG);
+        return;
+    }
+    if (ovf) part.reset();                           // a CTA could not attend all its kept rows
+    __syncthreads();                                 // every thread is done with the candidates
+    float *slots = reinterpret_cast<float *>(cbuf);  // the candidates are no longer needed
+    part.store(slots + warp * PSTRIDE);
+    __syncthreads();
+    const bool direct = count <= rest0;              // every kept row was attended by the collect pass
+    for (int d = tid; d < D; d += blockDim.x) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w2 = 0; w2 < FIN_WARPS; ++w2) M = fmaxf(M, slots[w2 * PSTRIDE]);
+        float L = 0.0f, O = 0.0f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w2 = 0; w2 < FIN_WARPS; ++w2) {
+                const float *sl = slots + w2 * PSTRIDE;
+                const float wg = sl[0] == -INFINITY ? 0.0f : exp2f(sl[0] - M);
+                L = fmaf(sl[1], wg, L);
+                O = fmaf(sl[POFF + d], wg, O);
+            }
+        }
+        if (direct) {
+            a.out[bh * D + d] = O * (L > 0.0f ? 1.0f / L : 0.0f);
+        } else {
+            hrec[POFF + d] = O;
+            if (d == 0) { hrec[0] = M; hrec[1] = L; }
+        }
     }
 }
 
