@@ -152,3 +152,56 @@ def test_ctx128k_b8_sampled_layers():
     # for every layer.
     for layer in (0, 29):
         _workload("ctx128k-b8-48layer", [0.9], layer=layer)
+
+
+# ------------------------------------------------------- staging overflow
+
+def _bins_f32(z):
+    """Level-1 bin of fp32 logits (sign, exponent, 4 mantissa bits; |z| below
+    2^-6 in the innermost bins): the selection's bin map, restated here to
+    check that this case reaches the overflow path."""
+    u = np.asarray(z, dtype=np.float32).view(np.uint32).astype(np.int64)
+    s = -(u >> 31)
+    k = np.clip((((u << 1) & 0xFFFFFFFF) >> 20) - (121 << 4), 0, 255)
+    return 256 + (k ^ s)
+
+
+@pytest.mark.slow
+def test_fused_staging_overflow():
+    """A 512K-token group where most tokens of each head lie above the
+    boundary bin: a collect CTA keeps more rows of a head than it can stage,
+    and finalize / the list pass attend that head's rows themselves."""
+    N = 524288
+    spec = synth.small_spec(B=1, H_q=8, H_kv=1, N=N, head_class=(1,), p=0.9, needles="none",
+                            name="overflow")
+    c = synth.make_case(spec)
+    g = torch.Generator().manual_seed(7)
+    # head 0's logits ~ N(4, 0.5^2): the mass-weighted 10 % quantile lies
+    # well below the mean, so most tokens sit in bins above the boundary bin
+    qi0 = oracle.query_index(np64(c.q)[0, 0], np64(c.W_q_idx)[0])
+    n0 = float(np.linalg.norm(qi0))
+    u = torch.tensor(qi0 / n0 * (4.0 * math.sqrt(128) / n0), dtype=torch.float32)
+    kid = u[None, :] + torch.randn(N, 16, generator=g) * (0.5 * math.sqrt(128) / n0)
+    c.kidx_cache[0, 0, :N] = kid.to(c.kidx_cache.dtype)
+    gc = GpuCase(c)
+    gc.append_current()
+    out, si, sc, sm = gc.step(0.9)
+    # the case must reach the path: some head keeps > 1024 rows above its
+    # boundary bin inside one collect CTA's token range
+    q = np64(c.q)
+    kidx = oracle_kidx(gc, "bf16", True)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    tiles = (N + 31) // 32
+    chunk = (tiles + sms - 1) // sms * 32
+    worst = 0
+    for h in range(8):
+        z = oracle.index_logits(oracle.query_index(q[0, h], np64(c.W_q_idx)[h]), kidx[0, 0, :N],
+                                1 / math.sqrt(128))
+        sel = oracle.topp_select(z, 0.9)
+        zb = z[sel.order[len(sel.kept) - 1]]
+        bins = _bins_f32(z)
+        above = bins > _bins_f32(np.array([zb]))[0]
+        per_cta = np.add.reduceat(above.astype(np.int64), np.arange(0, N, chunk))
+        worst = max(worst, int(per_cta.max()))
+    assert worst > 1024, f"case does not overflow the staging ({worst} rows)"
+    _compare(gc, out, si, sc, sm, 0.9)
