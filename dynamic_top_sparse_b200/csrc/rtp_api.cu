@@ -34,7 +34,7 @@ struct Layout {
     size_t end_range;       // local / dense
     size_t part_list;
     size_t end_list;        // sparse decode
-    size_t tilebin, lists, cands, part_sel, ovf, rest0;
+    size_t tilebin, lists, cands, part_sel, ovf;
     size_t total;           // topp_select / decode_step
 };
 
@@ -70,7 +70,6 @@ Layout make_layout(const rtp_dims *d) {
     // and the collect grid twice as many
     L.part_sel = o; o = align_up(o + 2 * std::max((size_t)num_sms(), BHkv) * GMAX * PSTRIDE * 4, 256);
     L.ovf = o; o = align_up(o + BHq * 4, 256);
-    L.rest0 = o; o = align_up(o + BHq * 4, 256);
     L.total = o;
     return L;
 }
@@ -142,6 +141,9 @@ struct Launcher {
     // it on the device (pdl_wait).  Only for kernels that call pdl_wait
     // before touching global memory.
     bool pdl = false;
+    // Launch the next kernels in thread-block clusters of this many CTAs
+    // along x (0: no clusters).
+    unsigned cluster_x = 0;
     // Inside stream capture an event becomes a timestamp node of the graph
     // only when recorded as external.
     cudaError_t record(void *ev, bool capturing) {
@@ -165,17 +167,28 @@ struct Launcher {
             capturing = cs == cudaStreamCaptureStatusActive;
             if (record(prof->ev_start[slot], capturing) != cudaSuccess) return RTP_ERR_CUDA;
         }
-        if (pdl) {
+        if (pdl || cluster_x) {
             cudaLaunchConfig_t cfg{};
             cfg.gridDim = grid;
             cfg.blockDim = block;
             cfg.dynamicSmemBytes = smem;
             cfg.stream = st;
-            cudaLaunchAttribute at[1];
-            at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            at[0].val.programmaticStreamSerializationAllowed = 1;
+            cudaLaunchAttribute at[2];
+            unsigned n = 0;
+            if (pdl) {
+                at[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+                at[n].val.programmaticStreamSerializationAllowed = 1;
+                ++n;
+            }
+            if (cluster_x) {
+                at[n].id = cudaLaunchAttributeClusterDimension;
+                at[n].val.clusterDim.x = cluster_x;
+                at[n].val.clusterDim.y = 1;
+                at[n].val.clusterDim.z = 1;
+                ++n;
+            }
             cfg.attrs = at;
-            cfg.numAttrs = 1;
+            cfg.numAttrs = n;
             if (cudaLaunchKernelEx(&cfg, kernel, args...) != cudaSuccess) return RTP_ERR_CUDA;
         } else {
             kernel<<<grid, block, smem, st>>>(args...);
@@ -248,7 +261,7 @@ int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s, const After
     RTP_TRY(ln.run("hist", scan_kernel<Src>, grid, dim3(SCAN_THREADS), s.a, s.w));
     RTP_TRY(ln.run("collect", collect_kernel<Src>, grid, dim3(COL_THREADS), s.a, s.w));
     if (after_collect) RTP_TRY(after_collect());
-    RTP_TRY(ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)),
+    RTP_TRY(ln.run("finalize", finalize_kernel, dim3(1u, (unsigned)(d->B * s.a.n_ret * s.a.G)),
                    dim3(FIN_THREADS), s.a, s.w));
     return RTP_OK;
 }
@@ -290,9 +303,14 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sm
     int rc = ln.run_smem("hist", scan_tma_kernel, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w);
     if (rc == RTP_OK) rc = ln.run_smem("collect", collect_mma_kernel, cl_grid, dim3(CL_THREADS), CL_SMEM, s.a, s.w);
     if (rc == RTP_OK && after_collect) rc = after_collect();
-    if (rc == RTP_OK)
-        rc = ln.run("finalize", finalize_kernel, dim3((unsigned)(d->B * s.a.n_ret * s.a.G)), dim3(FIN_THREADS),
+    if (rc == RTP_OK) {
+        // with the fused attention the CTAs of a head form a cluster
+        const unsigned K = s.a.q_rope ? (unsigned)FIN_CLUSTER : 1u;
+        ln.cluster_x = K > 1 ? K : 0u;
+        rc = ln.run("finalize", finalize_kernel, dim3(K, (unsigned)(d->B * s.a.n_ret * s.a.G)), dim3(FIN_THREADS),
                     s.a, s.w);
+        ln.cluster_x = 0;
+    }
     ln.pdl = pdl0;
     return rc;
 }
@@ -716,17 +734,7 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
                 s.a.out = out;
                 s.a.part_sel = reinterpret_cast<float *>(w + L.part_sel);
                 s.a.ovf = reinterpret_cast<uint32_t *>(w + L.ovf);
-                s.a.part_list = reinterpret_cast<float *>(w + L.part_list);
-                s.a.rest0 = reinterpret_cast<int32_t *>(w + L.rest0);
                 rc = select_from_index(ln, dims, s, local_ctas);
-                if (rc == RTP_OK) {
-                    // the kept rows the selection left (the boundary bin's), merged
-                    // with the selection's partial
-                    ln.pdl = true;                      // follows finalize_kernel
-                    rc = launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class,
-                                     out, w, L, asc, LIST_TAIL, s.a.rest0);
-                    ln.pdl = false;
-                }
                 if (side && cudaStreamWaitEvent(main, side->join, 0) != cudaSuccess && rc == RTP_OK)
                     rc = RTP_ERR_CUDA;
                 return rc;

@@ -260,10 +260,7 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
 // rest): LIST_FIRST writes partials only; LIST_REST adds the remaining rows
 // and merges everything.  Partials live in per-head slots: the first pass
 // uses slots [0, it_first), the second [it_first, it_first + it_rest).
-// LIST_TAIL follows a selection that attended most rows itself: slot 0
-// already holds their merged partial, `first` gives the first row left, and
-// heads with no rows left were written by the selection.
-enum ListPhase : int32_t { LIST_ALL = 0, LIST_FIRST = 1, LIST_REST = 2, LIST_TAIL = 3 };
+enum ListPhase : int32_t { LIST_ALL = 0, LIST_FIRST = 1, LIST_REST = 2 };
 
 struct ListArgs {
     int B, H_q, H_kv, G;
@@ -277,8 +274,7 @@ struct ListArgs {
     const void *v;
     const int32_t *lists;        // [B*H_q*N_max]
     const int32_t *counts;       // [B*H_q] kept rows per head (read by LIST_ALL and LIST_REST)
-    const int32_t *first;        // [B*H_q] rows of the collect pass (LIST_FIRST, LIST_REST) or first row
-                                 // left (LIST_TAIL), or null
+    const int32_t *first;        // [B*H_q] rows of the collect pass (LIST_FIRST, LIST_REST), or null
     int phase;
     float *out;
     float *part;                 // [B*H_q][LIST_SLOTS][PSTRIDE]
@@ -336,7 +332,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
                 } else if (a.phase == LIST_FIRST) {
                     const int nf = (int)__ldcg(a.first + bh);
                     if (okN && nf >= 1 && nf <= N) { rows = nf; it = list_items(nf); }
-                } else if (a.phase == LIST_REST) {
+                } else {
                     const int cnt = __ldcg(a.counts + bh);
                     const int nf = __ldcg(a.first + bh);
                     if (okN && cnt >= 1 && cnt <= N && nf >= 0 && nf <= cnt) {
@@ -344,15 +340,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
                         rows = cnt - nf;
                         slot0 = list_items(nf);
                         it = max(1, list_items(rows));       // at least one item: it merges the head
-                    }
-                } else {
-                    const int cnt = __ldcg(a.counts + bh);
-                    const int nf = __ldcg(a.first + bh);
-                    if (okN && cnt >= 1 && cnt <= N && nf >= 0 && nf < cnt) {
-                        row0 = nf;
-                        rows = cnt - nf;
-                        slot0 = 1;                          // slot 0: the selection's partial
-                        it = list_items(rows);
                     }
                 }
                 pre[hi] = it;
@@ -391,7 +378,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
     }
     const int total = pre[nh];
     // heads with nothing to attend over get zeros (and a status: invalid input)
-    if (blockIdx.x == 0 && (a.phase == LIST_ALL || a.phase == LIST_REST)) {
+    if (blockIdx.x == 0 && a.phase != LIST_FIRST) {
         for (int hi = warp; hi < nh; hi += ATT_THREADS / 32) {
             if (pre[hi + 1] != pre[hi]) continue;
             const int b = hi / a.n_rq, h = a.ret_h[hi % a.n_rq];
@@ -481,10 +468,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
         __syncthreads();
         float *hp = a.part + bh * (size_t)LIST_SLOTS * PSTRIDE;
         float *pp = hp + (size_t)slot * PSTRIDE;
-        // a head attended by this one item only (besides, for LIST_TAIL, the
-        // selection's partial in slot 0): normalise and write directly
-        const bool tail1 = a.phase == LIST_TAIL && nit == 1;
-        const bool direct = (a.phase != LIST_FIRST && nrec == 1) || tail1;
+        // a head attended by this one item only: normalise and write directly
+        const bool direct = a.phase != LIST_FIRST && nrec == 1;
         if (tid < D) {
             float M = -INFINITY;
             for (int w = 0; w < ATT_THREADS / 32; ++w) M = fmaxf(M, wm[w]);
@@ -494,17 +479,6 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
                     const float wg = wm[w] == -INFINITY ? 0.0f : exp2f(wm[w] - M);
                     ls = fmaf(wl[w], wg, ls);
                     os = fmaf(wo[w][tid], wg, os);
-                }
-            }
-            if (tail1) {
-                // fold in slot 0
-                const float m0 = __ldcg(hp), l0 = __ldcg(hp + 1), o0 = __ldcg(hp + POFF + tid);
-                const float Mt = fmaxf(M, m0);
-                if (Mt != -INFINITY) {
-                    const float w1 = M == -INFINITY ? 0.0f : exp2f(M - Mt);
-                    const float w0 = m0 == -INFINITY ? 0.0f : exp2f(m0 - Mt);
-                    ls = ls * w1 + l0 * w0;
-                    os = os * w1 + o0 * w0;
                 }
             }
             if (direct) {

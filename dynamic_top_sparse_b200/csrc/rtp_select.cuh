@@ -33,6 +33,8 @@
 
 #include <type_traits>
 
+#include <cooperative_groups.h>
+
 #include "rtp_common.cuh"
 
 namespace rtp {
@@ -183,9 +185,14 @@ struct SelArgs {
     float *out;                          // [B, H_q, D]
     float *part_sel;                     // [collect CTAs][GMAX][PSTRIDE]
     uint32_t *ovf;                       // [B*H_q]
-    float *part_list;                    // [B*H_q][LIST_SLOTS][PSTRIDE]: slot 0 = collect partials merged
-    int32_t *rest0;                      // [B*H_q] first list row left to the list pass
 };
+
+// Record `r` of a cluster (the same shared variable in CTA rank r); the CTA's
+// own copy when the kernel runs without clusters.
+__device__ __forceinline__ const float *cluster_rec(cooperative_groups::cluster_group &cl, float *rec, int r,
+                                                    int K) {
+    return K > 1 ? cl.map_shared_rank(rec, r) : rec;
+}
 
 // ---------------------------------------------------------------------------
 // fused sparse attention helpers
@@ -1354,6 +1361,7 @@ __device__ __forceinline__ float cand_logit(unsigned long long c) { return key_l
 constexpr int FIN_THREADS = 512;
 constexpr int FIN_WARPS = FIN_THREADS / 32;
 constexpr int FIN_CAP = 3072;             // candidates staged in shared memory
+constexpr int FIN_CLUSTER = 4;            // CTAs per head with the fused attention
 // Exact selection inside the boundary bin.  One CTA per retrieval head;
 // grid = (B * n_ret * G).  Candidate masses relative to the boundary bin's
 // upper edge U* are each in (e^-32, 1]; they are summed in fixed point with
@@ -1370,8 +1378,14 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     __shared__ unsigned s_base;
     __shared__ int s_digit;
     __shared__ unsigned s_dcnt;
+    __shared__ __align__(16) float s_crec[FIN_CLUSTER * PSTRIDE];   // the ranks' attention partials (fused)
     const int G = a.G;
-    const int hb = blockIdx.x;
+    // grid (K, heads): with the fused attention the K CTAs of a head form a
+    // cluster; each runs the (cheap, identical) selection, rank 0 writes its
+    // results, and the ranks split the attention and merge through DSMEM
+    const int K = gridDim.x;
+    const int rank = blockIdx.x;
+    const int hb = blockIdx.y;
     const int b = hb / (a.n_ret * G);
     const int gi = (hb / G) % a.n_ret;
     const int h = a.ret_g[gi] * G + hb % G;
@@ -1379,7 +1393,8 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     pdl_wait();
     pdl_trigger();
     // the collect pass is done with the histogram: clear it for the next call
-    for (int i = threadIdx.x; i < NBIN; i += blockDim.x) w.hist[bh * NBIN + i] = 0.0;
+    if (rank == 0)
+        for (int i = threadIdx.x; i < NBIN; i += blockDim.x) w.hist[bh * NBIN + i] = 0.0;
     // the head's resolve record and both counters in one round of loads
     const Resolve r = w.res[bh];
     const unsigned nc_all = w.cand_cnt[bh];
@@ -1397,26 +1412,25 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     if (a.q_rope) {
         const size_t y = (size_t)b * a.n_ret + gi;
         const float *recs = a.part_sel + (size_t)(hb % G) * PSTRIDE;
-        for (int x = warp; x < a.cl_ctas; x += 2 * FIN_WARPS) {
-            // two records in flight per warp
-            const float *r0 = recs + (y * a.cl_ctas + x) * GMAX * PSTRIDE;
-            const bool has1 = x + FIN_WARPS < a.cl_ctas;
-            const float *r1 = recs + (y * a.cl_ctas + (has1 ? x + FIN_WARPS : x)) * GMAX * PSTRIDE;
-            const float m0 = __ldcg(r0), l0 = __ldcg(r0 + 1), m1 = __ldcg(r1), l1 = __ldcg(r1 + 1);
-            const float4 o0 = __ldcg(reinterpret_cast<const float4 *>(r0 + POFF) + lane);
-            const float4 o1 = __ldcg(reinterpret_cast<const float4 *>(r1 + POFF) + lane);
-            const float ox0[4] = {o0.x, o0.y, o0.z, o0.w}, ox1[4] = {o1.x, o1.y, o1.z, o1.w};
-            part.add(m0, l0, ox0);
-            if (has1) part.add(m1, l1, ox1);
-        }
+        for (int x = rank * FIN_WARPS + warp; x < a.cl_ctas; x += K * FIN_WARPS)
+            part.load_add(recs + (y * a.cl_ctas + x) * GMAX * PSTRIDE);
     }
+    // fused attention: this head's query (scaled) with the first loads
+    float qx_f[4] = {0.f, 0.f, 0.f, 0.f};
+    if (a.q_rope) {
+        const float4 q4 = *reinterpret_cast<const float4 *>(a.q_rope + bh * D + 4 * lane);
+        qx_f[0] = q4.x * a.attn_scale_log2; qx_f[1] = q4.y * a.attn_scale_log2;
+        qx_f[2] = q4.z * a.attn_scale_log2; qx_f[3] = q4.w * a.attn_scale_log2;
+    }
+    unsigned long long fin_theta = ~0ull;            // kept boundary candidates: key >= fin_theta
     const unsigned nc = r.mode == MODE_NORMAL ? nc_all : 0u;
     int32_t *lst = a.lists + bh * a.N_max;
     int count = 0;
     float mass = 0.0f;
 
     if (r.mode == MODE_KEEP_ALL) {
-        for (int t = tid; t < r.N; t += blockDim.x) lst[t] = t;
+        if (rank == 0)
+            for (int t = tid; t < r.N; t += blockDim.x) lst[t] = t;
         count = r.N;
         mass = 1.0f;
     } else if (r.mode != MODE_NORMAL || nc == 0u) {
@@ -1556,7 +1570,8 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             if (lane == 0 && bal) wbase = atomicAdd(&s_base, (unsigned)__popc(bal));
             wbase = __shfl_sync(0xffffffffu, wbase, 0);
             if (k) {
-                lst[base0 + wbase + __popc(bal & lt)] = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
+                if (rank == 0)
+                    lst[base0 + wbase + __popc(bal & lt)] = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
                 kept += staged ? fbuf[c] : fx_of(v);
             }
         }
@@ -1565,35 +1580,68 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         if (lane == 0) atomicAdd(&s_kept, kept);
         __syncthreads();
         count = (int)(base0 + s_base);
+        fin_theta = theta;
         const double kept_mass = (double)s_kept / S * (double)ex2_sfu((Ub - r.R) * 1.4426950408889634f);
         mass = (float)((r.above + kept_mass) / r.Z);
     }
-    if (tid == 0) {
+    if (tid == 0 && rank == 0) {
         a.count_out[bh] = count;
         if (a.mass_out) a.mass_out[bh] = mass;
     }
     if (!a.q_rope) return;
 
-    // Fused attention: merge the collect CTAs' partials of this head into
-    // one record (slot 0 of the head's list partials); the rows the collect
-    // pass did not attend -- the boundary bin's, or all of them after a
-    // staging overflow -- are left to the list pass (rest0 = first of them).
-    // A head with no such rows gets its output here.
-    float *hrec = a.part_list + bh * (size_t)LIST_SLOTS * PSTRIDE;
-    const int rest0 = ovf ? 0 : (int)base0;
-    if (tid == 0) a.rest0[bh] = rest0;
+    // Fused attention: the kept rows the collect pass did not attend (the
+    // boundary bin's kept candidates, plus, after a staging overflow, the
+    // collect pass's rows) are split over the cluster's ranks and warps;
+    // each rank merges its warps and the collect records it folded into one
+    // partial, stores it into rank 0's shared memory, and rank 0 merges.
+    namespace cgr = cooperative_groups;
+    cgr::cluster_group cluster = cgr::this_cluster();
     if (count <= 0) {
         // nothing kept (invalid input): zeros and a status
-        for (int d = tid; d < D; d += blockDim.x) a.out[bh * D + d] = 0.0f;
-        if (tid == 0) set_status(w.status, RTP_ERR_DEVICE_ARG);
+        if (rank == 0) {
+            for (int d = tid; d < D; d += blockDim.x) a.out[bh * D + d] = 0.0f;
+            if (tid == 0) set_status(w.status, RTP_ERR_DEVICE_ARG);
+        }
         return;
     }
-    if (ovf) part.reset();                           // a CTA could not attend all its kept rows
+    if (ovf) part.reset();                           // a collect CTA could not attend all its kept rows
+    {
+        const size_t bg = (size_t)b * a.H_kv + (size_t)(h / G);
+        const __nv_bfloat16 *kb = a.k_cache + bg * a.N_max * D;
+        const __nv_bfloat16 *vb = a.v_cache + bg * a.N_max * D;
+        const int worker = rank * FIN_WARPS + warp, workers = K * FIN_WARPS;
+        if (ovf) {
+            // the collect pass's rows, from its list
+            for (int rb = worker * 8; rb < (int)base0; rb += workers * 8) {
+                const int id = lane < 8 && rb + lane < (int)base0 ? __ldcg(lst + rb + lane) : -1;
+                attend8(kb, vb, id, qx_f, part);
+            }
+        }
+        if (r.mode == MODE_KEEP_ALL) {
+            for (int rb = worker * 8; rb < count; rb += workers * 8) {
+                const int id = lane < 8 && rb + lane < count ? rb + lane : -1;
+                attend8(kb, vb, id, qx_f, part);
+            }
+        } else if (r.mode == MODE_NORMAL) {
+            // boundary-bin candidates at or above theta, eight candidate slots at a time
+            const bool staged = nc <= (unsigned)FIN_CAP;
+            for (int cb = worker * 8; cb < (int)nc; cb += workers * 8) {
+                int id = -1;
+                if (lane < 8 && cb + lane < (int)nc) {
+                    const unsigned long long v = staged ? cbuf[cb + lane] : __ldcg(cg + cb + lane);
+                    if (v >= fin_theta) id = (int)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
+                }
+                attend8(kb, vb, id, qx_f, part);
+            }
+        }
+    }
     __syncthreads();                                 // every thread is done with the candidates
     float *slots = reinterpret_cast<float *>(cbuf);  // the candidates are no longer needed
     part.store(slots + warp * PSTRIDE);
     __syncthreads();
-    const bool direct = count <= rest0;              // every kept row was attended by the collect pass
+    // this rank's partial goes into slot `rank` of rank 0's s_crec
+    float *dst = K > 1 ? cluster.map_shared_rank(s_crec, 0) + rank * PSTRIDE : s_crec;
     for (int d = tid; d < D; d += blockDim.x) {
         float M = -INFINITY;
 #pragma unroll
@@ -1608,11 +1656,24 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
                 O = fmaf(sl[POFF + d], wg, O);
             }
         }
-        if (direct) {
+        dst[POFF + d] = O;
+        if (d == 0) { dst[0] = M; dst[1] = L; }
+    }
+    if (K > 1) cluster.sync(); else __syncthreads();
+    if (rank == 0) {
+        for (int d = tid; d < D; d += blockDim.x) {
+            float M = -INFINITY;
+            for (int r2 = 0; r2 < K; ++r2) M = fmaxf(M, s_crec[r2 * PSTRIDE]);
+            float L = 0.0f, O = 0.0f;
+            if (M != -INFINITY) {
+                for (int r2 = 0; r2 < K; ++r2) {
+                    const float *rc = s_crec + r2 * PSTRIDE;
+                    const float wg = rc[0] == -INFINITY ? 0.0f : exp2f(rc[0] - M);
+                    L = fmaf(rc[1], wg, L);
+                    O = fmaf(rc[POFF + d], wg, O);
+                }
+            }
             a.out[bh * D + d] = O * (L > 0.0f ? 1.0f / L : 0.0f);
-        } else {
-            hrec[POFF + d] = O;
-            if (d == 0) { hrec[0] = M; hrec[1] = L; }
         }
     }
 }
