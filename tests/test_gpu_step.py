@@ -65,6 +65,10 @@ SMALL = [
     dict(B=2, H_q=8, H_kv=1, N=40, head_class=(1,), p=1e-9, seq_lens=[40, 2]),
     dict(B=1, H_q=6, H_kv=2, N=2049, head_class=(1, 0), p=0.99, needles="none"),
     dict(B=1, H_q=8, H_kv=1, N=4096, head_class=(1,), p=0.9, needle_scale=4.0, needles_per_head=40),
+    # bf16 index keys with fp32 caches: the selection on tensor cores, the
+    # attention in the separate list passes
+    dict(B=2, H_q=16, H_kv=2, N=6000, head_class=(1, 0), p=0.9, kv_dtype="f32", idx_dtype="bf16",
+         seq_lens=[6000, 1234]),
 ]
 
 
