@@ -50,9 +50,9 @@ Layout make_layout(const rtp_dims *d) {
     L.status = o; o += 256;
     L.arrive_range = o; o = align_up(o + BHkv * 4, 256);
     L.arrive_list = o; o = align_up(o + BHq * 4, 256);
-    L.cand_cnt = o; o = align_up(o + BHq * 4, 256);
-    L.list_cnt = o; o = align_up(o + BHq * 4, 256);
-    L.hist = o; o = align_up(o + BHq * NBIN * 8, 256);
+    L.cand_cnt = o; o = align_up(o + BHq * CNT_STRIDE * 4, 256);
+    L.list_cnt = o; o = align_up(o + BHq * CNT_STRIDE * 4, 256);
+    L.hist = o; o = align_up(o + BHq * HSTRIDE * 8, 256);
     L.ctrl_end = o;
     L.res = o; o = align_up(o + BHq * sizeof(Resolve), 256);
     L.qidx = o; o = align_up(o + BHq * R * 4, 256);
@@ -289,12 +289,12 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sm
     long long ctas = std::max(1LL, std::min(sms / std::max(groups, 1LL), tiles));
     s.a.chunk = (tiles + ctas - 1) / ctas * TILE;
     s.a.ctas = (int)((d->N_max + s.a.chunk - 1) / s.a.chunk);
-    // collect: one CTA per SM, the scan's ranges
-    const long long cl = s.a.ctas;
-    s.a.cl_chunk = (tiles + cl - 1) / cl * TILE;
-    s.a.cl_ctas = (int)((d->N_max + s.a.cl_chunk - 1) / s.a.cl_chunk);
+    // collect: the groups in pairs, one CTA per SM, the pair's tiles dealt
+    // round-robin over its CTAs
+    const long long pairs = (groups + PAIR - 1) / PAIR;
+    s.a.cl_ctas = (int)std::max(1LL, std::min(sms / pairs, PAIR * tiles));
     const dim3 grid((unsigned)s.a.ctas, (unsigned)groups);
-    const dim3 cl_grid((unsigned)s.a.cl_ctas, (unsigned)groups);
+    const dim3 cl_grid((unsigned)s.a.cl_ctas, (unsigned)pairs);
     // scan, collect and finalize wait on the device for their predecessor
     // (programmatic dependent launch), so each one's launch overlaps the
     // previous kernel's tail

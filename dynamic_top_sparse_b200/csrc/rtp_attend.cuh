@@ -274,7 +274,7 @@ struct ListArgs {
     const void *v;
     const int32_t *lists;        // [B*H_q*N_max]
     const int32_t *counts;       // [B*H_q] kept rows per head (read by LIST_ALL and LIST_REST)
-    const int32_t *first;        // [B*H_q] rows of the collect pass (LIST_FIRST, LIST_REST), or null
+    const int32_t *first;        // [B*H_q] at stride CNT_STRIDE: rows of the collect pass (LIST_FIRST, LIST_REST), or null
     int phase;
     float *out;
     float *part;                 // [B*H_q][LIST_SLOTS][PSTRIDE]
@@ -330,11 +330,11 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
                     const int cnt = __ldcg(a.counts + bh);
                     if (okN && cnt >= 1 && cnt <= N) { rows = cnt; it = list_items(cnt); }
                 } else if (a.phase == LIST_FIRST) {
-                    const int nf = (int)__ldcg(a.first + bh);
+                    const int nf = (int)__ldcg(a.first + bh * CNT_STRIDE);
                     if (okN && nf >= 1 && nf <= N) { rows = nf; it = list_items(nf); }
                 } else {
                     const int cnt = __ldcg(a.counts + bh);
-                    const int nf = __ldcg(a.first + bh);
+                    const int nf = __ldcg(a.first + bh * CNT_STRIDE);
                     if (okN && cnt >= 1 && cnt <= N && nf >= 0 && nf <= cnt) {
                         row0 = nf;
                         rows = cnt - nf;

@@ -171,6 +171,12 @@ __device__ __forceinline__ int list_items(int count) {
     return min(LIST_MAX_SPLIT, (count + LCH - 1) / LCH);
 }
 
+// Per-head counters of the selection (kept ids, boundary candidates) sit
+// one per 128-byte line: every collect CTA reserves space on them at about
+// the same moment, and counters sharing a line would queue those atomics on
+// one L2 slice.
+constexpr int CNT_STRIDE = 32;        // uint32 entries between consecutive heads' counters
+
 // Flash-decoding partial record of one head over a set of rows (log2
 // units): m = running max, l = sum of 2^(s - m), o[D] = unnormalised output.
 constexpr int PSTRIDE = D + 4;         // partial record: m, l, (2 unused), o[D]

@@ -53,6 +53,17 @@ enum ResolveMode : int32_t { MODE_NORMAL = 0, MODE_KEEP_ALL = 1, MODE_EMPTY = 2 
 constexpr int MB = 4;
 constexpr int E_LO = -6;
 constexpr int NBIN = 512;
+// Octaves: bins 16 s .. 16 s + 15 (one exponent of |z|, one sign) form
+// super-bin s; each head's histogram holds its NBIN bin sums followed by the
+// NSUP octave sums, so a resolve can read the 32 octave sums first and then
+// only the bins of the octave that holds the boundary.
+constexpr int NSUP = NBIN / 16;
+// The octave sums are kept in NREP replicas (a CTA adds to replica
+// blockIdx.x mod NREP; the resolve sums them): the scan's CTAs all add their
+// octave sums at the same moment, and one copy packed into two lines per
+// head queued ~1000 fp64 atomics per line.
+constexpr int NREP = 4;
+constexpr int HSTRIDE = NBIN + NREP * NSUP;   // doubles per head
 constexpr uint32_t BIN_BASE = (uint32_t)(127 + E_LO) << MB;   // k = (bits >> 19) - BIN_BASE
 constexpr float Z_LIMIT = 256.0f;   // logits beyond are reported (bins up to 16 nats wide stay resolvable)
 
@@ -62,6 +73,16 @@ __device__ __forceinline__ float ex2_sfu(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^y in fp64 range: 2^floor(y) exact (built from its exponent bits; 0 below
+// the normal range), 2^frac(y) by the SFU (relative error ~2^-22).  For
+// octave-level factors, which span far more than fp32's range.
+__device__ __forceinline__ double exp2_wide(double y) {
+    const double n = floor(y);
+    const int e = (int)fmax(fmin(n, 1023.0), -1023.0);
+    const double p2 = e < -1022 ? 0.0 : __longlong_as_double((long long)(e + 1023) << 52);
+    return (double)ex2_sfu((float)(y - n)) * p2;
 }
 
 // Per-CTA bin sums are kept in fixed point: FX_ONE units per unit of mass
@@ -131,6 +152,41 @@ __host__ __device__ __forceinline__ float bin_upper(int bin) {
     return -c.f;
 }
 
+// exp(U_b - U_octave(b)): a bin's mass relative to its octave's upper edge
+// per unit of mass relative to its own (a constant of the bin; the scans
+// tabulate it in shared memory while they stream).
+__device__ __forceinline__ double octave_factor(int bin) {
+    return exp2_wide((double)(bin_upper(bin) - bin_upper(bin | 15)) * 1.4426950408889634);
+}
+
+// A CTA's fixed-point bin sum v (< 2^52) times `unit` as a double, without
+// a conversion instruction: v OR-ed into the mantissa of 2^52 is exactly
+// 2^52 + v, and one fma removes the 2^52.
+__device__ __forceinline__ double fixed_to_double(unsigned long long v, double unit) {
+    return fma(__longlong_as_double((long long)(0x4330000000000000ull | v)), unit, -4503599627370496.0 * unit);
+}
+
+// Adds a CTA's bin sums of G heads to the histograms (gh0: the first head's;
+// heads HSTRIDE apart).  bin_mass(i) = mass of entry i = head * NBIN + bin
+// relative to the bin's upper edge; fac = the octave factors; rep = the
+// CTA's octave replica.  One atomic per non-empty bin; the loop is
+// warp-aligned (G * NBIN and blockDim are multiples of 32), so 16
+// consecutive lanes hold one octave, whose sum relative to the octave's
+// upper edge is formed across the half-warp (fixed order) and added to the
+// octave's replica slot.
+template <typename BinMass>
+__device__ __forceinline__ void flush_hist(double *gh0, int G, const double *fac, int rep, const BinMass &bin_mass) {
+    for (int i = threadIdx.x; i < G * NBIN; i += blockDim.x) {
+        const double m = bin_mass(i);
+        double *gh = gh0 + (size_t)(i / NBIN) * HSTRIDE;
+        if (m != 0.0) atomicAdd(gh + i % NBIN, m);
+        double x = m * fac[i % NBIN];
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+        if ((threadIdx.x & 15) == 0 && x != 0.0) atomicAdd(gh + NBIN + rep * NSUP + (i % NBIN) / 16, x);
+    }
+}
+
 struct Resolve {
     double Z;          // total mass, relative to exp(R)
     double above;      // mass of the bins above b*, same units
@@ -144,9 +200,9 @@ static_assert(sizeof(Resolve) == 40, "Resolve layout");
 
 struct SelWs {
     uint32_t *status;
-    uint32_t *cand_cnt;          // [B*H_q]
-    uint32_t *list_cnt;          // [B*H_q]
-    double *hist;                // [B*H_q][NBIN]
+    uint32_t *cand_cnt;          // [B*H_q] at stride CNT_STRIDE
+    uint32_t *list_cnt;          // [B*H_q] at stride CNT_STRIDE
+    double *hist;                // [B*H_q][HSTRIDE]: bin sums, then octave sums
     Resolve *res;                // [B*H_q]
     uint16_t *tilebin;           // [B*H_kv][ntile][GMAX]: per tile, 1 + largest bin of each head (0: none)
     unsigned long long *cands;   // [B*H_q][N_max]
@@ -159,8 +215,7 @@ struct SelArgs {
     int ntile;
     int ctas;                    // scan/collect CTAs per (b, g)
     long long chunk;             // tokens per CTA, multiple of TILE
-    int cl_ctas;                 // collect_mma_kernel CTAs per (b, g)
-    long long cl_chunk;          // its tokens per CTA, multiple of TILE
+    int cl_ctas;                 // collect_mma_kernel CTAs per pair of groups; the pair's tile i goes to CTA i mod cl_ctas
     const int32_t *seq_lens;
     int n_ret;
     int ret_g[MAX_RET_GROUPS];
@@ -183,7 +238,7 @@ struct SelArgs {
     const __nv_bfloat16 *v_cache;
     float attn_scale_log2;
     float *out;                          // [B, H_q, D]
-    float *part_sel;                     // [collect CTAs][GMAX][PSTRIDE]
+    float *part_sel;                     // [collect CTAs][2 GMAX][PSTRIDE] (pair-heads)
     uint32_t *ovf;                       // [B*H_q]
 };
 
@@ -233,6 +288,15 @@ struct WarpPart {
 // The warp attends up to 8 rows of one head: lane u < 8 holds row id `id`
 // (-1: none), all 16 row loads in flight before the dot products.  qx: the
 // lane's 4 query dims times the softmax scale times log2(e).
+// Pulls the K and V rows of one token (bf16, D = 128: two 128-byte lines
+// each) toward L2, so that a later gather of the row finds it there.
+__device__ __forceinline__ void prefetch_kv_l2(const __nv_bfloat16 *k_row, const __nv_bfloat16 *v_row) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(k_row));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(k_row + 64));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(v_row));
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(v_row + 64));
+}
+
 __device__ __forceinline__ void attend8(const __nv_bfloat16 *kb, const __nv_bfloat16 *vb, int id,
                                         const float (&qx)[4], WarpPart &p) {
     const int lane = threadIdx.x & 31;
@@ -278,14 +342,16 @@ __device__ __forceinline__ void attend8(const __nv_bfloat16 *kb, const __nv_bflo
     p.m = mn;
 }
 
-__device__ __forceinline__ int valid_len(const int32_t *seq_lens, int b, long long N_max,
-                                         uint32_t *status) {
-    int N = seq_lens[b];
+__device__ __forceinline__ int checked_len(int N, long long N_max, uint32_t *status) {
     if (N < 1 || (long long)N > N_max) {
         set_status(status, RTP_ERR_DEVICE_ARG);
         return 0;
     }
     return N;
+}
+__device__ __forceinline__ int valid_len(const int32_t *seq_lens, int b, long long N_max,
+                                         uint32_t *status) {
+    return checked_len(seq_lens[b], N_max, status);
 }
 
 // q_idx of the group's heads into shared memory.  Output o = h * R + j
@@ -504,57 +570,56 @@ template <typename Src> struct NeedsQ : std::true_type {};
 template <> struct NeedsQ<SrcBuffer> : std::false_type {};
 
 // ---------------------------------------------------------------------------
-// resolve one head's histogram (one warp): R = U(top bin), bin masses
-// S_b exp(U_b - R) in fp64, the boundary bin where the mass accumulated
-// from the top first reaches p Z.  Zeroes the histogram for the next call.
+// Resolve one head from its level-1 histogram `gh` (global memory, all of the
+// scan's CTAs done).  One warp, two rounds of loads: first the 32 octave
+// sums (lane s: octave s), which fix the total mass Z and the octave where
+// the mass accumulated from the top first reaches p Z; then the 16 bins of
+// that octave (lanes 0-15) and of the top octave (lanes 16-31).  R = upper
+// edge of the top non-empty bin; all masses are returned relative to it.  In
+// descending bin order b* is the first bin where the cumulative mass reaches
+// p Z; `above` is the mass of the bins before it and `target` what b* must
+// still supply (infinite: all of b*).  Every lane returns the same record.
+// Octave factors are taken in fp64 (octaves can lie hundreds of nats apart);
+// bin factors within the boundary octave use the same fp32 expression as
+// finalize.
 // ---------------------------------------------------------------------------
-// Resolve one head from its level-1 histogram `gh` (global memory, all of
-// the group's scan CTAs done).  One warp; lane l holds bins 16 l .. 16 l + 15
-// in registers (one round of loads).  Bin masses are taken relative to the
-// upper edge R of the top non-empty bin; in descending bin order the first
-// bin where the cumulative mass reaches p Z is b*, `above` is the mass of
-// the bins before it and `target` what b* must still supply (infinite: all
-// of b*).  Every lane returns the same record.
 __device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, float p, int N) {
-    constexpr int SEG = NBIN / 32;
     const int lane = threadIdx.x & 31;
-    // bin sums, rounded to fp32 (relative error 2^-24 per bin; the cut and
-    // the masses downstream are accurate to far better than 1e-5 of Z)
-    float v[SEG];
+    constexpr double L2E_D = 1.4426950408889634;
+    double ss = 0.0;
 #pragma unroll
-    for (int j = 0; j < SEG; j += 2) {
-        const double2 t = __ldcg(reinterpret_cast<const double2 *>(gh + lane * SEG + j));
-        v[j] = (float)t.x;
-        v[j + 1] = (float)t.y;
-    }
-    int top = -1, low = NBIN;
-#pragma unroll
-    for (int j = 0; j < SEG; ++j)
-        if (v[j] > 0.0f) { top = lane * SEG + j; low = min(low, lane * SEG + j); }
-    top = __reduce_max_sync(0xffffffffu, top);
-    low = __reduce_min_sync(0xffffffffu, low);
+    for (int q = 0; q < NREP; ++q) ss += __ldcg(gh + NBIN + q * NSUP + lane);
+    const unsigned ne = __ballot_sync(0xffffffffu, ss > 0.0);
     Resolve r;
     r.N = N;
-    if (top < 0 || N == 0) {
+    if (!ne || N == 0) {
         r.Z = 0; r.above = 0; r.target = 0; r.R = 0.f; r.bstar = -1; r.mode = MODE_EMPTY;
         return r;
     }
-    const float R = bin_upper(top);
-    double seg = 0.0;
-#pragma unroll
-    for (int j = 0; j < SEG; ++j) {
-        v[j] = v[j] > 0.0f ? v[j] * ex2_sfu((bin_upper(lane * SEG + j) - R) * 1.4426950408889634f) : 0.0f;
-        seg += (double)v[j];
-    }
-    // inclusive suffix sums over lanes: mass of this lane's bins and all above
-    double incl = seg;
+    const int stop = 31 - __clz(ne), slow = __ffs(ne) - 1;
+    const float R0 = bin_upper(16 * stop + 15);
+    // octave masses relative to R0, inclusive suffix sums from the top octave
+    const double ms = ss > 0.0 ? ss * exp2_wide((double)(bin_upper(16 * lane + 15) - R0) * L2E_D) : 0.0;
+    double incl = ms;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
         const double t = __shfl_down_sync(0xffffffffu, incl, o);
         if (lane + o < 32) incl += t;
     }
-    const double Z = __shfl_sync(0xffffffffu, incl, 0);
-    const double excl = incl - seg;
+    const double Z0 = __shfl_sync(0xffffffffu, incl, 0);
+    const double target0 = p >= 1.0f ? 0.0 : p <= 0.0f ? 0.0 : (double)p * Z0;
+    const unsigned hit = __ballot_sync(0xffffffffu, ms > 0.0 && incl >= target0);
+    // boundary octave (rounding kept p Z out of reach: the lowest octave)
+    const int sb = hit ? 31 - __clz(hit) : slow;
+    const double above0 = __shfl_sync(0xffffffffu, incl - ms, sb);
+    // second round: bins of the boundary octave and of the top octave
+    const int bin = lane < 16 ? 16 * sb + lane : 16 * stop + (lane - 16);
+    const double sv = __ldcg(gh + bin);
+    const unsigned nt = __ballot_sync(0xffffffffu, lane >= 16 && sv > 0.0) >> 16;
+    const int btop = 16 * stop + (nt ? 31 - __clz(nt) : 15);
+    const float R = bin_upper(btop);
+    const double sc = exp2_wide((double)(R0 - R) * L2E_D);       // R0 units -> R units (>= 1)
+    const double Z = Z0 * sc;
     r.Z = Z;
     r.R = R;
     if (p >= 1.0f) {
@@ -562,41 +627,26 @@ __device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, f
         return r;
     }
     const double target = p <= 0.0f ? 0.0 : (double)p * Z;
-    const unsigned hit = __ballot_sync(0xffffffffu, seg > 0.0 && incl >= target);
-    int bstar = -1;
-    double above = 0.0, tin = INFINITY;
-    if (hit) {
-        const int L = 31 - __clz(hit);            // highest bins first
-        if (lane == L) {
-            double cum = excl;
-            bool done = false;
+    // the boundary octave's bins relative to R (lane 15 = its highest bin),
+    // inclusive suffix sums on top of the octaves above
+    const double mb = lane < 16 && sv > 0.0
+                          ? sv * (double)ex2_sfu((bin_upper(bin) - R) * 1.4426950408889634f) : 0.0;
+    double incb = mb;
 #pragma unroll
-            for (int j = SEG - 1; j >= 0; --j) {
-                if (done || !(v[j] > 0.0f)) continue;
-                bstar = lane * SEG + j;           // if rounding never crosses, the last bin is kept whole
-                above = cum;
-                if (cum + (double)v[j] >= target) { tin = target - cum; done = true; }
-                else { cum += (double)v[j]; tin = INFINITY; }
-            }
-        }
-        bstar = __shfl_sync(0xffffffffu, bstar, L);
-        above = __shfl_sync(0xffffffffu, above, L);
-        tin = __shfl_sync(0xffffffffu, tin, L);
-    } else {
-        // rounding kept p Z out of reach: keep everything down to the lowest bin
-        double m_low = 0.0;
-#pragma unroll
-        for (int j = 0; j < SEG; ++j)
-            if (lane * SEG + j == low) m_low = (double)v[j];
-        m_low = __shfl_sync(0xffffffffu, m_low, low / SEG);
-        bstar = low;
-        above = Z - m_low;
-        tin = INFINITY;
+    for (int o = 1; o < 16; o <<= 1) {
+        const double t = __shfl_down_sync(0xffffffffu, incb, o);
+        if (lane + o < 16) incb += t;
     }
+    incb += above0 * sc;
+    const unsigned hb = __ballot_sync(0xffffffffu, lane < 16 && mb > 0.0 && incb >= target);
+    const unsigned nb = __ballot_sync(0xffffffffu, lane < 16 && mb > 0.0);
+    // b*: the highest bin whose cumulative mass reaches p Z; if rounding kept
+    // it out of reach, the octave's lowest non-empty bin, kept whole
+    const int L = hb ? 31 - __clz(hb) : nb ? __ffs(nb) - 1 : 0;
     r.mode = MODE_NORMAL;
-    r.bstar = bstar;
-    r.above = above;
-    r.target = tin;
+    r.bstar = 16 * sb + L;
+    r.above = __shfl_sync(0xffffffffu, incb - mb, L);
+    r.target = hb ? target - r.above : INFINITY;
     return r;
 }
 
@@ -612,6 +662,7 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(SelArgs a, SelWs w) 
     __shared__ __align__(16) float qs[GMAX * R];
     __shared__ __align__(16) uint32_t shl[2 * GMAX * NBIN];   // fixed-point bin sums: low words, then high words
     uint32_t *const shh = shl + GMAX * NBIN;
+    __shared__ double s_fac[NBIN];                               // octave factors
     __shared__ int s_err;
     const int b = blockIdx.y / a.n_ret;
     const int g = a.ret_g[blockIdx.y % a.n_ret];
@@ -622,11 +673,12 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(SelArgs a, SelWs w) 
     if (threadIdx.x == 0) s_err = 0;
     // this call's collect pass appends from zero
     if (blockIdx.x == 0 && threadIdx.x < G) {
-        w.cand_cnt[bh0 + threadIdx.x] = 0u;
-        w.list_cnt[bh0 + threadIdx.x] = 0u;
+        w.cand_cnt[(bh0 + threadIdx.x) * CNT_STRIDE] = 0u;
+        w.list_cnt[(bh0 + threadIdx.x) * CNT_STRIDE] = 0u;
         if (a.ovf) a.ovf[bh0 + threadIdx.x] = 0u;
     }
     for (int i = threadIdx.x; i < 2 * GMAX * NBIN; i += blockDim.x) shl[i] = 0u;
+    for (int i = threadIdx.x; i < NBIN; i += blockDim.x) s_fac[i] = octave_factor(i);
     if constexpr (NeedsQ<Src>::value) {
         project_query<(GMAX * R + SCAN_WARPS - 1) / SCAN_WARPS>(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D,
                                                                a.idx_scale, qs, G, warp, SCAN_WARPS);
@@ -702,11 +754,9 @@ __global__ void __launch_bounds__(SCAN_THREADS) scan_kernel(SelArgs a, SelWs w) 
     if (err) s_err = 1;
     __syncthreads();
     if (s_err && threadIdx.x == 0) set_status(w.status, RTP_ERR_RANGE);
-    for (int i = threadIdx.x; i < G * NBIN; i += blockDim.x) {
-        const uint32_t lo = shl[i], hi = shh[i];
-        if (lo | hi)
-            atomicAdd(&w.hist[bh0 * NBIN + i], ((double)hi * 4294967296.0 + (double)lo) * (1.0 / FX_ONE));
-    }
+    flush_hist(w.hist + bh0 * HSTRIDE, G, s_fac, blockIdx.x % NREP, [&](int i) {
+        return fixed_to_double(((unsigned long long)shh[i] << 32) | shl[i], 1.0 / FX_ONE);
+    });
 }
 
 // ---------------------------------------------------------------------------
@@ -754,10 +804,11 @@ __device__ __forceinline__ int scan_value(float z, uint32_t row, int &bin) {
 // Producer of a TMA ring (lane 0 of the producer warp): streams the index
 // keys of tokens [t_lo, t_hi) stage by stage into `ring` (ST_TOK tokens per
 // stage).  Waits are bounded: on a timeout it records RTP_ERR_TIMEOUT and
-// sets *abort.  Before returning it waits for its own copies still in flight.
+// sets *abort.  Returns the number of stages issued; ring_drain then waits
+// for the copies still in flight (none may land after the CTA exits).
 template <int NS>
-__device__ __forceinline__ void ring_produce(int t_lo, int t_hi, const __nv_bfloat16 *rows, uint8_t *ring,
-                                             uint64_t *full, uint64_t *empty, uint32_t *status, int *abort) {
+__device__ __forceinline__ int ring_produce(int t_lo, int t_hi, const __nv_bfloat16 *rows, uint8_t *ring,
+                                            uint64_t *full, uint64_t *empty, uint32_t *status, int *abort) {
     const int n_st = t_hi > t_lo ? (t_hi - t_lo + ST_TOK - 1) / ST_TOK : 0;
     int issued = 0;
     for (int it = 0; it < n_st; ++it) {
@@ -775,7 +826,10 @@ __device__ __forceinline__ void ring_produce(int t_lo, int t_hi, const __nv_bflo
         bulk_g2s(ring + st * ST_BYTES, rows + (size_t)tok0 * R, bytes, &full[st]);
         issued = it + 1;
     }
-    // no copy may still be landing in shared memory when the CTA exits
+    return issued;
+}
+template <int NS>
+__device__ __forceinline__ void ring_drain(uint64_t *full, int issued) {
     for (int it = max(0, issued - NS); it < issued; ++it)
         mbar_wait(&full[it % NS], (uint32_t)((it / NS) & 1));
 }
@@ -788,6 +842,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
     uint64_t *full = reinterpret_cast<uint64_t *>(dsm + NSTAGE * ST_BYTES + GMAX * NBIN * 12);
     uint64_t *empty = full + NSTAGE;
     __shared__ __align__(16) float qs[GMAX * R];
+    __shared__ double s_fac[NBIN];              // octave factors (the producer warp's idle lanes)
     __shared__ int s_err, s_abort;
     const int b = blockIdx.y / a.n_ret;
     const int g = a.ret_g[blockIdx.y % a.n_ret];
@@ -804,12 +859,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
     for (int i = threadIdx.x; i < GMAX * NBIN; i += blockDim.x) { h32[i] = 0u; h64[i] = 0ull; }
     pdl_wait();
     pdl_trigger();
-    // this call's collect pass appends from zero
-    if (blockIdx.x == 0 && threadIdx.x < G) {
-        w.cand_cnt[bh0 + threadIdx.x] = 0u;
-        w.list_cnt[bh0 + threadIdx.x] = 0u;
-        if (a.ovf) a.ovf[bh0 + threadIdx.x] = 0u;
-    }
     // the consumers' q_idx loads go out before the producer's first bulk copy
     QProj<(GMAX * R + TC_WARPS - 1) / TC_WARPS> qp;
     if (warp < TC_WARPS) qp.load(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D, G, warp, TC_WARPS);
@@ -821,14 +870,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
     const __nv_bfloat16 *rows = reinterpret_cast<const __nv_bfloat16 *>(a.kidx) + bg * a.N_max * R;
 
     if (warp == TC_WARPS) {
+        // lane 0 streams; once it has issued the last stage the other lanes
+        // fill the octave factor table (needed only by the flush) while lane
+        // 0 waits for its copies in flight
+        int issued = 0;
+        if (lane == 0) issued = ring_produce<NSTAGE>(t_lo, t_hi, rows, ring, full, empty, w.status, &s_abort);
+        __syncwarp();
         if (lane == 0)
-            ring_produce<NSTAGE>(t_lo, t_hi, rows, ring, full, empty, w.status, &s_abort);
+            ring_drain<NSTAGE>(full, issued);
+        else
+            for (int i = lane - 1; i < NBIN; i += 31) s_fac[i] = octave_factor(i);
     } else {
         // consumers: finish q_idx of the group (the producer is already streaming)
         qp.store(a.idx_scale, qs, G, warp, TC_WARPS);
         asm volatile("bar.sync 1, %0;" ::"r"(TC_WARPS * 32) : "memory");
-        if (blockIdx.x == 0)
+        // q_idx for the collect pass, and its counters from zero (these
+        // stores come after the barriers of the prologue, which would wait
+        // for them)
+        if (blockIdx.x == 0) {
             for (int i = threadIdx.x; i < G * R; i += TC_WARPS * 32) w.qidx[bh0 * R + i] = qs[i];
+            if (threadIdx.x < G) {
+                w.cand_cnt[(bh0 + threadIdx.x) * CNT_STRIDE] = 0u;
+                w.list_cnt[(bh0 + threadIdx.x) * CNT_STRIDE] = 0u;
+                if (a.ovf) a.ovf[bh0 + threadIdx.x] = 0u;
+            }
+        }
         SrcMma src;
         src.init(rows, a.N_max, qs, G);
         const int gid = lane >> 2, tig = lane & 3;
@@ -914,10 +980,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
     }
     __syncthreads();
     if (s_err && threadIdx.x == 0) set_status(w.status, RTP_ERR_RANGE);
-    for (int i = threadIdx.x; i < G * NBIN; i += blockDim.x) {
-        const unsigned long long v = h64[i] + h32[i];
-        if (v) atomicAdd(&w.hist[bh0 * NBIN + i], (double)v * (1.0 / FX18));
-    }
+    flush_hist(w.hist + bh0 * HSTRIDE, G, s_fac, blockIdx.x % NREP,
+               [&](int i) { return fixed_to_double(h64[i] + h32[i], 1.0 / FX18); });
 }
 
 // ---------------------------------------------------------------------------
@@ -965,7 +1029,7 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
     if (warp < GMAX) {
         int mode = MODE_EMPTY, bs = NBIN;
         if (warp < G) {
-            const Resolve r = resolve_head(w.hist + (bh0 + warp) * NBIN, a.p, N);
+            const Resolve r = resolve_head(w.hist + (bh0 + warp) * HSTRIDE, a.p, N);
             if (blockIdx.x == 0 && lane == 0) w.res[bh0 + warp] = r;
             mode = r.mode;
             bs = r.bstar;
@@ -1033,7 +1097,7 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
                             if (p < (unsigned)KCAP) {
                                 s_kbuf[h * KCAP + p] = t;
                             } else {
-                                const unsigned q = atomicAdd(&w.list_cnt[bh0 + h], 1u);
+                                const unsigned q = atomicAdd(&w.list_cnt[(bh0 + h) * CNT_STRIDE], 1u);
                                 a.lists[(bh0 + h) * a.N_max + q] = t;
                             }
                         } else if (zz >= s_clo[h]) {
@@ -1043,7 +1107,7 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
                             if (p < (unsigned)CCAP) {
                                 s_cbuf[h * CCAP + p] = key;
                             } else {
-                                const unsigned q = atomicAdd(&w.cand_cnt[bh0 + h], 1u);
+                                const unsigned q = atomicAdd(&w.cand_cnt[(bh0 + h) * CNT_STRIDE], 1u);
                                 w.cands[(bh0 + h) * a.N_max + q] = key;
                             }
                         }
@@ -1063,8 +1127,8 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
         const unsigned ncd = min(s_cc[warp], (unsigned)CCAP);
         unsigned kb = 0u, cb = 0u;
         if (lane == 0) {
-            if (nk) kb = atomicAdd(&w.list_cnt[bh], nk);
-            if (ncd) cb = atomicAdd(&w.cand_cnt[bh], ncd);
+            if (nk) kb = atomicAdd(&w.list_cnt[bh * CNT_STRIDE], nk);
+            if (ncd) cb = atomicAdd(&w.cand_cnt[bh * CNT_STRIDE], ncd);
         }
         kb = __shfl_sync(0xffffffffu, kb, 0);
         cb = __shfl_sync(0xffffffffu, cb, 0);
@@ -1074,128 +1138,152 @@ __global__ void __launch_bounds__(COL_THREADS) collect_kernel(SelArgs a, SelWs w
 }
 
 // ---------------------------------------------------------------------------
-// collect for bf16 index keys.  Every CTA first resolves the group's heads
-// from the finished histograms (warp h: head h; the group's first CTA
-// records them for finalize) while its other warps load q_idx and every warp
-// loads the scan's tile records of its first window.  Warp w then owns
-// tiles w, w + CL_WARPS, ... of the CTA's range, screened 32 at a time by
-// their records (a tile is needed when some head's largest bin in it
-// reaches b*); the needed ones are loaded CL_BATCH at a time, all loads in
-// flight, their logits recomputed with the scan's tensor-core arithmetic,
-// and kept ids (z above b*) and b*'s candidates staged per head.
-// grid = the scan's, CL_THREADS threads.
+// collect for bf16 index keys.  The retrieval groups are taken in pairs
+// (groups 2p and 2p + 1 in (b, g) order; with an odd count the last pair has
+// one): the CTAs of a pair share its tiles, so a group with many needed
+// tiles borrows its partner's CTAs.  Every CTA first resolves the pair's
+// heads from the finished histograms (warp w: pair-head w = head w mod GMAX
+// of the pair's group w / GMAX; the pair's first CTA records them for
+// finalize) while loading q_idx and the tile records of its first window.
+// The pair's tiles (its first group's, then its second's) are dealt to its
+// CTAs round-robin; warp w of a CTA takes its tiles w, w + CL_WARPS, ...,
+// screened 32 at a time by their records (a tile is needed when some head's
+// largest bin in it reaches b*).  The needed ones are loaded CL_BATCH at a
+// time, all loads in flight, and their logits recomputed with the scan's
+// tensor-core arithmetic; one compare per value finds those at or above the
+// floor of the head's boundary bin, and only these are sorted into kept ids
+// (z above b*) and b*'s candidates, staged per pair-head.
+// grid = (cl_ctas, pairs), CL_THREADS threads.
 // ---------------------------------------------------------------------------
 constexpr int CL_WARPS = 16;
 constexpr int CL_THREADS = CL_WARPS * 32;
 constexpr int CL_BATCH = 4;
-constexpr int CL_KCAP = 1024;     // kept ids staged per head per CTA
-static_assert(GMAX * D % CL_THREADS == 0 && GMAX * R <= CL_THREADS && CL_WARPS >= GMAX,
-              "collect prologue: load split, one resolving warp per head slot");
-// dynamic shared memory: staged kept ids, scaled q_rope of the group, and one
-// partial record per (warp, head) for the fused attention
-constexpr int CL_SMEM = GMAX * CL_KCAP * 4 + GMAX * D * 4 + CL_WARPS * GMAX * PSTRIDE * 4;
+constexpr int PAIR = 2;                    // retrieval groups per collect CTA
+constexpr int HP = PAIR * GMAX;            // pair-heads: group-in-pair * GMAX + head
+constexpr int CL_KCAP = 512;               // kept ids staged per pair-head per CTA
+constexpr int CL_SLOTS = 32;               // attention partial slots (one round of heads)
+static_assert(CL_WARPS == HP, "one resolving and one flushing warp per pair-head");
+static_assert(HP * D % CL_THREADS == 0 && HP * R <= CL_THREADS, "collect prologue load split");
+static_assert(CL_SLOTS >= CL_WARPS, "a round holds every warp's partial of any one head");
+// dynamic shared memory: staged kept ids and candidates, the scaled q_rope of
+// the pair's heads, and the attention partial slots
+constexpr int CL_SMEM = HP * CL_KCAP * 4 + HP * CCAP * 8 + HP * D * 4 + CL_SLOTS * PSTRIDE * 4;
 
 __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, SelWs w) {
     extern __shared__ __align__(16) uint8_t csm[];
-    int32_t *s_kbuf = reinterpret_cast<int32_t *>(csm);                       // [GMAX][CL_KCAP]
-    float *s_qr = reinterpret_cast<float *>(csm + GMAX * CL_KCAP * 4);         // [GMAX][D]
-    float *s_slot = s_qr + GMAX * D;                                            // [CL_WARPS][GMAX][PSTRIDE]
-    __shared__ __align__(16) float qs[GMAX * R];
-    __shared__ int s_bstar[GMAX];
-    __shared__ unsigned s_kc[GMAX], s_cc[GMAX];
-    __shared__ float s_khi[GMAX], s_clo[GMAX];      // keep: z > s_khi; candidate: s_clo <= z <= s_khi
-    __shared__ unsigned long long s_cbuf[GMAX * CCAP];
-    const int b = blockIdx.y / a.n_ret;
-    const int g = a.ret_g[blockIdx.y % a.n_ret];
+    int32_t *s_kbuf = reinterpret_cast<int32_t *>(csm);                                          // [HP][CL_KCAP]
+    unsigned long long *s_cbuf = reinterpret_cast<unsigned long long *>(csm + HP * CL_KCAP * 4);  // [HP][CCAP]
+    float *s_qr = reinterpret_cast<float *>(csm + HP * CL_KCAP * 4 + HP * CCAP * 8);              // [HP][D]
+    float *s_slot = s_qr + HP * D;                                                                  // [CL_SLOTS][PSTRIDE]
+    __shared__ __align__(16) float qs[PAIR][GMAX * R];
+    __shared__ int s_bstar[HP];
+    __shared__ unsigned s_kc[HP], s_cc[HP];
+    __shared__ float s_khi[HP], s_clo[HP];      // keep: z > s_khi; candidate: s_clo <= z <= s_khi
+    __shared__ Resolve s_res[HP];               // the pair's first CTA records them at the end
     const int G = a.G;
-    const size_t bg = (size_t)b * a.H_kv + g;
-    const size_t bh0 = (size_t)b * a.H_q + (size_t)g * G;
+    const int groups = a.B * a.n_ret;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (threadIdx.x < GMAX) { s_kc[threadIdx.x] = 0u; s_cc[threadIdx.x] = 0u; }
-    pdl_wait();
-    pdl_trigger();
-    const int N = valid_len(a.seq_lens, b, a.N_max, w.status);
-    const int t_lo = (int)((long long)blockIdx.x * a.cl_chunk);
-    const int t_hi = (int)min((long long)N, (long long)t_lo + a.cl_chunk);
-    const uint4 *recs = reinterpret_cast<const uint4 *>(w.tilebin + bg * a.ntile * GMAX);
-    // tile of lane `lane` in window `win` of this warp
-    auto tile_of = [&](int win) { return t_lo / TILE + warp + (win * 32 + lane) * CL_WARPS; };
-    const int ti_end = (t_hi + TILE - 1) / TILE;
-    uint4 rec = make_uint4(0u, 0u, 0u, 0u);
-    if (t_hi > t_lo && tile_of(0) < ti_end) rec = __ldcg(recs + tile_of(0));
-    // q_idx and (fused attention) the scaled q_rope of the group: loads first,
-    // stored to shared memory after the resolve
-    constexpr int QR_PER = GMAX * D / CL_THREADS;
-    const float qv = threadIdx.x < G * R ? w.qidx[bh0 * R + threadIdx.x] : 0.0f;
+    const int C = gridDim.x, cx = blockIdx.x;
+    // the pair's groups: group y = b * n_ret + i is (b, ret_g[i])
+    const int y0 = PAIR * blockIdx.y, y1 = y0 + 1;
+    const bool has1 = y1 < groups;
+    const int b0 = y0 / a.n_ret, b1 = has1 ? y1 / a.n_ret : b0;
+    const int g0 = a.ret_g[y0 % a.n_ret], g1 = has1 ? a.ret_g[y1 % a.n_ret] : g0;
+    const size_t bg0 = (size_t)b0 * a.H_kv + g0, bg1 = (size_t)b1 * a.H_kv + g1;
+    const size_t bh00 = (size_t)b0 * a.H_q + (size_t)g0 * G, bh01 = (size_t)b1 * a.H_q + (size_t)g1 * G;
+    // pair-head ph is valid when its group exists and its head is < G
+    auto ph_ok = [&](int ph) { return (ph < GMAX || has1) && ph % GMAX < G; };
+    auto ph_bh = [&](int ph) { return (ph < GMAX ? bh00 : bh01) + ph % GMAX; };
+    if (threadIdx.x < HP) { s_kc[threadIdx.x] = 0u; s_cc[threadIdx.x] = 0u; }
+    // inputs of the call (no earlier kernel writes them) load before the wait
+    const int n0 = a.seq_lens[b0], n1 = has1 ? a.seq_lens[b1] : 0;
+    constexpr int QR_PER = HP * D / CL_THREADS;
     float qrv[QR_PER];
 #pragma unroll
     for (int k = 0; k < QR_PER; ++k) {
-        const int i = threadIdx.x + k * CL_THREADS;
-        qrv[k] = a.q_rope && i < G * D ? a.q_rope[bh0 * D + i] : 0.0f;
+        const int i = threadIdx.x + k * CL_THREADS, ph = i / D;
+        qrv[k] = a.q_rope && ph_ok(ph) ? a.q_rope[ph_bh(ph) * D + i % D] : 0.0f;
+    }
+    pdl_wait();
+    pdl_trigger();
+    const int N0 = checked_len(n0, a.N_max, w.status);
+    const int N1 = has1 ? checked_len(n1, a.N_max, w.status) : 0;
+    const int nt0 = (N0 + TILE - 1) / TILE;
+    const int ntot = nt0 + (N1 + TILE - 1) / TILE;
+    const uint4 *recs0 = reinterpret_cast<const uint4 *>(w.tilebin + bg0 * a.ntile * GMAX);
+    const uint4 *recs1 = reinterpret_cast<const uint4 *>(w.tilebin + bg1 * a.ntile * GMAX);
+    // The pair's tile T (< ntot) is tile T of its first group, or T - nt0 of
+    // its second; tile T goes to CTA T mod C.  Tile of lane `lane` in window
+    // `win` of this warp:
+    auto tile_of = [&](int win) { return cx + C * (warp + (win * 32 + lane) * CL_WARPS); };
+    uint4 rec = make_uint4(0u, 0u, 0u, 0u);
+    {
+        const int T = tile_of(0);
+        if (T < ntot) rec = __ldcg(T < nt0 ? recs0 + T : recs1 + (T - nt0));
+    }
+    // q_idx of the pair's heads (the scan wrote it): loaded now, stored to
+    // shared memory after the resolve, with the scaled q_rope
+    float qv = 0.0f;
+    {
+        const int i = threadIdx.x, ph = i / R;
+        if (i < HP * R && ph_ok(ph)) qv = w.qidx[ph_bh(ph) * R + i % R];
     }
     {
         int bs = NBIN, mode = MODE_EMPTY;
-        if (warp < G) {
-            const Resolve r = resolve_head(w.hist + (bh0 + warp) * NBIN, a.p, N);
-            if (blockIdx.x == 0 && lane == 0) w.res[bh0 + warp] = r;
+        if (ph_ok(warp)) {
+            const size_t bh = ph_bh(warp);
+            const Resolve r = resolve_head(w.hist + bh * HSTRIDE, a.p, warp < GMAX ? N0 : N1);
+            if (cx == 0 && lane == 0) s_res[warp] = r;
             mode = r.mode;
             bs = r.bstar;
         }
-        if (lane == 0 && warp < GMAX) {
+        if (lane == 0) {
             // keep-all heads need no collect pass: finalize lists every token
             s_bstar[warp] = mode == MODE_NORMAL ? bs : NBIN;
             s_khi[warp] = mode == MODE_NORMAL ? bin_hi_incl(bs) : INFINITY;
             s_clo[warp] = mode == MODE_NORMAL ? bin_lo_incl(bs) : INFINITY;
         }
     }
-    if (threadIdx.x < G * R) qs[threadIdx.x] = qv;
+    if (threadIdx.x < HP * R) (&qs[0][0])[threadIdx.x] = qv;
 #pragma unroll
-    for (int k = 0; k < QR_PER; ++k) {
-        const int i = threadIdx.x + k * CL_THREADS;
-        if (i < G * D) s_qr[i] = qrv[k] * a.attn_scale_log2;
-    }
+    for (int k = 0; k < QR_PER; ++k) s_qr[threadIdx.x + k * CL_THREADS] = qrv[k] * a.attn_scale_log2;
     __syncthreads();
-    if (t_hi <= t_lo) {
-        // an empty range: empty partials for the fused attention
-        if (a.q_rope) {
-            const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
-            for (int i = threadIdx.x; i < G * PSTRIDE; i += blockDim.x) {
-                const int h = i / PSTRIDE, j = i % PSTRIDE;
-                a.part_sel[(cta * GMAX + h) * PSTRIDE + j] = j == 0 ? -INFINITY : 0.0f;
-            }
-        }
+    const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+    if (cx >= ntot) {
+        // no tile for this CTA: empty partials for the fused attention
+        if (cx == 0 && lane == 0 && ph_ok(warp)) w.res[ph_bh(warp)] = s_res[warp];
+        if (a.q_rope)
+            for (int i = threadIdx.x; i < HP * PSTRIDE; i += blockDim.x)
+                a.part_sel[cta * HP * PSTRIDE + i] = i % PSTRIDE == 0 ? -INFINITY : 0.0f;
         return;
     }
-    const __nv_bfloat16 *rows = reinterpret_cast<const __nv_bfloat16 *>(a.kidx) + bg * a.N_max * R;
-    SrcMma src;
-    src.init(rows, a.N_max, qs, G);
-    const int tig = lane & 3;
-    int bst[GMAX];
-#pragma unroll
-    for (int h = 0; h < GMAX; ++h) bst[h] = h < G ? s_bstar[h] : NBIN;
-    // thresholds of the lane's two head slots (heads 2 tig, 2 tig + 1):
-    // kept  khi < z < Z_LIMIT, candidate  clo <= z <= khi and z < Z_LIMIT,
-    // with khi and clo raised so that z > -Z_LIMIT too (|z| < Z_LIMIT is the
-    // binned range; -255.99998 is the smallest float above -Z_LIMIT)
-    float khi[2], clo[2];
-#pragma unroll
-    for (int sl = 0; sl < 2; ++sl) {
-        const int h = 2 * tig + sl;
-        khi[sl] = h < G ? fmaxf(s_khi[h], -Z_LIMIT) : INFINITY;
-        clo[sl] = h < G ? fmaxf(s_clo[h], -255.99998f) : INFINITY;
-    }
+    const __nv_bfloat16 *rows0 = reinterpret_cast<const __nv_bfloat16 *>(a.kidx) + bg0 * a.N_max * R;
+    const __nv_bfloat16 *rows1 = reinterpret_cast<const __nv_bfloat16 *>(a.kidx) + bg1 * a.N_max * R;
+    SrcMma src0, src1;
+    src0.init(rows0, a.N_max, qs[0], G);
+    src1.init(rows1, a.N_max, qs[1], G);
+    const int gid = lane >> 2, tig = lane & 3;
+    // thresholds of the lane's two head slots (heads 2 tig, 2 tig + 1) in
+    // either group: kept z > khi, candidate clo <= z <= khi
+    const float khi00 = s_khi[2 * tig], khi01 = s_khi[2 * tig + 1];
+    const float khi10 = s_khi[GMAX + 2 * tig], khi11 = s_khi[GMAX + 2 * tig + 1];
+    const float clo00 = s_clo[2 * tig], clo01 = s_clo[2 * tig + 1];
+    const float clo10 = s_clo[GMAX + 2 * tig], clo11 = s_clo[GMAX + 2 * tig + 1];
 
-    for (int win = 0; t_lo / TILE + warp + win * 32 * CL_WARPS < ti_end; ++win) {
-        if (win > 0) rec = tile_of(win) < ti_end ? __ldcg(recs + tile_of(win)) : make_uint4(0u, 0u, 0u, 0u);
-        // heads whose largest bin in lane's tile reaches their b*
+    for (int win = 0; cx + C * (warp + win * 32 * CL_WARPS) < ntot; ++win) {
+        const int T = tile_of(win);
+        const int tg = T < nt0 ? 0 : 1;                     // the lane's tile: group in pair, tile index
+        const int ti = T - (tg ? nt0 : 0);
+        if (win > 0) rec = T < ntot ? __ldcg(tg ? recs1 + ti : recs0 + ti) : make_uint4(0u, 0u, 0u, 0u);
+        // heads whose largest bin in the lane's tile reaches their b*
         const uint32_t rw[4] = {rec.x, rec.y, rec.z, rec.w};
         unsigned hm = 0u;
 #pragma unroll
         for (int h = 0; h < GMAX; ++h) {
             const int tbmax = (int)((rw[h >> 1] >> (16 * (h & 1))) & 0xffffu) - 1;
-            if (tbmax >= bst[h]) hm |= 1u << h;
+            if (tbmax >= s_bstar[tg * GMAX + h]) hm |= 1u << h;
         }
-        if (tile_of(win) >= ti_end) hm = 0u;
+        if (T >= ntot) hm = 0u;
         unsigned todo = __ballot_sync(0xffffffffu, hm != 0u);
         while (todo) {
             // up to CL_BATCH needed tiles, all loads in flight
@@ -1205,151 +1293,171 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
             for (int k = 0; k < CL_BATCH; ++k) {
                 sel[k] = todo ? __ffs(todo) - 1 : -1;
                 if (todo) todo &= todo - 1u;
-                if (sel[k] >= 0) src.load(__shfl_sync(0xffffffffu, tile_of(win), sel[k]) * TILE, f[k]);
+                if (sel[k] >= 0) {
+                    const int gk = __shfl_sync(0xffffffffu, tg, sel[k]);
+                    const int tb = __shfl_sync(0xffffffffu, ti, sel[k]) * TILE;
+                    if (gk) src1.load(tb, f[k]); else src0.load(tb, f[k]);
+                }
             }
 #pragma unroll
             for (int k = 0; k < CL_BATCH; ++k) {
                 if (sel[k] < 0) break;
-                const int tb = __shfl_sync(0xffffffffu, tile_of(win), sel[k]) * TILE;
+                const int gk = __shfl_sync(0xffffffffu, tg, sel[k]);
+                const int tb = __shfl_sync(0xffffffffu, ti, sel[k]) * TILE;
                 const unsigned hmask = __shfl_sync(0xffffffffu, hm, sel[k]);
                 float z[SrcMma::NV];
-                src.eval(f[k], z);
-                // fast pass: bit v of km / cm marks value v as kept / candidate
-                const float khi0 = (hmask >> (2 * tig)) & 1u ? khi[0] : INFINITY;
-                const float khi1 = (hmask >> (2 * tig + 1)) & 1u ? khi[1] : INFINITY;
-                const float clo0 = (hmask >> (2 * tig)) & 1u ? clo[0] : INFINITY;
-                const float clo1 = (hmask >> (2 * tig + 1)) & 1u ? clo[1] : INFINITY;
-                unsigned km = 0u, cm = 0u;
+                if (gk) src1.eval(f[k], z); else src0.eval(f[k], z);
+                // fast pass: bit v marks a value at or above the floor of its
+                // head's boundary bin (heads whose tile maximum reaches b*)
+                const float cl0 = (hmask >> (2 * tig)) & 1u ? (gk ? clo10 : clo00) : INFINITY;
+                const float cl1 = (hmask >> (2 * tig + 1)) & 1u ? (gk ? clo11 : clo01) : INFINITY;
+                unsigned mk = 0u;
 #pragma unroll
-                for (int v = 0; v < SrcMma::NV; ++v) {
-                    const float zz = z[v];
-                    const float kh = (v & 1) ? khi1 : khi0, cl = (v & 1) ? clo1 : clo0;
-                    km |= (unsigned)(zz > kh && zz < Z_LIMIT) << v;
-                    cm |= (unsigned)(zz >= cl && zz <= kh && zz < Z_LIMIT) << v;
-                }
-                if (t_hi - tb < TILE) {
+                for (int v = 0; v < SrcMma::NV; ++v) mk |= (unsigned)(z[v] >= ((v & 1) ? cl1 : cl0)) << v;
+                const int Ng = gk ? N1 : N0;
+                if (Ng - tb < TILE) {
 #pragma unroll
                     for (int v = 0; v < SrcMma::NV; ++v)
-                        if (tb + src.tok(v) >= t_hi) { km &= ~(1u << v); cm &= ~(1u << v); }
+                        if (tb + src0.tok(v) >= Ng) mk &= ~(1u << v);
                 }
-                // rare pass: stage the marked values
-                while (km | cm) {
-                    const int v = __ffs(km | cm) - 1;
-                    const bool kept = (km >> v) & 1u;
-                    km &= ~(1u << v);
-                    cm &= ~(1u << v);
-                    const int h = src.head(src.slot(v));
-                    const int t = tb + src.tok(v);
-                    if (kept) {
-                        const unsigned p = atomicAdd(&s_kc[h], 1u);
+                // rare pass: kept (above the bin) or candidate (in it), staged
+                const float kh0 = gk ? khi10 : khi00, kh1 = gk ? khi11 : khi01;
+                while (mk) {
+                    const int v = __ffs(mk) - 1;
+                    mk &= mk - 1u;
+                    float zv = 0.0f;                      // z[v] without dynamic register indexing
+#pragma unroll
+                    for (int u = 0; u < SrcMma::NV; ++u) zv = u == v ? z[u] : zv;
+                    const int h = src0.head(src0.slot(v));
+                    const int ph = gk * GMAX + h;
+                    const size_t bh = (gk ? bh01 : bh00) + h;
+                    const int t = tb + src0.tok(v);
+                    if (zv > ((v & 1) ? kh1 : kh0)) {
+                        const unsigned p = atomicAdd(&s_kc[ph], 1u);
                         if (p < (unsigned)CL_KCAP) {
-                            s_kbuf[h * CL_KCAP + p] = t;
+                            s_kbuf[ph * CL_KCAP + p] = t;
                         } else {
-                            const unsigned q = atomicAdd(&w.list_cnt[bh0 + h], 1u);
-                            a.lists[(bh0 + h) * a.N_max + q] = t;
+                            const unsigned q = atomicAdd(&w.list_cnt[bh * CNT_STRIDE], 1u);
+                            a.lists[bh * a.N_max + q] = t;
                         }
                     } else {
-                        float zv = 0.0f;                  // z[v] without dynamic register indexing
-#pragma unroll
-                        for (int u = 0; u < SrcMma::NV; ++u) zv = u == v ? z[u] : zv;
                         const unsigned long long key = ((unsigned long long)logit_key(zv + 0.0f) << 32) |
                                                        (unsigned long long)(0xffffffffu - (uint32_t)t);
-                        const unsigned p = atomicAdd(&s_cc[h], 1u);
+                        const unsigned p = atomicAdd(&s_cc[ph], 1u);
                         if (p < (unsigned)CCAP) {
-                            s_cbuf[h * CCAP + p] = key;
+                            s_cbuf[ph * CCAP + p] = key;
                         } else {
-                            const unsigned q = atomicAdd(&w.cand_cnt[bh0 + h], 1u);
-                            w.cands[(bh0 + h) * a.N_max + q] = key;
+                            const unsigned q = atomicAdd(&w.cand_cnt[bh * CNT_STRIDE], 1u);
+                            w.cands[bh * a.N_max + q] = key;
+                        }
+                        // finalize attends the candidates it keeps: their rows
+                        // start toward L2 now (there are few of them)
+                        if (a.q_rope) {
+                            const size_t row = ((gk ? bg1 : bg0) * a.N_max + t) * D;
+                            prefetch_kv_l2(a.k_cache + row, a.v_cache + row);
                         }
                     }
                 }
             }
         }
     }
-    // flush the staged ids: one global reservation per head and kind
+    // the staged ids go out with one global reservation per pair-head and
+    // kind (warp w: pair-head w); the reservations are taken here and used
+    // after the fused attention, which hides their round trip
     __syncthreads();
-    if (warp < G) {
-        const size_t bh = bh0 + warp;
-        const unsigned nk = min(s_kc[warp], (unsigned)CL_KCAP);
-        const unsigned ncd = min(s_cc[warp], (unsigned)CCAP);
-        unsigned kb = 0u, cb = 0u;
-        if (lane == 0) {
-            if (nk) kb = atomicAdd(&w.list_cnt[bh], nk);
-            if (ncd) cb = atomicAdd(&w.cand_cnt[bh], ncd);
-        }
+    const bool wok = ph_ok(warp);
+    const size_t wbh = ph_bh(warp);
+    unsigned kb = 0u, cb = 0u;
+    const unsigned nk = wok ? min(s_kc[warp], (unsigned)CL_KCAP) : 0u;
+    const unsigned ncd = wok ? min(s_cc[warp], (unsigned)CCAP) : 0u;
+    if (lane == 0) {
+        if (nk) kb = atomicAdd(&w.list_cnt[wbh * CNT_STRIDE], nk);
+        if (ncd) cb = atomicAdd(&w.cand_cnt[wbh * CNT_STRIDE], ncd);
+    }
+    auto flush_ids = [&]() {
+        // (a global store before a block barrier would make the barrier wait
+        // for it, so the resolve records go out here, at the end)
+        if (cx == 0 && lane == 0 && wok) w.res[wbh] = s_res[warp];
         kb = __shfl_sync(0xffffffffu, kb, 0);
         cb = __shfl_sync(0xffffffffu, cb, 0);
-        for (unsigned j = lane; j < nk; j += 32) a.lists[bh * a.N_max + kb + j] = s_kbuf[warp * CL_KCAP + j];
-        for (unsigned j = lane; j < ncd; j += 32) w.cands[bh * a.N_max + cb + j] = s_cbuf[warp * CCAP + j];
+        for (unsigned j = lane; j < nk; j += 32) a.lists[wbh * a.N_max + kb + j] = s_kbuf[warp * CL_KCAP + j];
+        for (unsigned j = lane; j < ncd; j += 32) w.cands[wbh * a.N_max + cb + j] = s_cbuf[warp * CCAP + j];
+    };
+    if (!a.q_rope) {
+        flush_ids();
+        return;
     }
-    if (!a.q_rope) return;
 
-    // Fused attention over the rows staged here: chunks of 8 rows, head by
-    // head, dealt round-robin to the warps; each warp keeps one running
-    // partial and files it under (warp, head) when its head changes.  A head
-    // whose staging overflowed is left to finalize (ovf flag, empty partial).
-    int cpre[GMAX + 1];
-    cpre[0] = 0;
+    // Fused attention over the rows staged here, in rounds of pair-heads
+    // whose partial slots fit CL_SLOTS.  A round's rows form chunks of 8 of
+    // one head (heads in order), dealt round-robin to the warps; a warp
+    // keeps one running partial and files it when its head changes, in the
+    // slot of the head numbered by the warp's first chunk in the head (the
+    // first CL_WARPS chunks of a head belong to distinct warps, so a head
+    // with c chunks fills min(c, CL_WARPS) slots, each once).  Every warp
+    // derives the round layout itself (lane h: pair-head h), so no block
+    // barrier -- which would wait for the reservations above -- precedes the
+    // attention.  A head whose staging overflowed is left to finalize (ovf
+    // flag, empty partial).
+    if (lane == 0 && wok && s_kc[warp] > (unsigned)CL_KCAP) a.ovf[wbh] = 1u;
+    const __nv_bfloat16 *kc0 = a.k_cache + bg0 * a.N_max * D, *kc1 = a.k_cache + bg1 * a.N_max * D;
+    const __nv_bfloat16 *vc0 = a.v_cache + bg0 * a.N_max * D, *vc1 = a.v_cache + bg1 * a.N_max * D;
+    const int nrow_l = lane < HP && ph_ok(lane) && s_kc[lane] <= (unsigned)CL_KCAP ? (int)s_kc[lane] : 0;
+    for (int h_lo = 0; h_lo < HP;) {
+        // lane h in [h_lo, HP): its chunks and slots, inclusive prefix sums
+        const int c = lane >= h_lo ? (nrow_l + 7) / 8 : 0;
+        const int sl = min(c, CL_WARPS);
+        int cs = c, ss = sl;
 #pragma unroll
-    for (int h = 0; h < GMAX; ++h) {
-        const int nkh = h < G && s_kc[h] <= (unsigned)CL_KCAP ? (int)s_kc[h] : 0;
-        cpre[h + 1] = cpre[h] + (nkh + 7) / 8;
-    }
-    if (threadIdx.x < G && s_kc[threadIdx.x] > (unsigned)CL_KCAP) a.ovf[bh0 + threadIdx.x] = 1u;
-    float *my = s_slot + warp * GMAX * PSTRIDE;
-    {
-        WarpPart e;
-        e.reset();
-#pragma unroll
-        for (int h = 0; h < GMAX; ++h) e.store(my + h * PSTRIDE);
-    }
-    __syncwarp();
-    const __nv_bfloat16 *kb = a.k_cache + bg * a.N_max * D;
-    const __nv_bfloat16 *vb = a.v_cache + bg * a.N_max * D;
-    WarpPart part;
-    part.reset();
-    int cur = -1;
-    float qx[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int k = warp; k < cpre[GMAX]; k += CL_WARPS) {
-        // head of chunk k and its first chunk (no dynamic register indexing)
-        int h = 0, c0 = 0;
-#pragma unroll
-        for (int j = 1; j <= GMAX; ++j)
-            if (cpre[j] <= k) { h = j; c0 = cpre[j]; }
-        if (h != cur) {
-            if (cur >= 0) part.store(my + cur * PSTRIDE);
-            part.reset();
-            cur = h;
-            const float4 q4 = *reinterpret_cast<const float4 *>(s_qr + h * D + 4 * lane);
-            qx[0] = q4.x; qx[1] = q4.y; qx[2] = q4.z; qx[3] = q4.w;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int tc = __shfl_up_sync(0xffffffffu, cs, o), ts = __shfl_up_sync(0xffffffffu, ss, o);
+            if (lane >= o) { cs += tc; ss += ts; }
         }
-        const int r = (k - c0) * 8 + lane;
-        const int id = lane < 8 && r < (int)s_kc[h] ? s_kbuf[h * CL_KCAP + r] : -1;
-        attend8(kb, vb, id, qx, part);
-    }
-    if (cur >= 0) part.store(my + cur * PSTRIDE);
-    __syncthreads();
-    // merge the warps' partials per head into this CTA's record of the head
-    const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
-    for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-        const int h = i / D, d = i % D;
-        float M = -INFINITY;
-#pragma unroll
-        for (int w2 = 0; w2 < CL_WARPS; ++w2) M = fmaxf(M, s_slot[(w2 * GMAX + h) * PSTRIDE]);
-        float L = 0.0f, O = 0.0f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int w2 = 0; w2 < CL_WARPS; ++w2) {
-                const float *sl = s_slot + (w2 * GMAX + h) * PSTRIDE;
-                const float wg = sl[0] == -INFINITY ? 0.0f : exp2f(sl[0] - M);
-                L = fmaf(sl[1], wg, L);
-                O = fmaf(sl[POFF + d], wg, O);
+        // the round: heads h_lo .. h_hi - 1, as many as fit (at least one)
+        const unsigned fit = __ballot_sync(0xffffffffu, lane >= h_lo && lane < HP && ss <= CL_SLOTS);
+        const int h_hi = 32 - __clz(fit);
+        const int nchunk = __shfl_sync(0xffffffffu, cs, h_hi - 1);
+        const int c0_l = cs - c, s0_l = ss - sl;          // lane's first chunk and slot
+        WarpPart part;
+        part.reset();
+        int cur = -1, kfirst = 0, cur_c0 = 0, cur_s0 = 0;
+        float qx[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int k = warp; k < nchunk; k += CL_WARPS) {
+            // the chunk's head: the last non-empty head of the round starting at or before k
+            const unsigned st = __ballot_sync(0xffffffffu, lane >= h_lo && lane < h_hi && c > 0 && c0_l <= k);
+            const int ph = 31 - __clz(st);
+            const int c0 = __shfl_sync(0xffffffffu, c0_l, ph), s0 = __shfl_sync(0xffffffffu, s0_l, ph);
+            if (ph != cur) {
+                if (cur >= 0) part.store(s_slot + (cur_s0 + kfirst - cur_c0) * PSTRIDE);
+                part.reset();
+                cur = ph;
+                kfirst = k;
+                cur_c0 = c0;
+                cur_s0 = s0;
+                const float4 q4 = *reinterpret_cast<const float4 *>(s_qr + ph * D + 4 * lane);
+                qx[0] = q4.x; qx[1] = q4.y; qx[2] = q4.z; qx[3] = q4.w;
             }
+            const int r = (k - c0) * 8 + lane;
+            const int id = lane < 8 && r < (int)s_kc[ph] ? s_kbuf[ph * CL_KCAP + r] : -1;
+            if (ph < GMAX) attend8(kc0, vc0, id, qx, part); else attend8(kc1, vc1, id, qx, part);
         }
-        float *rec = a.part_sel + (cta * GMAX + h) * PSTRIDE;
-        rec[POFF + d] = O;
-        if (d == 0) { rec[0] = M; rec[1] = L; }
+        if (cur >= 0) part.store(s_slot + (cur_s0 + kfirst - cur_c0) * PSTRIDE);
+        __syncthreads();
+        // merge each head's slots into this CTA's record of the head: one
+        // warp per head, lane l folding dims 4 l .. 4 l + 3 slot by slot
+        for (int ph = h_lo + warp; ph < h_hi; ph += CL_WARPS) {
+            const int s0 = __shfl_sync(0xffffffffu, s0_l, ph), s1 = __shfl_sync(0xffffffffu, ss, ph);
+            WarpPart acc;
+            acc.reset();
+            for (int q = s0; q < s1; ++q) acc.load_add(s_slot + q * PSTRIDE);
+            acc.store(a.part_sel + (cta * HP + ph) * PSTRIDE);
+        }
+        // the slots are reused only by a further round (no barrier after the
+        // last: it would wait for the record stores)
+        if (h_hi < HP) __syncthreads();
+        h_lo = h_hi;
     }
+    flush_ids();
 }
 
 // ---------------------------------------------------------------------------
@@ -1373,9 +1481,12 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     __shared__ uint32_t hfx32[256];
     __shared__ unsigned hcnt[256];
     __shared__ __align__(16) unsigned long long cbuf[FIN_CAP];
-    __shared__ uint32_t fbuf[FIN_CAP];
+    __shared__ __align__(16) uint32_t fbuf[FIN_CAP];
+    // ids of the kept candidates (staged case), compacted over the start of
+    // cbuf once the keys are read
+    int32_t *const s_kid = reinterpret_cast<int32_t *>(cbuf);
     __shared__ unsigned long long s_min, s_max, s_theta, s_excl, s_kept;
-    __shared__ unsigned s_base;
+    __shared__ unsigned s_base2, s_wcnt[FIN_WARPS];
     __shared__ int s_digit;
     __shared__ unsigned s_dcnt;
     __shared__ __align__(16) float s_crec[FIN_CLUSTER * PSTRIDE];   // the ranks' attention partials (fused)
@@ -1390,17 +1501,22 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     const int gi = (hb / G) % a.n_ret;
     const int h = a.ret_g[gi] * G + hb % G;
     const size_t bh = (size_t)b * a.H_q + h;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // fused attention: this head's query (scaled), an input of the call that
+    // no earlier kernel writes, loads before the wait
+    float qx_f[4] = {0.f, 0.f, 0.f, 0.f};
+    if (a.q_rope) {
+        const float4 q4 = *reinterpret_cast<const float4 *>(a.q_rope + bh * D + 4 * lane);
+        qx_f[0] = q4.x * a.attn_scale_log2; qx_f[1] = q4.y * a.attn_scale_log2;
+        qx_f[2] = q4.z * a.attn_scale_log2; qx_f[3] = q4.w * a.attn_scale_log2;
+    }
     pdl_wait();
     pdl_trigger();
-    // the collect pass is done with the histogram: clear it for the next call
-    if (rank == 0)
-        for (int i = threadIdx.x; i < NBIN; i += blockDim.x) w.hist[bh * NBIN + i] = 0.0;
     // the head's resolve record and both counters in one round of loads
     const Resolve r = w.res[bh];
-    const unsigned nc_all = w.cand_cnt[bh];
-    const unsigned base0 = w.list_cnt[bh];
+    const unsigned nc_all = w.cand_cnt[bh * CNT_STRIDE];
+    const unsigned base0 = w.list_cnt[bh * CNT_STRIDE];
     const unsigned ovf = a.q_rope ? a.ovf[bh] : 0u;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned long long *cg = w.cands + bh * a.N_max;
     // first candidate of each thread, loaded before the count is known (the
     // buffer holds N_max entries, so the read is in bounds)
@@ -1410,17 +1526,11 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     WarpPart part;
     part.reset();
     if (a.q_rope) {
+        // the records of this head's pair-head in every CTA of its pair
         const size_t y = (size_t)b * a.n_ret + gi;
-        const float *recs = a.part_sel + (size_t)(hb % G) * PSTRIDE;
+        const float *recs = a.part_sel + ((y % PAIR) * GMAX + (size_t)(hb % G)) * PSTRIDE;
         for (int x = rank * FIN_WARPS + warp; x < a.cl_ctas; x += K * FIN_WARPS)
-            part.load_add(recs + (y * a.cl_ctas + x) * GMAX * PSTRIDE);
-    }
-    // fused attention: this head's query (scaled) with the first loads
-    float qx_f[4] = {0.f, 0.f, 0.f, 0.f};
-    if (a.q_rope) {
-        const float4 q4 = *reinterpret_cast<const float4 *>(a.q_rope + bh * D + 4 * lane);
-        qx_f[0] = q4.x * a.attn_scale_log2; qx_f[1] = q4.y * a.attn_scale_log2;
-        qx_f[2] = q4.z * a.attn_scale_log2; qx_f[3] = q4.w * a.attn_scale_log2;
+            part.load_add(recs + ((y / PAIR) * a.cl_ctas + x) * HP * PSTRIDE);
     }
     unsigned long long fin_theta = ~0ull;            // kept boundary candidates: key >= fin_theta
     const unsigned nc = r.mode == MODE_NORMAL ? nc_all : 0u;
@@ -1429,8 +1539,6 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     float mass = 0.0f;
 
     if (r.mode == MODE_KEEP_ALL) {
-        if (rank == 0)
-            for (int t = tid; t < r.N; t += blockDim.x) lst[t] = t;
         count = r.N;
         mass = 1.0f;
     } else if (r.mode != MODE_NORMAL || nc == 0u) {
@@ -1447,7 +1555,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             const float m = ex2_sfu((cand_logit(v) - Ub) * 1.4426950408889634f);
             return (unsigned long long)((double)m * S);
         };
-        if (tid == 0) { s_min = ~0ull; s_max = 0ull; s_kept = 0ull; s_base = 0u; }
+        if (tid == 0) { s_min = ~0ull; s_max = 0ull; s_kept = 0ull; s_base2 = 0u; }
         __syncthreads();
         {
             unsigned long long lo = ~0ull, hi = 0ull;
@@ -1553,10 +1661,13 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
                 __syncthreads();
             }
         }
-        // kept = candidates at or above theta, appended after the ids the
-        // collect pass wrote (block-wide ranks, no global atomics)
+        // kept = candidates at or above theta: their count and mass, and
+        // (staged) their ids, compacted in candidate order -- the same order
+        // in every rank of the cluster, which split the list by position --
+        // for the attention and for the list append rank 0 makes at the end
         unsigned long long kept = 0ull;
         const unsigned lt = (1u << lane) - 1u;
+        unsigned kbase = 0u;                         // kept candidates before this chunk
         for (unsigned c0 = 0; c0 < nc; c0 += blockDim.x) {
             const unsigned c = c0 + tid;
             unsigned long long v = 0ull;
@@ -1566,29 +1677,62 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
                 k = v >= theta;
             }
             const unsigned bal = __ballot_sync(0xffffffffu, k);
-            unsigned wbase = 0u;
-            if (lane == 0 && bal) wbase = atomicAdd(&s_base, (unsigned)__popc(bal));
-            wbase = __shfl_sync(0xffffffffu, wbase, 0);
-            if (k) {
-                if (rank == 0)
-                    lst[base0 + wbase + __popc(bal & lt)] = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
-                kept += staged ? fbuf[c] : fx_of(v);
+            if (k) kept += staged ? fbuf[c] : fx_of(v);
+            if (lane == 0) s_wcnt[warp] = (unsigned)__popc(bal);
+            // every key of the chunk is read (id i lands on key i / 2, below
+            // c0 + blockDim.x / 2) and the warps' counts are in
+            __syncthreads();
+            unsigned before = 0u, total = 0u;
+#pragma unroll
+            for (int w2 = 0; w2 < FIN_WARPS; ++w2) {
+                const unsigned n = s_wcnt[w2];
+                before += w2 < warp ? n : 0u;
+                total += n;
             }
+            if (staged && k)
+                s_kid[kbase + before + __popc(bal & lt)] = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
+            kbase += total;
+            __syncthreads();                          // the counts are read before the next chunk
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(0xffffffffu, kept, o);
         if (lane == 0) atomicAdd(&s_kept, kept);
         __syncthreads();
-        count = (int)(base0 + s_base);
+        count = (int)(base0 + kbase);
         fin_theta = theta;
         const double kept_mass = (double)s_kept / S * (double)ex2_sfu((Ub - r.R) * 1.4426950408889634f);
         mass = (float)((r.above + kept_mass) / r.Z);
     }
-    if (tid == 0 && rank == 0) {
-        a.count_out[bh] = count;
-        if (a.mass_out) a.mass_out[bh] = mass;
+    // Rank 0's global writes go out last (a global store before a block or
+    // cluster barrier makes that barrier wait for it): count and mass, the
+    // kept ids (every token for keep-all; the kept boundary candidates after
+    // the collect pass's ids), and the cleared histogram for the next call.
+    auto finish = [&]() {
+        if (rank != 0) return;
+        if (tid == 0) {
+            a.count_out[bh] = count;
+            if (a.mass_out) a.mass_out[bh] = mass;
+        }
+        if (r.mode == MODE_KEEP_ALL) {
+            for (int t = tid; t < r.N; t += blockDim.x) lst[t] = t;
+        } else if (r.mode == MODE_NORMAL && nc > 0u) {
+            if (nc <= (unsigned)FIN_CAP) {
+                for (int i = tid; i < count - (int)base0; i += blockDim.x) lst[base0 + i] = s_kid[i];
+            } else {
+                for (unsigned c = tid; c < nc; c += blockDim.x) {
+                    const unsigned long long v = cg[c];
+                    if (v >= fin_theta)
+                        lst[base0 + atomicAdd(&s_base2, 1u)] =
+                            (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
+                }
+            }
+        }
+        for (int i = tid; i < HSTRIDE; i += blockDim.x) w.hist[bh * HSTRIDE + i] = 0.0;
+    };
+    if (!a.q_rope) {
+        finish();
+        return;
     }
-    if (!a.q_rope) return;
 
     // Fused attention: the kept rows the collect pass did not attend (the
     // boundary bin's kept candidates, plus, after a staging overflow, the
@@ -1603,6 +1747,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             for (int d = tid; d < D; d += blockDim.x) a.out[bh * D + d] = 0.0f;
             if (tid == 0) set_status(w.status, RTP_ERR_DEVICE_ARG);
         }
+        finish();
         return;
     }
     if (ovf) part.reset();                           // a collect CTA could not attend all its kept rows
@@ -1624,20 +1769,29 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
                 attend8(kb, vb, id, qx_f, part);
             }
         } else if (r.mode == MODE_NORMAL) {
-            // boundary-bin candidates at or above theta, eight candidate slots at a time
-            const bool staged = nc <= (unsigned)FIN_CAP;
-            for (int cb = worker * 8; cb < (int)nc; cb += workers * 8) {
-                int id = -1;
-                if (lane < 8 && cb + lane < (int)nc) {
-                    const unsigned long long v = staged ? cbuf[cb + lane] : __ldcg(cg + cb + lane);
-                    if (v >= fin_theta) id = (int)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
+            // boundary-bin candidates at or above theta: the compacted ids
+            // (staged), else eight candidate slots at a time
+            if (nc <= (unsigned)FIN_CAP) {
+                const int nk = count - (int)base0;
+                for (int rb = worker * 8; rb < nk; rb += workers * 8)
+                    attend8(kb, vb, lane < 8 && rb + lane < nk ? s_kid[rb + lane] : -1, qx_f, part);
+            } else {
+                for (int cb = worker * 8; cb < (int)nc; cb += workers * 8) {
+                    int id = -1;
+                    if (lane < 8 && cb + lane < (int)nc) {
+                        const unsigned long long v = __ldcg(cg + cb + lane);
+                        if (v >= fin_theta) id = (int)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
+                    }
+                    attend8(kb, vb, id, qx_f, part);
                 }
-                attend8(kb, vb, id, qx_f, part);
             }
         }
     }
-    __syncthreads();                                 // every thread is done with the candidates
-    float *slots = reinterpret_cast<float *>(cbuf);  // the candidates are no longer needed
+    // the warps' partials go into the mass buffer (no longer needed; the
+    // candidates stay for the list append at the end)
+    float *slots = reinterpret_cast<float *>(fbuf);
+    static_assert(FIN_WARPS * PSTRIDE <= FIN_CAP, "partial slots fit the mass buffer");
+    __syncthreads();                                 // every thread is done with the masses
     part.store(slots + warp * PSTRIDE);
     __syncthreads();
     // this rank's partial goes into slot `rank` of rank 0's s_crec
@@ -1676,6 +1830,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             a.out[bh * D + d] = O * (L > 0.0f ? 1.0f / L : 0.0f);
         }
     }
+    finish();
 }
 
 // ---------------------------------------------------------------------------
