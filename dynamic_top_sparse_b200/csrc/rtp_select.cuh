@@ -1470,6 +1470,7 @@ constexpr int FIN_THREADS = 512;
 constexpr int FIN_WARPS = FIN_THREADS / 32;
 constexpr int FIN_CAP = 3072;             // candidates staged in shared memory
 constexpr int FIN_CLUSTER = 4;            // CTAs per head with the fused attention
+constexpr int FIN_FOLD = 3;               // collect records a warp loads at once
 // Exact selection inside the boundary bin.  One CTA per retrieval head;
 // grid = (B * n_ret * G).  Candidate masses relative to the boundary bin's
 // upper edge U* are each in (e^-32, 1]; they are summed in fixed point with
@@ -1526,11 +1527,32 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     WarpPart part;
     part.reset();
     if (a.q_rope) {
-        // the records of this head's pair-head in every CTA of its pair
+        // the records of this head's pair-head in every CTA of its pair,
+        // FIN_FOLD per warp at a time with all their loads issued first (one
+        // round trip, not one per record)
         const size_t y = (size_t)b * a.n_ret + gi;
-        const float *recs = a.part_sel + ((y % PAIR) * GMAX + (size_t)(hb % G)) * PSTRIDE;
-        for (int x = rank * FIN_WARPS + warp; x < a.cl_ctas; x += K * FIN_WARPS)
-            part.load_add(recs + ((y / PAIR) * a.cl_ctas + x) * HP * PSTRIDE);
+        const float *recs = a.part_sel + ((y % PAIR) * GMAX + (size_t)(hb % G)) * PSTRIDE +
+                            (y / PAIR) * a.cl_ctas * HP * PSTRIDE;
+        for (int x0 = rank * FIN_WARPS + warp; x0 < a.cl_ctas; x0 += FIN_FOLD * K * FIN_WARPS) {
+            float mx[FIN_FOLD], lx[FIN_FOLD];
+            float4 ox[FIN_FOLD];
+#pragma unroll
+            for (int j = 0; j < FIN_FOLD; ++j) {
+                const int x = x0 + j * K * FIN_WARPS;
+                mx[j] = -INFINITY; lx[j] = 0.0f; ox[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (x < a.cl_ctas) {
+                    const float *rc = recs + (size_t)x * HP * PSTRIDE;
+                    mx[j] = rc[0];
+                    lx[j] = rc[1];
+                    ox[j] = *reinterpret_cast<const float4 *>(rc + POFF + 4 * lane);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < FIN_FOLD; ++j) {
+                const float o4[4] = {ox[j].x, ox[j].y, ox[j].z, ox[j].w};
+                part.add(mx[j], lx[j], o4);
+            }
+        }
     }
     unsigned long long fin_theta = ~0ull;            // kept boundary candidates: key >= fin_theta
     const unsigned nc = r.mode == MODE_NORMAL ? nc_all : 0u;
