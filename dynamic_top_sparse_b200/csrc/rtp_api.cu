@@ -88,6 +88,7 @@ size_t op_bytes(const Layout &L, int op) {
 }
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+bool aligned4(const void *p) { return ((uintptr_t)p & 3u) == 0; }
 
 int check_dims(const rtp_dims *d) {
     if (!d) return RTP_ERR_INVALID_ARG;
@@ -441,6 +442,17 @@ int noalloc_scratch(char *&out) {
     }
     out = static_cast<char *>(ptrs[dev]);
     return RTP_OK;
+}
+
+// Self-test of the bounded device-side wait: one thread waits on an
+// mbarrier that nothing completes (no copy is in flight on it), gives up
+// after WAIT_LIMIT_NS and records RTP_ERR_TIMEOUT.
+__global__ void wait_timeout_kernel(uint32_t *status) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1u);
+    fence_mbar_init();
+    if (!mbar_wait(&bar, 0u)) set_status(status, RTP_ERR_TIMEOUT);
 }
 
 }  // namespace
@@ -805,6 +817,12 @@ int rtp_prof_destroy(rtp_prof *prof) {
     prof->name = nullptr;
     prof->capacity = prof->count = 0;
     return RTP_OK;
+}
+
+int rtp_selftest_wait_timeout(int32_t *dev_status, rtp_stream_t stream) {
+    if (!dev_status || !aligned4(dev_status)) return RTP_ERR_INVALID_ARG;
+    wait_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(reinterpret_cast<uint32_t *>(dev_status));
+    return cudaGetLastError() == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
 }
 
 }  // extern "C"

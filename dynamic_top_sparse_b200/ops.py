@@ -41,7 +41,8 @@ OP_DECODE_STEP = 6
 EXPORTS = ("rtp_workspace_size", "rtp_workspace_init", "rtp_check", "rtp_error_string",
            "rtp_version", "rtp_append_index_keys", "rtp_index_scores", "rtp_topp_select",
            "rtp_sparse_decode", "rtp_local_decode", "rtp_dense_decode", "rtp_decode_step",
-           "rtp_prof_init", "rtp_prof_elapsed", "rtp_prof_destroy", "rtp_dense_decode_noalloc")
+           "rtp_prof_init", "rtp_prof_elapsed", "rtp_prof_destroy", "rtp_dense_decode_noalloc",
+           "rtp_selftest_wait_timeout")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20
 NOALLOC_MAX_GROUPS = 1024
@@ -97,6 +98,7 @@ _SIGS = {
     "rtp_prof_destroy": (ctypes.c_int, [ctypes.POINTER(Prof)]),
     "rtp_dense_decode_noalloc": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Opts), _P, _P, _P, _P, _P,
                                                 _P]),
+    "rtp_selftest_wait_timeout": (ctypes.c_int, [_P, _P]),
 }
 
 
@@ -274,6 +276,12 @@ def decode_step(dims: Dims, q, q_rope, k_cache, v_cache, kidx_cache, W_q_idx, he
                               _ptr(q_rope), _ptr(k_cache), _ptr(v_cache), _ptr(kidx_cache), _ptr(W_q_idx),
                               _hc(head_class), float(p), int(window), int(n_sink), _ptr(out), ws.ptr,
                               ws.nbytes, _stream()), "rtp_decode_step")
+
+
+def selftest_wait_timeout(dev_status):
+    """Launch the bounded-wait self-test: its one waiting thread gives up
+    after 0.2 s and writes RTP_ERR_TIMEOUT into the zeroed device int32."""
+    _ck(lib().rtp_selftest_wait_timeout(_ptr(dev_status), _stream()), "rtp_selftest_wait_timeout")
 
 
 def dense_decode_noalloc(dims: Dims, q_rope, k_cache, v_cache, out, dev_status=None, opts: Opts | None = None):

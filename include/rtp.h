@@ -301,6 +301,19 @@ RTP_API int rtp_dense_decode_noalloc(const rtp_dims *dims, const rtp_opts *opts,
                                      const void *k_cache, const void *v_cache, float *out,
                                      int32_t *dev_status, rtp_stream_t stream);
 
+/* Self-test of failure detection (no counterpart in the pages).  The
+ * library's device-side waits -- the index scan's waits on its own bulk
+ * copies -- are bounded: after 0.2 s a waiting kernel records
+ * RTP_ERR_TIMEOUT and returns, and the context stays usable.  This call
+ * launches one kernel whose single waiting thread waits on a barrier that
+ * nothing completes, so its wait runs out by construction (about 0.2 s of
+ * device time) and it writes RTP_ERR_TIMEOUT into *dev_status (a device
+ * int32, 4-byte aligned, which the caller zeroes first: the first error
+ * written wins).  Returns RTP_ERR_INVALID_ARG for a null or misaligned
+ * pointer, RTP_ERR_CUDA if the launch fails, else RTP_OK (asynchronous:
+ * read dev_status after synchronising the stream). */
+RTP_API int rtp_selftest_wait_timeout(int32_t *dev_status, rtp_stream_t stream);
+
 /* Launch accounting helpers (see rtp_prof). */
 RTP_API int rtp_prof_init(rtp_prof *prof, int32_t capacity);
 RTP_API int rtp_prof_elapsed(const rtp_prof *prof, int32_t slot, float *ms);

@@ -75,3 +75,17 @@ def test_append_bad_position_reports():
     ops.append_index_keys(gc.dims, gc.k_new, gc.Wk, pos, gc.hc, gc.kidx, gc.ws)
     assert gc.ws.check() == ops.RTP_ERR_DEVICE_ARG
     assert torch.equal(gc.kidx[1], before[1])
+
+
+def test_bounded_wait_runs_out_and_context_stays_usable():
+    """A device-side wait that nothing ends gives up after its bound and
+    reports RTP_ERR_TIMEOUT; the next step on the same context is correct."""
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    ops.selftest_wait_timeout(st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == ops.RTP_ERR_TIMEOUT
+    gc = _case()
+    out = torch.zeros((2, 8, 128), device="cuda")
+    ops.decode_step(gc.dims, gc.q, gc.q_rope, gc.k, gc.v, gc.kidx, gc.Wq, gc.hc, 0.9, 64, 4, out, gc.ws)
+    assert gc.ws.check() == 0
+    assert torch.isfinite(out).all()
