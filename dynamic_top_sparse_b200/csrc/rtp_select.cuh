@@ -658,7 +658,7 @@ constexpr int SCAN_THREADS = 512;
 constexpr int SCAN_WARPS = SCAN_THREADS / 32;
 
 template <typename Src>
-__global__ void __launch_bounds__(SCAN_THREADS, 1) scan_kernel(SelArgs a, SelWs w) {
+__global__ void __launch_bounds__(SCAN_THREADS, 2) scan_kernel(SelArgs a, SelWs w) {
     __shared__ __align__(16) float qs[GMAX * R];
     __shared__ __align__(16) uint32_t shl[2 * GMAX * NBIN];   // fixed-point bin sums: low words, then high words
     uint32_t *const shh = shl + GMAX * NBIN;
@@ -1008,7 +1008,7 @@ constexpr int KCAP = 256;     // kept ids staged per head per CTA
 constexpr int CCAP = 128;     // candidates staged per head per CTA
 
 template <typename Src>
-__global__ void __launch_bounds__(COL_THREADS, 1) collect_kernel(SelArgs a, SelWs w) {
+__global__ void __launch_bounds__(COL_THREADS, 2) collect_kernel(SelArgs a, SelWs w) {
     __shared__ __align__(16) float qs[GMAX * R];
     __shared__ int s_bstar[GMAX];
     __shared__ int s_mode[GMAX];
