@@ -20,12 +20,16 @@
  *
  * The threshold is found without sorting (same summary, Method section 5:
  * sort-free histogram threshold and bandwidth-optimised sparse decode): one
- * streaming pass over the index keys gives each head's softmax statistics
- * (max m, sum Z); tokens with z < m + ln(Z (1 - p) / N) - 1 carry less than
- * (1 - p) / N of the mass each and can never be kept; the remaining
- * candidates are ranked by an exact radix select on the order-preserving
- * bits of z (then the token id), with per-digit mass histograms, down to
- * the boundary token.
+ * streaming pass over the index keys builds, per head, a histogram of
+ * softmax mass over the fp32 bits of z (512 bins: sign, exponent and 4
+ * mantissa bits, each bin's mass kept relative to its upper edge, plus
+ * per-octave sums); from it, the boundary bin -- where the mass accumulated
+ * from the top first reaches p Z -- and Z itself.  Tokens above that bin
+ * are kept outright; the tokens inside it are ranked by an exact radix
+ * select on the order-preserving bits of z (then the token id), with
+ * per-digit mass histograms, down to the boundary token.  The binned range
+ * is |z| < 256: a logit outside it, or not finite, is reported as
+ * RTP_ERR_RANGE.
  *
  * Conventions shared by every call
  *   - Tensor pointers are DEVICE pointers owned by the caller, dense
@@ -205,8 +209,8 @@ RTP_API int rtp_index_scores(const rtp_dims *dims, const rtp_opts *opts, const f
  *   count_out [B, H_q] int32:   |S| (>= 1)
  *   mass_out  [B, H_q] fp32:    mass of S (optional, NULL: not written)
  * p >= 1 keeps all N_b tokens; p <= 0 keeps the top token; p NaN is
- * RTP_ERR_INVALID_ARG.  A logit that is not finite is skipped and reported
- * as RTP_ERR_RANGE.
+ * RTP_ERR_INVALID_ARG.  A logit that is not finite or has |z| >= 256 is
+ * reported as RTP_ERR_RANGE (the call's outputs are then unspecified).
  */
 RTP_API int rtp_topp_select(const rtp_dims *dims, const float *z, const uint8_t *head_class,
                     float p, int32_t *idx_out, int32_t *count_out, float *mass_out,
