@@ -230,8 +230,8 @@ struct SelArgs {
     float *mass_out;             // [B*H_q] or null
     // Fused sparse attention of a decode step (bf16 caches); q_rope null = off.
     // Every collect CTA attends the rows it kept and writes one partial per
-    // head of its group; finalize attends the boundary bin's kept rows and
-    // merges.  A head whose kept rows overflowed a CTA's staging is attended
+    // head of its pair of groups; finalize attends the boundary bin's kept
+    // rows and merges.  A head whose kept rows overflowed a CTA's staging is attended
     // wholly by finalize (ovf flag).
     const float *q_rope;                 // [B, H_q, D]
     const __nv_bfloat16 *k_cache;        // [B, H_kv, N_max, D]
@@ -1471,12 +1471,14 @@ constexpr int FIN_WARPS = FIN_THREADS / 32;
 constexpr int FIN_CAP = 3072;             // candidates staged in shared memory
 constexpr int FIN_CLUSTER = 4;            // CTAs per head with the fused attention
 constexpr int FIN_FOLD = 3;               // collect records a warp loads at once
-// Exact selection inside the boundary bin.  One CTA per retrieval head;
-// grid = (B * n_ret * G).  Candidate masses relative to the boundary bin's
-// upper edge U* are each in (e^-32, 1]; they are summed in fixed point with
-// S = 2^62 / nc units per unit of mass, so sums stay below 2^62 and do not
-// depend on the order of the adds.  The head's level-1 histogram is cleared
-// here for the next call.
+// Exact selection inside the boundary bin.  One CTA per retrieval head, or
+// a cluster of FIN_CLUSTER CTAs per head with the fused attention (each
+// rank runs the same selection); grid = (1 or FIN_CLUSTER, B * n_ret * G).
+// Candidate masses relative to the boundary bin's upper edge U* are each in
+// (e^-32, 1]; they are summed in fixed point with S = (2^31 - 1) / nc
+// (staged in shared memory) or 2^62 / nc units per unit of mass, so sums
+// cannot wrap and do not depend on the order of the adds.  Rank 0 clears
+// the head's level-1 histogram for the next call, last.
 __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs w) {
     __shared__ unsigned long long hfx[256];
     __shared__ uint32_t hfx32[256];
