@@ -274,7 +274,9 @@ struct ListArgs {
     const void *v;
     const int32_t *lists;        // [B*H_q*N_max]
     const int32_t *counts;       // [B*H_q] kept rows per head (read by LIST_ALL and LIST_REST)
-    const int32_t *first;        // [B*H_q] at stride CNT_STRIDE: rows of the collect pass (LIST_FIRST, LIST_REST), or null
+    // [B*H_q] at stride CNT_STRIDE: rows of the collect pass (LIST_FIRST,
+    // LIST_REST), or null
+    const int32_t *first;
     int phase;
     float *out;
     float *part;                 // [B*H_q][LIST_SLOTS][PSTRIDE]

@@ -215,7 +215,7 @@ struct SelArgs {
     int ntile;
     int ctas;                    // scan/collect CTAs per (b, g)
     long long chunk;             // tokens per CTA, multiple of TILE
-    int cl_ctas;                 // collect_mma_kernel CTAs per pair of groups; the pair's tile i goes to CTA i mod cl_ctas
+    int cl_ctas;                 // collect_mma_kernel CTAs per pair of groups (tile i -> CTA i mod cl_ctas)
     const int32_t *seq_lens;
     int n_ret;
     int ret_g[MAX_RET_GROUPS];
@@ -231,8 +231,8 @@ struct SelArgs {
     // Fused sparse attention of a decode step (bf16 caches); q_rope null = off.
     // Every collect CTA attends the rows it kept and writes one partial per
     // head of its pair of groups; finalize attends the boundary bin's kept
-    // rows and merges.  A head whose kept rows overflowed a CTA's staging is attended
-    // wholly by finalize (ovf flag).
+    // rows and merges.  A head whose kept rows overflowed a CTA's staging is
+    // attended wholly by finalize (ovf flag).
     const float *q_rope;                 // [B, H_q, D]
     const __nv_bfloat16 *k_cache;        // [B, H_kv, N_max, D]
     const __nv_bfloat16 *v_cache;
@@ -1102,7 +1102,8 @@ __global__ void __launch_bounds__(COL_THREADS, 2) collect_kernel(SelArgs a, SelW
                             }
                         } else if (zz >= s_clo[h]) {
                             const unsigned long long key =
-                                ((unsigned long long)logit_key(zz) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)t);
+                                ((unsigned long long)logit_key(zz) << 32) |
+                                (unsigned long long)(0xffffffffu - (uint32_t)t);
                             const unsigned p = atomicAdd(&s_cc[h], 1u);
                             if (p < (unsigned)CCAP) {
                                 s_cbuf[h * CCAP + p] = key;
@@ -1174,7 +1175,7 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
     int32_t *s_kbuf = reinterpret_cast<int32_t *>(csm);                                          // [HP][CL_KCAP]
     unsigned long long *s_cbuf = reinterpret_cast<unsigned long long *>(csm + HP * CL_KCAP * 4);  // [HP][CCAP]
     float *s_qr = reinterpret_cast<float *>(csm + HP * CL_KCAP * 4 + HP * CCAP * 8);              // [HP][D]
-    float *s_slot = s_qr + HP * D;                                                                  // [CL_SLOTS][PSTRIDE]
+    float *s_slot = s_qr + HP * D;                                                        // [CL_SLOTS][PSTRIDE]
     __shared__ __align__(16) float qs[PAIR][GMAX * R];
     __shared__ int s_bstar[HP];
     __shared__ unsigned s_kc[HP], s_cc[HP];
