@@ -138,3 +138,5 @@ def test_other_calls_reject_bad_arguments(L):
                                    None) == ops.RTP_ERR_INVALID_ARG
     assert L.rtp_workspace_init(None, 100, None) == ops.RTP_ERR_WORKSPACE
     assert L.rtp_check(None, None) == ops.RTP_ERR_WORKSPACE
+    assert L.rtp_selftest_wait_timeout(None, None) == ops.RTP_ERR_INVALID_ARG
+    assert L.rtp_selftest_wait_timeout(FAKE + 2, None) == ops.RTP_ERR_INVALID_ARG     # misaligned
