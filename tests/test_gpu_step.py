@@ -71,6 +71,9 @@ SMALL = [
     # attention in the separate list passes
     dict(B=2, H_q=16, H_kv=2, N=6000, head_class=(1, 0), p=0.9, kv_dtype="f32", idx_dtype="bf16",
          seq_lens=[6000, 1234]),
+    # flat logits, ~20 % of 64K kept per head: dozens of kept rows per head
+    # in every collect CTA, so its attention runs in several rounds of slots
+    dict(B=1, H_q=16, H_kv=2, N=65536, head_class=(1, 1), p=0.2, needles="none"),
 ]
 
 
