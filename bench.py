@@ -27,6 +27,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from dynamic_top_sparse_b200 import ops, synth  # noqa: E402
+from dynamic_top_sparse_b200.dist import allreduce_max, barrier  # noqa: E402
 
 METRIC = "sparse decode attention steps/s and achieved HBM GB/s (% peak) at 64K-1M ctx"
 L2_BYTES = 126 * 2 ** 20
@@ -523,21 +524,6 @@ def run_reference(args, rank, world):
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "note": "the CPU oracle (numpy fp64), timed on host cores over a bounded sample"}
-
-
-# -------------------------------------------------------------- distributed
-
-def barrier(world):
-    if world > 1:
-        torch.distributed.barrier()
-
-
-def allreduce_max(x, world, dev):
-    if world == 1:
-        return x
-    t = torch.tensor([x], dtype=torch.float64, device=dev)
-    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    return float(t.item())
 
 
 def main():
