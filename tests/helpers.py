@@ -9,9 +9,9 @@ import torch
 import oracle
 from dynamic_top_sparse_b200 import ops, synth
 
-# Tolerances.  Sets: the spec rule -- bit-exact except tokens whose
-# oracle cumulative mass (strictly before them, descending order) lies within
-# MASS_TOL of p; the kept set's oracle mass must reach p - MASS_TOL.
+# Tolerances.  Sets: bit-exact except tokens whose oracle cumulative mass
+# (strictly before them, descending order) lies within MASS_TOL of p; the
+# kept set's oracle mass must reach p - MASS_TOL.
 MASS_TOL = 1e-5
 # Attention output vs the oracle over its own kept set (bf16 caches, fp32
 # accumulation).
@@ -40,7 +40,8 @@ def gpu_set(sel_idx: torch.Tensor, sel_count: torch.Tensor, b: int, h: int) -> n
 
 
 def check_selection(ids: np.ndarray, sel: oracle.Selection, p: float, where: str = ""):
-    """North-star set rule plus the mass floor.  Returns (n_diff, mass)."""
+    """The set rule (bit-exact except tokens within MASS_TOL of the p
+    boundary) plus the mass floor.  Returns (n_diff, mass)."""
     assert ids.size >= 1, f"{where}: empty kept set"
     assert np.unique(ids).size == ids.size, f"{where}: duplicate ids"
     n = sel.pi.shape[0]

@@ -25,7 +25,7 @@ def _declared():
     return sorted(set(re.findall(r"RTP_API[^;(]*?\b(rtp_\w+)\s*\(", src)))
 
 
-def test_header_declares_the_north_star_calls():
+def test_header_declares_the_step_calls():
     names = set(_declared())
     for n in ("rtp_append_index_keys", "rtp_index_scores", "rtp_topp_select", "rtp_sparse_decode",
               "rtp_local_decode", "rtp_decode_step", "rtp_dense_decode", "rtp_workspace_size",
