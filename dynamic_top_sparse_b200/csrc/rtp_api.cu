@@ -365,7 +365,7 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
     long long want = ((long long)per_sm * num_sms() + (long long)d->B * a.n_grp - 1) / ((long long)d->B * a.n_grp);
     if (max_ctas > 0) want = std::max(1LL, (long long)max_ctas / ((long long)d->B * a.n_grp));
     a.n_split = (int)std::max(1LL, std::min(want, std::min(chunks, (long long)RANGE_SPLIT_MAX)));
-    a.scale_log2 = attn_scale * 1.4426950408889634f;
+    a.scale_log2 = attn_scale * L2E;
     a.q = q; a.k = k; a.v = v; a.out = out;
     a.part = reinterpret_cast<float *>(ws + L.part_range);
     a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_range);
@@ -400,7 +400,7 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
     for (int h = 0; h < d->H_q; ++h)
         if (hc[h / a.G] == RTP_HEAD_RETRIEVAL) a.ret_h[a.n_rq++] = h;
     if (a.n_rq == 0) return RTP_OK;
-    a.scale_log2 = attn_scale * 1.4426950408889634f;
+    a.scale_log2 = attn_scale * L2E;
     a.q = q; a.k = k; a.v = v; a.lists = lists; a.counts = counts; a.out = out;
     a.first = first;
     a.phase = phase;
@@ -656,7 +656,7 @@ int rtp_dense_decode_noalloc(const rtp_dims *dims, const rtp_opts *opts, const f
     const long long chunks = (dims->N_max + 255) / 256;
     const long long want = (2LL * num_sms() + groups - 1) / groups;
     a.n_split = (int)std::max(1LL, std::min({want, chunks, cap, (long long)RANGE_SPLIT_MAX}));
-    a.scale_log2 = scale_or_default(opts ? opts->attn_scale : 0.f) * 1.4426950408889634f;
+    a.scale_log2 = scale_or_default(opts ? opts->attn_scale : 0.f) * L2E;
     a.q = q_rope; a.k = k_cache; a.v = v_cache; a.out = out;
     a.part = reinterpret_cast<float *>(scr + NOALLOC_PART_OFF);
     a.arrive = reinterpret_cast<uint32_t *>(scr + NOALLOC_ARRIVE_OFF);
@@ -742,7 +742,7 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
                 s.a.q_rope = q_rope;
                 s.a.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
                 s.a.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
-                s.a.attn_scale_log2 = asc * 1.4426950408889634f;
+                s.a.attn_scale_log2 = asc * L2E;
                 s.a.out = out;
                 s.a.part_sel = reinterpret_cast<float *>(w + L.part_sel);
                 s.a.ovf = reinterpret_cast<uint32_t *>(w + L.ovf);

@@ -12,7 +12,6 @@ namespace rtp {
 constexpr int D = 128;          // head dim
 constexpr int R = 16;           // indexer dim
 constexpr int GMAX = 8;         // largest GQA group handled in one tile
-constexpr int WARP = 32;
 
 // ---------------------------------------------------------------------------
 // status word (first 4 bytes of the workspace): the first error wins
@@ -153,11 +152,6 @@ __device__ __forceinline__ float warp_sum(float v) {
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    return v;
-}
-__device__ __forceinline__ double warp_sum_d(double v) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     return v;
 }
 

@@ -43,7 +43,8 @@ constexpr int SC_THREADS = 256;
 constexpr int SC_WARPS = SC_THREADS / 32;
 constexpr int TILE = 32;                   // tokens per warp tile
 constexpr int MAX_RET_GROUPS = 64;
-constexpr float L2E = 1.4426950408889634f;
+constexpr float L2E = 1.4426950408889634f;     // log2(e)
+constexpr double L2E_D = 1.4426950408889634;
 
 enum ResolveMode : int32_t { MODE_NORMAL = 0, MODE_KEEP_ALL = 1, MODE_EMPTY = 2 };
 
@@ -101,16 +102,7 @@ __device__ __forceinline__ int bin_and_fx(float z, uint32_t &fx) {
     k = min(max(k, 0), 255);
     const uint32_t eb = (uint32_t)(k + (int)BIN_BASE + 1 + s) << (23 - MB);
     const float U = __uint_as_float(eb | ((uint32_t)s & 0x80000000u));
-    fx = __float2uint_rn(ex2_sfu((z - U) * 1.4426950408889634f) * FX_ONE);
-    return 256 + (k ^ s);
-}
-
-// Bin only (same arithmetic as bin_and_fx).
-__device__ __forceinline__ int logit_bin(float z) {
-    const uint32_t u = __float_as_uint(z);
-    const int s = (int)u >> 31;
-    int k = (int)((u << 1) >> (24 - MB)) - (int)BIN_BASE;
-    k = min(max(k, 0), 255);
+    fx = __float2uint_rn(ex2_sfu((z - U) * L2E) * FX_ONE);
     return 256 + (k ^ s);
 }
 
@@ -156,7 +148,7 @@ __host__ __device__ __forceinline__ float bin_upper(int bin) {
 // per unit of mass relative to its own (a constant of the bin; the scans
 // tabulate it in shared memory while they stream).
 __device__ __forceinline__ double octave_factor(int bin) {
-    return exp2_wide((double)(bin_upper(bin) - bin_upper(bin | 15)) * 1.4426950408889634);
+    return exp2_wide((double)(bin_upper(bin) - bin_upper(bin | 15)) * L2E_D);
 }
 
 // A CTA's fixed-point bin sum v (< 2^52) times `unit` as a double, without
@@ -585,7 +577,6 @@ template <> struct NeedsQ<SrcBuffer> : std::false_type {};
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, float p, int N) {
     const int lane = threadIdx.x & 31;
-    constexpr double L2E_D = 1.4426950408889634;
     double ss = 0.0;
 #pragma unroll
     for (int q = 0; q < NREP; ++q) ss += __ldcg(gh + NBIN + q * NSUP + lane);
@@ -630,7 +621,7 @@ __device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, f
     // the boundary octave's bins relative to R (lane 15 = its highest bin),
     // inclusive suffix sums on top of the octaves above
     const double mb = lane < 16 && sv > 0.0
-                          ? sv * (double)ex2_sfu((bin_upper(bin) - R) * 1.4426950408889634f) : 0.0;
+                          ? sv * (double)ex2_sfu((bin_upper(bin) - R) * L2E) : 0.0;
     double incb = mb;
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) {
@@ -795,7 +786,7 @@ __device__ __forceinline__ int scan_value(float z, uint32_t row, int &bin) {
     const int kr = (int)((u << 1) >> (24 - MB)) - (int)BIN_BASE;
     const int k = max(kr, 0) & 255;
     const uint32_t eb = ((uint32_t)(k + (int)BIN_BASE + 1 + s) << (23 - MB)) | (u & 0x80000000u);
-    const uint32_t fx = __float2uint_rn(ex2_sfu(fmaf(z - __uint_as_float(eb), 1.4426950408889634f, 18.0f)));
+    const uint32_t fx = __float2uint_rn(ex2_sfu(fmaf(z - __uint_as_float(eb), L2E, 18.0f)));
     bin = 256 + (k ^ s);
     asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row + 4u * (uint32_t)bin), "r"(fx) : "memory");
     return kr;
@@ -987,20 +978,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
 // ---------------------------------------------------------------------------
 // collect: kept ids above b*, candidates in b*.  grid as scan.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void warp_append(bool c, int h, unsigned lane_lt, uint32_t *cnt_base,
-                                            unsigned &pos) {
-    const unsigned act = __ballot_sync(0xffffffffu, c);
-    if (!act) return;
-    if (c) {
-        const unsigned grp = __match_any_sync(act, h);
-        const int leader = __ffs(grp) - 1;
-        unsigned base = 0;
-        if ((threadIdx.x & 31) == leader) base = atomicAdd(&cnt_base[h], (unsigned)__popc(grp));
-        base = __shfl_sync(grp, base, leader);
-        pos = base + __popc(grp & lane_lt);
-    }
-}
-
 constexpr int COL_THREADS = 512;
 constexpr int COL_WARPS = COL_THREADS / 32;
 
@@ -1577,7 +1554,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         const bool staged = nc <= (unsigned)FIN_CAP;
         const double S = staged ? (double)(0x7fffffffu / nc) : ldexp(1.0, 62) / (double)nc;
         auto fx_of = [&](unsigned long long v) -> unsigned long long {
-            const float m = ex2_sfu((cand_logit(v) - Ub) * 1.4426950408889634f);
+            const float m = ex2_sfu((cand_logit(v) - Ub) * L2E);
             return (unsigned long long)((double)m * S);
         };
         if (tid == 0) { s_min = ~0ull; s_max = 0ull; s_kept = 0ull; s_base2 = 0u; }
@@ -1603,7 +1580,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             }
         }
         __syncthreads();
-        const double tS = r.target / (double)ex2_sfu((Ub - r.R) * 1.4426950408889634f) * S;
+        const double tS = r.target / (double)ex2_sfu((Ub - r.R) * L2E) * S;
         unsigned long long T = !(tS < 9.0e18) ? ~0ull : (unsigned long long)llrint(tS);
         const unsigned long long diff = s_min ^ s_max;
         unsigned long long theta = s_min;          // one candidate (or all equal): keep all
@@ -1725,7 +1702,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         __syncthreads();
         count = (int)(base0 + kbase);
         fin_theta = theta;
-        const double kept_mass = (double)s_kept / S * (double)ex2_sfu((Ub - r.R) * 1.4426950408889634f);
+        const double kept_mass = (double)s_kept / S * (double)ex2_sfu((Ub - r.R) * L2E);
         mass = (float)((r.above + kept_mass) / r.Z);
     }
     // Rank 0's global writes go out last (a global store before a block or
