@@ -4,9 +4,10 @@ step; 48 layers per step for the 48-layer workload) on synthetic caches.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload ctx512k] [--p P]
     python bench.py --impl reference ...   # the CPU oracle, timed on host cores
 
-Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) are independent
-replicas of the workload per rank (the step shards by sequence and KV head
-with no data exchange): value = steps of all ranks / max rank time.
+Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) give every rank
+sequences of its own, seeded per rank, of the same workload shape (the step
+shards by sequence and KV head with no data exchange): value = steps of all
+ranks / max rank time.
 """
 from __future__ import annotations
 
@@ -27,7 +28,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from dynamic_top_sparse_b200 import ops, synth  # noqa: E402
-from dynamic_top_sparse_b200.dist import allreduce_max, barrier  # noqa: E402
+from dynamic_top_sparse_b200.dist import allreduce_max, barrier, rank_seed  # noqa: E402
 
 METRIC = "sparse decode attention steps/s and achieved HBM GB/s (% peak) at 64K-1M ctx"
 L2_BYTES = 126 * 2 ** 20
@@ -220,7 +221,8 @@ def index_bytes(spec, layers):
 # ------------------------------------------------------------------ our arm
 
 def run_ours(args, rank, world, dev):
-    spec, layers0 = build_workload(args.workload)
+    # each rank serves sequences of its own (rank 0's are the single-GPU workload)
+    spec, layers0 = build_workload(args.workload, seed=rank_seed(0, rank))
     if args.p is not None:
         spec.p = args.p
     p = spec.p

@@ -1,8 +1,6 @@
 """Comparison helpers shared by the GPU parity tests (test infrastructure)."""
 from __future__ import annotations
 
-import math
-
 import numpy as np
 import torch
 
@@ -116,15 +114,6 @@ class GpuCase:
         st = self.ws.check()
         assert st == 0, f"device status {st}: {ops.error_string(st)}"
         return out, sel_idx, sel_cnt, sel_mass
-
-
-def oracle_inputs(gc: GpuCase, kidx_override=None):
-    """Host fp64 copies of the case tensors (the oracle's own inputs)."""
-    c = gc.c
-    kidx = c.kidx_cache if kidx_override is None else kidx_override
-    return dict(q=np64(c.q), q_rope=None if c.q_rope is None else np64(c.q_rope),
-                k=np64(c.k_cache), v=np64(c.v_cache), kidx=np64(kidx) if isinstance(kidx, torch.Tensor) else kidx,
-                Wq=np64(c.W_q_idx), Wk=np64(c.W_k_idx), seq=c.seq_lens.cpu().numpy())
 
 
 def oracle_kidx(gc: GpuCase, idx_dtype: str, with_current: bool):

@@ -8,7 +8,7 @@ import torch
 
 import oracle
 from dynamic_top_sparse_b200 import ops, synth
-from tests.helpers import (MASS_TOL, OUT_TOL_SAME_SET, GpuCase, check_selection, np64,
+from tests.helpers import (OUT_TOL_SAME_SET, GpuCase, check_selection, np64,
                            within)
 
 pytestmark = pytest.mark.gpu

@@ -1,9 +1,7 @@
 """Device-side error reporting: bad device-resident arguments and logits out
 of the binned range are recorded in the workspace status word and returned
 by rtp_check(); the kernels skip the offending work (no fault, no hang)."""
-import math
 
-import numpy as np
 import pytest
 import torch
 

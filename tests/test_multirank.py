@@ -67,3 +67,10 @@ def test_shard_units_partition(B, H_kv, world):
 def test_shard_units_rejects_bad_rank():
     with pytest.raises(ValueError):
         rdist.shard_units(2, 2, 2, 2)
+
+
+def test_rank_seeds_are_distinct_and_rank0_keeps_the_base():
+    seeds = [rdist.rank_seed(0, r) for r in range(8)]
+    assert seeds[0] == 0                      # rank 0 serves the single-GPU workload
+    assert len(set(seeds)) == 8
+    assert not set(seeds) & {rdist.rank_seed(1, r) for r in range(8)}
