@@ -8,4 +8,4 @@ from .rtpurbo import (HEAD_LOCAL, HEAD_RETRIEVAL, Selection, StepResult,  # noqa
                       append_index_keys, attend, decode_step, default_scale,
                       dense_decode, descending_order, index_logits, local_rows,
                       project_index_key, query_index, round_to, round_to_bf16,
-                      round_to_f32, softmax_mass, topp_select)
+                      round_to_f32, softmax_mass, topk_select, topp_select)

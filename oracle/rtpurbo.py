@@ -206,6 +206,27 @@ def topp_select(z: np.ndarray, p: float) -> Selection:
     return Selection(kept=order[:keep], order=order, excl=excl, pi=pi)
 
 
+def topk_select(z: np.ndarray, k: int) -> Selection:
+    """The k tokens with the largest scores: the fixed-budget selection that
+    the summary's Method section 3 ("dynamic top-p vs static top-k") sets
+    the top-p rule against.  The first min(k, N) tokens of the same
+    descending order as topp_select (equal scores by ascending index); a
+    budget below one token is an error (attention over no rows is
+    undefined).
+    """
+    k = int(k)
+    if k < 1:
+        raise ValueError("k < 1")
+    z = np.asarray(z, np.float64)
+    n = z.shape[0]
+    if n == 0:
+        raise ValueError("no tokens")
+    order = descending_order(z)
+    pi = softmax_mass(z)
+    excl = np.concatenate(([0.0], np.cumsum(pi[order])[:-1]))
+    return Selection(kept=order[:min(k, n)], order=order, excl=excl, pi=pi)
+
+
 # ---------------------------------------------------------------------------
 # a6 / a7: attention over a set of rows
 # ---------------------------------------------------------------------------
@@ -248,7 +269,7 @@ class StepResult:
 def decode_step(q, q_rope, k_cache, v_cache, kidx_cache, W_q_idx, head_class,
                 seq_lens, p: float, window: int, n_sink: int,
                 idx_scale: float | None = None, attn_scale: float | None = None,
-                heads=None) -> StepResult:
+                heads=None, topk: int | None = None) -> StepResult:
     """One decode step of one layer.
 
     q: [B, H_q, d] pre-RoPE query (indexer input); q_rope: [B, H_q, d]
@@ -258,7 +279,8 @@ def decode_step(q, q_rope, k_cache, v_cache, kidx_cache, W_q_idx, head_class,
 
     Query head h belongs to KV head h // (H_q // H_kv).  Local heads attend
     over local_rows(); retrieval heads score every cached token with the
-    indexer, keep the top-p set, and attend exactly over those rows.
+    indexer, keep the top-p set (or, with ``topk``, the top-k set; p is then
+    unused), and attend exactly over those rows.
     ``heads`` optionally restricts the computation to a list of (b, h).
     """
     q = np.asarray(q, np.float64)
@@ -278,7 +300,7 @@ def decode_step(q, q_rope, k_cache, v_cache, kidx_cache, W_q_idx, head_class,
         V = v_cache[b, g, :N]
         if head_class[g] == HEAD_RETRIEVAL:
             z = index_logits(query_index(q[b, h], W_q_idx[h]), kidx_cache[b, g, :N], isc)
-            sel = topp_select(z, p)
+            sel = topp_select(z, p) if topk is None else topk_select(z, topk)
             res.selections[(b, h)] = sel
             res.z[(b, h)] = z
             rows = sel.kept

@@ -361,3 +361,80 @@ def test_needle_margin_in_index_space():
         assert abs(np.median(z[nd]) - lift) < 1.5
         # background keys ~ N(0, I_r): logit std is |q_idx| / sqrt(d)
         assert abs(bg.std() / (np.linalg.norm(qi) / math.sqrt(128)) - 1.0) < 0.1
+
+
+# ------------------------------------------- static top-k (the fixed budget)
+
+@pytest.mark.parametrize("seed", range(30))
+def test_topk_bruteforce(seed):
+    """Among all k-subsets the kept set has the largest mass; every kept
+    score is >= every dropped one; at the k-th score the lowest indices
+    are the ones kept."""
+    g = np.random.default_rng(100 + seed)
+    n = int(g.integers(1, 11))
+    z = (g.integers(-2, 3, n) * 0.7) if seed % 2 == 0 else g.normal(0, 1.5, n)
+    z = np.asarray(z, np.float64)
+    k = int(g.integers(1, n + 2))
+    ez = np.array([math.exp(v - max(z)) for v in z])
+    pi = ez / math.fsum(ez)
+    sel = oracle.topk_select(z, k)
+    kept = sel.kept.tolist()
+    assert len(kept) == min(k, n) and len(set(kept)) == len(kept)
+    best = max(math.fsum(pi[list(c)]) for c in itertools.combinations(range(n), min(k, n)))
+    assert abs(math.fsum(pi[kept]) - best) < 1e-12
+    dropped = [i for i in range(n) if i not in kept]
+    if dropped:
+        assert min(z[kept]) >= max(z[dropped])
+        edge = min(z[kept])
+        tied_kept = sorted(i for i in kept if z[i] == edge)
+        tied_all = sorted(i for i in range(n) if z[i] == edge)
+        assert tied_kept == tied_all[:len(tied_kept)]
+
+
+def test_topk_closed_forms():
+    z = np.array([0.1, 3.0, -1.0, 3.0, 2.9])
+    assert oracle.topk_select(z, 1).kept.tolist() == [1]            # argmax, lowest index
+    assert sorted(oracle.topk_select(z, 5).kept.tolist()) == [0, 1, 2, 3, 4]
+    assert sorted(oracle.topk_select(z, 99).kept.tolist()) == [0, 1, 2, 3, 4]
+    assert oracle.topk_select(np.full(50, -0.3), 7).kept.tolist() == list(range(7))
+    for bad in (0, -3):
+        with pytest.raises(ValueError):
+            oracle.topk_select(z, bad)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_topk_with_the_topp_size_is_the_topp_set(seed):
+    """The top-p set is a prefix of the descending order, so the top-k set
+    of its size is the same set."""
+    g = np.random.default_rng(200 + seed)
+    z = g.normal(0, 2.0, 3000)
+    p = float(g.uniform(0.1, 0.99))
+    a = oracle.topp_select(z, p).kept
+    b = oracle.topk_select(z, len(a)).kept
+    assert set(a.tolist()) == set(b.tolist())
+
+
+def test_step_with_topk_attends_the_k_best_index_scores():
+    """The step with a budget k equals masked dense attention over the k
+    tokens of largest index score (ranked here with Python's sort), and
+    with k >= N equals dense attention."""
+    g = np.random.default_rng(21)
+    B, H_q, H_kv, d, r, N = 1, 4, 2, 16, 4, 29
+    q = g.normal(0, 1, (B, H_q, d))
+    K = g.normal(0, 1, (B, H_kv, N, d))
+    V = g.normal(0, 1, (B, H_kv, N, d))
+    kidx = g.normal(0, 1, (B, H_kv, N, r))
+    W = g.normal(0, 0.3, (H_q, r, d))
+    hc = np.array([1, 1], np.uint8)
+    sc = 1 / math.sqrt(d)
+    for k in (1, 5, N, N + 3):
+        res = oracle.decode_step(q, None, K, V, kidx, W, hc, [N], p=0.5, window=4, n_sink=1, topk=k)
+        for h in range(H_q):
+            gq = h // 2
+            qi = [sum(W[h, j, i] * q[0, h, i] for i in range(d)) for j in range(r)]
+            zs = [sc * sum(qi[j] * kidx[0, gq, t, j] for j in range(r)) for t in range(N)]
+            best = sorted(range(N), key=lambda t: (-zs[t], t))[:min(k, N)]
+            mask = np.zeros(N, bool)
+            mask[best] = True
+            ref = _masked_dense_attention(q[0, h], K[0, gq], V[0, gq], mask, sc)
+            np.testing.assert_allclose(res.out[0, h], ref, rtol=0, atol=1e-12)
