@@ -1,0 +1,55 @@
+"""Host-side arithmetic of bench.py (CPU): the step's required bytes, the
+numerator of its roofline."""
+import types
+
+import numpy as np
+import pytest
+import torch
+
+import bench
+from dynamic_top_sparse_b200 import synth
+
+
+def _layer(lens, hc, H_q):
+    case = types.SimpleNamespace(seq_lens=torch.tensor(lens, dtype=torch.int32))
+    return types.SimpleNamespace(case=case, hc=np.asarray(hc, np.uint8), H_q=H_q)
+
+
+def _spec(B, N, p=0.9, kv="bf16", idx="bf16"):
+    return synth.Spec("t", B=B, H_q=8, H_kv=2, N=N, kv_dtype=kv, idx_dtype=idx, p=p, window=16, n_sink=4)
+
+
+def test_required_bytes_counts_the_group_union_once():
+    """Group 0 retrieval (query heads 0-3), group 1 local; two sequences.
+    Kept rows of the group's heads overlap: their union is read once."""
+    spec = _spec(B=2, N=100)
+    L = _layer([100, 60], [1, 0], 8)
+    idx = np.full((2, 8, 100), -1, np.int32)
+    cnt = np.zeros((2, 8), np.int32)
+    kept = {(0, 0): [5, 6, 7], (0, 1): [6, 7, 8], (0, 2): [99], (0, 3): [5],
+            (1, 0): [0], (1, 1): [0], (1, 2): [0], (1, 3): [59, 58]}
+    for (b, h), ids in kept.items():
+        idx[b, h, :len(ids)] = ids
+        cnt[b, h] = len(ids)
+    got = bench.required_bytes(spec, [L], [(idx, cnt)])
+    kidx = (100 + 60) * 16 * 2                      # index keys of the retrieval group, bf16
+    rows = (5 + 3) * 2 * 128 * 2                    # unions {5,6,7,8,99} and {0,58,59}: K and V rows
+    local = (4 + 16) * 2 * 128 * 2 * 2              # 4 sinks + 16 window rows, both sequences
+    wq = 4 * 16 * 128 * 4                           # W_q_idx of the 4 retrieval query heads, fp32
+    assert got == kidx + rows + local + wq
+
+
+def test_required_bytes_short_sequence_reads_each_local_row_once():
+    """N below window + sinks: every row once, not sinks and window twice."""
+    spec = _spec(B=1, N=10)
+    L = _layer([10], [0, 0], 8)
+    got = bench.required_bytes(spec, [L], [(np.zeros((1, 8, 10), np.int32), np.zeros((1, 8), np.int32))])
+    assert got == 2 * 10 * 2 * 128 * 2
+
+
+@pytest.mark.parametrize("p", [1.0, 1.5])
+def test_required_bytes_keep_all_reads_every_row(p):
+    spec = _spec(B=1, N=50, p=p, kv="f32", idx="f32")
+    L = _layer([50], [1, 1], 8)
+    got = bench.required_bytes(spec, [L], None)
+    assert got == 2 * (50 * 16 * 4 + 50 * 2 * 128 * 4) + 8 * 16 * 128 * 4
