@@ -53,3 +53,50 @@ def test_required_bytes_keep_all_reads_every_row(p):
     L = _layer([50], [1, 1], 8)
     got = bench.required_bytes(spec, [L], None)
     assert got == 2 * (50 * 16 * 4 + 50 * 2 * 128 * 4) + 8 * 16 * 128 * 4
+
+
+class _FakeNvml:
+    """Reads only: clocks and clock-event reason words from fixed lists."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self, clocks, reasons, fail_init=False):
+        self._c, self._r, self._fail = iter(clocks), iter(reasons), fail_init
+
+    def nvmlInit(self):
+        if self._fail:
+            raise RuntimeError("no driver")
+
+    def nvmlDeviceGetHandleByPciBusId(self, bus):
+        raise RuntimeError("by index instead")
+
+    def nvmlDeviceGetHandleByIndex(self, i):
+        return ("gpu", i)
+
+    def nvmlDeviceGetMaxClockInfo(self, h, which):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, which):
+        return next(self._c)
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return next(self._r)
+
+
+def test_clock_report_decodes_reasons_and_takes_the_median(monkeypatch):
+    import sys
+    fake = _FakeNvml([1965, 1965, 1800, 1965, 1300], [0x1, 0x4, 0x0, 0x4 | 0x20, 0x8])
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    c = bench.Clocks(0)
+    for _ in range(5):
+        c._sample()
+    rep = c.report()
+    assert rep["sm_mhz"] == 1965 and rep["sm_max_mhz"] == 1965 and rep["samples"] == 5
+    # gpu_idle is not a slowdown; the others are named as NVML defines the bits
+    assert rep["reasons"] == ["hw_slowdown", "sw_power_cap", "sw_thermal_slowdown"]
+
+
+def test_clock_report_without_nvml(monkeypatch):
+    import sys
+    monkeypatch.setitem(sys.modules, "pynvml", _FakeNvml([], [], fail_init=True))
+    rep = bench.Clocks(0).report()
+    assert rep["sm_mhz"] is None and rep["reasons"] == [] and "NVML" in rep["note"]
