@@ -100,3 +100,21 @@ def test_clock_report_without_nvml(monkeypatch):
     monkeypatch.setitem(sys.modules, "pynvml", _FakeNvml([], [], fail_init=True))
     rep = bench.Clocks(0).report()
     assert rep["sm_mhz"] is None and rep["reasons"] == [] and "NVML" in rep["note"]
+
+
+def test_recorded_traffic_is_used_only_while_the_scan_sources_are_unchanged(tmp_path, monkeypatch):
+    import json
+    import shutil
+    src = tmp_path / "dynamic_top_sparse_b200" / "csrc"
+    src.mkdir(parents=True)
+    for name in bench.SCAN_SOURCES:
+        shutil.copy(f"{bench.ROOT}/dynamic_top_sparse_b200/csrc/{name}", src / name)
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    rec = {"records": [{"kernel": "hist", "workload": "w", "csrc": bench.csrc_hash(), "bytes_per_launch": 123}]}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    assert bench.traffic_for("hist", "w") == 123
+    assert bench.traffic_for("hist", "other workload") is None
+    with open(src / bench.SCAN_SOURCES[-1], "a") as f:
+        f.write("\n// edited\n")
+    assert bench.traffic_for("hist", "w") is None
