@@ -118,3 +118,29 @@ def test_recorded_traffic_is_used_only_while_the_scan_sources_are_unchanged(tmp_
     with open(src / bench.SCAN_SOURCES[-1], "a") as f:
         f.write("\n// edited\n")
     assert bench.traffic_for("hist", "w") is None
+
+
+def test_reference_arm_under_two_ranks_prints_one_line_from_rank0():
+    """The reference arm (the oracle on host cores) launched like the
+    multi-GPU bench: rank 0 prints one JSON line, the other rank exits 0
+    without output."""
+    import json
+    import os
+    import socket
+    import subprocess
+    import sys
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--steps", "3", "--warmup", "3", "--workload", "ctx4k-fp32", "--cpu-seconds", "1"]
+    r = subprocess.run(cmd, cwd=bench.ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] == 1
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["value"] == rec["value"]
