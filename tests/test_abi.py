@@ -140,3 +140,14 @@ def test_other_calls_reject_bad_arguments(L):
     assert L.rtp_check(None, None) == ops.RTP_ERR_WORKSPACE
     assert L.rtp_selftest_wait_timeout(None, None) == ops.RTP_ERR_INVALID_ARG
     assert L.rtp_selftest_wait_timeout(FAKE + 2, None) == ops.RTP_ERR_INVALID_ARG     # misaligned
+
+
+def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
+    """No CPU fallback: with the library missing every call raises."""
+    from dynamic_top_sparse_b200 import ops
+    monkeypatch.setattr(ops, "_lib", None)
+    monkeypatch.setattr(ops, "LIB_PATH", str(tmp_path / "librtp.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        ops.lib()
+    with pytest.raises(RuntimeError, match="missing"):
+        ops.error_string(0)
