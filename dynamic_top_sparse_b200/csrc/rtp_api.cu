@@ -365,6 +365,10 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
     long long want = ((long long)per_sm * num_sms() + (long long)d->B * a.n_grp - 1) / ((long long)d->B * a.n_grp);
     if (max_ctas > 0) want = std::max(1LL, (long long)max_ctas / ((long long)d->B * a.n_grp));
     a.n_split = (int)std::max(1LL, std::min(want, std::min(chunks, (long long)RANGE_SPLIT_MAX)));
+    // Slots are indexed by (b, g) at a fixed stride, not by this launch's
+    // split count: the local and the dense retrieval launches of one step run
+    // at the same time on two streams with different n_split.
+    a.slots = RANGE_SPLIT_MAX;
     a.scale_log2 = attn_scale * L2E;
     a.q = q; a.k = k; a.v = v; a.out = out;
     a.part = reinterpret_cast<float *>(ws + L.part_range);
@@ -656,6 +660,7 @@ int rtp_dense_decode_noalloc(const rtp_dims *dims, const rtp_opts *opts, const f
     const long long chunks = (dims->N_max + 255) / 256;
     const long long want = (2LL * num_sms() + groups - 1) / groups;
     a.n_split = (int)std::max(1LL, std::min({want, chunks, cap, (long long)RANGE_SPLIT_MAX}));
+    a.slots = a.n_split;
     a.scale_log2 = scale_or_default(opts ? opts->attn_scale : 0.f) * L2E;
     a.q = q_rope; a.k = k_cache; a.v = v_cache; a.out = out;
     a.part = reinterpret_cast<float *>(scr + NOALLOC_PART_OFF);

@@ -83,12 +83,13 @@ struct RangeArgs {
     int dense;
     int window, n_sink;
     int n_split;
+    int slots;          // partial slots reserved per KV group (>= n_split)
     float scale_log2;
     const float *q;
     const void *k;
     const void *v;
     float *out;
-    float *part;        // [B*H_kv][n_split][GMAX][PSTRIDE]
+    float *part;        // [B*H_kv][slots][GMAX][PSTRIDE]
     uint32_t *arrive;   // [B*H_kv]
     uint32_t *status;
 };
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) atomicAdd(&O[h][lane * 4 + i], acc[h][i]);
     __syncthreads();
-    float *pp = a.part + (bg * a.n_split + blockIdx.x) * GMAX * PSTRIDE;
+    float *pp = a.part + (bg * a.slots + blockIdx.x) * GMAX * PSTRIDE;
     for (int i = tid; i < G * PSTRIDE; i += blockDim.x) {
         const int h = i / PSTRIDE, e = i % PSTRIDE;
         pp[i] = e == 0 ? s_m[h] : (e == 1 ? s_l[h] : (e < POFF ? 0.0f : O[h][e - POFF]));
@@ -247,7 +248,7 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    merge_partials(a.part + bg * a.n_split * GMAX * PSTRIDE, n_active, GMAX * PSTRIDE, G, a.out + bh0 * D);
+    merge_partials(a.part + bg * a.slots * GMAX * PSTRIDE, n_active, GMAX * PSTRIDE, G, a.out + bh0 * D);
     if (tid == 0) a.arrive[bg] = 0;
 }
 

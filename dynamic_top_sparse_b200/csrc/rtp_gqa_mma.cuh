@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a
         s_o[warp][gid][32 * tig + 16 + j] = o[j][1];
     }
     __syncthreads();
-    float *pp = a.part + (bg * a.n_split + blockIdx.x) * GMAX * PSTRIDE;
+    float *pp = a.part + (bg * a.slots + blockIdx.x) * GMAX * PSTRIDE;
     for (int i = tid; i < G * D; i += blockDim.x) {
         const int h = i / D, d = i % D;
         float M = -INFINITY;
@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    merge_partials(a.part + bg * a.n_split * GMAX * PSTRIDE, n_active, GMAX * PSTRIDE, G, a.out + bh0 * D);
+    merge_partials(a.part + bg * a.slots * GMAX * PSTRIDE, n_active, GMAX * PSTRIDE, G, a.out + bh0 * D);
     if (tid == 0) a.arrive[bg] = 0;
 }
 

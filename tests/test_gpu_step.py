@@ -99,6 +99,44 @@ def test_step_p_one_equals_dense():
     _compare(gc, out, None, None, None, 1.0, with_current=False)
 
 
+def _p_ge_one_mixed(gc: GpuCase, heads=None, repeats=20):
+    """p >= 1 with local and retrieval heads in one step: the local heads'
+    window attention and the retrieval heads' dense attention run at the
+    same time on two streams, each split over CTAs with its own split count.
+    Every head against the oracle's step (p >= 1 keeps every token), the
+    retrieval heads also against the oracle's dense attention, and the same
+    output, bit for bit, on every repeat over one workspace."""
+    c = gc.c
+    G = gc.H_q // gc.H_kv
+    ret = [(b, h) for (b, h) in (heads or [(b, h) for b in range(gc.B) for h in range(gc.H_q)])
+           if c.head_class[h // G] == oracle.HEAD_RETRIEVAL]
+    dense = oracle.dense_decode(np64(c.q_rope if c.q_rope is not None else c.q), np32(c.k_cache),
+                                np32(c.v_cache), c.seq_lens.cpu().numpy(), heads=ret)
+    for p in (1.0, 1.5):
+        first, _, _, _ = gc.step(p, want_sel=False)
+        _compare(gc, first, None, None, None, p, heads=heads, with_current=False)
+        o = first.cpu().numpy()
+        for b, h in ret:
+            within(o[b, h], dense[b, h], OUT_TOL, f"p={p} b={b} h={h} vs dense")
+        for _ in range(repeats):
+            again, _, _, _ = gc.step(p, want_sel=False)
+            assert torch.equal(again, first), f"p={p}: output changed on a repeat"
+
+
+@pytest.mark.parametrize("hc", [(1, 0), (0, 1, 1, 0)])
+def test_step_p_ge_one_mixed_heads_small(hc):
+    spec = synth.small_spec(B=2, H_q=8 * len(hc), H_kv=len(hc), N=20000, head_class=hc,
+                            seq_lens=[20000, 9000], window=4096, n_sink=4)
+    _p_ge_one_mixed(GpuCase(synth.make_case(spec)))
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("key", ["ctx64k", "ctx512k"])
+def test_step_p_ge_one_mixed_heads(key):
+    gc = GpuCase(synth.make_case(key, device="cuda"))
+    _p_ge_one_mixed(gc)
+
+
 def test_step_repeatable_on_one_workspace():
     spec = synth.small_spec(B=2, H_q=16, H_kv=2, N=6000, head_class=(1, 0))
     gc = GpuCase(synth.make_case(spec))
