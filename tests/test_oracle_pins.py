@@ -55,6 +55,13 @@ def test_golden_bf16_rounding(golden_dir):
         assert y == float(c["y"]), c
 
 
+def test_golden_f32_rounding(golden_dir):
+    fx = _load(golden_dir, "f32_rounding.json")
+    for c in fx["cases"]:
+        y = float(oracle.round_to(np.array([float(c["x"])]), "f32")[0])
+        assert y == float(c["y"]), c
+
+
 def test_bf16_rounding_matches_torch_cast():
     """fp32 -> bf16 rounding of torch's cast (round to nearest even) agrees
     with the oracle on fp32 inputs (single rounding from fp32)."""
@@ -308,7 +315,8 @@ def test_index_projection_selector():
                                [3.0, 1.0, 5.0], rtol=0, atol=0)
 
 
-def test_append_index_keys_rows_and_rounding():
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_append_index_keys_rows_and_rounding(dtype, golden_dir):
     g = np.random.default_rng(8)
     B, H_kv, N_max, d, r, T = 2, 2, 10, 8, 3, 2
     W = np.zeros((H_kv, r, d))
@@ -317,14 +325,20 @@ def test_append_index_keys_rows_and_rounding():
     W[:, 2, 7] = 0.5
     k = g.normal(0, 1, (B, H_kv, T, d))
     cache = np.full((B, H_kv, N_max, r), -7.0)
-    out = oracle.append_index_keys(cache, k, W, [3, 8], "bf16", head_class=[1, 0])
+    # one key of the f32 cache carries a hand-worked rounding case: 1 + 3*2^-24
+    # is halfway between two fp32 values and goes to the even one, 1 + 2^-22
+    k[0, 0, 0, 1] = 1 + 3 * 2.0 ** -24
+    out = oracle.append_index_keys(cache, k, W, [3, 8], dtype, head_class=[1, 0])
+    rnd = oracle.round_to_bf16 if dtype == "bf16" else oracle.round_to_f32
     for b, p0 in enumerate([3, 8]):
-        exp = oracle.round_to_bf16(np.stack([k[b, 0, :, 1], k[b, 0, :, 3], 0.5 * k[b, 0, :, 7]], -1))
+        exp = rnd(np.stack([k[b, 0, :, 1], k[b, 0, :, 3], 0.5 * k[b, 0, :, 7]], -1))
         np.testing.assert_array_equal(out[b, 0, p0:p0 + T], exp)
         mask = np.ones(N_max, bool)
         mask[p0:p0 + T] = False
         assert np.all(out[b, 0, mask] == -7.0)
         assert np.all(out[b, 1] == -7.0)      # local head untouched
+    # bf16: 1 + 3*2^-24 is far below the halfway point 1 + 2^-8, so it is 1
+    assert out[0, 0, 3, 0] == (1 + 2.0 ** -22 if dtype == "f32" else 1.0)
 
 
 # ------------------------------------------------------ synthetic workloads
