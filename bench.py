@@ -180,10 +180,13 @@ def build_workload(key: str, seed: int = 0):
     return spec, layers
 
 
-def required_bytes(spec, layers, sel):
-    """Algorithmic bytes a step must read: index keys of retrieval heads,
-    the union of kept K/V rows per KV group, window+sink rows of local
-    heads, and the query projector of retrieval heads."""
+def required_bytes(spec, layers, sel, p=None):
+    """Algorithmic bytes a step must read: index keys of retrieval heads
+    (only when a threshold is computed, p < 1), the union of kept K/V rows
+    per KV group (every row at p >= 1), window+sink rows of local heads, and
+    the query projector of retrieval heads (only when selecting)."""
+    p = spec.p if p is None else p
+    selecting = p < 1.0
     total = 0
     kv_el = 2 if spec.kv_dtype == "bf16" else 4
     ix_el = 2 if spec.idx_dtype == "bf16" else 4
@@ -194,10 +197,12 @@ def required_bytes(spec, layers, sel):
             N = lens[b]
             for g in range(L.hc.shape[0]):
                 if L.hc[g] == synth.HEAD_RETRIEVAL:
-                    total += N * spec.r * ix_el
-                    if spec.p >= 1.0 or sel is None:
+                    if not selecting or sel is None:
                         total += N * 2 * spec.d * kv_el
+                        if selecting:
+                            total += N * spec.r * ix_el
                     else:
+                        total += N * spec.r * ix_el
                         idx, cnt = sel[li]
                         u = set()
                         for h in range(g * G, (g + 1) * G):
@@ -206,33 +211,54 @@ def required_bytes(spec, layers, sel):
                 else:
                     rows = min(N, spec.n_sink) + (N - max(min(N, spec.n_sink), N - spec.window))
                     total += rows * 2 * spec.d * kv_el
-        n_rq = sum(G for g in range(L.hc.shape[0]) if L.hc[g] == synth.HEAD_RETRIEVAL)
-        total += n_rq * spec.r * spec.d * 4
+        if selecting:
+            n_rq = sum(G for g in range(L.hc.shape[0]) if L.hc[g] == synth.HEAD_RETRIEVAL)
+            total += n_rq * spec.r * spec.d * 4
     return total
 
 
 def index_bytes(spec, layers):
+    """Index keys the scan reads per step (every layer's retrieval groups)."""
     ix_el = 2 if spec.idx_dtype == "bf16" else 4
-    L = layers[0]
-    n_ret = int((L.hc == synth.HEAD_RETRIEVAL).sum())
-    return spec.B * n_ret * spec.N * spec.r * ix_el
+    tot = 0
+    for L in layers:
+        n_ret = int((L.hc == synth.HEAD_RETRIEVAL).sum())
+        tot += n_ret * int(L.case.seq_lens.sum()) * spec.r * ix_el
+    return tot
+
+
+def replicas_for(spec, req, max_replicas):
+    """Rotating cache replicas so that K steps in a row read >= 3 x L2 of
+    distinct required bytes (one replica when a step alone exceeds that)."""
+    if spec.layers > 1:
+        return 1
+    return max(1, min(max_replicas, math.ceil(3 * L2_BYTES / max(req, 1))))
 
 
 # ------------------------------------------------------------------ our arm
 
-def run_ours(args, rank, world, dev):
-    # each rank serves sequences of its own (rank 0's are the single-GPU workload)
-    spec, layers0 = build_workload(args.workload, seed=rank_seed(0, rank))
-    if args.p is not None:
-        spec.p = args.p
-    p = spec.p
-    one_step_bytes = None
-    out = torch.empty((spec.B, spec.H_q, spec.d), device=dev)
-    ws = ops.Workspace(layers0[0].dims)
+class Bench:
+    """One workload on this rank: its layers, rotating replicas, a workspace
+    and the step through the C ABI."""
 
-    def step(layers, prof=None, sel=None):
+    def __init__(self, key, seed, dev):
+        self.key = key
+        self.spec, self.layers0 = build_workload(key, seed=seed)
+        self.dev = dev
+        self.out = torch.empty((self.spec.B, self.spec.H_q, self.spec.d), device=dev)
+        self.ws = ops.Workspace(self.layers0[0].dims)
+        self.reps = [self.layers0]
+        self.stream = torch.cuda.Stream()
+
+    def set_replicas(self, n):
+        while len(self.reps) < n:
+            self.reps.append([L.clone_caches() for L in self.layers0])
+        self.reps = self.reps[:n]
+
+    def step(self, layers, p, prof=None, sel=None):
+        spec = self.spec
         for li, L in enumerate(layers):
-            ops.append_index_keys(L.dims, L.k_new, L.Wk, L.pos, L.hc, L.kidx, ws)
+            ops.append_index_keys(L.dims, L.k_new, L.Wk, L.pos, L.hc, L.kidx, self.ws)
             opts = None
             if prof is not None or sel is not None:
                 kw = {}
@@ -240,184 +266,302 @@ def run_ours(args, rank, world, dev):
                     kw = dict(sel_idx=sel[li][0], sel_count=sel[li][1])
                 opts = ops.make_opts(prof=prof, **kw)
             ops.decode_step(L.dims, L.q, L.q_rope, L.k, L.v, L.kidx, L.Wq, L.hc, p, spec.window,
-                            spec.n_sink, out, ws, opts)
+                            spec.n_sink, self.out, self.ws, opts)
 
-    # kept sets of one step -> required bytes
-    sel = [(torch.full((spec.B, spec.H_q, L.k.shape[2]), -1, dtype=torch.int32, device=dev),
-            torch.zeros((spec.B, spec.H_q), dtype=torch.int32, device=dev)) for L in layers0]
-    step(layers0, sel=sel)
-    st = ws.check()
-    if st:
-        raise RuntimeError(f"device status {st}: {ops.error_string(st)}")
-    req = required_bytes(spec, layers0, [(a.cpu().numpy(), b.cpu().numpy()) for a, b in sel])
-    kept = [[int(x) for x in b.cpu().numpy().ravel() if x > 0] for _, b in sel]
-    del sel
-
-    # rotating replicas so that no step reads what the previous ones left in L2
-    n_rep = 1 if spec.layers > 1 else max(1, math.ceil(3 * L2_BYTES / max(req, 1)))
-    n_rep = min(n_rep, args.max_replicas)
-    reps = [layers0] + [[L.clone_caches() for L in layers0] for _ in range(n_rep - 1)]
-
-    # launches per step (all kernels)
-    pr_all = ops.Profiler(256)
-    step(reps[0], prof=pr_all)
-    torch.cuda.synchronize()
-    # rtp_append_index_keys takes no options, so its one launch per layer is
-    # not in the profiler's count
-    launches_per_step = pr_all.p.count + len(layers0)
-    pr_all.close()
-
-    # CUDA graph per replica
-    graphs = []
-    s = torch.cuda.Stream()
-    s.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(s):
-        for R in reps:
-            step(R)
-    torch.cuda.current_stream().wait_stream(s)
-    torch.cuda.synchronize()
-    for R in reps:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step(R)
-        graphs.append(g)
-    torch.cuda.synchronize()
-
-    for i in range(args.warmup):
-        graphs[i % n_rep].replay()
-    torch.cuda.synchronize()
-
-    clocks = Clocks(dev.index)
-    barrier(world)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with clocks:
-        e0.record()
-        for i in range(args.steps):
-            graphs[i % n_rep].replay()
-        e1.record()
-        torch.cuda.synchronize()
-    barrier(world)
-    ms = e0.elapsed_time(e1)
-    ms_max = allreduce_max(ms, world, dev)
-    ms_per_step = ms_max / args.steps
-    value = world * args.steps / (ms_max / 1e3)
-
-    # per-kernel device times: the step captured with event-record nodes
-    # around every kernel (one graph per replica, distinct event slots),
-    # replayed with a sync after each replay to read the slots
-    per_step_slots = launches_per_step + 4
-    pr = ops.Profiler(per_step_slots * n_rep)
-    pgraphs = []
-    for R in reps:
-        g = torch.cuda.CUDAGraph()
-        first = pr.p.count
-        with torch.cuda.graph(g):
-            step(R, prof=pr)
-        pgraphs.append((g, first, pr.p.count))
-    torch.cuda.synchronize()
-    n_prof = max(1, min(args.steps, args.prof_steps))
-    breakdown = {}
-    for i in range(n_prof + n_rep):
-        g, lo, hi = pgraphs[i % n_rep]
-        g.replay()
-        torch.cuda.synchronize()
-        if i < n_rep:
-            continue          # first pass over each graph: warm-up
-        for slot in range(lo, hi):
-            name = pr.p.name[slot].decode()
-            ms_ = ctypes_elapsed(pr, slot)
-            breakdown.setdefault(name, []).append(ms_)
-    pr.close()
-    hist_ms = breakdown.get("hist", [])
-    breakdown = {k: {"avg_ms": float(np.mean(v)), "launches_per_step": len(v) / n_prof}
-                 for k, v in breakdown.items()}
-    hist_avg_ms = float(np.mean(hist_ms)) if hist_ms else None
-    hbm_peak, peak_src = peaks()
-    idx_b = index_bytes(spec, layers0)
-    achieved = idx_b / (hist_avg_ms * 1e-3) / 1e9 if hist_avg_ms else None
-    workload = spec.name
-
-    # dense decode over the same caches
-    dgraphs = []
-    dense_out = torch.empty_like(out)
-
-    def dense_step(layers):
+    def dense_step(self, layers, out):
         for L in layers:
-            ops.dense_decode(L.dims, L.q_rope if L.q_rope is not None else L.q, L.k, L.v, dense_out, ws)
+            ops.dense_decode(L.dims, L.q_rope if L.q_rope is not None else L.q, L.k, L.v, out, self.ws)
 
-    with torch.cuda.stream(s):
-        for R in reps:
-            dense_step(R)
-    torch.cuda.synchronize()
-    for R in reps:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            dense_step(R)
-        dgraphs.append(g)
-    n_dense = max(3, min(args.steps, args.dense_steps))
-    for i in range(3):
-        dgraphs[i % n_rep].replay()
-    torch.cuda.synchronize()
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    d0.record()
-    for i in range(n_dense):
-        dgraphs[i % n_rep].replay()
-    d1.record()
-    torch.cuda.synchronize()
-    dense_ms = d0.elapsed_time(d1) / n_dense
+    def check(self):
+        st = self.ws.check()
+        if st:
+            raise RuntimeError(f"device status {st}: {ops.error_string(st)}")
 
-    # end to end: pinned host inputs -> device, graph, result -> host
-    e2e = None
-    if not args.no_e2e:
-        hq = [torch.empty(L.q.shape, dtype=L.q.dtype, pin_memory=True) for L in reps[0]]
-        hqr = [torch.empty(L.q.shape, dtype=L.q.dtype, pin_memory=True) for L in reps[0]]
-        hk = [torch.empty(L.k_new.shape, dtype=L.k_new.dtype, pin_memory=True) for L in reps[0]]
-        for i, L in enumerate(reps[0]):
+    def selection(self, p):
+        """Kept sets of one step -> (required bytes, kept counts per layer)."""
+        spec = self.spec
+        if p >= 1.0:
+            self.step(self.layers0, p)
+            self.check()
+            return required_bytes(spec, self.layers0, None, p), []
+        sel = [(torch.full((spec.B, spec.H_q, L.k.shape[2]), -1, dtype=torch.int32, device=self.dev),
+                torch.zeros((spec.B, spec.H_q), dtype=torch.int32, device=self.dev)) for L in self.layers0]
+        self.step(self.layers0, p, sel=sel)
+        self.check()
+        req = required_bytes(spec, self.layers0, [(a.cpu().numpy(), b.cpu().numpy()) for a, b in sel], p)
+        kept = [[int(x) for x in b.cpu().numpy().ravel() if x > 0] for _, b in sel]
+        return req, kept
+
+    def capture(self, fn):
+        """One CUDA graph per replica of fn(replica)."""
+        with torch.cuda.stream(self.stream):
+            self.stream.wait_stream(torch.cuda.current_stream())
+            for R in self.reps:
+                fn(R)
+        torch.cuda.current_stream().wait_stream(self.stream)
+        torch.cuda.synchronize()
+        graphs = []
+        for R in self.reps:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                fn(R)
+            graphs.append(g)
+        torch.cuda.synchronize()
+        return graphs
+
+    def time_graphs(self, graphs, steps, warmup, world, clocks=None):
+        """Device ms per step over `steps` replays (max over ranks)."""
+        n = len(graphs)
+        for i in range(warmup):
+            graphs[i % n].replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ctx = clocks if clocks is not None else _Null()
+        with ctx:
+            e0.record()
+            for i in range(steps):
+                graphs[i % n].replay()
+            e1.record()
+            torch.cuda.synchronize()
+        barrier(world)
+        return allreduce_max(e0.elapsed_time(e1), world, self.dev) / steps
+
+    def launches_per_step(self, p):
+        pr = ops.Profiler(1024)
+        self.step(self.reps[0], p, prof=pr)
+        torch.cuda.synchronize()
+        # rtp_append_index_keys takes no options, so its one launch per layer
+        # is not in the profiler's count
+        n = pr.p.count + len(self.layers0)
+        pr.close()
+        return n
+
+    def breakdown(self, p, n_prof, per_step_slots):
+        """Per-kernel device times: the step captured with event-record nodes
+        around every kernel (one graph per replica, distinct event slots),
+        replayed with a sync after each replay to read the slots."""
+        n_rep = len(self.reps)
+        pr = ops.Profiler(per_step_slots * n_rep)
+        pgraphs = []
+        for R in self.reps:
+            g = torch.cuda.CUDAGraph()
+            first = pr.p.count
+            with torch.cuda.graph(g):
+                self.step(R, p, prof=pr)
+            pgraphs.append((g, first, pr.p.count))
+        torch.cuda.synchronize()
+        times = {}
+        for i in range(n_prof + n_rep):
+            g, lo, hi = pgraphs[i % n_rep]
+            g.replay()
+            torch.cuda.synchronize()
+            if i < n_rep:
+                continue          # first pass over each graph: warm-up
+            for slot in range(lo, hi):
+                times.setdefault(pr.p.name[slot].decode(), []).append(ctypes_elapsed(pr, slot))
+        pr.close()
+        del pgraphs
+        return times
+
+    def dense_ms(self, steps, world):
+        dense_out = torch.empty_like(self.out)
+        graphs = self.capture(lambda R: self.dense_step(R, dense_out))
+        ms = self.time_graphs(graphs, steps, 3, world)
+        del graphs
+        return ms
+
+    def free(self):
+        self.reps = []
+        self.layers0 = []
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+
+
+class _Null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def kept_stats(kept):
+    flat = [x for k in kept for x in k]
+    if not flat:
+        return {"min": 0, "max": 0, "mean": 0.0}
+    return {"min": min(flat), "max": max(flat), "mean": float(np.mean(flat))}
+
+
+def measure_point(bn, p, steps, warmup, world, hbm_peak, max_replicas, n_prof, clocks=None):
+    """One (workload, p) point: step time, required bytes and their rate,
+    the scan kernel's rate and the per-kernel times."""
+    spec = bn.spec
+    req, kept = bn.selection(p)
+    bn.set_replicas(replicas_for(spec, req, max_replicas))
+    lps = bn.launches_per_step(p)
+    graphs = bn.capture(lambda R: bn.step(R, p))
+    ms = bn.time_graphs(graphs, steps, warmup, world, clocks)
+    del graphs
+    times = bn.breakdown(p, n_prof, lps + 4)
+    hist = times.get("hist", [])
+    # one scan launch per layer: its time per launch, and the index keys of
+    # one layer's retrieval groups per launch
+    hist_ms = float(np.mean(hist)) if hist else None
+    idx_b = index_bytes(spec, bn.layers0) // max(1, len(bn.layers0)) if p < 1.0 else 0
+    scan_gbs = idx_b / (hist_ms * 1e-3) / 1e9 if hist_ms else None
+    gbs = req / (ms * 1e-3) / 1e9
+    n_rep = len(bn.reps)
+    return {
+        "p": p, "ms_per_step": ms, "steps_per_s": 1e3 / ms, "required_bytes_per_step": int(req),
+        "achieved_gbs": gbs, "pct_peak": gbs / hbm_peak, "pct_of_8tbs": gbs / 8000.0,
+        "scan": {"gbs": scan_gbs, "frac": scan_gbs / hbm_peak if scan_gbs else None,
+                 "avg_launch_ms": hist_ms, "bytes_per_launch": idx_b},
+        "kernels": {k: {"avg_ms": float(np.mean(v)), "launches_per_step": len(v) / n_prof}
+                    for k, v in times.items()},
+        "kept_rows_per_retrieval_head": kept_stats(kept),
+        "launches_per_step": lps,
+        "replicas": n_rep,
+        "l2": f"rotating {n_rep} cache replicas ({n_rep} x {req / 1e6:.1f} MB >= 3 x L2)" if n_rep > 1
+        else f"{spec.layers} layer(s) per step ({req / 1e6:.0f} MB > L2)" if req > 3 * L2_BYTES
+        else f"1 replica ({req / 1e6:.1f} MB per step)",
+    }
+
+
+def e2e_measure(bn, p, graphs, steps, world):
+    """End to end through the C ABI from pinned host memory: every step
+    copies its q, q_rope and new key from the host, runs the C-ABI calls
+    (rtp_append_index_keys + rtp_decode_step per layer) and copies the
+    output back.  Three forms: a host wait after every step; double-buffered
+    host buffers with one wait per `depth` steps (a decode loop that does
+    not block on each step); and the per-step-wait form with the calls
+    replayed from a CUDA graph."""
+    n_rep = len(bn.reps)
+    L0 = bn.reps[0]
+
+    def pinned_like(t):
+        return torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+
+    bufs = []
+    for _ in range(2):
+        hq = [pinned_like(L.q) for L in L0]
+        hqr = [pinned_like(L.q) for L in L0]
+        hk = [pinned_like(L.k_new) for L in L0]
+        for i, L in enumerate(L0):
             hq[i].copy_(L.q)
             hqr[i].copy_(L.q_rope if L.q_rope is not None else L.q)
             hk[i].copy_(L.k_new)
-        hout = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-        n_e2e = max(3, min(args.steps, args.e2e_steps))
-        h2d = sum(t.numel() * t.element_size() for t in hq + hk) + (
-            sum(t.numel() * t.element_size() for t in hqr) if reps[0][0].q_rope is not None else 0)
-        d2h = hout.numel() * hout.element_size()
+        bufs.append((hq, hqr, hk, pinned_like(bn.out)))
+    has_rope = L0[0].q_rope is not None
+    hq, hqr, hk, hout = bufs[0]
+    h2d = sum(t.numel() * t.element_size() for t in hq + hk) + (
+        sum(t.numel() * t.element_size() for t in hqr) if has_rope else 0)
+    d2h = hout.numel() * hout.element_size()
 
-        def e2e_step(i, use_graph):
-            R = reps[i % n_rep]
-            for j, L in enumerate(R):
-                L.q.copy_(hq[j], non_blocking=True)
-                if L.q_rope is not None:
-                    L.q_rope.copy_(hqr[j], non_blocking=True)
-                L.k_new.copy_(hk[j], non_blocking=True)
-            if use_graph:
-                graphs[i % n_rep].replay()
-            else:
-                step(R)
-            hout.copy_(out, non_blocking=True)
+    def one(i, use_graph, wait):
+        hq, hqr, hk, hout = bufs[i % 2]
+        R = bn.reps[i % n_rep]
+        for j, L in enumerate(R):
+            L.q.copy_(hq[j], non_blocking=True)
+            if has_rope:
+                L.q_rope.copy_(hqr[j], non_blocking=True)
+            L.k_new.copy_(hk[j], non_blocking=True)
+        if use_graph:
+            graphs[i % n_rep].replay()
+        else:
+            bn.step(R, p)
+        hout.copy_(bn.out, non_blocking=True)
+        if wait:
             torch.cuda.current_stream().synchronize()
 
-        def e2e_time(use_graph):
-            for i in range(3):
-                e2e_step(i, use_graph)
-            barrier(world)
-            x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            x0.record()
-            for i in range(n_e2e):
-                e2e_step(i, use_graph)
-            x1.record()
-            torch.cuda.synchronize()
-            e2e_ms = allreduce_max(x0.elapsed_time(x1), world, dev)
-            return world * n_e2e / (e2e_ms / 1e3)
+    def run(use_graph, depth):
+        for i in range(3):
+            one(i, use_graph, True)
+        barrier(world)
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record()
+        for i in range(steps):
+            one(i, use_graph, (i + 1) % depth == 0)
+        x1.record()
+        torch.cuda.synchronize()
+        return world * steps / (allreduce_max(x0.elapsed_time(x1), world, bn.dev) / 1e3)
 
-        e2e = {"value": e2e_time(False), "unit": "steps/s", "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "steps": n_e2e,
-               "note": "per step: pinned host q/q_rope/k_new -> device, the C-ABI calls "
-                       "(rtp_append_index_keys + rtp_decode_step per layer), out -> host, sync",
-               "graph_value": e2e_time(True),
-               "graph_note": "the same with the step's C-ABI calls captured once in a CUDA graph and replayed"}
+    depth = 64
+    pipelined = run(False, depth)
+    per_step = run(False, 1)
+    graph_step = run(True, 1)
+    return {"value": pipelined, "unit": "steps/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": steps,
+            "note": f"per step: pinned host q/q_rope/k_new -> device, the C-ABI calls "
+                    f"(rtp_append_index_keys + rtp_decode_step per layer), out -> pinned host; "
+                    f"double-buffered host buffers, one host wait per {depth} steps",
+            "sync_value": per_step,
+            "sync_note": "the same with a host wait after every step",
+            "graph_value": graph_step,
+            "graph_note": "the per-step-wait form with the step's C-ABI calls captured once in a "
+                          "CUDA graph and replayed"}
 
-    step_gbs = req / (ms_per_step * 1e-3) / 1e9
+
+# workloads measured beside the headline line, in the same run
+SWEEP = (("ctx64k", (0.9,)), ("ctx1m", (0.8, 0.9, 0.95, 1.0)), ("ctx128k-b8-48layer", (0.9,)))
+
+
+def measure_workload(key, ps, args, rank, world, dev, hbm_peak):
+    bn = Bench(key, rank_seed(0, rank), dev)
+    try:
+        pts = {}
+        for p in ps:
+            pts[str(p)] = measure_point(bn, p, args.sweep_steps, args.warmup, world, hbm_peak,
+                                        args.max_replicas, min(args.prof_steps, 50))
+        dense = bn.dense_ms(max(3, min(args.sweep_steps, args.dense_steps)), world)
+        spec = bn.spec
+        for v in pts.values():
+            v["dense_ms_per_step"] = dense
+            v["speedup_sparse_vs_dense"] = dense / v["ms_per_step"]
+        return {"workload": spec.name, "B": spec.B, "ctx": spec.N, "layers": spec.layers,
+                "dense_bytes_per_step": int(sum(2 * L.k.numel() * L.k.element_size() for L in bn.layers0)),
+                "points": pts}
+    finally:
+        bn.free()
+        del bn
+        torch.cuda.empty_cache()
+
+
+def run_ours(args, rank, world, dev):
+    # each rank serves sequences of its own (rank 0's are the single-GPU workload)
+    hbm_peak, peak_src = peaks()
+    bn = Bench(args.workload, rank_seed(0, rank), dev)
+    spec = bn.spec
+    if args.p is not None:
+        spec.p = args.p
+    p = spec.p
+    clocks = Clocks(dev.index)
+    pt = measure_point(bn, p, args.steps, args.warmup, world, hbm_peak, args.max_replicas,
+                       max(1, min(args.steps, args.prof_steps)), clocks)
+    ms_per_step = pt["ms_per_step"]
+    value = world / (ms_per_step * 1e-3)
+    dense_ms = bn.dense_ms(max(3, min(args.steps, args.dense_steps)), world)
+
+    e2e = None
+    if not args.no_e2e:
+        graphs = bn.capture(lambda R: bn.step(R, p))
+        e2e = e2e_measure(bn, p, graphs, max(3, min(args.steps, args.e2e_steps)), world)
+        del graphs
+    dense_bytes = int(sum(2 * L.k.numel() * L.k.element_size() for L in bn.layers0))
+    n_rep = pt["replicas"]
+    workload = spec.name
+    bn.free()
+    del bn
+
+    sweep = {}
+    if not args.no_sweep:
+        for key, ps in SWEEP:
+            if key == args.workload:
+                continue
+            sweep[key] = measure_workload(key, ps, args, rank, world, dev, hbm_peak)
+
+    sc = pt["scan"]
     res = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -425,32 +569,30 @@ def run_ours(args, rank, world, dev):
         "config": {"workload": workload, "key": args.workload, "B": spec.B, "ctx": spec.N, "H_q": spec.H_q,
                    "H_kv": spec.H_kv, "d": spec.d, "r": spec.r, "layers": spec.layers, "p": p,
                    "window": spec.window, "n_sink": spec.n_sink, "cache_dtype": spec.kv_dtype,
-                   "index_dtype": spec.idx_dtype, "accumulate": "f32",
-                   "l2": f"rotating {n_rep} cache replicas per rank ({n_rep} x {req / 1e6:.1f} MB >= 3 x L2)"
-                   if n_rep > 1 else f"{spec.layers} distinct layers per step ({req / 1e6:.0f} MB > L2)",
+                   "index_dtype": spec.idx_dtype, "accumulate": "f32", "l2": pt["l2"],
                    "timing": "CUDA graph replays, CUDA events, max over ranks",
                    "parallelism": f"replicas x{world} (independent sequences per rank)"},
-        "required_bytes_per_step": int(req),
-        "achieved_gbs": step_gbs,
-        "pct_peak": step_gbs / hbm_peak,
-        "pct_of_8tbs": step_gbs / 8000.0,
-        "kept_rows_per_retrieval_head": {"min": min(min(k) for k in kept if k) if any(kept) else 0,
-                                         "max": max(max(k) for k in kept if k) if any(kept) else 0,
-                                         "mean": float(np.mean([x for k in kept for x in k])) if any(kept) else 0},
+        "required_bytes_per_step": pt["required_bytes_per_step"],
+        "achieved_gbs": pt["achieved_gbs"],
+        "pct_peak": pt["pct_peak"],
+        "pct_of_8tbs": pt["pct_of_8tbs"],
+        "kept_rows_per_retrieval_head": pt["kept_rows_per_retrieval_head"],
         "roofline": {"bound": "hbm", "kernel": "hist (index-key scan + mass histogram)",
-                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
-                     "frac": (achieved / hbm_peak) if achieved else None,
+                     "achieved": sc["gbs"], "peak": hbm_peak, "unit": "GB/s",
+                     "frac": sc["frac"],
                      "traffic": traffic_for("hist", workload),
-                     "bytes_per_launch": idx_b, "avg_launch_ms": hist_avg_ms,
+                     "bytes_per_launch": sc["bytes_per_launch"], "avg_launch_ms": sc["avg_launch_ms"],
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
                      else "fallback 6650 GB/s"},
         "dense": {"ms_per_step": dense_ms, "speedup_sparse_vs_dense": dense_ms / ms_per_step,
-                  "bytes_per_step": int(sum(2 * L.k.numel() * L.k.element_size() for L in reps[0]))},
-        "kernels": breakdown,
-        "gpu_launches": int(launches_per_step * args.steps),
-        "launches_per_step": launches_per_step,
+                  "bytes_per_step": dense_bytes},
+        "kernels": pt["kernels"],
+        "gpu_launches": int(pt["launches_per_step"] * args.steps),
+        "launches_per_step": pt["launches_per_step"],
+        "replicas": n_rep,
         "clocks": clocks.report(),
         "e2e": e2e,
+        "workloads": sweep,
         "pages_context": {"decode_speedup_1M_H20": 2.01, "prefill_speedup_1M_H20": 9.36},
     }
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -542,7 +684,10 @@ def main():
     ap.add_argument("--prof-steps", type=int, default=200)
     ap.add_argument("--dense-steps", type=int, default=200)
     ap.add_argument("--e2e-steps", type=int, default=2000)
-    ap.add_argument("--max-replicas", type=int, default=16)
+    ap.add_argument("--max-replicas", type=int, default=64)
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="measure only --workload (no other workloads in the same run)")
+    ap.add_argument("--sweep-steps", type=int, default=400)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -550,6 +695,9 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world:
+        sys.exit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch N > 1 ranks with "
+                 f"torch.distributed.run --nproc-per-node N")
     if args.impl == "reference":
         res = run_reference(args, rank, world)
         if res is not None:

@@ -49,10 +49,40 @@ def test_required_bytes_short_sequence_reads_each_local_row_once():
 
 @pytest.mark.parametrize("p", [1.0, 1.5])
 def test_required_bytes_keep_all_reads_every_row(p):
+    """p >= 1 keeps every token without a threshold: the step reads every
+    K/V row of the retrieval groups and neither index keys nor W_q_idx."""
     spec = _spec(B=1, N=50, p=p, kv="f32", idx="f32")
     L = _layer([50], [1, 1], 8)
     got = bench.required_bytes(spec, [L], None)
-    assert got == 2 * (50 * 16 * 4 + 50 * 2 * 128 * 4) + 8 * 16 * 128 * 4
+    assert got == 2 * 50 * 2 * 128 * 4
+    # the p argument overrides the workload's own
+    assert bench.required_bytes(_spec(B=1, N=50, p=0.5, kv="f32", idx="f32"), [L], None, p) == got
+
+
+def test_index_bytes_per_layer_and_sequence_lengths():
+    """Index keys the scan reads: retrieval groups x the sequences' own
+    lengths, summed over layers."""
+    spec = _spec(B=2, N=100)
+    la = _layer([100, 60], [1, 0], 8)
+    lb = _layer([100, 60], [1, 1], 8)
+    assert bench.index_bytes(spec, [la, lb]) == (1 + 2) * 160 * 16 * 2
+
+
+def test_replicas_cover_three_l2():
+    spec = _spec(B=1, N=100)
+    assert bench.replicas_for(spec, 8_500_000, 64) == 47      # 3 x 126 MiB / 8.5 MB
+    assert bench.replicas_for(spec, 8_500_000, 16) == 16
+    assert bench.replicas_for(spec, 2_000_000_000, 64) == 1
+    spec.layers = 48
+    assert bench.replicas_for(spec, 1000, 64) == 1
+
+
+def test_gpus_must_match_world_size(monkeypatch):
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    monkeypatch.setattr("sys.argv", ["bench.py", "--gpus", "8"])
+    with pytest.raises(SystemExit) as e:
+        bench.main()
+    assert "WORLD_SIZE=1" in str(e.value)
 
 
 class _FakeNvml:
