@@ -1,6 +1,7 @@
 // C ABI of librtp.so: argument checks, workspace layout and kernel launches
 // for the RTPurbo sparse decode step.  Contract: include/rtp.h.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdlib>
 #include <cstdio>
@@ -435,16 +436,20 @@ namespace {
 constexpr size_t NOALLOC_ARRIVE_OFF = 256;                       // after the status word
 constexpr size_t NOALLOC_PART_OFF = 256 + RTP_NOALLOC_MAX_GROUPS * 4;
 
+// The address is cached per device in an atomic slot: threads that make
+// their first call at the same time may both look it up, and both store the
+// same value.  The cache assumes the device is not reset (cudaDeviceReset)
+// after the first call; the array's address would then change.
 int noalloc_scratch(char *&out) {
-    static void *ptrs[64] = {nullptr};
+    static std::atomic<void *> ptrs[64];
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
-    if (!ptrs[dev]) {
-        void *p = nullptr;
+    void *p = ptrs[dev].load(std::memory_order_acquire);
+    if (!p) {
         if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return RTP_ERR_CUDA;
-        ptrs[dev] = p;
+        ptrs[dev].store(p, std::memory_order_release);
     }
-    out = static_cast<char *>(ptrs[dev]);
+    out = static_cast<char *>(p);
     return RTP_OK;
 }
 

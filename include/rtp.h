@@ -293,8 +293,9 @@ RTP_API int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const fl
  * RTP_NOALLOC_MAX_GROUPS (the partials would not fit), before any launch.
  *
  * The first call on a device, with that device current, looks up the
- * array's device address (cudaGetSymbolAddress); make that first call
- * before any stream capture.  All calls share the one array and it keeps
+ * array's device address (cudaGetSymbolAddress) and keeps it for the
+ * process; make that first call before any stream capture, and do not
+ * reset the device (cudaDeviceReset) after it.  All calls share the one array and it keeps
  * the last call's contents: each call clears the part that must start at
  * zero, and calls whose executions overlap on the GPU (different streams,
  * no ordering between them) race on it -- order them on one stream.

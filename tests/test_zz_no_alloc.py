@@ -5,8 +5,9 @@ in the process (this file is collected last on purpose)."""
 import pytest
 import torch
 
+import oracle
 from dynamic_top_sparse_b200 import ops, synth
-from tests.helpers import OUT_TOL_SAME_SET, GpuCase
+from tests.helpers import OUT_TOL, OUT_TOL_SAME_SET, GpuCase, np32, np64, within
 
 pytestmark = pytest.mark.gpu
 
@@ -34,6 +35,8 @@ def test_noalloc_matches_dense_two_calls(kvdt):
     ref = torch.zeros((2, 16, 128), device="cuda")
     ops.dense_decode(gc.dims, gc.q_rope, gc.k, gc.v, ref, gc.ws)
     assert gc.ws.check() == 0
+    c = gc.c
+    exact = oracle.dense_decode(np64(c.q_rope), np32(c.k_cache), np32(c.v_cache), c.seq_lens.cpu().numpy())
     st = torch.full((1,), -1, dtype=torch.int32, device="cuda")
     for call in range(2):
         out = torch.full((2, 16, 128), float("nan"), device="cuda")
@@ -43,6 +46,8 @@ def test_noalloc_matches_dense_two_calls(kvdt):
         assert torch.isfinite(out).all(), f"call {call}"
         err = _max_abs(out, ref)
         assert err <= OUT_TOL_SAME_SET, f"call {call}: max abs diff {err}"
+        # and the oracle's dense attention over the same caches
+        within(out.cpu().numpy(), exact, OUT_TOL, f"call {call} vs oracle")
 
 
 def test_noalloc_status_is_per_call():
