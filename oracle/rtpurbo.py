@@ -326,3 +326,40 @@ def dense_decode(q_rope, k_cache, v_cache, seq_lens, attn_scale: float | None = 
         g = h // G
         out[b, h] = attend(q_rope[b, h], k_cache[b, g, :N], v_cache[b, g, :N], np.arange(N), asc)
     return out
+
+
+# ---------------------------------------------------------------------------
+# prefill
+# ---------------------------------------------------------------------------
+
+def prefill_attention(q, k_cache, v_cache, head_class, pos0, window: int, n_sink: int,
+                      attn_scale: float | None = None, rows_of=None) -> np.ndarray:
+    """Attention of a prompt's query tokens during prefill (summary, Method
+    section 1: local heads keep a sliding window with attention sinks at
+    every step, retrieval heads keep the full KV cache).
+
+    q: [B, H_q, T, d] post-RoPE queries of T consecutive prompt tokens; query
+    i of sequence b sits at position P = pos0[b] + i.  It sees the cached
+    tokens 0..P (its own key included: causal), so it is the decode step's
+    attention with N = P + 1 tokens: a local head attends over
+    local_rows(P + 1, window, n_sink), a retrieval head over all P + 1
+    tokens.  ``rows_of`` optionally restricts the work to a list of
+    (b, h, i); the other outputs stay NaN.  Returns [B, H_q, T, d] fp64.
+    """
+    q = np.asarray(q, np.float64)
+    B, H_q, T, d = q.shape
+    H_kv = k_cache.shape[1]
+    G = H_q // H_kv
+    asc = default_scale(d) if attn_scale is None else attn_scale
+    out = np.full((B, H_q, T, d), np.nan)
+    todo = rows_of if rows_of is not None else [(b, h, i) for b in range(B) for h in range(H_q)
+                                                for i in range(T)]
+    for b, h, i in todo:
+        g = h // G
+        n = int(pos0[b]) + i + 1
+        if head_class[g] == HEAD_RETRIEVAL:
+            rows = np.arange(n)
+        else:
+            rows = local_rows(n, window, n_sink)
+        out[b, h, i] = attend(q[b, h, i], k_cache[b, g, :n], v_cache[b, g, :n], rows, asc)
+    return out

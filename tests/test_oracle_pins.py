@@ -452,3 +452,59 @@ def test_step_with_topk_attends_the_k_best_index_scores():
             mask[best] = True
             ref = _masked_dense_attention(q[0, h], K[0, gq], V[0, gq], mask, sc)
             np.testing.assert_allclose(res.out[0, h], ref, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------------ prefill pins
+
+def _prefill_case(seed, B=2, H_q=4, H_kv=2, T=6, d=8, pos0=(3, 0)):
+    g = np.random.default_rng(seed)
+    N_max = max(pos0) + T
+    q = g.normal(0, 1, (B, H_q, T, d))
+    K = g.normal(0, 1, (B, H_kv, N_max, d))
+    V = g.normal(0, 1, (B, H_kv, N_max, d))
+    return q, K, V, np.asarray(pos0)
+
+
+@pytest.mark.parametrize("window,n_sink", [(3, 1), (1, 0), (2, 2), (100, 0)])
+def test_prefill_matches_explicit_causal_window_mask(window, n_sink):
+    """Each query against the explicit mask: key position j is visible to
+    the query at position P when j <= P and, for a local head, j < n_sink
+    or P - j < window (loops, no shared helper)."""
+    q, K, V, pos0 = _prefill_case(5)
+    hc = np.array([0, 1], np.uint8)
+    out = oracle.prefill_attention(q, K, V, hc, pos0, window, n_sink)
+    B, H_q, T, d = q.shape
+    for b in range(B):
+        for h in range(H_q):
+            g = h // 2
+            for i in range(T):
+                P = int(pos0[b]) + i
+                mask = np.array([j <= P and (hc[g] == 1 or j < n_sink or P - j < window)
+                                 for j in range(K.shape[2])])
+                ref = _masked_dense_attention(q[b, h, i], K[b, g], V[b, g], mask, 1 / math.sqrt(d))
+                np.testing.assert_allclose(out[b, h, i], ref, rtol=0, atol=1e-12)
+
+
+def test_prefill_last_query_is_the_decode_step():
+    """The last prompt token's attention is the decode step's attention over
+    the same cache (p = 1 keeps every token of a retrieval head)."""
+    q, K, V, pos0 = _prefill_case(6, T=5, pos0=(7, 2))
+    B, H_q, T, d = q.shape
+    hc = np.array([1, 0], np.uint8)
+    out = oracle.prefill_attention(q, K, V, hc, pos0, 3, 1)
+    lens = pos0 + T
+    kidx = np.random.default_rng(1).normal(0, 1, (B, 2, K.shape[2], 4))
+    W = np.random.default_rng(2).normal(0, 1, (H_q, 4, d))
+    dec = oracle.decode_step(q[:, :, T - 1], None, K, V, kidx, W, hc, lens, 1.0, 3, 1)
+    np.testing.assert_allclose(out[:, :, T - 1], dec.out, rtol=0, atol=1e-12)
+
+
+def test_prefill_first_position_returns_v0_and_wide_window_is_causal():
+    q, K, V, pos0 = _prefill_case(7, pos0=(0, 4))
+    loc = oracle.prefill_attention(q, K, V, np.array([0, 0], np.uint8), pos0, 10**6, 0)
+    ret = oracle.prefill_attention(q, K, V, np.array([1, 1], np.uint8), pos0, 3, 1)
+    full = oracle.prefill_attention(q, K, V, np.array([1, 1], np.uint8), pos0, 1, 0)
+    np.testing.assert_allclose(loc, full, rtol=0, atol=1e-12)      # a window past position 0 is all causal rows
+    np.testing.assert_allclose(ret, full, rtol=0, atol=1e-12)      # retrieval heads ignore window and sinks
+    for h in range(q.shape[1]):
+        np.testing.assert_array_equal(loc[0, h, 0], K[0, h // 2, 0] * 0 + V[0, h // 2, 0])
