@@ -528,6 +528,92 @@ def measure_workload(key, ps, args, rank, world, dev, hbm_peak):
         torch.cuda.empty_cache()
 
 
+def local_pairs(n: int, window: int, n_sink: int) -> int:
+    """Rows a local head attends over at a step with n cached tokens."""
+    s = min(n_sink, n)
+    return s + (n - max(s, n - window))
+
+
+def prefill_pairs(pos0: int, T: int, window: int, n_sink: int, local: bool) -> int:
+    """(query, key) pairs of one head's causal prefill attention over prompt
+    tokens at positions pos0 .. pos0 + T - 1."""
+    if not local:
+        a, b = pos0 + 1, pos0 + T
+        return (a + b) * T // 2
+    return sum(local_pairs(P + 1, window, n_sink) for P in range(pos0, pos0 + T))
+
+
+def measure_prefill(args, world, dev):
+    """Prefill of a whole 64K-token prompt in the 64K workload's shape (32 q /
+    4 KV heads, KV0 retrieval, window 4096 + 4 sinks): the prompt's index
+    keys (rtp_append_index_keys, T = N) and its causal attention
+    (rtp_prefill_attention), against the same attention with every head
+    keeping the full cache.  Tensor-bound: FLOPs = 4 d per (query, key)
+    pair (q.k and p.v)."""
+    spec = synth.spec_for("ctx64k")
+    B, H_q, H_kv, N, d = 1, spec.H_q, spec.H_kv, spec.N, spec.d
+    G = H_q // H_kv
+    hc = np.array([1, 0, 0, 0], np.uint8)
+    g = torch.Generator(device=dev).manual_seed(rank_seed(17, 0))
+    q = torch.randn(B, H_q, N, d, generator=g, device=dev).to(torch.bfloat16)
+    k = torch.randn(B, H_kv, N, d, generator=g, device=dev).to(torch.bfloat16)
+    v = torch.randn(B, H_kv, N, d, generator=g, device=dev).to(torch.bfloat16)
+    W = torch.randn(H_kv, spec.r, d, generator=g, device=dev) / math.sqrt(d)
+    kidx = torch.zeros(B, H_kv, N, spec.r, dtype=torch.bfloat16, device=dev)
+    seq = torch.full((B,), N, dtype=torch.int32, device=dev)
+    pos0 = torch.zeros(B, dtype=torch.int32, device=dev)
+    dims = ops.make_dims(B, H_q, H_kv, N, seq, ops.RTP_BF16, ops.RTP_BF16)
+    ws = ops.Workspace(dims)
+    out = torch.empty(B, H_q, N, d, device=dev)
+
+    def timed(fn, n):
+        fn()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(n):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        return allreduce_max(e0.elapsed_time(e1), world, dev) / n
+
+    n = max(2, args.prefill_steps)
+    ms_rtp = timed(lambda: ops.prefill_attention(dims, q, pos0, k, v, hc, spec.window, spec.n_sink, out, ws), n)
+    ms_full = timed(lambda: ops.prefill_attention(dims, q, pos0, k, v, np.ones(H_kv, np.uint8), spec.window,
+                                                  spec.n_sink, out, ws), n)
+    ms_keys = timed(lambda: ops.append_index_keys(dims, k, W, pos0, hc, kidx, ws), max(n, 20))
+    if ws.check():
+        raise RuntimeError("prefill: device status set")
+    pairs = sum(G * prefill_pairs(0, N, spec.window, spec.n_sink, hc[gi] == 0) for gi in range(H_kv))
+    pairs_full = H_q * prefill_pairs(0, N, spec.window, spec.n_sink, False)
+    fl, fl_full = 4 * d * pairs, 4 * d * pairs_full
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            tf_peak, tf_src = float(json.load(f)["bf16_tflops"]), "measured bf16_tflops (cuBLAS burst)"
+    except Exception:
+        tf_peak, tf_src = 1590.0, "fallback 1590 TFLOP/s"
+    ret = int(hc.sum())
+    key_bytes = B * ret * N * (d * 2 + spec.r * 2)
+    res = {
+        "workload": f"prefill of a {N}-token prompt, B1, 32q/4kv, KV0 retrieval (full causal), "
+                    f"KV1-3 local (window {spec.window} + {spec.n_sink} sinks), bf16",
+        "attention_ms": ms_rtp, "flops": fl, "tflops": fl / (ms_rtp * 1e-3) / 1e12,
+        "full_attention_ms": ms_full, "full_flops": fl_full,
+        "full_tflops": fl_full / (ms_full * 1e-3) / 1e12,
+        "speedup_vs_full": ms_full / ms_rtp,
+        "roofline": {"bound": "tensor", "achieved": fl / (ms_rtp * 1e-3) / 1e12, "peak": tf_peak,
+                     "unit": "TFLOP/s", "frac": fl / (ms_rtp * 1e-3) / 1e12 / tf_peak,
+                     "peak_source": tf_src},
+        "index_keys_ms": ms_keys, "index_keys_gbs": key_bytes / (ms_keys * 1e-3) / 1e9,
+        "index_keys_bytes": key_bytes,
+        "steps": n,
+    }
+    del q, k, v, kidx, out
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, rank, world, dev):
     # each rank serves sequences of its own (rank 0's are the single-GPU workload)
     hbm_peak, peak_src = peaks()
@@ -561,6 +647,8 @@ def run_ours(args, rank, world, dev):
                 continue
             sweep[key] = measure_workload(key, ps, args, rank, world, dev, hbm_peak)
 
+    prefill = None if args.no_prefill else measure_prefill(args, world, dev)
+
     sc = pt["scan"]
     res = {
         "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
@@ -593,6 +681,7 @@ def run_ours(args, rank, world, dev):
         "clocks": clocks.report(),
         "e2e": e2e,
         "workloads": sweep,
+        "prefill": prefill,
         "pages_context": {"decode_speedup_1M_H20": 2.01, "prefill_speedup_1M_H20": 9.36},
     }
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -688,6 +777,8 @@ def main():
     ap.add_argument("--no-sweep", action="store_true",
                     help="measure only --workload (no other workloads in the same run)")
     ap.add_argument("--sweep-steps", type=int, default=400)
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--prefill-steps", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -14,6 +14,7 @@
 #include "rtp_attend.cuh"
 #include "rtp_append.cuh"
 #include "rtp_gqa_mma.cuh"
+#include "rtp_prefill.cuh"
 
 using namespace rtp;
 
@@ -84,6 +85,7 @@ size_t op_bytes(const Layout &L, int op) {
         case RTP_OP_SPARSE_DECODE: return L.end_list;
         case RTP_OP_TOPP_SELECT:
         case RTP_OP_DECODE_STEP: return L.total;
+        case RTP_OP_PREFILL: return L.status + 256;
         default: return 0;
     }
 }
@@ -636,6 +638,48 @@ int rtp_dense_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_
     Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
     return launch_range(ln, dims, q_rope, k_cache, v_cache, nullptr, -1, true, 1, 0, out, (char *)ws, L,
                         scale_or_default(opts ? opts->attn_scale : 0.f));
+}
+
+int rtp_prefill_attention(const rtp_dims *dims, const rtp_opts *opts, const void *q, int32_t T,
+                          const int32_t *pos0, const void *k_cache, const void *v_cache,
+                          const uint8_t *head_class, int32_t window, int32_t n_sink, float *out, void *ws,
+                          size_t ws_bytes, rtp_stream_t stream) {
+    RTP_TRY(check_dims(dims));
+    if (!q || !pos0 || !k_cache || !v_cache || !out) return RTP_ERR_INVALID_ARG;
+    if (T < 1 || T > dims->N_max || window < 1 || n_sink < 0) return RTP_ERR_INVALID_ARG;
+    if (dims->kv_dtype != RTP_BF16) return RTP_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) || !aligned4(pos0))
+        return RTP_ERR_INVALID_ARG;
+    RTP_TRY(check_head_class(dims, head_class));
+    RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_PREFILL));
+    static bool attr_set[64] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
+    if (!attr_set[dev]) {
+        if (cudaFuncSetAttribute(prefill_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM) !=
+            cudaSuccess)
+            return RTP_ERR_CUDA;
+        attr_set[dev] = true;
+    }
+    // head classes go to the device through the kernel parameters
+    PrefillArgs a{};
+    a.B = dims->B; a.H_q = dims->H_q; a.H_kv = dims->H_kv; a.G = dims->H_q / dims->H_kv;
+    a.N_max = dims->N_max; a.T = T;
+    a.nsub = std::max(1, PF_WARPS / a.G);
+    a.n_qblk = (T + 16 * a.nsub - 1) / (16 * a.nsub);
+    a.seq_lens = dims->seq_lens; a.pos0 = pos0;
+    for (int g = 0; g < dims->H_kv; ++g) a.hc[g] = head_class[g];
+    a.window = window; a.n_sink = n_sink;
+    a.scale_log2 = scale_or_default(opts ? opts->attn_scale : 0.f) * L2E;
+    a.q = static_cast<const __nv_bfloat16 *>(q);
+    a.k = static_cast<const __nv_bfloat16 *>(k_cache);
+    a.v = static_cast<const __nv_bfloat16 *>(v_cache);
+    a.out = out;
+    a.status = reinterpret_cast<uint32_t *>(static_cast<char *>(ws));
+    if ((long long)a.n_qblk > 0x7fffffffLL) return RTP_ERR_UNSUPPORTED;
+    Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
+    return ln.run_smem("prefill_attn", prefill_attn_kernel, dim3((unsigned)a.n_qblk, (unsigned)(dims->B * dims->H_kv)),
+                       dim3(PF_THREADS), PF_SMEM, a);
 }
 
 int rtp_dense_decode_noalloc(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,

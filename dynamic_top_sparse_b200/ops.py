@@ -37,12 +37,13 @@ OP_SPARSE_DECODE = 3
 OP_LOCAL_DECODE = 4
 OP_DENSE_DECODE = 5
 OP_DECODE_STEP = 6
+OP_PREFILL = 7
 
 EXPORTS = ("rtp_workspace_size", "rtp_workspace_init", "rtp_check", "rtp_error_string",
            "rtp_version", "rtp_append_index_keys", "rtp_index_scores", "rtp_topp_select",
            "rtp_sparse_decode", "rtp_local_decode", "rtp_dense_decode", "rtp_decode_step",
            "rtp_prof_init", "rtp_prof_elapsed", "rtp_prof_destroy", "rtp_dense_decode_noalloc",
-           "rtp_selftest_wait_timeout")
+           "rtp_selftest_wait_timeout", "rtp_prefill_attention")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20
 NOALLOC_MAX_GROUPS = 1024
@@ -99,6 +100,9 @@ _SIGS = {
     "rtp_dense_decode_noalloc": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Opts), _P, _P, _P, _P, _P,
                                                 _P]),
     "rtp_selftest_wait_timeout": (ctypes.c_int, [_P, _P]),
+    "rtp_prefill_attention": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Opts), _P, ctypes.c_int32, _P,
+                                             _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P, _P,
+                                             ctypes.c_size_t, _P]),
 }
 
 
@@ -276,6 +280,17 @@ def decode_step(dims: Dims, q, q_rope, k_cache, v_cache, kidx_cache, W_q_idx, he
                               _ptr(q_rope), _ptr(k_cache), _ptr(v_cache), _ptr(kidx_cache), _ptr(W_q_idx),
                               _hc(head_class), float(p), int(window), int(n_sink), _ptr(out), ws.ptr,
                               ws.nbytes, _stream()), "rtp_decode_step")
+
+
+def prefill_attention(dims: Dims, q, pos0, k_cache, v_cache, head_class, window: int, n_sink: int, out,
+                      ws: Workspace, opts: Opts | None = None):
+    """Causal prefill attention of T prompt tokens per sequence (q [B, H_q, T, d]
+    bf16, pos0 [B] int32 device positions of token 0, out [B, H_q, T, d] fp32)."""
+    T = q.shape[2]
+    _ck(lib().rtp_prefill_attention(ctypes.byref(dims), ctypes.byref(opts) if opts else None, _ptr(q), int(T),
+                                    _ptr(pos0), _ptr(k_cache), _ptr(v_cache), _hc(head_class), int(window),
+                                    int(n_sink), _ptr(out), ws.ptr, ws.nbytes, _stream()),
+        "rtp_prefill_attention")
 
 
 def selftest_wait_timeout(dev_status):

@@ -102,7 +102,8 @@ enum {
     RTP_OP_SPARSE_DECODE = 3,
     RTP_OP_LOCAL_DECODE = 4,
     RTP_OP_DENSE_DECODE = 5,
-    RTP_OP_DECODE_STEP = 6 /* covers every other op */
+    RTP_OP_DECODE_STEP = 6, /* covers every other op */
+    RTP_OP_PREFILL = 7
 };
 
 /* Shapes of one layer.  d must be 128 and r must be 16 on this path. */
@@ -272,6 +273,34 @@ RTP_API int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const fl
                     const void *kidx_cache, const float *W_q_idx,
                     const uint8_t *head_class, float p, int32_t window, int32_t n_sink,
                     float *out, void *ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * Prefill attention of a prompt (gist.science technical summary, Method
+ * section 1: local heads keep a sliding window with attention sinks,
+ * retrieval heads keep the full KV cache; arXiv abstract: only retrieval
+ * heads keep the full cache).  The T prompt tokens of sequence b sit at
+ * positions pos0[b] .. pos0[b] + T - 1 and their keys and values are
+ * already in the caches (write them first; the index keys of the prompt
+ * come from rtp_append_index_keys with the same T).  The token at position
+ * P attends causally, exactly, over
+ *   local KV heads:     the rows j <= P with j < n_sink or P - j < window
+ *                       (the decode step's set for N = P + 1);
+ *   retrieval KV heads: every row j <= P.
+ *   q    [B, H_q, T, d] bf16, post-RoPE queries of the prompt tokens
+ *   pos0 [B] int32 DEVICE array: position of prompt token 0
+ *   k_cache, v_cache [B, H_kv, N_max, d] bf16 (dims->kv_dtype == RTP_BF16)
+ *   out  [B, H_q, T, d] fp32
+ * Needs 0 <= pos0[b] and pos0[b] + T <= seq_lens[b] <= N_max (else
+ * RTP_ERR_DEVICE_ARG in the status word and zeros for that sequence);
+ * window >= 1, n_sink >= 0, 1 <= T <= N_max.  Workspace:
+ * rtp_workspace_size(dims, RTP_OP_PREFILL) bytes (the status word only).
+ * Softmax scale opts->attn_scale (0: 1/sqrt(d)).  A kv_dtype of RTP_F32 is
+ * RTP_ERR_UNSUPPORTED.
+ */
+RTP_API int rtp_prefill_attention(const rtp_dims *dims, const rtp_opts *opts, const void *q, int32_t T,
+                                  const int32_t *pos0, const void *k_cache, const void *v_cache,
+                                  const uint8_t *head_class, int32_t window, int32_t n_sink, float *out,
+                                  void *ws, size_t ws_bytes, rtp_stream_t stream);
 
 /*
  * Dense decode without a caller workspace.  (The paper has no counterpart:

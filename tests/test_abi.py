@@ -136,6 +136,21 @@ def test_other_calls_reject_bad_arguments(L):
                                    None) == ops.RTP_ERR_INVALID_ARG
     assert L.rtp_append_index_keys(ctypes.byref(d), FAKE, 70000, FAKE, FAKE, hc, FAKE, FAKE, big,
                                    None) == ops.RTP_ERR_INVALID_ARG
+    # prefill: prompt length, window, cache type, workspace
+    pf = L.rtp_prefill_attention
+    assert pf(ctypes.byref(d), None, FAKE, 0, FAKE, FAKE, FAKE, hc, 16, 4, FAKE, FAKE, big,
+              None) == ops.RTP_ERR_INVALID_ARG
+    assert pf(ctypes.byref(d), None, FAKE, 70000, FAKE, FAKE, FAKE, hc, 16, 4, FAKE, FAKE, big,
+              None) == ops.RTP_ERR_INVALID_ARG
+    assert pf(ctypes.byref(d), None, FAKE, 8, FAKE, FAKE, FAKE, hc, 0, 4, FAKE, FAKE, big,
+              None) == ops.RTP_ERR_INVALID_ARG
+    assert pf(ctypes.byref(d), None, None, 8, FAKE, FAKE, FAKE, hc, 16, 4, FAKE, FAKE, big,
+              None) == ops.RTP_ERR_INVALID_ARG
+    assert pf(ctypes.byref(_dims(ops, kv_dtype=ops.RTP_F32)), None, FAKE, 8, FAKE, FAKE, FAKE, hc, 16, 4,
+              FAKE, FAKE, big, None) == ops.RTP_ERR_UNSUPPORTED
+    assert pf(ctypes.byref(d), None, FAKE, 8, FAKE, FAKE, FAKE, hc, 16, 4, FAKE, FAKE, 100,
+              None) == ops.RTP_ERR_WORKSPACE
+    assert L.rtp_workspace_size(ctypes.byref(d), ops.OP_PREFILL) == 256
     assert L.rtp_workspace_init(None, 100, None) == ops.RTP_ERR_WORKSPACE
     assert L.rtp_check(None, None) == ops.RTP_ERR_WORKSPACE
     assert L.rtp_selftest_wait_timeout(None, None) == ops.RTP_ERR_INVALID_ARG

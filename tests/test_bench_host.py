@@ -174,3 +174,16 @@ def test_reference_arm_under_two_ranks_prints_one_line_from_rank0():
     assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
     assert rec["cpu_baseline"]["kind"] == "oracle" and rec["cpu_baseline"]["cores"] == 1
     assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["e2e"]["value"] == rec["value"]
+
+
+def test_prefill_pairs_closed_forms():
+    """Causal pairs: T tokens from position 0 see 1 + 2 + ... + T keys; a
+    local head's tokens see min(P + 1, window + sinks) keys once the
+    window has passed the sinks."""
+    assert bench.prefill_pairs(0, 10, 4, 1, False) == 55
+    assert bench.prefill_pairs(5, 3, 4, 1, False) == 6 + 7 + 8
+    # window 4, 1 sink: positions 0..9 see 1, 2, 3, 4, 5, then 5 each
+    assert bench.prefill_pairs(0, 10, 4, 1, True) == 1 + 2 + 3 + 4 + 5 * 6
+    assert bench.local_pairs(3, 100, 4) == 3
+    assert bench.local_pairs(1000, 4096, 4) == 1000
+    assert bench.local_pairs(65536, 4096, 4) == 4100
