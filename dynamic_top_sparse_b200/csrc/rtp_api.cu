@@ -529,23 +529,32 @@ int rtp_append_index_keys(const rtp_dims *dims, const void *k_pre, int32_t T, co
     unsigned long long mask = head_class ? ret_mask(dims, head_class)
                                          : (dims->H_kv >= 64 ? ~0ull : ((1ull << dims->H_kv) - 1));
     Launcher ln{(cudaStream_t)stream, nullptr};
-    const dim3 grid((unsigned)((T + APP_WARPS - 1) / APP_WARPS), (unsigned)(dims->B * dims->H_kv));
-    const dim3 block(APP_WARPS * 32);
+    // the append waits on the device for the previous kernel of the stream,
+    // so its launch overlaps that kernel's tail
+    ln.pdl = true;
+    // about two CTAs per SM over all (b, g); runs of APP_TOK tokens
+    const long long units = (long long)dims->B * dims->H_kv;
+    const long long per_bg = std::max(1LL, 2LL * num_sms() / units);
+    long long tpc = std::max<long long>(APP_TOK, (T + per_bg - 1) / per_bg);
+    tpc = (tpc + APP_TOK - 1) / APP_TOK * APP_TOK;
+    const dim3 grid((unsigned)((T + tpc - 1) / tpc), (unsigned)units);
+    const dim3 block(APP_THREADS);
+    const int tp = (int)tpc;
     const bool kb = dims->kv_dtype == RTP_BF16, ib = dims->idx_dtype == RTP_BF16;
     if (kb && ib)
         return ln.run("append", append_kernel<__nv_bfloat16, __nv_bfloat16>, grid, block,
                       (const __nv_bfloat16 *)k_pre, W_k_idx, pos, (__nv_bfloat16 *)kidx_cache,
-                      dims->H_kv, (int)T, (long long)dims->N_max, mask, status);
+                      dims->H_kv, (int)T, tp, (long long)dims->N_max, mask, status);
     if (kb && !ib)
         return ln.run("append", append_kernel<__nv_bfloat16, float>, grid, block,
                       (const __nv_bfloat16 *)k_pre, W_k_idx, pos, (float *)kidx_cache, dims->H_kv,
-                      (int)T, (long long)dims->N_max, mask, status);
+                      (int)T, tp, (long long)dims->N_max, mask, status);
     if (!kb && ib)
         return ln.run("append", append_kernel<float, __nv_bfloat16>, grid, block,
                       (const float *)k_pre, W_k_idx, pos, (__nv_bfloat16 *)kidx_cache, dims->H_kv,
-                      (int)T, (long long)dims->N_max, mask, status);
+                      (int)T, tp, (long long)dims->N_max, mask, status);
     return ln.run("append", append_kernel<float, float>, grid, block, (const float *)k_pre, W_k_idx,
-                  pos, (float *)kidx_cache, dims->H_kv, (int)T, (long long)dims->N_max, mask, status);
+                  pos, (float *)kidx_cache, dims->H_kv, (int)T, tp, (long long)dims->N_max, mask, status);
 }
 
 int rtp_index_scores(const rtp_dims *dims, const rtp_opts *opts, const float *q,
