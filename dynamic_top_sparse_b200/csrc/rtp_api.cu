@@ -768,8 +768,19 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
     if (any_local && s.a.n_ret > 0) {
         int max_ctas = 0;
         if (selecting) {
+            // SMs for the local heads in proportion to their bytes against
+            // the selection's (the index keys, read by the scan and again by
+            // the collect pass); both move about the same bytes per SM and
+            // microsecond.  At least LOCAL_SMS, at most half the GPU.
             const int groups = dims->B * (dims->H_kv - s.a.n_ret);
-            local_ctas = groups * std::max(1, LOCAL_SMS / groups);
+            const double kv_el = dims->kv_dtype == RTP_BF16 ? 2.0 : 4.0;
+            const double ix_el = dims->idx_dtype == RTP_BF16 ? 2.0 : 4.0;
+            const double rows = std::min<double>((double)dims->N_max, (double)window + (double)n_sink);
+            const double lb = (double)groups * rows * 2.0 * D * kv_el;
+            const double sb = 2.0 * dims->B * s.a.n_ret * (double)dims->N_max * R * ix_el;
+            int want = (int)std::lround(num_sms() * lb / std::max(1.0, lb + sb));
+            want = std::max(LOCAL_SMS, std::min(want, num_sms() / 2));
+            local_ctas = groups * std::max(1, want / groups);
             local_ctas = std::min(local_ctas, num_sms() / 2);
             max_ctas = local_ctas;
         }
