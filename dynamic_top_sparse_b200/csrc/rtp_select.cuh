@@ -792,6 +792,55 @@ __device__ __forceinline__ int scan_value(float z, uint32_t row, int &bin) {
     return kr;
 }
 
+// The two head slots of one token at once: scan_value's bin arithmetic on
+// the top 16 bits of both floats (sign, exponent and the top MB mantissa
+// bits all sit there, and so does the upper edge of a bin) packed into one
+// register and worked in 16-bit halves.  Per half: a = exponent and top MB
+// mantissa bits of |z|; kc = a clamped to [BIN_BASE, BIN_BASE + 255]; nm =
+// 0xffff where z < 0; bin = kc - BIN_BASE + 256 (z >= 0) or BIN_BASE + 255 -
+// kc (z < 0), computed as (kc ^ nm) minus P_POS or P_NEG; the bin's upper
+// edge has top bits (kc + 1) << 3 (z >= 0) or kc << 3 | 0x8000 (z < 0).  No
+// half carries into or borrows from the other.  amax keeps the largest a of
+// each slot (above A_OK: out of range or not finite), bmax the largest bin.
+// Same bins and edges as scan_value for every value in range.
+static_assert(MB == 4, "scan_pair's packed layout assumes 4 mantissa bits per bin");
+constexpr uint32_t P_POS = (uint32_t)BIN_BASE - 256u;
+constexpr uint32_t P_NEG = 65535u - ((uint32_t)BIN_BASE + 255u);
+constexpr uint32_t A_OK = (uint32_t)BIN_BASE + (uint32_t)KMAX_OK;
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ void scan_pair(float z0, float z1, uint32_t row0, uint32_t row1, uint32_t &amax,
+                                          uint32_t &bmax) {
+    const uint32_t h = prmt(__float_as_uint(z0), __float_as_uint(z1), 0x7632u);   // [top(z1) : top(z0)]
+    const uint32_t a = (h >> 3) & 0x0fff0fffu;
+    amax = max_u16x2(amax, a);
+    const uint32_t kc = min_u16x2(max_u16x2(a, (uint32_t)BIN_BASE * 0x10001u), ((uint32_t)BIN_BASE + 255u) * 0x10001u);
+    const uint32_t nm = prmt(h, 0u, 0xbb99u);              // each half: its sign bit replicated
+    // (the mask changes no bin; it keeps every address inside the head's row
+    // whatever the halves hold)
+    const uint32_t bin2 = ((kc ^ nm) - (P_POS * 0x10001u + (nm & ((P_NEG - P_POS) * 0x10001u)))) & 0x01ff01ffu;
+    bmax = max_u16x2(bmax, bin2);
+    const uint32_t hu = (kc << 3) + (nm & 0x7ff87ff8u) + 0x00080008u;
+    const float U0 = __uint_as_float(hu << 16), U1 = __uint_as_float(hu & 0xffff0000u);
+    const uint32_t fx0 = __float2uint_rn(ex2_sfu(fmaf(z0 - U0, L2E, 18.0f)));
+    const uint32_t fx1 = __float2uint_rn(ex2_sfu(fmaf(z1 - U1, L2E, 18.0f)));
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row0 + 4u * (bin2 & 0xffffu)), "r"(fx0) : "memory");
+    asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row1 + 4u * (bin2 >> 16)), "r"(fx1) : "memory");
+}
+
 // Producer of a TMA ring (lane 0 of the producer warp): streams the index
 // keys of tokens [t_lo, t_hi) stage by stage into `ring` (ST_TOK tokens per
 // stage).  Waits are bounded: on a timeout it records RTP_ERR_TIMEOUT and
@@ -892,6 +941,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
         const uint32_t hrow0 = smem_u32(h32 + (2 * tig) * NBIN), hrow1 = smem_u32(h32 + (2 * tig + 1) * NBIN);
         const bool full_group = G == GMAX;
         int kmax = 0;
+        uint32_t amax = 0u;                // packed largest exponent bits per slot (scan_pair)
         uint32_t *tbin = reinterpret_cast<uint32_t *>(w.tilebin + bg * a.ntile * GMAX);
 
         // One 32-token tile: logits on the tensor cores, level-1 masses into
@@ -905,16 +955,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
                     f.a[i][r] = *reinterpret_cast<const uint2 *>(tile + (16 * i + gid + 8 * r) * (R * 2) + 8 * tig);
             float z[SrcMma::NV];
             src.eval(f, z);
-            int tmax[2] = {-1, -1};
+            // the lane's largest bin per head slot, both slots in one word:
+            // (1 + max bin) per 16-bit half (0: no value)
+            uint32_t pk;
             if (nvalid >= TILE && full_group) {
+                // value v is slot v & 1 of its token: pairs (v, v + 1)
+                uint32_t bmax = 0u;
 #pragma unroll
-                for (int v = 0; v < SrcMma::NV; ++v) {
-                    const int sl = v & 1;
-                    int bin;
-                    kmax = max(kmax, scan_value(z[v] + 0.0f, sl ? hrow1 : hrow0, bin));
-                    tmax[sl] = max(tmax[sl], bin);
-                }
+                for (int v = 0; v < SrcMma::NV; v += 2)
+                    scan_pair(z[v] + 0.0f, z[v + 1] + 0.0f, hrow0, hrow1, amax, bmax);
+                pk = bmax + 0x00010001u;
             } else {
+                int tmax[2] = {-1, -1};
 #pragma unroll
                 for (int v = 0; v < SrcMma::NV; ++v) {
                     const int sl = v & 1;
@@ -923,9 +975,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
                     kmax = max(kmax, scan_value(z[v] + 0.0f, sl ? hrow1 : hrow0, bin));
                     tmax[sl] = max(tmax[sl], bin);
                 }
+                pk = (uint32_t)(tmax[0] + 1) | ((uint32_t)(tmax[1] + 1) << 16);
             }
-            // both head slots in one word: (1 + max bin) per 16-bit half
-            uint32_t pk = (uint32_t)(tmax[0] + 1) | ((uint32_t)(tmax[1] + 1) << 16);
+            // max over the warp's lanes of the same slots
 #pragma unroll
             for (int o = 4; o < 32; o <<= 1) {
                 const uint32_t other = __shfl_xor_sync(0xffffffffu, pk, o);
@@ -967,7 +1019,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
                 asm volatile("bar.sync 1, %0;" ::"r"(TC_WARPS * 32) : "memory");
             }
         }
-        if (kmax > KMAX_OK) s_err = 1;
+        if (kmax > KMAX_OK || max(amax & 0xffffu, amax >> 16) > A_OK) s_err = 1;
     }
     __syncthreads();
     if (s_err && threadIdx.x == 0) set_status(w.status, RTP_ERR_RANGE);
