@@ -991,12 +991,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
         bool dead = false;
         int st = 0, phase = 0, spill_in = SPILL_STAGES;
         for (int it = 0; it < n_st; ++it) {
-            if (!dead) dead = *(volatile int *)&s_abort != 0;
-            if (!dead && !mbar_wait(&full[st], (uint32_t)phase)) {
+            // one decision for the warp, so scan_tile (tensor cores, full-warp
+            // shuffles) runs with all 32 lanes or none; every lane waits on
+            // the barrier itself (its own acquire of the stage)
+            int live = dead ? 0 : (*(volatile int *)&s_abort == 0);
+            live = __shfl_sync(0xffffffffu, live, 0);
+            if (live && !mbar_wait(&full[st], (uint32_t)phase)) {
                 set_status(w.status, RTP_ERR_TIMEOUT);
                 s_abort = 1;
-                dead = true;
+                live = 0;
             }
+            dead = !__all_sync(0xffffffffu, live);
             if (!dead) {
                 const int tb0 = t_lo + it * ST_TOK + warp * TILE;
                 const uint8_t *tiles = ring + st * ST_BYTES + warp * (TILE * R * 2);
