@@ -180,13 +180,13 @@ def build_workload(key: str, seed: int = 0):
     return spec, layers
 
 
-def required_bytes(spec, layers, sel, p=None):
+def required_bytes(spec, layers, sel, p=None, topk=0):
     """Algorithmic bytes a step must read: index keys of retrieval heads
-    (only when a threshold is computed, p < 1), the union of kept K/V rows
+    (only when a threshold is computed: p < 1 or static top-k), the union of kept K/V rows
     per KV group (every row at p >= 1), window+sink rows of local heads, and
     the query projector of retrieval heads (only when selecting)."""
     p = spec.p if p is None else p
-    selecting = p < 1.0
+    selecting = topk > 0 or p < 1.0
     total = 0
     kv_el = 2 if spec.kv_dtype == "bf16" else 4
     ix_el = 2 if spec.idx_dtype == "bf16" else 4
@@ -255,16 +255,17 @@ class Bench:
             self.reps.append([L.clone_caches() for L in self.layers0])
         self.reps = self.reps[:n]
 
-    def step(self, layers, p, prof=None, sel=None):
+    def step(self, layers, p, prof=None, sel=None, topk=0):
+        """One step of every layer: top-p with p, or static top-k when topk > 0."""
         spec = self.spec
         for li, L in enumerate(layers):
             ops.append_index_keys(L.dims, L.k_new, L.Wk, L.pos, L.hc, L.kidx, self.ws)
             opts = None
-            if prof is not None or sel is not None:
+            if prof is not None or sel is not None or topk:
                 kw = {}
                 if sel is not None:
                     kw = dict(sel_idx=sel[li][0], sel_count=sel[li][1])
-                opts = ops.make_opts(prof=prof, **kw)
+                opts = ops.make_opts(prof=prof, topk=topk, **kw)
             ops.decode_step(L.dims, L.q, L.q_rope, L.k, L.v, L.kidx, L.Wq, L.hc, p, spec.window,
                             spec.n_sink, self.out, self.ws, opts)
 
@@ -277,18 +278,19 @@ class Bench:
         if st:
             raise RuntimeError(f"device status {st}: {ops.error_string(st)}")
 
-    def selection(self, p):
+    def selection(self, p, topk=0):
         """Kept sets of one step -> (required bytes, kept counts per layer)."""
         spec = self.spec
-        if p >= 1.0:
+        if p >= 1.0 and not topk:
             self.step(self.layers0, p)
             self.check()
             return required_bytes(spec, self.layers0, None, p), []
         sel = [(torch.full((spec.B, spec.H_q, L.k.shape[2]), -1, dtype=torch.int32, device=self.dev),
                 torch.zeros((spec.B, spec.H_q), dtype=torch.int32, device=self.dev)) for L in self.layers0]
-        self.step(self.layers0, p, sel=sel)
+        self.step(self.layers0, p, sel=sel, topk=topk)
         self.check()
-        req = required_bytes(spec, self.layers0, [(a.cpu().numpy(), b.cpu().numpy()) for a, b in sel], p)
+        req = required_bytes(spec, self.layers0, [(a.cpu().numpy(), b.cpu().numpy()) for a, b in sel], p,
+                             topk)
         kept = [[int(x) for x in b.cpu().numpy().ravel() if x > 0] for _, b in sel]
         return req, kept
 
@@ -328,9 +330,9 @@ class Bench:
         barrier(world)
         return allreduce_max(e0.elapsed_time(e1), world, self.dev) / steps
 
-    def launches_per_step(self, p):
+    def launches_per_step(self, p, topk=0):
         pr = ops.Profiler(1024)
-        self.step(self.reps[0], p, prof=pr)
+        self.step(self.reps[0], p, prof=pr, topk=topk)
         torch.cuda.synchronize()
         # rtp_append_index_keys takes no options, so its one launch per layer
         # is not in the profiler's count
@@ -338,7 +340,7 @@ class Bench:
         pr.close()
         return n
 
-    def breakdown(self, p, n_prof, per_step_slots):
+    def breakdown(self, p, n_prof, per_step_slots, topk=0):
         """Per-kernel device times: the step captured with event-record nodes
         around every kernel (one graph per replica, distinct event slots),
         replayed with a sync after each replay to read the slots."""
@@ -349,7 +351,7 @@ class Bench:
             g = torch.cuda.CUDAGraph()
             first = pr.p.count
             with torch.cuda.graph(g):
-                self.step(R, p, prof=pr)
+                self.step(R, p, prof=pr, topk=topk)
             pgraphs.append((g, first, pr.p.count))
         torch.cuda.synchronize()
         times = {}
@@ -394,27 +396,28 @@ def kept_stats(kept):
     return {"min": min(flat), "max": max(flat), "mean": float(np.mean(flat))}
 
 
-def measure_point(bn, p, steps, warmup, world, hbm_peak, max_replicas, n_prof, clocks=None):
-    """One (workload, p) point: step time, required bytes and their rate,
-    the scan kernel's rate and the per-kernel times."""
+def measure_point(bn, p, steps, warmup, world, hbm_peak, max_replicas, n_prof, clocks=None, topk=0):
+    """One (workload, p) point -- or static top-k with topk > 0: step time,
+    required bytes and their rate, the scan kernel's rate and the per-kernel
+    times."""
     spec = bn.spec
-    req, kept = bn.selection(p)
+    req, kept = bn.selection(p, topk)
     bn.set_replicas(replicas_for(spec, req, max_replicas))
-    lps = bn.launches_per_step(p)
-    graphs = bn.capture(lambda R: bn.step(R, p))
+    lps = bn.launches_per_step(p, topk)
+    graphs = bn.capture(lambda R: bn.step(R, p, topk=topk))
     ms = bn.time_graphs(graphs, steps, warmup, world, clocks)
     del graphs
-    times = bn.breakdown(p, n_prof, lps + 4)
+    times = bn.breakdown(p, n_prof, lps + 4, topk)
     hist = times.get("hist", [])
     # one scan launch per layer: its time per launch, and the index keys of
     # one layer's retrieval groups per launch
     hist_ms = float(np.mean(hist)) if hist else None
-    idx_b = index_bytes(spec, bn.layers0) // max(1, len(bn.layers0)) if p < 1.0 else 0
+    idx_b = index_bytes(spec, bn.layers0) // max(1, len(bn.layers0)) if (p < 1.0 or topk) else 0
     scan_gbs = idx_b / (hist_ms * 1e-3) / 1e9 if hist_ms else None
     gbs = req / (ms * 1e-3) / 1e9
     n_rep = len(bn.reps)
     return {
-        "p": p, "ms_per_step": ms, "steps_per_s": 1e3 / ms, "required_bytes_per_step": int(req),
+        "p": None if topk else p, "topk": topk or None, "ms_per_step": ms, "steps_per_s": 1e3 / ms, "required_bytes_per_step": int(req),
         "achieved_gbs": gbs, "pct_peak": gbs / hbm_peak, "pct_of_8tbs": gbs / 8000.0,
         "scan": {"gbs": scan_gbs, "frac": scan_gbs / hbm_peak if scan_gbs else None,
                  "avg_launch_ms": hist_ms, "bytes_per_launch": idx_b},
@@ -502,6 +505,9 @@ def e2e_measure(bn, p, graphs, steps, world):
             "graph_note": "the per-step-wait form with the step's C-ABI calls captured once in a "
                           "CUDA graph and replayed"}
 
+
+# static top-k budget measured beside the headline's top-p (tokens per head)
+TOPK_BUDGET = 2048
 
 # workloads measured beside the headline line, in the same run
 SWEEP = (("ctx64k", (0.9,)), ("ctx1m", (0.8, 0.9, 0.95, 1.0)), ("ctx128k-b8-48layer", (0.9,)))
@@ -628,6 +634,13 @@ def run_ours(args, rank, world, dev):
     ms_per_step = pt["ms_per_step"]
     value = world / (ms_per_step * 1e-3)
     dense_ms = bn.dense_ms(max(3, min(args.steps, args.dense_steps)), world)
+    # static top-k on the same caches, beside top-p: the fixed budget of
+    # TOPK_BUDGET tokens per head
+    topk_pt = measure_point(bn, p, args.sweep_steps, args.warmup, world, hbm_peak, args.max_replicas,
+                            min(args.prof_steps, 50), topk=TOPK_BUDGET)
+    topk_pt["dense_ms_per_step"] = dense_ms
+    topk_pt["speedup_sparse_vs_dense"] = dense_ms / topk_pt["ms_per_step"]
+    bn.set_replicas(pt["replicas"])
 
     e2e = None
     if not args.no_e2e:
@@ -680,6 +693,7 @@ def run_ours(args, rank, world, dev):
         "replicas": n_rep,
         "clocks": clocks.report(),
         "e2e": e2e,
+        "topk": topk_pt,
         "workloads": sweep,
         "prefill": prefill,
         "pages_context": {"decode_speedup_1M_H20": 2.01, "prefill_speedup_1M_H20": 9.36},

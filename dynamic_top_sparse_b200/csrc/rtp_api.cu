@@ -280,7 +280,9 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sm
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
     if (!attr_set[dev]) {
-        if (cudaFuncSetAttribute(scan_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM) !=
+        if (cudaFuncSetAttribute(scan_tma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(scan_tma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM) !=
                 cudaSuccess ||
             cudaFuncSetAttribute(collect_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CL_SMEM) !=
                 cudaSuccess)
@@ -304,7 +306,8 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sm
     // previous kernel's tail
     const bool pdl0 = ln.pdl;
     ln.pdl = true;
-    int rc = ln.run_smem("hist", scan_tma_kernel, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w);
+    int rc = s.a.topk > 0 ? ln.run_smem("hist", scan_tma_kernel<true>, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w)
+                          : ln.run_smem("hist", scan_tma_kernel<false>, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w);
     if (rc == RTP_OK) rc = ln.run_smem("collect", collect_mma_kernel, cl_grid, dim3(CL_THREADS), CL_SMEM, s.a, s.w);
     if (rc == RTP_OK && after_collect) rc = after_collect();
     if (rc == RTP_OK) {
@@ -602,6 +605,26 @@ int rtp_topp_select(const rtp_dims *dims, const float *z, const uint8_t *head_cl
     return launch_select<SrcBuffer>(ln, dims, s);
 }
 
+int rtp_topk_select(const rtp_dims *dims, const float *z, const uint8_t *head_class, int32_t k,
+                    int32_t *idx_out, int32_t *count_out, void *ws, size_t ws_bytes, rtp_stream_t stream) {
+    RTP_TRY(check_dims(dims));
+    if (!z || !idx_out || !count_out || k < 1) return RTP_ERR_INVALID_ARG;
+    if (!aligned16(z)) return RTP_ERR_INVALID_ARG;
+    RTP_TRY(check_head_class(dims, head_class));
+    RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_TOPP_SELECT));
+    const Layout L = make_layout(dims);
+    SelPlan s = make_sel(dims, head_class, (char *)ws, L);
+    if (s.a.n_ret == 0) return RTP_OK;
+    s.a.z = z;
+    s.a.p = 0.0f;           // not used with topk
+    s.a.topk = k;
+    s.a.lists = idx_out;
+    s.a.count_out = count_out;
+    s.a.mass_out = nullptr;
+    Launcher ln{(cudaStream_t)stream, nullptr};
+    return launch_select<SrcBuffer>(ln, dims, s);
+}
+
 int rtp_sparse_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
                       const void *k_cache, const void *v_cache, const int32_t *idx,
                       const int32_t *count, const uint8_t *head_class, float *out, void *ws,
@@ -763,7 +786,9 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
     // joined at its end.  Beside the selection they get a few SMs of their
     // own (the selection kernels take one CTA per SM on the rest), so that
     // neither waits for the other's CTAs to drain.
-    const bool selecting = s.a.n_ret > 0 && p < 1.0f;
+    const int topk = opts ? opts->topk : 0;
+    if (topk < 0) return RTP_ERR_INVALID_ARG;
+    const bool selecting = s.a.n_ret > 0 && (topk > 0 || p < 1.0f);
     int local_ctas = 0;
     if (any_local && s.a.n_ret > 0) {
         int max_ctas = 0;
@@ -797,7 +822,7 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
     }
     int rc = RTP_OK;
     if (s.a.n_ret > 0) {
-        if (p >= 1.0f) {
+        if (!selecting) {
             // every token is kept: the retrieval heads' attention is dense
             rc = launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_RETRIEVAL, true, 1, 0,
                               out, w, L, asc);
@@ -807,6 +832,7 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
             s.a.Wq = W_q_idx;
             s.a.idx_scale = isc;
             s.a.p = p;
+            s.a.topk = topk;
             s.a.lists = opts && opts->sel_idx ? opts->sel_idx : reinterpret_cast<int32_t *>(w + L.lists);
             s.a.count_out = opts && opts->sel_count ? opts->sel_count : reinterpret_cast<int32_t *>(w + L.counts);
             s.a.mass_out = opts ? opts->sel_mass : nullptr;

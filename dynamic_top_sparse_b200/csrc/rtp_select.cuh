@@ -212,6 +212,10 @@ struct SelArgs {
     int n_ret;
     int ret_g[MAX_RET_GROUPS];
     float p;
+    // > 0: keep the topk largest logits of each head instead of the top-p
+    // set (static top-k, the fixed budget Method section 3 sets top-p
+    // against): every token counts one unit where top-p counts its mass
+    int topk;
     float idx_scale;
     const float *q;              // [B, H_q, D] pre-RoPE queries
     const float *Wq;             // [H_q, R, D]
@@ -575,7 +579,10 @@ template <> struct NeedsQ<SrcBuffer> : std::false_type {};
 // bin factors within the boundary octave use the same fp32 expression as
 // finalize.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, float p, int N) {
+// With topk > 0 the histogram holds token counts (every octave factor is 1)
+// and the target is min(topk, N) tokens; counts are exact in fp64.
+__device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, float p, int N, int topk) {
+    const bool cnt = topk > 0;
     const int lane = threadIdx.x & 31;
     double ss = 0.0;
 #pragma unroll
@@ -590,7 +597,8 @@ __device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, f
     const int stop = 31 - __clz(ne), slow = __ffs(ne) - 1;
     const float R0 = bin_upper(16 * stop + 15);
     // octave masses relative to R0, inclusive suffix sums from the top octave
-    const double ms = ss > 0.0 ? ss * exp2_wide((double)(bin_upper(16 * lane + 15) - R0) * L2E_D) : 0.0;
+    const double ms = ss > 0.0 ? (cnt ? ss : ss * exp2_wide((double)(bin_upper(16 * lane + 15) - R0) * L2E_D))
+                               : 0.0;
     double incl = ms;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -598,7 +606,7 @@ __device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, f
         if (lane + o < 32) incl += t;
     }
     const double Z0 = __shfl_sync(0xffffffffu, incl, 0);
-    const double target0 = p >= 1.0f ? 0.0 : p <= 0.0f ? 0.0 : (double)p * Z0;
+    const double target0 = cnt ? (double)min(topk, N) : p >= 1.0f ? 0.0 : p <= 0.0f ? 0.0 : (double)p * Z0;
     const unsigned hit = __ballot_sync(0xffffffffu, ms > 0.0 && incl >= target0);
     // boundary octave (rounding kept p Z out of reach: the lowest octave)
     const int sb = hit ? 31 - __clz(hit) : slow;
@@ -609,19 +617,19 @@ __device__ __forceinline__ Resolve resolve_head(const double *__restrict__ gh, f
     const unsigned nt = __ballot_sync(0xffffffffu, lane >= 16 && sv > 0.0) >> 16;
     const int btop = 16 * stop + (nt ? 31 - __clz(nt) : 15);
     const float R = bin_upper(btop);
-    const double sc = exp2_wide((double)(R0 - R) * L2E_D);       // R0 units -> R units (>= 1)
+    const double sc = cnt ? 1.0 : exp2_wide((double)(R0 - R) * L2E_D);   // R0 units -> R units (>= 1)
     const double Z = Z0 * sc;
     r.Z = Z;
     r.R = R;
-    if (p >= 1.0f) {
+    if (cnt ? topk >= N : p >= 1.0f) {
         r.mode = MODE_KEEP_ALL; r.bstar = -1; r.above = 0; r.target = 0;
         return r;
     }
-    const double target = p <= 0.0f ? 0.0 : (double)p * Z;
+    const double target = cnt ? (double)topk : p <= 0.0f ? 0.0 : (double)p * Z;
     // the boundary octave's bins relative to R (lane 15 = its highest bin),
     // inclusive suffix sums on top of the octaves above
     const double mb = lane < 16 && sv > 0.0
-                          ? sv * (double)ex2_sfu((bin_upper(bin) - R) * L2E) : 0.0;
+                          ? (cnt ? sv : sv * (double)ex2_sfu((bin_upper(bin) - R) * L2E)) : 0.0;
     double incb = mb;
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) {
@@ -669,7 +677,7 @@ __global__ void __launch_bounds__(SCAN_THREADS, 2) scan_kernel(SelArgs a, SelWs 
         if (a.ovf) a.ovf[bh0 + threadIdx.x] = 0u;
     }
     for (int i = threadIdx.x; i < 2 * GMAX * NBIN; i += blockDim.x) shl[i] = 0u;
-    for (int i = threadIdx.x; i < NBIN; i += blockDim.x) s_fac[i] = octave_factor(i);
+    for (int i = threadIdx.x; i < NBIN; i += blockDim.x) s_fac[i] = a.topk ? 1.0 : octave_factor(i);
     if constexpr (NeedsQ<Src>::value) {
         project_query<(GMAX * R + SCAN_WARPS - 1) / SCAN_WARPS>(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D,
                                                                a.idx_scale, qs, G, warp, SCAN_WARPS);
@@ -708,6 +716,7 @@ __global__ void __launch_bounds__(SCAN_THREADS, 2) scan_kernel(SelArgs a, SelWs 
                 err |= !(fabsf(zz) < Z_LIMIT);
                 uint32_t fx;
                 const int bin = bin_and_fx(zz, fx);
+                if (a.topk) fx = (uint32_t)FX_ONE;
                 uint32_t *cell = &shl[src.head(sl) * NBIN + bin];
                 const uint32_t old = atomicAdd(cell, fx);
                 if (old + fx < old) atomicAdd(cell + GMAX * NBIN, 1u);
@@ -723,6 +732,7 @@ __global__ void __launch_bounds__(SCAN_THREADS, 2) scan_kernel(SelArgs a, SelWs 
                 if (!(fabsf(zz) < Z_LIMIT)) { err = 1; continue; }
                 uint32_t fx;
                 const int bin = bin_and_fx(zz, fx);
+                if (a.topk) fx = (uint32_t)FX_ONE;
                 uint32_t *cell = &shl[h * NBIN + bin];
                 const uint32_t old = atomicAdd(cell, fx);
                 if (old + fx < old) atomicAdd(cell + GMAX * NBIN, 1u);
@@ -779,14 +789,17 @@ static_assert((long long)SPILL_STAGES * ST_TOK * 266240LL < 4294967296LL, "bin c
 // shared address `row` (32-bit, bins of 4 bytes) and returns the raw
 // (unclamped) k, whose maximum the caller checks once (k > KMAX_OK: z out
 // of range or not finite).  The clamped bin index is returned in `bin`.
+// CNT (static top-k): every value adds one unit, 2^18, instead of its mass.
 constexpr int KMAX_OK = (int)((127 + 7) << MB) + 15 - (int)BIN_BASE;   // |z| < 256
+constexpr uint32_t CNT_UNIT = 1u << 18;
+template <bool CNT>
 __device__ __forceinline__ int scan_value(float z, uint32_t row, int &bin) {
     const uint32_t u = __float_as_uint(z);
     const int s = (int)u >> 31;                                          // 0 or -1
     const int kr = (int)((u << 1) >> (24 - MB)) - (int)BIN_BASE;
     const int k = max(kr, 0) & 255;
     const uint32_t eb = ((uint32_t)(k + (int)BIN_BASE + 1 + s) << (23 - MB)) | (u & 0x80000000u);
-    const uint32_t fx = __float2uint_rn(ex2_sfu(fmaf(z - __uint_as_float(eb), L2E, 18.0f)));
+    const uint32_t fx = CNT ? CNT_UNIT : __float2uint_rn(ex2_sfu(fmaf(z - __uint_as_float(eb), L2E, 18.0f)));
     bin = 256 + (k ^ s);
     asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row + 4u * (uint32_t)bin), "r"(fx) : "memory");
     return kr;
@@ -822,6 +835,7 @@ __device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
     asm("min.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
 }
+template <bool CNT>
 __device__ __forceinline__ void scan_pair(float z0, float z1, uint32_t row0, uint32_t row1, uint32_t &amax,
                                           uint32_t &bmax) {
     const uint32_t h = prmt(__float_as_uint(z0), __float_as_uint(z1), 0x7632u);   // [top(z1) : top(z0)]
@@ -835,8 +849,8 @@ __device__ __forceinline__ void scan_pair(float z0, float z1, uint32_t row0, uin
     bmax = max_u16x2(bmax, bin2);
     const uint32_t hu = (kc << 3) + (nm & 0x7ff87ff8u) + 0x00080008u;
     const float U0 = __uint_as_float(hu << 16), U1 = __uint_as_float(hu & 0xffff0000u);
-    const uint32_t fx0 = __float2uint_rn(ex2_sfu(fmaf(z0 - U0, L2E, 18.0f)));
-    const uint32_t fx1 = __float2uint_rn(ex2_sfu(fmaf(z1 - U1, L2E, 18.0f)));
+    const uint32_t fx0 = CNT ? CNT_UNIT : __float2uint_rn(ex2_sfu(fmaf(z0 - U0, L2E, 18.0f)));
+    const uint32_t fx1 = CNT ? CNT_UNIT : __float2uint_rn(ex2_sfu(fmaf(z1 - U1, L2E, 18.0f)));
     asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row0 + 4u * (bin2 & 0xffffu)), "r"(fx0) : "memory");
     asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row1 + 4u * (bin2 >> 16)), "r"(fx1) : "memory");
 }
@@ -874,6 +888,7 @@ __device__ __forceinline__ void ring_drain(uint64_t *full, int issued) {
         mbar_wait(&full[it % NS], (uint32_t)((it / NS) & 1));
 }
 
+template <bool CNT>
 __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelWs w) {
     extern __shared__ __align__(128) uint8_t dsm[];
     uint8_t *ring = dsm;
@@ -919,7 +934,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
         if (lane == 0)
             ring_drain<NSTAGE>(full, issued);
         else
-            for (int i = lane - 1; i < NBIN; i += 31) s_fac[i] = octave_factor(i);
+            for (int i = lane - 1; i < NBIN; i += 31) s_fac[i] = CNT ? 1.0 : octave_factor(i);
     } else {
         // consumers: finish q_idx of the group (the producer is already streaming)
         qp.store(a.idx_scale, qs, G, warp, TC_WARPS);
@@ -963,7 +978,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
                 uint32_t bmax = 0u;
 #pragma unroll
                 for (int v = 0; v < SrcMma::NV; v += 2)
-                    scan_pair(z[v] + 0.0f, z[v + 1] + 0.0f, hrow0, hrow1, amax, bmax);
+                    scan_pair<CNT>(z[v] + 0.0f, z[v + 1] + 0.0f, hrow0, hrow1, amax, bmax);
                 pk = bmax + 0x00010001u;
             } else {
                 int tmax[2] = {-1, -1};
@@ -972,7 +987,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
                     const int sl = v & 1;
                     if (2 * tig + sl >= G || src.tok(v) >= nvalid) continue;
                     int bin;
-                    kmax = max(kmax, scan_value(z[v] + 0.0f, sl ? hrow1 : hrow0, bin));
+                    kmax = max(kmax, scan_value<CNT>(z[v] + 0.0f, sl ? hrow1 : hrow0, bin));
                     tmax[sl] = max(tmax[sl], bin);
                 }
                 pk = (uint32_t)(tmax[0] + 1) | ((uint32_t)(tmax[1] + 1) << 16);
@@ -1063,7 +1078,7 @@ __global__ void __launch_bounds__(COL_THREADS, 2) collect_kernel(SelArgs a, SelW
     if (warp < GMAX) {
         int mode = MODE_EMPTY, bs = NBIN;
         if (warp < G) {
-            const Resolve r = resolve_head(w.hist + (bh0 + warp) * HSTRIDE, a.p, N);
+            const Resolve r = resolve_head(w.hist + (bh0 + warp) * HSTRIDE, a.p, N, a.topk);
             if (blockIdx.x == 0 && lane == 0) w.res[bh0 + warp] = r;
             mode = r.mode;
             bs = r.bstar;
@@ -1267,7 +1282,7 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
         int bs = NBIN, mode = MODE_EMPTY;
         if (ph_ok(warp)) {
             const size_t bh = ph_bh(warp);
-            const Resolve r = resolve_head(w.hist + bh * HSTRIDE, a.p, warp < GMAX ? N0 : N1);
+            const Resolve r = resolve_head(w.hist + bh * HSTRIDE, a.p, warp < GMAX ? N0 : N1, a.topk);
             if (cx == 0 && lane == 0) s_res[warp] = r;
             mode = r.mode;
             bs = r.bstar;
@@ -1610,7 +1625,11 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         // mass keeps >= 19 bits).  Otherwise 64-bit, S = 2^62 / nc.
         const bool staged = nc <= (unsigned)FIN_CAP;
         const double S = staged ? (double)(0x7fffffffu / nc) : ldexp(1.0, 62) / (double)nc;
+        // static top-k: every candidate weighs one unit and the target is a
+        // whole number of units (exact integers)
+        const unsigned long long unit = (unsigned long long)S;
         auto fx_of = [&](unsigned long long v) -> unsigned long long {
+            if (a.topk > 0) return unit;
             const float m = ex2_sfu((cand_logit(v) - Ub) * L2E);
             return (unsigned long long)((double)m * S);
         };
@@ -1638,7 +1657,8 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         }
         __syncthreads();
         const double tS = r.target / (double)ex2_sfu((Ub - r.R) * L2E) * S;
-        unsigned long long T = !(tS < 9.0e18) ? ~0ull : (unsigned long long)llrint(tS);
+        unsigned long long T = a.topk > 0 ? (r.target < (double)nc ? (unsigned long long)r.target * unit : ~0ull)
+                               : !(tS < 9.0e18) ? ~0ull : (unsigned long long)llrint(tS);
         const unsigned long long diff = s_min ^ s_max;
         unsigned long long theta = s_min;          // one candidate (or all equal): keep all
         if (diff != 0ull) {
@@ -1759,7 +1779,8 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         __syncthreads();
         count = (int)(base0 + kbase);
         fin_theta = theta;
-        const double kept_mass = (double)s_kept / S * (double)ex2_sfu((Ub - r.R) * L2E);
+        const double kept_mass = a.topk > 0 ? (double)(s_kept / unit)
+                                            : (double)s_kept / S * (double)ex2_sfu((Ub - r.R) * L2E);
         mass = (float)((r.above + kept_mass) / r.Z);
     }
     // Rank 0's global writes go out last (a global store before a block or

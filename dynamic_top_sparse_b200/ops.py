@@ -40,7 +40,7 @@ OP_DECODE_STEP = 6
 OP_PREFILL = 7
 
 EXPORTS = ("rtp_workspace_size", "rtp_workspace_init", "rtp_check", "rtp_error_string",
-           "rtp_version", "rtp_append_index_keys", "rtp_index_scores", "rtp_topp_select",
+           "rtp_version", "rtp_append_index_keys", "rtp_index_scores", "rtp_topp_select", "rtp_topk_select",
            "rtp_sparse_decode", "rtp_local_decode", "rtp_dense_decode", "rtp_decode_step",
            "rtp_prof_init", "rtp_prof_elapsed", "rtp_prof_destroy", "rtp_dense_decode_noalloc",
            "rtp_selftest_wait_timeout", "rtp_prefill_attention")
@@ -66,7 +66,7 @@ class Prof(ctypes.Structure):
 class Opts(ctypes.Structure):
     _fields_ = [("idx_scale", ctypes.c_float), ("attn_scale", ctypes.c_float),
                 ("sel_idx", ctypes.c_void_p), ("sel_count", ctypes.c_void_p),
-                ("sel_mass", ctypes.c_void_p), ("prof", ctypes.POINTER(Prof))]
+                ("sel_mass", ctypes.c_void_p), ("prof", ctypes.POINTER(Prof)), ("topk", ctypes.c_int32)]
 
 
 _lib = None
@@ -83,6 +83,8 @@ _SIGS = {
     "rtp_index_scores": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Opts), _P, _P, _P, _P, _P,
                                         _P, ctypes.c_size_t, _P]),
     "rtp_topp_select": (ctypes.c_int, [ctypes.POINTER(Dims), _P, _P, ctypes.c_float, _P, _P, _P, _P,
+                                       ctypes.c_size_t, _P]),
+    "rtp_topk_select": (ctypes.c_int, [ctypes.POINTER(Dims), _P, _P, ctypes.c_int32, _P, _P, _P,
                                        ctypes.c_size_t, _P]),
     "rtp_sparse_decode": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Opts), _P, _P, _P, _P, _P,
                                          _P, _P, _P, ctypes.c_size_t, _P]),
@@ -225,8 +227,8 @@ class Profiler:
 
 
 def make_opts(idx_scale=0.0, attn_scale=0.0, sel_idx=None, sel_count=None, sel_mass=None,
-              prof: Profiler | None = None) -> Opts:
-    o = Opts(idx_scale, attn_scale, _ptr(sel_idx), _ptr(sel_count), _ptr(sel_mass), None)
+              prof: Profiler | None = None, topk: int = 0) -> Opts:
+    o = Opts(idx_scale, attn_scale, _ptr(sel_idx), _ptr(sel_count), _ptr(sel_mass), None, int(topk))
     if prof is not None:
         o.prof = ctypes.pointer(prof.p)
     return o
@@ -252,6 +254,11 @@ def topp_select(dims: Dims, z, head_class, p: float, idx_out, count_out, mass_ou
     _ck(lib().rtp_topp_select(ctypes.byref(dims), _ptr(z), _hc(head_class), float(p), _ptr(idx_out),
                               _ptr(count_out), _ptr(mass_out), ws.ptr, ws.nbytes, _stream()),
         "rtp_topp_select")
+
+
+def topk_select(dims: Dims, z, head_class, k: int, idx_out, count_out, ws: Workspace):
+    _ck(lib().rtp_topk_select(ctypes.byref(dims), _ptr(z), _hc(head_class), int(k), _ptr(idx_out),
+                              _ptr(count_out), ws.ptr, ws.nbytes, _stream()), "rtp_topk_select")
 
 
 def sparse_decode(dims: Dims, q_rope, k_cache, v_cache, idx, count, head_class, out, ws: Workspace,

@@ -145,8 +145,15 @@ typedef struct rtp_opts {
                                  retrieval head, first sel_count entries,
                                  order unspecified                          */
     int32_t *sel_count;       /* [B, H_q]: |S_h| (retrieval heads only)      */
-    float *sel_mass;          /* [B, H_q]: index-softmax mass of S_h         */
+    float *sel_mass;          /* [B, H_q]: index-softmax mass of S_h (with
+                                 topk: the kept fraction of the N_b tokens) */
     rtp_prof *prof;           /* optional launch accounting                 */
+    /* rtp_decode_step only: > 0 selects static top-k instead of top-p for
+     * the retrieval heads (Method section 3 sets the dynamic top-p rule
+     * against this fixed budget): each head keeps its topk tokens of
+     * largest index logit (equal logits: lower index first), all N_b when
+     * topk >= N_b; p is then not used.  0: top-p. */
+    int32_t topk;
 } rtp_opts;
 
 /* Workspace bytes `op` needs for these shapes (0 on invalid dims).  The
@@ -216,6 +223,25 @@ RTP_API int rtp_index_scores(const rtp_dims *dims, const rtp_opts *opts, const f
 RTP_API int rtp_topp_select(const rtp_dims *dims, const float *z, const uint8_t *head_class,
                     float p, int32_t *idx_out, int32_t *count_out, float *mass_out,
                     void *ws, size_t ws_bytes, rtp_stream_t stream);
+
+/*
+ * Static top-k selection from given logits (gist.science technical summary,
+ * Method section 3: the fixed budget that the dynamic top-p rule is set
+ * against): for each retrieval head the k tokens of largest z (equal z:
+ * lower index first), or all N_b tokens when k >= N_b.
+ *   z         [B, H_q, N_max] fp32 logits (local heads' rows not read)
+ *   idx_out   [B, H_q, N_max] int32: the set in the first count entries,
+ *             any order
+ *   count_out [B, H_q] int32: min(k, N_b)
+ * k < 1 is RTP_ERR_INVALID_ARG; logits out of the binned range or not
+ * finite as for rtp_topp_select.  Workspace: the size rtp_topp_select needs
+ * (RTP_OP_TOPP_SELECT).  The same level-1 histogram and boundary-bin radix
+ * select as top-p, with every token counting one unit instead of its mass,
+ * so the kept set is exact.
+ */
+RTP_API int rtp_topk_select(const rtp_dims *dims, const float *z, const uint8_t *head_class, int32_t k,
+                            int32_t *idx_out, int32_t *count_out, void *ws, size_t ws_bytes,
+                            rtp_stream_t stream);
 
 /*
  * a6 -- sparse decode (Method section 5): exact softmax attention of each

@@ -136,6 +136,13 @@ def test_other_calls_reject_bad_arguments(L):
                                    None) == ops.RTP_ERR_INVALID_ARG
     assert L.rtp_append_index_keys(ctypes.byref(d), FAKE, 70000, FAKE, FAKE, hc, FAKE, FAKE, big,
                                    None) == ops.RTP_ERR_INVALID_ARG
+    for kk in (0, -5):
+        assert L.rtp_topk_select(ctypes.byref(d), FAKE, hc, kk, FAKE, FAKE, FAKE, big,
+                                 None) == ops.RTP_ERR_INVALID_ARG
+    assert L.rtp_topk_select(ctypes.byref(d), None, hc, 8, FAKE, FAKE, FAKE, big, None) == ops.RTP_ERR_INVALID_ARG
+    assert L.rtp_topk_select(ctypes.byref(d), FAKE + 4, hc, 8, FAKE, FAKE, FAKE, big,
+                             None) == ops.RTP_ERR_INVALID_ARG
+    assert L.rtp_topk_select(ctypes.byref(d), FAKE, hc, 8, FAKE, FAKE, FAKE, 100, None) == ops.RTP_ERR_WORKSPACE
     # prefill: prompt length, window, cache type, workspace
     pf = L.rtp_prefill_attention
     assert pf(ctypes.byref(d), None, FAKE, 0, FAKE, FAKE, FAKE, hc, 16, 4, FAKE, FAKE, big,
