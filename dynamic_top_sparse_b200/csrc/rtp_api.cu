@@ -224,6 +224,8 @@ void plan_chunks(SelArgs &a, long long N_max) {
     long long ctas = (2LL * num_sms() + groups - 1) / groups;
     const long long tiles = (N_max + TILE - 1) / TILE;
     ctas = std::max(1LL, std::min({ctas, tiles, (long long)SCAN_CTAS_MAX}));
+    // at most MAX_CTA_TOKENS tokens per CTA (its 64-bit wide-bin sums cannot wrap)
+    ctas = std::max(ctas, (tiles * TILE + MAX_CTA_TOKENS - 1) / MAX_CTA_TOKENS);
     long long chunk = (tiles + ctas - 1) / ctas * TILE;
     ctas = (N_max + chunk - 1) / chunk;
     a.ctas = (int)ctas;
@@ -293,6 +295,7 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sm
     const long long tiles = (d->N_max + TILE - 1) / TILE;
     const long long sms = std::max(1LL, (long long)num_sms() - std::max(0, reserve_sms));
     long long ctas = std::max(1LL, std::min(sms / std::max(groups, 1LL), tiles));
+    ctas = std::max(ctas, (tiles * TILE + MAX_CTA_TOKENS - 1) / MAX_CTA_TOKENS);
     s.a.chunk = (tiles + ctas - 1) / ctas * TILE;
     s.a.ctas = (int)((d->N_max + s.a.chunk - 1) / s.a.chunk);
     // collect: the groups in pairs, one CTA per SM, the pair's tiles dealt
@@ -390,7 +393,7 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
 int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
                 const int32_t *lists, const int32_t *counts, const uint8_t *hc, float *out,
                 char *ws, const Layout &L, float attn_scale, int phase = LIST_ALL,
-                const int32_t *first = nullptr) {
+                const int32_t *first = nullptr, const uint32_t *spill = nullptr) {
     static int attr_set[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
@@ -413,6 +416,7 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
     a.scale_log2 = attn_scale * L2E;
     a.q = q; a.k = k; a.v = v; a.lists = lists; a.counts = counts; a.out = out;
     a.first = first;
+    a.spill = spill;
     a.phase = phase;
     a.part = reinterpret_cast<float *>(ws + L.part_list);
     a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_list);
@@ -421,7 +425,8 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
         std::min<long long>(LIST_MAX_SPLIT, (d->N_max + LCH - 1) / LCH);
     const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(max_items, 2LL * num_sms()));
     const size_t smem = list_smem_bytes(d->B * a.n_rq, d->B);
-    const char *name = phase == LIST_FIRST ? "sparse_attn_first" : "sparse_attn";
+    const char *name = phase == LIST_FIRST ? "sparse_attn_first" : phase == LIST_SPILL ? "sparse_attn_spill"
+                                                                                       : "sparse_attn";
     if (d->kv_dtype == RTP_BF16)
         return ln.run_smem(name, list_attn_kernel<__nv_bfloat16>, dim3(grid), dim3(ATT_THREADS), smem, a);
     return ln.run_smem(name, list_attn_kernel<float>, dim3(grid), dim3(ATT_THREADS), smem, a);
@@ -846,7 +851,22 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
                 s.a.out = out;
                 s.a.part_sel = reinterpret_cast<float *>(w + L.part_sel);
                 s.a.ovf = reinterpret_cast<uint32_t *>(w + L.ovf);
+                // heads that keep many rows beyond what the collect pass
+                // attended are finished by a list pass over every SM (a
+                // 4-CTA cluster per head would take long over them); it is
+                // needed only when a head can keep more than FIN_SPILL rows
+                const bool can_spill = dims->N_max > FIN_SPILL;
+                s.a.spill_rows = can_spill ? FIN_SPILL : 0;
+                s.a.part_list = reinterpret_cast<float *>(w + L.part_list);
                 rc = select_from_index(ln, dims, s, local_ctas);
+                if (rc == RTP_OK && can_spill) {
+                    const bool pdl0 = ln.pdl;
+                    ln.pdl = true;
+                    rc = launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out,
+                                     w, L, asc, LIST_SPILL, reinterpret_cast<const int32_t *>(w + L.list_cnt),
+                                     s.a.ovf);
+                    ln.pdl = pdl0;
+                }
                 if (side && cudaStreamWaitEvent(main, side->join, 0) != cudaSuccess && rc == RTP_OK)
                     rc = RTP_ERR_CUDA;
                 return rc;

@@ -261,7 +261,11 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
 // rest): LIST_FIRST writes partials only; LIST_REST adds the remaining rows
 // and merges everything.  Partials live in per-head slots: the first pass
 // uses slots [0, it_first), the second [it_first, it_first + it_rest).
-enum ListPhase : int32_t { LIST_ALL = 0, LIST_FIRST = 1, LIST_REST = 2 };
+// LIST_SPILL finishes the heads that the fused step's finalize handed over
+// (their kept rows were too many for its cluster to attend quickly): flag
+// spill[bh] = 2 (the rows from first[bh] on) or 3 (every row), finalize's
+// partial in slot 0; heads without a flag are left alone.
+enum ListPhase : int32_t { LIST_ALL = 0, LIST_FIRST = 1, LIST_REST = 2, LIST_SPILL = 3 };
 
 struct ListArgs {
     int B, H_q, H_kv, G;
@@ -278,6 +282,7 @@ struct ListArgs {
     // [B*H_q] at stride CNT_STRIDE: rows of the collect pass (LIST_FIRST,
     // LIST_REST), or null
     const int32_t *first;
+    const uint32_t *spill;       // [B*H_q] hand-over flags (LIST_SPILL)
     int phase;
     float *out;
     float *part;                 // [B*H_q][LIST_SLOTS][PSTRIDE]
@@ -335,6 +340,16 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
                 } else if (a.phase == LIST_FIRST) {
                     const int nf = (int)__ldcg(a.first + bh * CNT_STRIDE);
                     if (okN && nf >= 1 && nf <= N) { rows = nf; it = list_items(nf); }
+                } else if (a.phase == LIST_SPILL) {
+                    const uint32_t fl = __ldcg(a.spill + bh);
+                    const int cnt = fl >= SPILL_FROM_FIRST ? __ldcg(a.counts + bh) : 0;
+                    const int nf = fl == SPILL_FROM_FIRST ? __ldcg(a.first + bh * CNT_STRIDE) : 0;
+                    if (okN && fl >= SPILL_FROM_FIRST && cnt >= 1 && cnt <= N && nf >= 0 && nf <= cnt) {
+                        row0 = nf;
+                        rows = cnt - nf;
+                        slot0 = 1;                                   // finalize's partial
+                        it = max(1, list_items(rows));
+                    }
                 } else {
                     const int cnt = __ldcg(a.counts + bh);
                     const int nf = __ldcg(a.first + bh * CNT_STRIDE);
@@ -385,6 +400,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
         for (int hi = warp; hi < nh; hi += ATT_THREADS / 32) {
             if (pre[hi + 1] != pre[hi]) continue;
             const int b = hi / a.n_rq, h = a.ret_h[hi % a.n_rq];
+            if (a.phase == LIST_SPILL && __ldcg(a.spill + (size_t)b * a.H_q + h) < SPILL_FROM_FIRST) continue;
             float *o = a.out + ((size_t)b * a.H_q + h) * D + lane * 4;
             o[0] = o[1] = o[2] = o[3] = 0.0f;
             if (lane == 0) set_status(a.status, RTP_ERR_DEVICE_ARG);

@@ -160,6 +160,9 @@ __device__ __forceinline__ float warp_max(float v) {
 constexpr int LCH = 64;
 constexpr int LIST_MAX_SPLIT = 64;
 constexpr int LIST_SLOTS = 2 * LIST_MAX_SPLIT;   // partial record slots per head
+// Flags by which the fused step's finalize hands a head's remaining rows to
+// a list pass: the rows from the collect pass's count on, or every row.
+constexpr uint32_t SPILL_FROM_FIRST = 2u, SPILL_ALL_ROWS = 3u;
 __device__ __forceinline__ int list_items(int count) {
     if (count <= 0) return 0;
     return min(LIST_MAX_SPLIT, (count + LCH - 1) / LCH);

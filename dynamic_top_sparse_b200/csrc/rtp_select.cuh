@@ -158,6 +158,35 @@ __device__ __forceinline__ double fixed_to_double(unsigned long long v, double u
     return fma(__longlong_as_double((long long)(0x4330000000000000ull | v)), unit, -4503599627370496.0 * unit);
 }
 
+// The same for a 64-bit fixed-point sum: its two 32-bit halves, each exact,
+// added with one rounding.
+__device__ __forceinline__ double wide_fixed_to_double(unsigned long long v, double unit) {
+    return fixed_to_double(v >> 32, 4294967296.0 * unit) + fixed_to_double(v & 0xffffffffull, unit);
+}
+
+// Wide bins.  A bin spans 1/16 of an octave of |z|, so from |z| = 32 on it is
+// 2 to 8 nats wide and a value near its bottom weighs e^-8 of its upper
+// edge: at 2^18 or 2^20 units per unit of mass such a term keeps only a
+// few bits.  The scans add the values of these bins (k in [K_WIDE, K_TOP],
+// |z| in [32, 256), both signs: NWIDE bins per head) to separate 64-bit
+// counters at 2^38 units per unit of mass instead: an fp32 term times 2^38
+// converts exactly, so every term keeps fp32's relative precision, and the
+// sums stay below 2^64 for up to 2^25 values of one bin in one CTA.
+constexpr int K_WIDE = (int)((127 + 5) << MB) - (int)BIN_BASE;      // |z| >= 32
+constexpr int K_TOP = (int)((127 + 7) << MB) + 15 - (int)BIN_BASE;  // |z| < 256
+constexpr int NWK = K_TOP - K_WIDE + 1;                            // wide k values per sign
+constexpr int NWIDE = 2 * NWK;
+constexpr float WIDE_Z = 32.0f;
+constexpr float FX38_EXP2 = 38.0f;
+constexpr double FX38_UNIT = 1.0 / 274877906944.0;                  // 2^-38
+constexpr long long MAX_CTA_TOKENS = 1ll << 24;                     // per scan CTA
+// slot of a bin among the head's wide counters, or -1
+__host__ __device__ __forceinline__ int wide_slot(int bin) {
+    const int k = bin >= 256 ? bin - 256 : 255 - bin;
+    if (k < K_WIDE || k > K_TOP) return -1;
+    return (bin >= 256 ? 0 : NWK) + (k - K_WIDE);
+}
+
 // Adds a CTA's bin sums of G heads to the histograms (gh0: the first head's;
 // heads HSTRIDE apart).  bin_mass(i) = mass of entry i = head * NBIN + bin
 // relative to the bin's upper edge; fac = the octave factors; rep = the
@@ -236,6 +265,13 @@ struct SelArgs {
     float *out;                          // [B, H_q, D]
     float *part_sel;                     // [collect CTAs][2 GMAX][PSTRIDE] (pair-heads)
     uint32_t *ovf;                       // [B*H_q]
+    // Hand-over of large heads: a head whose rows left to finalize exceed
+    // spill_rows (> 0) is not attended by finalize's cluster; finalize
+    // stores its partial in slot 0 of the head's list partials (part_list)
+    // and flags the head in ovf (SPILL_FROM_FIRST / SPILL_ALL_ROWS) for a
+    // list pass over all SMs.
+    int spill_rows;
+    float *part_list;                    // [B*H_q][LIST_SLOTS][PSTRIDE]
 };
 
 // Record `r` of a cluster (the same shared variable in CTA rank r); the CTA's
@@ -661,6 +697,7 @@ __global__ void __launch_bounds__(SCAN_THREADS, 2) scan_kernel(SelArgs a, SelWs 
     __shared__ __align__(16) float qs[GMAX * R];
     __shared__ __align__(16) uint32_t shl[2 * GMAX * NBIN];   // fixed-point bin sums: low words, then high words
     uint32_t *const shh = shl + GMAX * NBIN;
+    __shared__ unsigned long long shw[GMAX * NWIDE];             // wide bins, 2^38 fixed point
     __shared__ double s_fac[NBIN];                               // octave factors
     __shared__ int s_err;
     const int b = blockIdx.y / a.n_ret;
@@ -677,7 +714,24 @@ __global__ void __launch_bounds__(SCAN_THREADS, 2) scan_kernel(SelArgs a, SelWs 
         if (a.ovf) a.ovf[bh0 + threadIdx.x] = 0u;
     }
     for (int i = threadIdx.x; i < 2 * GMAX * NBIN; i += blockDim.x) shl[i] = 0u;
+    for (int i = threadIdx.x; i < GMAX * NWIDE; i += blockDim.x) shw[i] = 0ull;
     for (int i = threadIdx.x; i < NBIN; i += blockDim.x) s_fac[i] = a.topk ? 1.0 : octave_factor(i);
+    // one value's mass into its head's bin counters
+    auto add_value = [&](int h, float zz) -> int {
+        uint32_t fx;
+        const int bin = bin_and_fx(zz, fx);
+        const int wsl = a.topk ? -1 : wide_slot(bin);
+        if (wsl >= 0) {
+            atomicAdd(&shw[h * NWIDE + wsl],
+                      (unsigned long long)__float2ull_rn(ex2_sfu(fmaf(zz - bin_upper(bin), L2E, FX38_EXP2))));
+            return bin;
+        }
+        if (a.topk) fx = (uint32_t)FX_ONE;
+        uint32_t *cell = &shl[h * NBIN + bin];
+        const uint32_t old = atomicAdd(cell, fx);
+        if (old + fx < old) atomicAdd(cell + GMAX * NBIN, 1u);
+        return bin;
+    };
     if constexpr (NeedsQ<Src>::value) {
         project_query<(GMAX * R + SCAN_WARPS - 1) / SCAN_WARPS>(a.q + bh0 * D, a.Wq + (size_t)g * G * R * D,
                                                                a.idx_scale, qs, G, warp, SCAN_WARPS);
@@ -714,12 +768,7 @@ __global__ void __launch_bounds__(SCAN_THREADS, 2) scan_kernel(SelArgs a, SelWs 
                 const int sl = src.slot(v);
                 const float zz = z[v] + 0.0f;      // folds -0 onto +0
                 err |= !(fabsf(zz) < Z_LIMIT);
-                uint32_t fx;
-                const int bin = bin_and_fx(zz, fx);
-                if (a.topk) fx = (uint32_t)FX_ONE;
-                uint32_t *cell = &shl[src.head(sl) * NBIN + bin];
-                const uint32_t old = atomicAdd(cell, fx);
-                if (old + fx < old) atomicAdd(cell + GMAX * NBIN, 1u);
+                const int bin = add_value(src.head(sl), zz);
                 tmax[sl] = max(tmax[sl], bin);
             }
         } else {
@@ -730,12 +779,7 @@ __global__ void __launch_bounds__(SCAN_THREADS, 2) scan_kernel(SelArgs a, SelWs 
                 if (h >= G || src.tok(v) >= nvalid) continue;
                 const float zz = z[v] + 0.0f;
                 if (!(fabsf(zz) < Z_LIMIT)) { err = 1; continue; }
-                uint32_t fx;
-                const int bin = bin_and_fx(zz, fx);
-                if (a.topk) fx = (uint32_t)FX_ONE;
-                uint32_t *cell = &shl[h * NBIN + bin];
-                const uint32_t old = atomicAdd(cell, fx);
-                if (old + fx < old) atomicAdd(cell + GMAX * NBIN, 1u);
+                const int bin = add_value(h, zz);
                 tmax[sl] = max(tmax[sl], bin);
             }
         }
@@ -756,7 +800,9 @@ __global__ void __launch_bounds__(SCAN_THREADS, 2) scan_kernel(SelArgs a, SelWs 
     __syncthreads();
     if (s_err && threadIdx.x == 0) set_status(w.status, RTP_ERR_RANGE);
     flush_hist(w.hist + bh0 * HSTRIDE, G, s_fac, blockIdx.x % NREP, [&](int i) {
-        return fixed_to_double(((unsigned long long)shh[i] << 32) | shl[i], 1.0 / FX_ONE);
+        const int wsl = wide_slot(i % NBIN);
+        const double m = fixed_to_double(((unsigned long long)shh[i] << 32) | shl[i], 1.0 / FX_ONE);
+        return wsl < 0 ? m : m + wide_fixed_to_double(shw[(i / NBIN) * NWIDE + wsl], FX38_UNIT);
     });
 }
 
@@ -779,7 +825,13 @@ constexpr int ST_BYTES = ST_TOK * R * 2;                 // bf16 index keys
 constexpr int NSTAGE = 3;
 constexpr int SPILL_STAGES = 10;                         // 15360 tokens
 constexpr float FX18 = 262144.0f;                        // 2^18
-constexpr int TC_SMEM = NSTAGE * ST_BYTES + GMAX * NBIN * 4 + GMAX * NBIN * 8 + 2 * NSTAGE * 8;
+// shared memory: the ring, the 32-bit and 64-bit bin sums, the wide bins'
+// 64-bit sums, then the ring's mbarriers
+constexpr int TC_OFF_H64 = NSTAGE * ST_BYTES + GMAX * NBIN * 4;
+constexpr int TC_OFF_HW = TC_OFF_H64 + GMAX * NBIN * 8;
+constexpr int TC_OFF_BAR = TC_OFF_HW + GMAX * NWIDE * 8;
+constexpr int TC_SMEM = TC_OFF_BAR + 2 * NSTAGE * 8;
+static_assert(TC_OFF_H64 % 8 == 0 && TC_OFF_HW % 8 == 0 && TC_OFF_BAR % 8 == 0, "8-byte aligned regions");
 // largest single add: 2^18 e^(2^-6) < 266240 (values of the k = 0 bins may
 // sit slightly above the bin's upper edge)
 static_assert((long long)SPILL_STAGES * ST_TOK * 266240LL < 4294967296LL, "bin counters would wrap");
@@ -790,6 +842,14 @@ static_assert((long long)SPILL_STAGES * ST_TOK * 266240LL < 4294967296LL, "bin c
 // (unclamped) k, whose maximum the caller checks once (k > KMAX_OK: z out
 // of range or not finite).  The clamped bin index is returned in `bin`.
 // CNT (static top-k): every value adds one unit, 2^18, instead of its mass.
+// The fixed-point value round(v) of v in [0, 2^22) is taken with one fp32 add
+// of 1.5 * 2^23 (the sum's unit in the last place is 1, so the add rounds v
+// to the nearest integer, ties to even, like a conversion instruction) and
+// one integer subtract of the sum's constant high bits, which keeps the
+// conversion off the pipe that also serves ex2.
+__device__ __forceinline__ uint32_t round_fx(float v) {
+    return __float_as_uint(v + 12582912.0f) - 0x4B400000u;
+}
 constexpr int KMAX_OK = (int)((127 + 7) << MB) + 15 - (int)BIN_BASE;   // |z| < 256
 constexpr uint32_t CNT_UNIT = 1u << 18;
 template <bool CNT>
@@ -799,9 +859,31 @@ __device__ __forceinline__ int scan_value(float z, uint32_t row, int &bin) {
     const int kr = (int)((u << 1) >> (24 - MB)) - (int)BIN_BASE;
     const int k = max(kr, 0) & 255;
     const uint32_t eb = ((uint32_t)(k + (int)BIN_BASE + 1 + s) << (23 - MB)) | (u & 0x80000000u);
-    const uint32_t fx = CNT ? CNT_UNIT : __float2uint_rn(ex2_sfu(fmaf(z - __uint_as_float(eb), L2E, 18.0f)));
+    const uint32_t fx = CNT ? CNT_UNIT : round_fx(ex2_sfu(fmaf(z - __uint_as_float(eb), L2E, 18.0f)));
     bin = 256 + (k ^ s);
     asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row + 4u * (uint32_t)bin), "r"(fx) : "memory");
+    return kr;
+}
+
+// scan_value for a tile that holds values of |z| >= 32: the values of the
+// wide bins go to their 64-bit counters at `wrow` (2^38 fixed point), the
+// others as in scan_value.
+__device__ __forceinline__ int scan_value_wide(float z, uint32_t row, uint32_t wrow, int &bin) {
+    const uint32_t u = __float_as_uint(z);
+    const int s = (int)u >> 31;                                          // 0 or -1
+    const int kr = (int)((u << 1) >> (24 - MB)) - (int)BIN_BASE;
+    const int k = max(kr, 0) & 255;
+    const uint32_t eb = ((uint32_t)(k + (int)BIN_BASE + 1 + s) << (23 - MB)) | (u & 0x80000000u);
+    const float d = z - __uint_as_float(eb);
+    bin = 256 + (k ^ s);
+    if (k >= K_WIDE && kr <= K_TOP) {
+        const unsigned long long fx = __float2ull_rn(ex2_sfu(fmaf(d, L2E, FX38_EXP2)));
+        const uint32_t slot = (uint32_t)((s ? NWK : 0) + (k - K_WIDE));
+        asm volatile("red.shared.add.u64 [%0], %1;" ::"r"(wrow + 8u * slot), "l"(fx) : "memory");
+    } else {
+        const uint32_t fx = round_fx(ex2_sfu(fmaf(d, L2E, 18.0f)));
+        asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row + 4u * (uint32_t)bin), "r"(fx) : "memory");
+    }
     return kr;
 }
 
@@ -849,8 +931,8 @@ __device__ __forceinline__ void scan_pair(float z0, float z1, uint32_t row0, uin
     bmax = max_u16x2(bmax, bin2);
     const uint32_t hu = (kc << 3) + (nm & 0x7ff87ff8u) + 0x00080008u;
     const float U0 = __uint_as_float(hu << 16), U1 = __uint_as_float(hu & 0xffff0000u);
-    const uint32_t fx0 = CNT ? CNT_UNIT : __float2uint_rn(ex2_sfu(fmaf(z0 - U0, L2E, 18.0f)));
-    const uint32_t fx1 = CNT ? CNT_UNIT : __float2uint_rn(ex2_sfu(fmaf(z1 - U1, L2E, 18.0f)));
+    const uint32_t fx0 = CNT ? CNT_UNIT : round_fx(ex2_sfu(fmaf(z0 - U0, L2E, 18.0f)));
+    const uint32_t fx1 = CNT ? CNT_UNIT : round_fx(ex2_sfu(fmaf(z1 - U1, L2E, 18.0f)));
     asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row0 + 4u * (bin2 & 0xffffu)), "r"(fx0) : "memory");
     asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(row1 + 4u * (bin2 >> 16)), "r"(fx1) : "memory");
 }
@@ -893,8 +975,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
     extern __shared__ __align__(128) uint8_t dsm[];
     uint8_t *ring = dsm;
     uint32_t *h32 = reinterpret_cast<uint32_t *>(dsm + NSTAGE * ST_BYTES);
-    unsigned long long *h64 = reinterpret_cast<unsigned long long *>(dsm + NSTAGE * ST_BYTES + GMAX * NBIN * 4);
-    uint64_t *full = reinterpret_cast<uint64_t *>(dsm + NSTAGE * ST_BYTES + GMAX * NBIN * 12);
+    unsigned long long *h64 = reinterpret_cast<unsigned long long *>(dsm + TC_OFF_H64);
+    unsigned long long *hw = reinterpret_cast<unsigned long long *>(dsm + TC_OFF_HW);
+    uint64_t *full = reinterpret_cast<uint64_t *>(dsm + TC_OFF_BAR);
     uint64_t *empty = full + NSTAGE;
     __shared__ __align__(16) float qs[GMAX * R];
     __shared__ double s_fac[NBIN];              // octave factors (the producer warp's idle lanes)
@@ -912,6 +995,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
         fence_mbar_init();
     }
     for (int i = threadIdx.x; i < GMAX * NBIN; i += blockDim.x) { h32[i] = 0u; h64[i] = 0ull; }
+    for (int i = threadIdx.x; i < GMAX * NWIDE; i += blockDim.x) hw[i] = 0ull;
     pdl_wait();
     pdl_trigger();
     // the consumers' q_idx loads go out before the producer's first bulk copy
@@ -954,6 +1038,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
         src.init(rows, a.N_max, qs, G);
         const int gid = lane >> 2, tig = lane & 3;
         const uint32_t hrow0 = smem_u32(h32 + (2 * tig) * NBIN), hrow1 = smem_u32(h32 + (2 * tig + 1) * NBIN);
+        const uint32_t hwrow0 = smem_u32(hw + (2 * tig) * NWIDE), hwrow1 = smem_u32(hw + (2 * tig + 1) * NWIDE);
         const bool full_group = G == GMAX;
         int kmax = 0;
         uint32_t amax = 0u;                // packed largest exponent bits per slot (scan_pair)
@@ -973,7 +1058,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
             // the lane's largest bin per head slot, both slots in one word:
             // (1 + max bin) per 16-bit half (0: no value)
             uint32_t pk;
-            if (nvalid >= TILE && full_group) {
+            // a tile with a value of |z| >= 32 (or not finite) anywhere in
+            // the warp takes the per-value path with the wide bins' counters
+            bool wide = false;
+            if constexpr (!CNT) {
+                float zm = 0.0f;
+#pragma unroll
+                for (int v = 0; v < SrcMma::NV; ++v) zm = fmaxf(zm, fabsf(z[v]));
+                wide = __any_sync(0xffffffffu, !(zm < WIDE_Z));
+            }
+            if (wide) {
+                int tmax[2] = {-1, -1};
+#pragma unroll
+                for (int v = 0; v < SrcMma::NV; ++v) {
+                    const int sl = v & 1;
+                    if (2 * tig + sl >= G || src.tok(v) >= nvalid) continue;
+                    int bin;
+                    kmax = max(kmax, scan_value_wide(z[v] + 0.0f, sl ? hrow1 : hrow0, sl ? hwrow1 : hwrow0, bin));
+                    tmax[sl] = max(tmax[sl], bin);
+                }
+                pk = (uint32_t)(tmax[0] + 1) | ((uint32_t)(tmax[1] + 1) << 16);
+            } else if (nvalid >= TILE && full_group) {
                 // value v is slot v & 1 of its token: pairs (v, v + 1)
                 uint32_t bmax = 0u;
 #pragma unroll
@@ -1044,7 +1149,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
     __syncthreads();
     if (s_err && threadIdx.x == 0) set_status(w.status, RTP_ERR_RANGE);
     flush_hist(w.hist + bh0 * HSTRIDE, G, s_fac, blockIdx.x % NREP,
-               [&](int i) { return fixed_to_double(h64[i] + h32[i], 1.0 / FX18); });
+               [&](int i) {
+                   const int wsl = wide_slot(i % NBIN);
+                   const double m = fixed_to_double(h64[i] + h32[i], 1.0 / FX18);
+                   return wsl < 0 ? m : m + wide_fixed_to_double(hw[(i / NBIN) * NWIDE + wsl], FX38_UNIT);
+               });
 }
 
 // ---------------------------------------------------------------------------
@@ -1521,6 +1630,7 @@ constexpr int FIN_WARPS = FIN_THREADS / 32;
 constexpr int FIN_CAP = 3072;             // candidates staged in shared memory
 constexpr int FIN_CLUSTER = 4;            // CTAs per head with the fused attention
 constexpr int FIN_FOLD = 3;               // collect records a warp loads at once
+constexpr int FIN_SPILL = 2048;           // rows above which finalize hands a head to the list pass
 // Exact selection inside the boundary bin.  One CTA per retrieval head, or
 // a cluster of FIN_CLUSTER CTAs per head with the fused attention (each
 // rank runs the same selection); grid = (1 or FIN_CLUSTER, B * n_ret * G).
@@ -1607,6 +1717,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         }
     }
     unsigned long long fin_theta = ~0ull;            // kept boundary candidates: key >= fin_theta
+    bool fin_staged = false;                         // the kept candidates' ids are compacted in s_kid
     const unsigned nc = r.mode == MODE_NORMAL ? nc_all : 0u;
     int32_t *lst = a.lists + bh * a.N_max;
     int count = 0;
@@ -1623,7 +1734,11 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         // Staged candidates: 32-bit fixed point, S = floor((2^31 - 1) / nc)
         // units per unit of mass (sums cannot wrap; with nc <= FIN_CAP each
         // mass keeps >= 19 bits).  Otherwise 64-bit, S = 2^62 / nc.
-        const bool staged = nc <= (unsigned)FIN_CAP;
+        // (a wide boundary bin -- |z| >= 32, terms down to e^-8 of its edge --
+        // always takes the 64-bit path: 32-bit units would leave such terms
+        // too few bits)
+        const bool staged = nc <= (unsigned)FIN_CAP && wide_slot(r.bstar) < 0;
+        fin_staged = staged;
         const double S = staged ? (double)(0x7fffffffu / nc) : ldexp(1.0, 62) / (double)nc;
         // static top-k: every candidate weighs one unit and the target is a
         // whole number of units (exact integers)
@@ -1787,16 +1902,18 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     // cluster barrier makes that barrier wait for it): count and mass, the
     // kept ids (every token for keep-all; the kept boundary candidates after
     // the collect pass's ids), and the cleared histogram for the next call.
+    bool spill = false;
     auto finish = [&]() {
         if (rank != 0) return;
         if (tid == 0) {
             a.count_out[bh] = count;
             if (a.mass_out) a.mass_out[bh] = mass;
+            if (spill) a.ovf[bh] = (ovf || r.mode == MODE_KEEP_ALL) ? SPILL_ALL_ROWS : SPILL_FROM_FIRST;
         }
         if (r.mode == MODE_KEEP_ALL) {
             for (int t = tid; t < r.N; t += blockDim.x) lst[t] = t;
         } else if (r.mode == MODE_NORMAL && nc > 0u) {
-            if (nc <= (unsigned)FIN_CAP) {
+            if (fin_staged) {
                 for (int i = tid; i < count - (int)base0; i += blockDim.x) lst[base0 + i] = s_kid[i];
             } else {
                 for (unsigned c = tid; c < nc; c += blockDim.x) {
@@ -1832,6 +1949,13 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     }
     if (ovf) part.reset();                           // a collect CTA could not attend all its kept rows
     {
+        // rows this cluster would attend: hand them over to the list pass
+        // when there are many (the same decision in every rank)
+        const long long att = (r.mode == MODE_KEEP_ALL ? (long long)count : (long long)count - base0) +
+                              (ovf ? (long long)base0 : 0LL);
+        spill = a.spill_rows > 0 && att > (long long)a.spill_rows;
+    }
+    if (!spill) {
         const size_t bg = (size_t)b * a.H_kv + (size_t)(h / G);
         const __nv_bfloat16 *kb = a.k_cache + bg * a.N_max * D;
         const __nv_bfloat16 *vb = a.v_cache + bg * a.N_max * D;
@@ -1851,7 +1975,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         } else if (r.mode == MODE_NORMAL) {
             // boundary-bin candidates at or above theta: the compacted ids
             // (staged), else eight candidate slots at a time
-            if (nc <= (unsigned)FIN_CAP) {
+            if (fin_staged) {
                 const int nk = count - (int)base0;
                 for (int rb = worker * 8; rb < nk; rb += workers * 8)
                     attend8(kb, vb, lane < 8 && rb + lane < nk ? s_kid[rb + lane] : -1, qx_f, part);
@@ -1907,7 +2031,14 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
                     O = fmaf(rc[POFF + d], wg, O);
                 }
             }
-            a.out[bh * D + d] = O * (L > 0.0f ? 1.0f / L : 0.0f);
+            if (spill) {
+                // the list pass adds the remaining rows and merges
+                float *pl = a.part_list + bh * (size_t)LIST_SLOTS * PSTRIDE;
+                pl[POFF + d] = O;
+                if (d == 0) { pl[0] = M; pl[1] = L; }
+            } else {
+                a.out[bh * D + d] = O * (L > 0.0f ? 1.0f / L : 0.0f);
+            }
         }
     }
     finish();

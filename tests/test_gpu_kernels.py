@@ -124,6 +124,33 @@ def test_topp_select(kind, N, p):
         assert abs(float(mass[0, h]) - float(sel.pi[ids].sum())) < 1e-5
 
 
+@pytest.mark.parametrize("lift", [40.0, 100.0, 200.0])
+@pytest.mark.parametrize("p", [0.5, 0.9, 0.99])
+def test_topp_select_large_logits(lift, p):
+    """Logits far from 0, where a level-1 bin spans several nats: peaked
+    heads shifted up by `lift` nats (the softmax is unchanged, the bins are
+    not) and a wide N(0, 40^2) spread.  The set rule and the mass within
+    1e-5 hold over the whole accepted range |z| < 256."""
+    H, N = 8, 4097
+    zs = [synth.random_logits(H, N, "peaked", seed=int(lift)) + lift,
+          np.clip(synth.random_logits(H, N, "wide", seed=int(lift)) * 5.0, -250.0, 250.0)]
+    for z in zs:
+        z = z.astype(np.float32)
+        seq = torch.tensor([N], dtype=torch.int32).cuda()
+        dims = _dims(1, H, 1, N, seq)
+        ws = ops.Workspace(dims)
+        idx = torch.full((1, H, N), -1, dtype=torch.int32, device="cuda")
+        cnt = torch.zeros((1, H), dtype=torch.int32, device="cuda")
+        mass = torch.zeros((1, H), dtype=torch.float32, device="cuda")
+        ops.topp_select(dims, torch.from_numpy(z).cuda().view(1, H, N), [1], p, idx, cnt, mass, ws)
+        assert ws.check() == 0
+        for h in range(H):
+            sel = oracle.topp_select(z[h].astype(np.float64), p)
+            ids = idx[0, h, : int(cnt[0, h])].cpu().numpy()
+            check_selection(ids, sel, p, f"lift={lift} p={p} h={h}")
+            assert abs(float(mass[0, h]) - float(sel.pi[ids].sum())) < 1e-5
+
+
 def test_topp_select_ragged_batch_and_reuse():
     """Ragged lengths across a batch, several heads per group, two calls on
     the same workspace give the same sets."""

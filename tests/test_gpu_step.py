@@ -137,6 +137,60 @@ def test_step_p_ge_one_mixed_heads(key):
     _p_ge_one_mixed(gc)
 
 
+@pytest.mark.parametrize("c_scale", [10.0, 25.0])
+def test_step_large_index_logits(c_scale):
+    """Index logits scaled by c_scale (idx_scale = c_scale / sqrt(d)): the
+    needles sit near 40-200 nats and the background spreads over +-10 nats,
+    where the level-1 bins are several nats wide."""
+    spec = synth.small_spec(B=2, H_q=16, H_kv=2, N=5000, head_class=(1, 0), seq_lens=[5000, 2500],
+                            needles_per_head=6, needle_scale=2.0)
+    gc = GpuCase(synth.make_case(spec))
+    gc.append_current()
+    isc = c_scale / math.sqrt(128)
+    for p in (0.5, 0.9, 0.999):
+        out, si, sc, sm = gc.step(p, idx_scale=isc)
+        c = gc.c
+        kidx = oracle_kidx(gc, "bf16", True)
+        q, qr = np64(c.q), np64(c.q_rope)
+        K, V, Wq = np32(c.k_cache), np32(c.v_cache), np64(c.W_q_idx)
+        tau = 1 / math.sqrt(128)
+        o = out.cpu().numpy()
+        for b in range(2):
+            N = int(c.seq_lens[b])
+            for h in range(8):                 # the retrieval group
+                z = oracle.index_logits(oracle.query_index(q[b, h], Wq[h]), kidx[b, 0, :N], isc)
+                assert np.max(np.abs(z)) > 32.0
+                sel = oracle.topp_select(z, p)
+                ids = gpu_set(si, sc, b, h)
+                _, mass = check_selection(ids, sel, p, f"c={c_scale} p={p} b={b} h={h}")
+                assert abs(float(sm[b, h]) - mass) < 1e-5
+                within(o[b, h], oracle.attend(qr[b, h], K[b, 0, :N], V[b, 0, :N], sel.kept, tau), OUT_TOL,
+                       f"c={c_scale} p={p} b={b} h={h}")
+
+
+@pytest.mark.parametrize("p", [0.3, 0.9])
+def test_step_flat_logits_hand_over(p):
+    """Every index key equal: all tokens share one logit, the boundary bin
+    holds every token and the kept set is the first ceil(p N) tokens by
+    index -- thousands of boundary rows, more than finalize attends itself,
+    so the list pass over every SM finishes those heads."""
+    spec = synth.small_spec(B=2, H_q=16, H_kv=2, N=19999, head_class=(1, 0), seq_lens=[19999, 7001],
+                            needles="none")
+    c = synth.make_case(spec)
+    c.kidx_cache[:, 0] = c.kidx_cache[:, 0, :1].clone()          # row 0's key everywhere
+    c.k_pre_new = c.k_pre_new.clone()
+    gc = GpuCase(c)
+    out, si, sc, sm = gc.step(p)                                 # no append: the current key stays equal
+    G = 8
+    for b in range(2):
+        N = int(c.seq_lens[b])
+        for h in range(G):
+            n = int(sc[b, h])
+            assert n == math.ceil(float(np.float32(p)) * N), (b, h, n)      # p N is 0.1 - 0.9 off an integer
+            assert sorted(gpu_set(si, sc, b, h).tolist()) == list(range(n))
+    _compare(gc, out, si, sc, sm, p, with_current=False)
+
+
 def test_step_repeatable_on_one_workspace():
     spec = synth.small_spec(B=2, H_q=16, H_kv=2, N=6000, head_class=(1, 0))
     gc = GpuCase(synth.make_case(spec))

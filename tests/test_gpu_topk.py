@@ -120,6 +120,9 @@ STEP = [
     (dict(B=1, H_q=32, H_kv=4, N=9000, head_class=(0, 1, 1, 0), window=256, n_sink=0), 1),
     (dict(B=2, H_q=8, H_kv=1, N=3000, head_class=(1,), seq_lens=[3000, 40]), 500),
     (dict(B=1, H_q=8, H_kv=2, N=2000, head_class=(1, 1), needles="none"), 2500),     # k > N: every token
+    # k > N with more rows than finalize attends itself: the list pass takes them
+    (dict(B=2, H_q=8, H_kv=1, N=6000, head_class=(1,), needles="none", seq_lens=[6000, 3000]), 10 ** 6),
+    (dict(B=1, H_q=8, H_kv=1, N=20000, head_class=(1,), needles="none"), 9000),
     (dict(B=2, H_q=4, H_kv=4, N=3000, head_class=(1, 0, 1, 0), kv_dtype="f32", idx_dtype="f32"), 300),
     (dict(B=2, H_q=16, H_kv=2, N=6000, head_class=(1, 0), kv_dtype="f32", idx_dtype="bf16"), 2048),
 ]
