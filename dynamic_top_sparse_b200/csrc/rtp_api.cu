@@ -432,6 +432,22 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
     return ln.run_smem(name, list_attn_kernel<float>, dim3(grid), dim3(ATT_THREADS), smem, a);
 }
 
+int launch_force(Launcher &ln, const rtp_dims *d, int32_t *lists, int32_t *counts, const uint8_t *hc, int window,
+                 int n_sink, char *ws, const Layout &L) {
+    ForceArgs a{};
+    a.B = d->B; a.H_q = d->H_q; a.G = d->H_q / d->H_kv;
+    a.N_max = d->N_max; a.seq_lens = d->seq_lens;
+    a.n_rq = 0;
+    for (int h = 0; h < d->H_q; ++h)
+        if (hc[h / a.G] == RTP_HEAD_RETRIEVAL) a.ret_h[a.n_rq++] = h;
+    if (a.n_rq == 0) return RTP_OK;
+    a.window = window; a.n_sink = n_sink;
+    a.lists = lists; a.counts = counts;
+    a.status = reinterpret_cast<uint32_t *>(ws + L.status);
+    const size_t smem = fr_smem_bytes(std::min<long long>(d->N_max, (long long)window + n_sink));
+    return ln.run_smem("force_rows", force_rows_kernel, dim3((unsigned)(d->B * a.n_rq)), dim3(FR_THREADS), smem, a);
+}
+
 }  // namespace
 
 // Scratch of rtp_dense_decode_noalloc: one fixed array per device, so
@@ -793,6 +809,9 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
     // neither waits for the other's CTAs to drain.
     const int topk = opts ? opts->topk : 0;
     if (topk < 0) return RTP_ERR_INVALID_ARG;
+    const bool force_local = opts && opts->force_local;
+    if (force_local && std::min<long long>(dims->N_max, (long long)window + n_sink) > FR_MAX_ROWS)
+        return RTP_ERR_UNSUPPORTED;
     const bool selecting = s.a.n_ret > 0 && (topk > 0 || p < 1.0f);
     int local_ctas = 0;
     if (any_local && s.a.n_ret > 0) {
@@ -841,7 +860,20 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
             s.a.lists = opts && opts->sel_idx ? opts->sel_idx : reinterpret_cast<int32_t *>(w + L.lists);
             s.a.count_out = opts && opts->sel_count ? opts->sel_count : reinterpret_cast<int32_t *>(w + L.counts);
             s.a.mass_out = opts ? opts->sel_mass : nullptr;
-            const bool fused = dims->kv_dtype == RTP_BF16 && dims->idx_dtype == RTP_BF16;
+            const bool fused = dims->kv_dtype == RTP_BF16 && dims->idx_dtype == RTP_BF16 && !force_local;
+            if (force_local) {
+                // selection alone, then each retrieval head's list united
+                // with the sink and window rows, then attention over the lists
+                s.a.ovf = nullptr;
+                rc = select_from_index(ln, dims, s, local_ctas);
+                if (rc == RTP_OK) rc = launch_force(ln, dims, s.a.lists, s.a.count_out, head_class, window, n_sink, w, L);
+                if (rc == RTP_OK)
+                    rc = launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out,
+                                     w, L, asc, LIST_ALL);
+                if (side && cudaStreamWaitEvent(main, side->join, 0) != cudaSuccess && rc == RTP_OK)
+                    rc = RTP_ERR_CUDA;
+                return rc;
+            }
             if (fused) {
                 // the sparse attention runs inside collect and finalize
                 s.a.q_rope = q_rope;

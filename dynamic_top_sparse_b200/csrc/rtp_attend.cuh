@@ -524,4 +524,62 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Forced local rows for retrieval heads: each retrieval head's kept list
+// S_h (the first counts[bh] entries) becomes S_h united with the sink and
+// window rows L of the sequence (the local heads' set).  One CTA per
+// retrieval head: a bitmap over L's rows in shared memory marks the kept
+// ids that fall in L, then the unmarked rows of L are appended.
+// grid = (B * n_rq), FR_THREADS threads, dynamic smem = fr_smem_bytes(L_max).
+// ---------------------------------------------------------------------------
+constexpr int FR_THREADS = 256;
+constexpr int FR_MAX_ROWS = 48 * 1024 * 8;       // |L| covered by the bitmap (48 KB)
+__host__ __device__ constexpr size_t fr_smem_bytes(long long rows) {
+    return (size_t)((rows + 31) / 32) * 4;
+}
+struct ForceArgs {
+    int B, H_q, G;
+    long long N_max;
+    const int32_t *seq_lens;
+    int n_rq;
+    int ret_h[MAX_RET_Q];
+    int window, n_sink;
+    int32_t *lists;              // [B*H_q*N_max]
+    int32_t *counts;             // [B*H_q]
+    uint32_t *status;
+};
+__global__ void __launch_bounds__(FR_THREADS) force_rows_kernel(ForceArgs a) {
+    extern __shared__ uint32_t fbm[];
+    __shared__ unsigned s_add;
+    pdl_wait();
+    pdl_trigger();
+    const int hi = blockIdx.x;
+    const int b = hi / a.n_rq, h = a.ret_h[hi % a.n_rq];
+    const size_t bh = (size_t)b * a.H_q + h;
+    const int N = a.seq_lens[b];
+    const int cnt = __ldcg(a.counts + bh);
+    if (N < 1 || (long long)N > a.N_max || cnt < 0 || cnt > N) return;     // reported by the step's kernels
+    const int s1 = min(a.n_sink, N);
+    const int w0 = max(s1, N - a.window);
+    const int nl = s1 + (N - w0);                                          // |L|
+    const int words = (nl + 31) / 32;
+    for (int i = threadIdx.x; i < words; i += blockDim.x) fbm[i] = 0u;
+    if (threadIdx.x == 0) s_add = 0u;
+    __syncthreads();
+    int32_t *lst = a.lists + bh * a.N_max;
+    for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+        const int t = __ldcg(lst + i);
+        const int li = t < s1 ? t : (t >= w0 && t < N ? s1 + (t - w0) : -1);
+        if (li >= 0) atomicOr(&fbm[li >> 5], 1u << (li & 31));
+    }
+    __syncthreads();
+    for (int li = threadIdx.x; li < nl; li += blockDim.x) {
+        if (fbm[li >> 5] & (1u << (li & 31))) continue;
+        const int t = li < s1 ? li : w0 + (li - s1);
+        lst[cnt + atomicAdd(&s_add, 1u)] = t;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) a.counts[bh] = cnt + (int)s_add;
+}
+
 }  // namespace rtp

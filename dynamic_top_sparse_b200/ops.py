@@ -66,7 +66,8 @@ class Prof(ctypes.Structure):
 class Opts(ctypes.Structure):
     _fields_ = [("idx_scale", ctypes.c_float), ("attn_scale", ctypes.c_float),
                 ("sel_idx", ctypes.c_void_p), ("sel_count", ctypes.c_void_p),
-                ("sel_mass", ctypes.c_void_p), ("prof", ctypes.POINTER(Prof)), ("topk", ctypes.c_int32)]
+                ("sel_mass", ctypes.c_void_p), ("prof", ctypes.POINTER(Prof)), ("topk", ctypes.c_int32),
+                ("force_local", ctypes.c_int32)]
 
 
 _lib = None
@@ -227,8 +228,9 @@ class Profiler:
 
 
 def make_opts(idx_scale=0.0, attn_scale=0.0, sel_idx=None, sel_count=None, sel_mass=None,
-              prof: Profiler | None = None, topk: int = 0) -> Opts:
-    o = Opts(idx_scale, attn_scale, _ptr(sel_idx), _ptr(sel_count), _ptr(sel_mass), None, int(topk))
+              prof: Profiler | None = None, topk: int = 0, force_local: bool = False) -> Opts:
+    o = Opts(idx_scale, attn_scale, _ptr(sel_idx), _ptr(sel_count), _ptr(sel_mass), None, int(topk),
+             1 if force_local else 0)
     if prof is not None:
         o.prof = ctypes.pointer(prof.p)
     return o

@@ -154,6 +154,14 @@ typedef struct rtp_opts {
      * largest index logit (equal logits: lower index first), all N_b when
      * topk >= N_b; p is then not used.  0: top-p. */
     int32_t topk;
+    /* rtp_decode_step only: nonzero unites each retrieval head's kept set
+     * with the local heads' rows (sinks [0, n_sink) and the window of the
+     * last `window` positions): S_h u L.  A serving option beside the
+     * method (Method section 1 keeps sinks and window for local heads only);
+     * the selection itself is unchanged.  sel_idx / sel_count then describe
+     * the union, sel_mass the selected set alone.  Needs
+     * min(N_max, window + n_sink) <= 393216, else RTP_ERR_UNSUPPORTED. */
+    int32_t force_local;
 } rtp_opts;
 
 /* Workspace bytes `op` needs for these shapes (0 on invalid dims).  The

@@ -269,7 +269,7 @@ class StepResult:
 def decode_step(q, q_rope, k_cache, v_cache, kidx_cache, W_q_idx, head_class,
                 seq_lens, p: float, window: int, n_sink: int,
                 idx_scale: float | None = None, attn_scale: float | None = None,
-                heads=None, topk: int | None = None) -> StepResult:
+                heads=None, topk: int | None = None, force_local: bool = False) -> StepResult:
     """One decode step of one layer.
 
     q: [B, H_q, d] pre-RoPE query (indexer input); q_rope: [B, H_q, d]
@@ -280,7 +280,10 @@ def decode_step(q, q_rope, k_cache, v_cache, kidx_cache, W_q_idx, head_class,
     Query head h belongs to KV head h // (H_q // H_kv).  Local heads attend
     over local_rows(); retrieval heads score every cached token with the
     indexer, keep the top-p set (or, with ``topk``, the top-k set; p is then
-    unused), and attend exactly over those rows.
+    unused), and attend exactly over those rows.  With ``force_local`` a
+    retrieval head attends over its kept set united with the local heads'
+    rows (a serving option beside the method: sinks and window kept for every
+    head).
     ``heads`` optionally restricts the computation to a list of (b, h).
     """
     q = np.asarray(q, np.float64)
@@ -304,6 +307,8 @@ def decode_step(q, q_rope, k_cache, v_cache, kidx_cache, W_q_idx, head_class,
             res.selections[(b, h)] = sel
             res.z[(b, h)] = z
             rows = sel.kept
+            if force_local:
+                rows = np.union1d(rows, local_rows(N, window, n_sink))
         else:
             rows = local_rows(N, window, n_sink)
         out[b, h] = attend(q_rope[b, h], K, V, rows, asc)

@@ -98,7 +98,8 @@ class GpuCase:
         pos = (self.seq - 1).to(torch.int32)
         ops.append_index_keys(self.dims, self.k_new, self.Wk, pos, self.hc, self.kidx, self.ws)
 
-    def step(self, p, window=None, n_sink=None, want_sel=True, out=None, topk=0, idx_scale=0.0):
+    def step(self, p, window=None, n_sink=None, want_sel=True, out=None, topk=0, idx_scale=0.0,
+             force_local=False):
         window = self.c.window if window is None else window
         n_sink = self.c.n_sink if n_sink is None else n_sink
         dev = self.q.device
@@ -108,7 +109,8 @@ class GpuCase:
             sel_idx = torch.full((self.B, self.H_q, self.N_max), -1, dtype=torch.int32, device=dev)
             sel_cnt = torch.zeros((self.B, self.H_q), dtype=torch.int32, device=dev)
             sel_mass = torch.zeros((self.B, self.H_q), dtype=torch.float32, device=dev)
-        opts = ops.make_opts(idx_scale=idx_scale, sel_idx=sel_idx, sel_count=sel_cnt, sel_mass=sel_mass, topk=topk)
+        opts = ops.make_opts(idx_scale=idx_scale, sel_idx=sel_idx, sel_count=sel_cnt, sel_mass=sel_mass, topk=topk,
+                             force_local=force_local)
         ops.decode_step(self.dims, self.q, self.q_rope, self.k, self.v, self.kidx, self.Wq, self.hc, p,
                         window, n_sink, out, self.ws, opts)
         st = self.ws.check()

@@ -107,6 +107,16 @@ def test_decode_step_rejects_bad_arguments(L):
     assert _step(L, ops, d, ws=0) == ops.RTP_ERR_WORKSPACE
     assert _step(L, ops, d, ws=FAKE + 128) == ops.RTP_ERR_WORKSPACE
     assert _step(L, ops, d, ws_bytes=1024) == ops.RTP_ERR_WORKSPACE
+    # options: a negative top-k budget; forced local rows beyond the bitmap's reach
+    opts = ops.Opts(0.0, 0.0, None, None, None, None, -1, 0)
+    arr = (ctypes.c_uint8 * 4)(1, 0, 0, 0)
+    ws_b = ops.workspace_size(d) or (1 << 40)
+    assert L.rtp_decode_step(ctypes.byref(d), ctypes.byref(opts), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, arr, 0.9,
+                             4096, 4, FAKE, FAKE, ws_b, None) == ops.RTP_ERR_INVALID_ARG
+    big = _dims(ops, N_max=1 << 20)
+    opts = ops.Opts(0.0, 0.0, None, None, None, None, 0, 1)
+    assert L.rtp_decode_step(ctypes.byref(big), ctypes.byref(opts), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, arr, 0.9,
+                             500000, 4, FAKE, FAKE, 1 << 40, None) == ops.RTP_ERR_UNSUPPORTED
     assert L.rtp_decode_step(None, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0.9, 1, 0, FAKE, FAKE,
                              1 << 40, None) == ops.RTP_ERR_INVALID_ARG
 

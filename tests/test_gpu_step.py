@@ -191,6 +191,64 @@ def test_step_flat_logits_hand_over(p):
     _compare(gc, out, si, sc, sm, p, with_current=False)
 
 
+FORCE = [
+    dict(B=2, H_q=16, H_kv=2, N=5000, head_class=(1, 0), seq_lens=[5000, 300], window=256, n_sink=4),
+    dict(B=1, H_q=32, H_kv=4, N=9000, head_class=(0, 1, 1, 0), window=1000, n_sink=0),
+    dict(B=2, H_q=8, H_kv=2, N=3000, head_class=(1, 1), kv_dtype="f32", idx_dtype="f32", window=64, n_sink=70),
+]
+
+
+def _check_forced(gc: GpuCase, p, out, si, sc, sm, heads=None):
+    c = gc.c
+    kidx = oracle_kidx(gc, c.spec.idx_dtype, True)
+    q = np64(c.q)
+    qr = q if c.q_rope is None else np64(c.q_rope)
+    K, V, Wq = np32(c.k_cache), np32(c.v_cache), np64(c.W_q_idx)
+    tau = 1 / math.sqrt(128)
+    G = gc.H_q // gc.H_kv
+    o = out.cpu().numpy()
+    todo = heads if heads is not None else [(b, h) for b in range(gc.B) for h in range(gc.H_q)]
+    for b, h in todo:
+        N = int(c.seq_lens[b])
+        g = h // G
+        loc = oracle.local_rows(N, c.window, c.n_sink)
+        if c.head_class[g] != oracle.HEAD_RETRIEVAL:
+            within(o[b, h], oracle.attend(qr[b, h], K[b, g, :N], V[b, g, :N], loc, tau), OUT_TOL, f"{b},{h}")
+            continue
+        z = oracle.index_logits(oracle.query_index(q[b, h], Wq[h]), kidx[b, g, :N], tau)
+        sel = oracle.topp_select(z, p)
+        ref_rows = np.union1d(sel.kept, loc)
+        ids = gpu_set(si, sc, b, h)
+        assert np.unique(ids).size == ids.size, f"{b},{h}: duplicate rows"
+        assert set(loc.tolist()) <= set(ids.tolist()), f"{b},{h}: a sink or window row is missing"
+        diff = set(ref_rows.tolist()) ^ set(ids.tolist())
+        amb = set(sel.ambiguous(p, 1e-5).tolist())
+        assert diff <= amb, f"{b},{h}: {len(diff - amb)} rows differ outside the mass window"
+        assert float(sm[b, h]) >= p - 1e-5
+        within(o[b, h], oracle.attend(qr[b, h], K[b, g, :N], V[b, g, :N], ref_rows, tau), OUT_TOL, f"{b},{h}")
+        within(o[b, h], oracle.attend(qr[b, h], K[b, g, :N], V[b, g, :N], ids, tau), OUT_TOL_SAME_SET,
+               f"{b},{h} (same rows)")
+
+
+@pytest.mark.parametrize("k", range(len(FORCE)))
+def test_step_force_local(k):
+    """force_local: each retrieval head attends over its top-p set united
+    with the sink and window rows."""
+    gc = GpuCase(synth.make_case(synth.small_spec(**FORCE[k], name=f"force{k}")))
+    gc.append_current()
+    for p in (0.5, 0.9):
+        out, si, sc, sm = gc.step(p, force_local=True)
+        _check_forced(gc, p, out, si, sc, sm)
+
+
+@pytest.mark.slow
+def test_step_force_local_ctx512k():
+    gc = GpuCase(synth.make_case("ctx512k", device="cuda"))
+    gc.append_current()
+    out, si, sc, sm = gc.step(0.9, force_local=True)
+    _check_forced(gc, 0.9, out, si, sc, sm)
+
+
 def test_step_repeatable_on_one_workspace():
     spec = synth.small_spec(B=2, H_q=16, H_kv=2, N=6000, head_class=(1, 0))
     gc = GpuCase(synth.make_case(spec))

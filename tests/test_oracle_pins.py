@@ -508,3 +508,28 @@ def test_prefill_first_position_returns_v0_and_wide_window_is_causal():
     np.testing.assert_allclose(ret, full, rtol=0, atol=1e-12)      # retrieval heads ignore window and sinks
     for h in range(q.shape[1]):
         np.testing.assert_array_equal(loc[0, h, 0], K[0, h // 2, 0] * 0 + V[0, h // 2, 0])
+
+
+def test_force_local_unites_kept_set_with_sinks_and_window():
+    """force_local: a retrieval head attends over its top-p set plus the
+    sink and window rows, each row once (checked against the explicit union
+    and an explicit mask)."""
+    g = np.random.default_rng(21)
+    B, H_q, H_kv, d, r, N = 1, 2, 1, 8, 4, 40
+    q = g.normal(0, 1, (B, H_q, d))
+    K = g.normal(0, 1, (B, H_kv, N, d))
+    V = g.normal(0, 1, (B, H_kv, N, d))
+    kidx = g.normal(0, 1, (B, H_kv, N, r))
+    W = g.normal(0, 1, (H_q, r, d))
+    hc = np.array([1], np.uint8)
+    for p in (1e-9, 0.5):
+        plain = oracle.decode_step(q, None, K, V, kidx, W, hc, [N], p, 5, 2)
+        forced = oracle.decode_step(q, None, K, V, kidx, W, hc, [N], p, 5, 2, force_local=True)
+        for h in range(H_q):
+            kept = set(plain.selections[(0, h)].kept.tolist())
+            rows = kept | {0, 1} | set(range(N - 5, N))
+            mask = np.array([t in rows for t in range(N)])
+            ref = _masked_dense_attention(q[0, h], K[0, 0], V[0, 0], mask, 1 / math.sqrt(d))
+            np.testing.assert_allclose(forced.out[0, h], ref, rtol=0, atol=1e-12)
+            if p == 1e-9:
+                assert len(kept) == 1
