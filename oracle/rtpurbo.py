@@ -139,8 +139,15 @@ def query_index(q_pre: np.ndarray, W_q_idx_h: np.ndarray) -> np.ndarray:
 
 
 def index_logits(q_idx: np.ndarray, kidx_rows: np.ndarray, scale: float) -> np.ndarray:
-    """z_t = scale * (q_idx . k_idx_t) for each cached row t ([N, r])."""
-    return scale * (np.asarray(kidx_rows, np.float64) @ np.asarray(q_idx, np.float64))
+    """z_t = scale * (q_idx . k_idx_t) for each cached row t ([N, r]).
+
+    Each row's dot product is summed the same way (an elementwise product
+    reduced along the row), so equal keys give exactly equal scores and the
+    tie rule decides between them; a blocked matrix-vector product may round
+    rows of different blocks differently."""
+    k = np.asarray(kidx_rows, np.float64)
+    q = np.asarray(q_idx, np.float64)
+    return scale * np.sum(k * q[None, :], axis=1)
 
 
 # ---------------------------------------------------------------------------

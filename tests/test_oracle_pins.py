@@ -533,3 +533,15 @@ def test_force_local_unites_kept_set_with_sinks_and_window():
             np.testing.assert_allclose(forced.out[0, h], ref, rtol=0, atol=1e-12)
             if p == 1e-9:
                 assert len(kept) == 1
+
+
+@pytest.mark.parametrize("N,p", [(19999, 0.3), (7001, 0.9), (40000, 0.50001)])
+def test_equal_index_keys_tie_and_keep_the_first_tokens(N, p):
+    """Every index key equal: the scores tie exactly (not merely to
+    rounding), so the kept set is the first ceil(p N) tokens by index."""
+    g = np.random.default_rng(N)
+    kidx = np.broadcast_to(g.normal(0, 1, 16), (N, 16)).copy()
+    q = g.normal(0, 1, 16)
+    z = oracle.index_logits(q, kidx, 1 / math.sqrt(128))
+    assert np.unique(z).size == 1
+    assert oracle.topp_select(z, p).kept.tolist() == list(range(math.ceil(p * N)))
