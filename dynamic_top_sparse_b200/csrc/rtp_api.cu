@@ -211,6 +211,34 @@ struct Launcher {
 
 float scale_or_default(float s) { return s > 0.0f ? s : 1.0f / std::sqrt((float)D); }
 
+// Paged K/V option: checked on the host, then turned into the kernels' row map.
+int check_kv(const rtp_dims *d, const rtp_opts *opts) {
+    const rtp_kv_pages *pg = opts ? opts->kv_pages : nullptr;
+    if (!pg) return RTP_OK;
+    if (!pg->block_table || ((uintptr_t)pg->block_table & 3u)) return RTP_ERR_INVALID_ARG;
+    const int ps = pg->page_size;
+    if (ps < 16 || ps > (1 << 20) || (ps & (ps - 1))) return RTP_ERR_INVALID_ARG;
+    if (pg->num_pages < 1 || pg->max_pages < 1) return RTP_ERR_INVALID_ARG;
+    if ((long long)pg->max_pages * ps < d->N_max) return RTP_ERR_INVALID_ARG;
+    return RTP_OK;
+}
+KvMap make_kv(const rtp_dims *d, const rtp_opts *opts, void *status) {
+    KvMap m{};
+    m.H_kv = d->H_kv;
+    m.N_max = d->N_max;
+    m.status = static_cast<uint32_t *>(status);
+    const rtp_kv_pages *pg = opts ? opts->kv_pages : nullptr;
+    if (pg) {
+        m.table = pg->block_table;
+        int sh = 0;
+        while ((1 << sh) < pg->page_size) ++sh;
+        m.page_shift = sh;
+        m.max_pages = pg->max_pages;
+        m.num_pages = pg->num_pages;
+    }
+    return m;
+}
+
 // ----------------------------------------------------------------- selection
 struct SelPlan {
     SelArgs a;
@@ -356,7 +384,7 @@ int side_stream(Side *&out, int slot = 0) {
 // ----------------------------------------------------------------- attention
 int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
                  const uint8_t *hc, int want_class, bool dense, int window, int n_sink, float *out,
-                 char *ws, const Layout &L, float attn_scale, int max_ctas = 0) {
+                 char *ws, const Layout &L, float attn_scale, int max_ctas = 0, const KvMap *kv = nullptr) {
     RangeArgs a{};
     a.B = d->B; a.H_q = d->H_q; a.H_kv = d->H_kv; a.G = d->H_q / d->H_kv;
     a.N_max = d->N_max; a.seq_lens = d->seq_lens;
@@ -383,6 +411,7 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
     a.part = reinterpret_cast<float *>(ws + L.part_range);
     a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_range);
     a.status = reinterpret_cast<uint32_t *>(ws + L.status);
+    a.kv = kv ? *kv : make_kv(d, nullptr, a.status);
     const dim3 grid((unsigned)a.n_split, (unsigned)(d->B * a.n_grp));
     const char *name = dense ? "dense_attn" : "local_attn";
     if (d->kv_dtype == RTP_BF16)
@@ -393,7 +422,7 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
 int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
                 const int32_t *lists, const int32_t *counts, const uint8_t *hc, float *out,
                 char *ws, const Layout &L, float attn_scale, int phase = LIST_ALL,
-                const int32_t *first = nullptr, const uint32_t *spill = nullptr) {
+                const int32_t *first = nullptr, const uint32_t *spill = nullptr, const KvMap *kv = nullptr) {
     static int attr_set[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
@@ -421,6 +450,7 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
     a.part = reinterpret_cast<float *>(ws + L.part_list);
     a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_list);
     a.status = reinterpret_cast<uint32_t *>(ws + L.status);
+    a.kv = kv ? *kv : make_kv(d, nullptr, a.status);
     const long long max_items = (long long)d->B * a.n_rq *
         std::min<long long>(LIST_MAX_SPLIT, (d->N_max + LCH - 1) / LCH);
     const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(max_items, 2LL * num_sms()));
@@ -656,10 +686,12 @@ int rtp_sparse_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q
         return RTP_ERR_INVALID_ARG;
     RTP_TRY(check_head_class(dims, head_class));
     RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_SPARSE_DECODE));
+    RTP_TRY(check_kv(dims, opts));
     const Layout L = make_layout(dims);
+    const KvMap kv = make_kv(dims, opts, (char *)ws + L.status);
     Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
     return launch_list(ln, dims, q_rope, k_cache, v_cache, idx, count, head_class, out, (char *)ws, L,
-                       scale_or_default(opts ? opts->attn_scale : 0.f));
+                       scale_or_default(opts ? opts->attn_scale : 0.f), LIST_ALL, nullptr, nullptr, &kv);
 }
 
 int rtp_local_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
@@ -673,10 +705,12 @@ int rtp_local_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_
         return RTP_ERR_INVALID_ARG;
     RTP_TRY(check_head_class(dims, head_class));
     RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_LOCAL_DECODE));
+    RTP_TRY(check_kv(dims, opts));
     const Layout L = make_layout(dims);
+    const KvMap kv = make_kv(dims, opts, (char *)ws + L.status);
     Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
     return launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
-                        n_sink, out, (char *)ws, L, scale_or_default(opts ? opts->attn_scale : 0.f));
+                        n_sink, out, (char *)ws, L, scale_or_default(opts ? opts->attn_scale : 0.f), 0, &kv);
 }
 
 int rtp_dense_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope,
@@ -687,10 +721,12 @@ int rtp_dense_decode(const rtp_dims *dims, const rtp_opts *opts, const float *q_
     if (!aligned16(q_rope) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return RTP_ERR_INVALID_ARG;
     RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_DENSE_DECODE));
+    RTP_TRY(check_kv(dims, opts));
     const Layout L = make_layout(dims);
+    const KvMap kv = make_kv(dims, opts, (char *)ws + L.status);
     Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
     return launch_range(ln, dims, q_rope, k_cache, v_cache, nullptr, -1, true, 1, 0, out, (char *)ws, L,
-                        scale_or_default(opts ? opts->attn_scale : 0.f));
+                        scale_or_default(opts ? opts->attn_scale : 0.f), 0, &kv);
 }
 
 int rtp_prefill_attention(const rtp_dims *dims, const rtp_opts *opts, const void *q, int32_t T,
@@ -705,6 +741,7 @@ int rtp_prefill_attention(const rtp_dims *dims, const rtp_opts *opts, const void
         return RTP_ERR_INVALID_ARG;
     RTP_TRY(check_head_class(dims, head_class));
     RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_PREFILL));
+    RTP_TRY(check_kv(dims, opts));
     static bool attr_set[64] = {false};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
@@ -729,6 +766,7 @@ int rtp_prefill_attention(const rtp_dims *dims, const rtp_opts *opts, const void
     a.v = static_cast<const __nv_bfloat16 *>(v_cache);
     a.out = out;
     a.status = reinterpret_cast<uint32_t *>(static_cast<char *>(ws));
+    a.kv = make_kv(dims, opts, a.status);
     if ((long long)a.n_qblk > 0x7fffffffLL) return RTP_ERR_UNSUPPORTED;
     Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
     return ln.run_smem("prefill_attn", prefill_attn_kernel, dim3((unsigned)a.n_qblk, (unsigned)(dims->B * dims->H_kv)),
@@ -742,6 +780,7 @@ int rtp_dense_decode_noalloc(const rtp_dims *dims, const rtp_opts *opts, const f
     if (!q_rope || !k_cache || !v_cache || !out) return RTP_ERR_INVALID_ARG;
     if (!aligned16(q_rope) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out))
         return RTP_ERR_INVALID_ARG;
+    RTP_TRY(check_kv(dims, opts));
     const long long groups = (long long)dims->B * dims->H_kv;
     if (groups > RTP_NOALLOC_MAX_GROUPS) return RTP_ERR_WORKSPACE;
     char *scr = nullptr;
@@ -768,6 +807,7 @@ int rtp_dense_decode_noalloc(const rtp_dims *dims, const rtp_opts *opts, const f
     a.part = reinterpret_cast<float *>(scr + NOALLOC_PART_OFF);
     a.arrive = reinterpret_cast<uint32_t *>(scr + NOALLOC_ARRIVE_OFF);
     a.status = reinterpret_cast<uint32_t *>(scr);
+    a.kv = make_kv(dims, opts, scr);
     Launcher ln{st, opts ? opts->prof : nullptr};
     const dim3 grid((unsigned)a.n_split, (unsigned)groups);
     if (dims->kv_dtype == RTP_BF16) {
@@ -793,8 +833,10 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
         return RTP_ERR_INVALID_ARG;
     RTP_TRY(check_head_class(dims, head_class));
     RTP_TRY(check_ws(dims, ws, ws_bytes, RTP_OP_DECODE_STEP));
+    RTP_TRY(check_kv(dims, opts));
     const Layout L = make_layout(dims);
     char *w = (char *)ws;
+    const KvMap kv = make_kv(dims, opts, w + L.status);
     Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
     const float asc = scale_or_default(opts ? opts->attn_scale : 0.f);
     const float isc = scale_or_default(opts ? opts->idx_scale : 0.f);
@@ -838,18 +880,18 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
         if (cudaStreamWaitEvent(side->st, side->fork, 0) != cudaSuccess) return RTP_ERR_CUDA;
         Launcher lside{side->st, ln.prof};
         RTP_TRY(launch_range(lside, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
-                             n_sink, out, w, L, asc, max_ctas));
+                             n_sink, out, w, L, asc, max_ctas, &kv));
         if (cudaEventRecord(side->join, side->st) != cudaSuccess) return RTP_ERR_CUDA;
     } else if (any_local) {
         RTP_TRY(launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window,
-                             n_sink, out, w, L, asc));
+                             n_sink, out, w, L, asc, 0, &kv));
     }
     int rc = RTP_OK;
     if (s.a.n_ret > 0) {
         if (!selecting) {
             // every token is kept: the retrieval heads' attention is dense
             rc = launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_RETRIEVAL, true, 1, 0,
-                              out, w, L, asc);
+                              out, w, L, asc, 0, &kv);
         } else {
             s.a.kidx = kidx_cache;
             s.a.q = q;
@@ -869,7 +911,7 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
                 if (rc == RTP_OK) rc = launch_force(ln, dims, s.a.lists, s.a.count_out, head_class, window, n_sink, w, L);
                 if (rc == RTP_OK)
                     rc = launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out,
-                                     w, L, asc, LIST_ALL);
+                                     w, L, asc, LIST_ALL, nullptr, nullptr, &kv);
                 if (side && cudaStreamWaitEvent(main, side->join, 0) != cudaSuccess && rc == RTP_OK)
                     rc = RTP_ERR_CUDA;
                 return rc;
@@ -879,6 +921,7 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
                 s.a.q_rope = q_rope;
                 s.a.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
                 s.a.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
+                s.a.kv = kv;
                 s.a.attn_scale_log2 = asc * L2E;
                 s.a.out = out;
                 s.a.part_sel = reinterpret_cast<float *>(w + L.part_sel);
@@ -896,7 +939,7 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
                     ln.pdl = true;
                     rc = launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out,
                                      w, L, asc, LIST_SPILL, reinterpret_cast<const int32_t *>(w + L.list_cnt),
-                                     s.a.ovf);
+                                     s.a.ovf, &kv);
                     ln.pdl = pdl0;
                 }
                 if (side && cudaStreamWaitEvent(main, side->join, 0) != cudaSuccess && rc == RTP_OK)
@@ -914,7 +957,7 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
                 if (cudaStreamWaitEvent(side2->st, side2->fork, 0) != cudaSuccess) return RTP_ERR_CUDA;
                 Launcher l2{side2->st, ln.prof};
                 RTP_TRY(launch_list(l2, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out,
-                                    w, L, asc, LIST_FIRST, first));
+                                    w, L, asc, LIST_FIRST, first, nullptr, &kv));
                 if (cudaEventRecord(side2->join, side2->st) != cudaSuccess) return RTP_ERR_CUDA;
                 return RTP_OK;
             };
@@ -922,7 +965,7 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
             if (side2 && cudaStreamWaitEvent(main, side2->join, 0) != cudaSuccess && rc == RTP_OK) rc = RTP_ERR_CUDA;
             if (rc == RTP_OK)
                 rc = launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, out,
-                                 w, L, asc, LIST_REST, first);
+                                 w, L, asc, LIST_REST, first, nullptr, &kv);
         }
     }
     if (side && cudaStreamWaitEvent(main, side->join, 0) != cudaSuccess && rc == RTP_OK) rc = RTP_ERR_CUDA;

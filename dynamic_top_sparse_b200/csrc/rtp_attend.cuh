@@ -92,6 +92,7 @@ struct RangeArgs {
     float *part;        // [B*H_kv][slots][GMAX][PSTRIDE]
     uint32_t *arrive;   // [B*H_kv]
     uint32_t *status;
+    KvMap kv;           // row addressing of k / v
 };
 
 template <typename KT>
@@ -131,8 +132,8 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
     if (tid < GMAX) { s_m[tid] = -INFINITY; s_l[tid] = 0.0f; }
     __syncthreads();
 
-    const KT *kb = reinterpret_cast<const KT *>(a.k) + bg * a.N_max * D;
-    const KT *vb = reinterpret_cast<const KT *>(a.v) + bg * a.N_max * D;
+    const KT *kc = reinterpret_cast<const KT *>(a.k);
+    const KT *vc = reinterpret_cast<const KT *>(a.v);
     float acc[GMAX][4];
 #pragma unroll
     for (int h = 0; h < GMAX; ++h)
@@ -146,9 +147,9 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
             float s[GMAX];
 #pragma unroll
             for (int h = 0; h < GMAX; ++h) s[h] = 0.0f;
-            if (j < hi) {
-                const long long row = j < s1 ? j : w0 + (j - s1);
-                const KT *kr = kb + row * D;
+            const long long kr_row = j < hi ? kv_row(a.kv, b, g, j < s1 ? j : w0 + (j - s1)) : -1LL;
+            if (kr_row >= 0) {
+                const KT *kr = kc + kr_row * D;
 #pragma unroll 4
                 for (int piece = 0; piece < D / 8; ++piece) {
                     float kx[8];
@@ -213,9 +214,9 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
 #pragma unroll 8
             for (int i = 0; i < nr; ++i) {
                 const long long j = rbase + i;
-                const long long row = j < s1 ? j : w0 + (j - s1);
-                float vx[4];
-                Row<KT>::load4(vb + row * D + lane * 4, vx);
+                const long long row = kv_row(a.kv, b, g, j < s1 ? j : w0 + (j - s1));
+                float vx[4] = {0.f, 0.f, 0.f, 0.f};
+                if (row >= 0) Row<KT>::load4(vc + row * D + lane * 4, vx);
 #pragma unroll
                 for (int h = 0; h < GMAX; ++h) {
                     if (h < G) {
@@ -288,6 +289,7 @@ struct ListArgs {
     float *part;                 // [B*H_q][LIST_SLOTS][PSTRIDE]
     uint32_t *arrive;            // [B*H_q]
     uint32_t *status;
+    KvMap kv;                    // row addressing of k / v
 };
 
 // Dynamic shared memory of list_attn_kernel: per head the item prefix, the
@@ -430,23 +432,25 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
         const float4 q4 = *reinterpret_cast<const float4 *>(a.q + bh * D + lane * 4);
         const float qx[4] = {q4.x * a.scale_log2, q4.y * a.scale_log2, q4.z * a.scale_log2,
                              q4.w * a.scale_log2};
-        const KT *kb = reinterpret_cast<const KT *>(a.k) + ((size_t)b * a.H_kv + g) * a.N_max * D;
-        const KT *vb = reinterpret_cast<const KT *>(a.v) + ((size_t)b * a.H_kv + g) * a.N_max * D;
+        const KT *kc = reinterpret_cast<const KT *>(a.k);
+        const KT *vc = reinterpret_cast<const KT *>(a.v);
         const int32_t *lst = a.lists + bh * a.N_max;
         float m = -INFINITY, l = 0.0f, o[4] = {0.f, 0.f, 0.f, 0.f};
         constexpr int U = 8;       // rows per warp per pass: all their K/V loads in flight
         for (int rb = r0 + warp * U; rb < r1; rb += (ATT_THREADS / 32) * U) {
             int myid = -1;
             if (lane < U && rb + lane < r1) myid = __ldcg(lst + rb + lane);
+            // lanes 0-7: the cache row of their token (-1: none or invalid)
+            const long long myrow = myid >= 0 && myid < N ? kv_row(a.kv, b, g, myid) : -1LL;
             float kx[U][4], vx[U][4];
             bool ok[U];
 #pragma unroll
             for (int u = 0; u < U; ++u) {
-                const int t = __shfl_sync(0xffffffffu, myid, u);
-                ok[u] = rb + u < r1 && t >= 0 && t < N;
+                const long long r = __shfl_sync(0xffffffffu, myrow, u);
+                ok[u] = rb + u < r1 && r >= 0;
                 if (ok[u]) {
-                    Row<KT>::load4(kb + (size_t)t * D + lane * 4, kx[u]);
-                    Row<KT>::load4(vb + (size_t)t * D + lane * 4, vx[u]);
+                    Row<KT>::load4(kc + r * D + lane * 4, kx[u]);
+                    Row<KT>::load4(vc + r * D + lane * 4, vx[u]);
                 } else {
 #pragma unroll
                     for (int i = 0; i < 4; ++i) kx[u][i] = vx[u][i] = 0.0f;

@@ -180,6 +180,30 @@ constexpr int PSTRIDE = D + 4;         // partial record: m, l, (2 unused), o[D]
 constexpr int POFF = 4;                // offset of o[] in a record (16-byte aligned)
 static_assert(PSTRIDE % 4 == 0 && POFF % 4 == 0, "partial records must keep o[] 16-byte aligned");
 
+// ---------------------------------------------------------------------------
+// K/V row addressing.  Contiguous caches hold token t of (sequence b, KV
+// head g) at row (b H_kv + g) N_max + t.  Paged caches (table != null) are
+// pools [num_pages][H_kv][page][D]: token t of sequence b lives in page
+// table[b max_pages + t / page] at slot t % page (page = 2^page_shift).  A
+// page number outside the pool is reported (RTP_ERR_DEVICE_ARG) and the row
+// reads as missing (-1).
+// ---------------------------------------------------------------------------
+struct KvMap {
+    const int32_t *table;
+    int page_shift, max_pages, num_pages;
+    int H_kv;
+    long long N_max;
+    uint32_t *status;
+};
+__device__ __forceinline__ long long kv_row(const KvMap &m, int b, int g, long long t) {
+    if (!m.table) return ((long long)b * m.H_kv + g) * m.N_max + t;
+    const long long j = t >> m.page_shift;
+    if (j >= m.max_pages) { set_status(m.status, RTP_ERR_DEVICE_ARG); return -1; }
+    const int pg = __ldg(m.table + (long long)b * m.max_pages + j);
+    if (pg < 0 || pg >= m.num_pages) { set_status(m.status, RTP_ERR_DEVICE_ARG); return -1; }
+    return (((long long)pg * m.H_kv + g) << m.page_shift) + (t & ((1LL << m.page_shift) - 1));
+}
+
 // Flash-decoding partial of one head over a set of rows.
 struct Partial {
     float m;        // max logit (-inf when empty)

@@ -101,11 +101,13 @@ __global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a
             qa[2][kk][0] = bf16x2(l[0], l[1]); qa[2][kk][1] = bf16x2(l[2], l[3]);
         }
     }
-    const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(a.k) + bg * a.N_max * D;
-    const __nv_bfloat16 *vb = reinterpret_cast<const __nv_bfloat16 *>(a.v) + bg * a.N_max * D;
+    const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(a.k);
+    const __nv_bfloat16 *vb = reinterpret_cast<const __nv_bfloat16 *>(a.v);
+    // cache row of range position j (past the end: a valid row, masked
+    // below; a page outside the pool is reported and read as row 0)
     auto row_of = [&](long long j) -> long long {
-        j = j < hi ? j : hi - 1;                  // past the end: reuse a valid row (masked below)
-        return j < s1 ? j : w0 + (j - s1);
+        j = j < hi ? j : hi - 1;
+        return max(0LL, kv_row(a.kv, b, g, j < s1 ? j : w0 + (j - s1)));
     };
 
     float m_run = -INFINITY, l_run = 0.0f;        // head gid (shared by the 4 lanes of gid)

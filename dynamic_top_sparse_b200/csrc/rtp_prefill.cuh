@@ -49,6 +49,7 @@ struct PrefillArgs {
     const __nv_bfloat16 *v;
     float *out;                  // [B, H_q, T, D]
     uint32_t *status;
+    KvMap kv;                    // row addressing of k / v
 };
 
 __device__ __forceinline__ void pf_cp_async16(void *dst, const void *src) {
@@ -114,7 +115,6 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_attn_kernel(PrefillArgs
     const int G = a.G;
     const int N = a.seq_lens[b];
     const int p0 = a.pos0[b];
-    const size_t bg = (size_t)b * a.H_kv + g;
     const int t_lo = qb * BQ;                                // first prompt token of the block
     const int t_hi = min(a.T, t_lo + BQ);                    // past the last
     const int hw = warp / a.nsub;                            // this warp's head within the group
@@ -134,8 +134,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_attn_kernel(PrefillArgs
     const TileRanges tr = prefill_tiles(P0, P1, local, a.window, a.n_sink);
     const int n_tiles = tr.count();
 
-    const __nv_bfloat16 *kb = a.k + bg * a.N_max * D;
-    const __nv_bfloat16 *vb = a.v + bg * a.N_max * D;
+
     // stage tile i: 64 rows of K then of V, 16 bytes per thread per copy;
     // rows past P1 repeat row P1 (finite; masked below)
     auto stage = [&](int i, int s) {
@@ -144,9 +143,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) prefill_attn_kernel(PrefillArgs
 #pragma unroll
         for (int c = tid; c < PF_BK * (D * 2 / 16); c += PF_THREADS) {
             const int r = c >> 4, piece = c & 15;
-            const long long row = min(key0 + r, P1);
-            pf_cp_async16(ks + r * PF_PITCH + piece * 16, kb + row * D + piece * 8);
-            pf_cp_async16(vs + r * PF_PITCH + piece * 16, vb + row * D + piece * 8);
+            const long long row = max(0LL, kv_row(a.kv, b, g, min(key0 + r, P1)));
+            pf_cp_async16(ks + r * PF_PITCH + piece * 16, a.k + row * D + piece * 8);
+            pf_cp_async16(vs + r * PF_PITCH + piece * 16, a.v + row * D + piece * 8);
         }
     };
     if (n_tiles > 0) stage(0, 0);

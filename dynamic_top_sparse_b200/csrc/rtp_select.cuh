@@ -259,8 +259,9 @@ struct SelArgs {
     // rows and merges.  A head whose kept rows overflowed a CTA's staging is
     // attended wholly by finalize (ovf flag).
     const float *q_rope;                 // [B, H_q, D]
-    const __nv_bfloat16 *k_cache;        // [B, H_kv, N_max, D]
+    const __nv_bfloat16 *k_cache;        // [B, H_kv, N_max, D], or page pools (kv)
     const __nv_bfloat16 *v_cache;
+    KvMap kv;                            // row addressing of k_cache / v_cache
     float attn_scale_log2;
     float *out;                          // [B, H_q, D]
     float *part_sel;                     // [collect CTAs][2 GMAX][PSTRIDE] (pair-heads)
@@ -329,18 +330,19 @@ __device__ __forceinline__ void prefetch_kv_l2(const __nv_bfloat16 *k_row, const
     asm volatile("prefetch.global.L2 [%0];" ::"l"(v_row + 64));
 }
 
-__device__ __forceinline__ void attend8(const __nv_bfloat16 *kb, const __nv_bfloat16 *vb, int id,
-                                        const float (&qx)[4], WarpPart &p) {
+__device__ __forceinline__ void attend8(const __nv_bfloat16 *kc, const __nv_bfloat16 *vc, const KvMap &km, int b,
+                                        int g, int id, const float (&qx)[4], WarpPart &p) {
     const int lane = threadIdx.x & 31;
     float kx[8][4], vx[8][4];
     bool ok[8];
+    const long long ro = id >= 0 ? kv_row(km, b, g, id) : -1LL;    // lanes 0-7: their token's row
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-        const int t = __shfl_sync(0xffffffffu, id, u);
-        ok[u] = t >= 0;
+        const long long r = __shfl_sync(0xffffffffu, ro, u);
+        ok[u] = r >= 0;
         if (ok[u]) {
-            Row<__nv_bfloat16>::load4(kb + (size_t)t * D + lane * 4, kx[u]);
-            Row<__nv_bfloat16>::load4(vb + (size_t)t * D + lane * 4, vx[u]);
+            Row<__nv_bfloat16>::load4(kc + r * D + lane * 4, kx[u]);
+            Row<__nv_bfloat16>::load4(vc + r * D + lane * 4, vx[u]);
         } else {
 #pragma unroll
             for (int i = 0; i < 4; ++i) kx[u][i] = vx[u][i] = 0.0f;
@@ -1512,8 +1514,8 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
                         // finalize attends the candidates it keeps: their rows
                         // start toward L2 now (there are few of them)
                         if (a.q_rope) {
-                            const size_t row = ((gk ? bg1 : bg0) * a.N_max + t) * D;
-                            prefetch_kv_l2(a.k_cache + row, a.v_cache + row);
+                            const long long row = kv_row(a.kv, gk ? b1 : b0, gk ? g1 : g0, t);
+                            if (row >= 0) prefetch_kv_l2(a.k_cache + row * D, a.v_cache + row * D);
                         }
                     }
                 }
@@ -1559,8 +1561,7 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
     // attention.  A head whose staging overflowed is left to finalize (ovf
     // flag, empty partial).
     if (lane == 0 && wok && s_kc[warp] > (unsigned)CL_KCAP) a.ovf[wbh] = 1u;
-    const __nv_bfloat16 *kc0 = a.k_cache + bg0 * a.N_max * D, *kc1 = a.k_cache + bg1 * a.N_max * D;
-    const __nv_bfloat16 *vc0 = a.v_cache + bg0 * a.N_max * D, *vc1 = a.v_cache + bg1 * a.N_max * D;
+
     const int nrow_l = lane < HP && ph_ok(lane) && s_kc[lane] <= (unsigned)CL_KCAP ? (int)s_kc[lane] : 0;
     for (int h_lo = 0; h_lo < HP;) {
         // lane h in [h_lo, HP): its chunks and slots, inclusive prefix sums
@@ -1598,7 +1599,8 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
             }
             const int r = (k - c0) * 8 + lane;
             const int id = lane < 8 && r < (int)s_kc[ph] ? s_kbuf[ph * CL_KCAP + r] : -1;
-            if (ph < GMAX) attend8(kc0, vc0, id, qx, part); else attend8(kc1, vc1, id, qx, part);
+            if (ph < GMAX) attend8(a.k_cache, a.v_cache, a.kv, b0, g0, id, qx, part);
+            else attend8(a.k_cache, a.v_cache, a.kv, b1, g1, id, qx, part);
         }
         if (cur >= 0) part.store(s_slot + (cur_s0 + kfirst - cur_c0) * PSTRIDE);
         __syncthreads();
@@ -1956,21 +1958,19 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         spill = a.spill_rows > 0 && att > (long long)a.spill_rows;
     }
     if (!spill) {
-        const size_t bg = (size_t)b * a.H_kv + (size_t)(h / G);
-        const __nv_bfloat16 *kb = a.k_cache + bg * a.N_max * D;
-        const __nv_bfloat16 *vb = a.v_cache + bg * a.N_max * D;
+        const int g = h / G;
         const int worker = rank * FIN_WARPS + warp, workers = K * FIN_WARPS;
         if (ovf) {
             // the collect pass's rows, from its list
             for (int rb = worker * 8; rb < (int)base0; rb += workers * 8) {
                 const int id = lane < 8 && rb + lane < (int)base0 ? __ldcg(lst + rb + lane) : -1;
-                attend8(kb, vb, id, qx_f, part);
+                attend8(a.k_cache, a.v_cache, a.kv, b, g, id, qx_f, part);
             }
         }
         if (r.mode == MODE_KEEP_ALL) {
             for (int rb = worker * 8; rb < count; rb += workers * 8) {
                 const int id = lane < 8 && rb + lane < count ? rb + lane : -1;
-                attend8(kb, vb, id, qx_f, part);
+                attend8(a.k_cache, a.v_cache, a.kv, b, g, id, qx_f, part);
             }
         } else if (r.mode == MODE_NORMAL) {
             // boundary-bin candidates at or above theta: the compacted ids
@@ -1978,7 +1978,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             if (fin_staged) {
                 const int nk = count - (int)base0;
                 for (int rb = worker * 8; rb < nk; rb += workers * 8)
-                    attend8(kb, vb, lane < 8 && rb + lane < nk ? s_kid[rb + lane] : -1, qx_f, part);
+                    attend8(a.k_cache, a.v_cache, a.kv, b, g, lane < 8 && rb + lane < nk ? s_kid[rb + lane] : -1, qx_f, part);
             } else {
                 for (int cb = worker * 8; cb < (int)nc; cb += workers * 8) {
                     int id = -1;
@@ -1986,7 +1986,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
                         const unsigned long long v = __ldcg(cg + cb + lane);
                         if (v >= fin_theta) id = (int)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
                     }
-                    attend8(kb, vb, id, qx_f, part);
+                    attend8(a.k_cache, a.v_cache, a.kv, b, g, id, qx_f, part);
                 }
             }
         }

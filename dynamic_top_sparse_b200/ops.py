@@ -63,11 +63,16 @@ class Prof(ctypes.Structure):
                 ("name", ctypes.POINTER(ctypes.c_char_p)), ("filter", ctypes.c_char_p)]
 
 
+class KvPages(ctypes.Structure):
+    _fields_ = [("block_table", ctypes.c_void_p), ("page_size", ctypes.c_int32), ("max_pages", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
 class Opts(ctypes.Structure):
     _fields_ = [("idx_scale", ctypes.c_float), ("attn_scale", ctypes.c_float),
                 ("sel_idx", ctypes.c_void_p), ("sel_count", ctypes.c_void_p),
                 ("sel_mass", ctypes.c_void_p), ("prof", ctypes.POINTER(Prof)), ("topk", ctypes.c_int32),
-                ("force_local", ctypes.c_int32)]
+                ("force_local", ctypes.c_int32), ("kv_pages", ctypes.POINTER(KvPages))]
 
 
 _lib = None
@@ -228,15 +233,28 @@ class Profiler:
 
 
 def make_opts(idx_scale=0.0, attn_scale=0.0, sel_idx=None, sel_count=None, sel_mass=None,
-              prof: Profiler | None = None, topk: int = 0, force_local: bool = False) -> Opts:
+              prof: Profiler | None = None, topk: int = 0, force_local: bool = False,
+              kv_pages: KvPages | None = None) -> Opts:
     o = Opts(idx_scale, attn_scale, _ptr(sel_idx), _ptr(sel_count), _ptr(sel_mass), None, int(topk),
-             1 if force_local else 0)
+             1 if force_local else 0, None)
+    if kv_pages is not None:
+        o.kv_pages = ctypes.pointer(kv_pages)
+        o._keep = kv_pages                     # the struct must outlive the options
     if prof is not None:
         o.prof = ctypes.pointer(prof.p)
     return o
 
 
 # ---------------------------------------------------------------- entry points
+
+def kv_pages(block_table, page_size: int, num_pages: int) -> KvPages:
+    """Paged K/V description: block_table [B, max_pages] int32 on the device."""
+    if block_table.dtype != torch.int32 or block_table.dim() != 2:
+        raise ValueError("block_table must be a 2-D int32 tensor")
+    pg = KvPages(_ptr(block_table), int(page_size), int(block_table.shape[1]), int(num_pages), 0)
+    pg._table = block_table                    # keep the table alive with the struct
+    return pg
+
 
 def append_index_keys(dims: Dims, k_pre, W_k_idx, pos, head_class, kidx_cache, ws: Workspace):
     T = k_pre.shape[2]

@@ -135,6 +135,24 @@ typedef struct rtp_prof {
     const char *filter;
 } rtp_prof;
 
+/* Paged K/V caches (a serving layout beside the method): k_cache and
+ * v_cache are pools of num_pages pages, each [H_kv, page_size, d] in the
+ * cache dtype (pool layout [num_pages, H_kv, page_size, d]); token t of
+ * sequence b sits in page block_table[b * max_pages + t / page_size] at slot
+ * t % page_size.  block_table is a DEVICE int32 array [B, max_pages];
+ * page_size is a power of two in [16, 2^20]; max_pages * page_size >=
+ * N_max.  A page number outside [0, num_pages) is reported by rtp_check()
+ * as RTP_ERR_DEVICE_ARG (the outputs it touches are then unspecified).
+ * The index-key cache stays contiguous ([B, H_kv, N_max, r]: 1/8 of the
+ * K/V bytes per token at r = 16, d = 128). */
+typedef struct rtp_kv_pages {
+    const int32_t *block_table;
+    int32_t page_size;
+    int32_t max_pages;
+    int32_t num_pages;
+    int32_t reserved;
+} rtp_kv_pages;
+
 /* Options; pass NULL for all defaults. */
 typedef struct rtp_opts {
     float idx_scale;          /* index logit scale; 0 -> 1/sqrt(d)          */
@@ -162,6 +180,10 @@ typedef struct rtp_opts {
      * the union, sel_mass the selected set alone.  Needs
      * min(N_max, window + n_sink) <= 393216, else RTP_ERR_UNSUPPORTED. */
     int32_t force_local;
+    /* Paged K/V caches (NULL: contiguous [B, H_kv, N_max, d]); honoured by
+     * rtp_decode_step, rtp_sparse_decode, rtp_local_decode,
+     * rtp_dense_decode, rtp_dense_decode_noalloc and rtp_prefill_attention. */
+    const rtp_kv_pages *kv_pages;
 } rtp_opts;
 
 /* Workspace bytes `op` needs for these shapes (0 on invalid dims).  The

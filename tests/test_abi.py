@@ -153,6 +153,13 @@ def test_other_calls_reject_bad_arguments(L):
     assert L.rtp_topk_select(ctypes.byref(d), FAKE + 4, hc, 8, FAKE, FAKE, FAKE, big,
                              None) == ops.RTP_ERR_INVALID_ARG
     assert L.rtp_topk_select(ctypes.byref(d), FAKE, hc, 8, FAKE, FAKE, FAKE, 100, None) == ops.RTP_ERR_WORKSPACE
+    # paged K/V: page size a power of two >= 16, a table, enough pages per sequence
+    for ps, mp, npg, tab in ((24, 4096, 10, FAKE), (8, 8192, 10, FAKE), (16, 10, 10, FAKE), (16, 4096, 0, FAKE),
+                             (16, 4096, 10, 0), (16, 4096, 10, FAKE + 2)):
+        pg = ops.KvPages(tab, ps, mp, npg, 0)
+        o = ops.Opts(0.0, 0.0, None, None, None, None, 0, 0, ctypes.pointer(pg))
+        assert L.rtp_dense_decode(ctypes.byref(d), ctypes.byref(o), FAKE, FAKE, FAKE, FAKE, FAKE, big,
+                                  None) == ops.RTP_ERR_INVALID_ARG, (ps, mp, npg)
     # prefill: prompt length, window, cache type, workspace
     pf = L.rtp_prefill_attention
     assert pf(ctypes.byref(d), None, FAKE, 0, FAKE, FAKE, FAKE, hc, 16, 4, FAKE, FAKE, big,
