@@ -415,7 +415,8 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
     const dim3 grid((unsigned)a.n_split, (unsigned)(d->B * a.n_grp));
     const char *name = dense ? "dense_attn" : "local_attn";
     if (d->kv_dtype == RTP_BF16)
-        return ln.run(name, gqa_mma_attn_kernel, grid, dim3(GQ_THREADS), a);
+        return a.kv.table ? ln.run(name, gqa_mma_attn_kernel<true>, grid, dim3(GQ_THREADS), a)
+                          : ln.run(name, gqa_mma_attn_kernel<false>, grid, dim3(GQ_THREADS), a);
     return ln.run(name, range_attn_kernel<float>, grid, dim3(ATT_THREADS), a);
 }
 
@@ -811,7 +812,11 @@ int rtp_dense_decode_noalloc(const rtp_dims *dims, const rtp_opts *opts, const f
     Launcher ln{st, opts ? opts->prof : nullptr};
     const dim3 grid((unsigned)a.n_split, (unsigned)groups);
     if (dims->kv_dtype == RTP_BF16) {
-        RTP_TRY(ln.run("dense_attn", gqa_mma_attn_kernel, grid, dim3(GQ_THREADS), a));
+        if (a.kv.table) {
+            RTP_TRY(ln.run("dense_attn", gqa_mma_attn_kernel<true>, grid, dim3(GQ_THREADS), a));
+        } else {
+            RTP_TRY(ln.run("dense_attn", gqa_mma_attn_kernel<false>, grid, dim3(GQ_THREADS), a));
+        }
     } else {
         RTP_TRY(ln.run("dense_attn", range_attn_kernel<float>, grid, dim3(ATT_THREADS), a));
     }

@@ -56,6 +56,9 @@ __device__ __forceinline__ void split3(float x, float &hi, float &mid, float &lo
     lo = r - mid;
 }
 
+// PAGED: rows through the block table of a page pool (a.kv.table), else
+// contiguous.
+template <bool PAGED>
 __global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a) {
     __shared__ float s_m[GQ_WARPS][GMAX], s_l[GQ_WARPS][GMAX];
     __shared__ float s_o[GQ_WARPS][GMAX][D];
@@ -105,9 +108,12 @@ __global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a
     const __nv_bfloat16 *vb = reinterpret_cast<const __nv_bfloat16 *>(a.v);
     // cache row of range position j (past the end: a valid row, masked
     // below; a page outside the pool is reported and read as row 0)
+    const long long base = (long long)bg * a.N_max;
     auto row_of = [&](long long j) -> long long {
         j = j < hi ? j : hi - 1;
-        return max(0LL, kv_row(a.kv, b, g, j < s1 ? j : w0 + (j - s1)));
+        const long long t = j < s1 ? j : w0 + (j - s1);
+        if constexpr (PAGED) return max(0LL, kv_row(a.kv, b, g, t));
+        return base + t;
     };
 
     float m_run = -INFINITY, l_run = 0.0f;        // head gid (shared by the 4 lanes of gid)
