@@ -54,6 +54,16 @@
  *   - Argument errors are detected on the host, before any launch, and
  *     returned; nothing is launched then.  Errors found on the device are
  *     recorded in the workspace status word and returned by rtp_check().
+ *   - State kept by the library (created on first use, held until exit):
+ *     per device, the SM count and whether each kernel's shared-memory
+ *     attribute is set; per host thread and device, two side streams with
+ *     their fork/join events, on which rtp_decode_step runs the local
+ *     heads (and, for fp32 caches, the first list pass) beside the
+ *     selection.  Two rtp_decode_step calls issued from one host thread on
+ *     different caller streams share those side streams, so the second
+ *     call's side work queues behind the first's; issue concurrent steps
+ *     from different host threads.  rtp_dense_decode_noalloc's scratch array
+ *     is described at that call.
  */
 #ifndef RTP_H_
 #define RTP_H_

@@ -305,12 +305,41 @@ def test_ctx1m_p_sweep():
 
 
 @pytest.mark.slow
-def test_ctx128k_b8_sampled_layers():
-    # the 48-layer workload runs 48 layers x 8 sequences; the oracle checks two layers
-    # fully (all 8 sequences, all heads) and the launch shape is the same
-    # for every layer.
-    for layer in (0, 29):
-        _workload("ctx128k-b8-48layer", [0.9], layer=layer)
+def test_ctx128k_b8_full_48_layer_step():
+    """The whole 48-layer step as the bench runs it: all 48 layers resident
+    (~110 GB), each layer's index-key append and decode step in turn on one
+    workspace; four layers spread across depth are checked in full (8
+    sequences x 32 heads each) against the oracle."""
+    import types
+
+    import bench
+    spec, layers = bench.build_workload("ctx128k-b8-48layer")
+    ws = ops.Workspace(layers[0].dims)
+    check = (0, 15, 31, 47)
+    results = {}
+    for li, L in enumerate(layers):
+        ops.append_index_keys(L.dims, L.k_new, L.Wk, L.pos, L.hc, L.kidx, ws)
+        out = torch.full((spec.B, spec.H_q, spec.d), float("nan"), device="cuda")
+        sel = None
+        if li in check:
+            sel = (torch.full((spec.B, spec.H_q, L.k.shape[2]), -1, dtype=torch.int32, device="cuda"),
+                   torch.zeros((spec.B, spec.H_q), dtype=torch.int32, device="cuda"),
+                   torch.zeros((spec.B, spec.H_q), device="cuda"))
+        opts = ops.make_opts(sel_idx=sel[0], sel_count=sel[1], sel_mass=sel[2]) if sel else None
+        ops.decode_step(L.dims, L.q, L.q_rope, L.k, L.v, L.kidx, L.Wq, L.hc, spec.p, spec.window, spec.n_sink, out,
+                        ws, opts)
+        if sel:
+            results[li] = (out, *sel)
+    st = ws.check()
+    assert st == 0, ops.error_string(st)
+    for li in check:
+        case = layers[li].case
+        gc = types.SimpleNamespace(c=case, B=spec.B, H_q=spec.H_q, H_kv=spec.H_kv)
+        out, si, sc, sm = results[li]
+        _compare(gc, out, si, sc, sm, spec.p)
+        del gc
+    del layers, results
+    torch.cuda.empty_cache()
 
 
 # ------------------------------------------------------- staging overflow
