@@ -78,15 +78,25 @@ def test_paged_decode_calls_match_contiguous(i):
         assert st == 0, ops.error_string(st)
         return out
 
-    # dense and local decode: the same arithmetic in the same order
+    # dense and local decode: bf16 caches take the same arithmetic in the
+    # same order (bit-exact); the fp32-cache kernel sums its warps'
+    # accumulators with shared-memory atomics, in no fixed order
+    exact = gc.k.dtype == torch.bfloat16
+
+    def same(x, y, what):
+        if exact:
+            assert torch.equal(x, y), what
+        else:
+            within(x.cpu().numpy(), y.cpu().numpy(), 1e-6, what)
+
     a = run(lambda o: ops.dense_decode(gc.dims, qr, gc.k, gc.v, o, gc.ws))
     b = run(lambda o: ops.dense_decode(gc.dims, qr, kp, vp, o, gc.ws, popt))
-    assert torch.equal(a, b)
+    same(a, b, "dense")
     a = run(lambda o: ops.local_decode(gc.dims, qr, gc.k, gc.v, gc.hc, c.window, c.n_sink, o, gc.ws))
     b = run(lambda o: ops.local_decode(gc.dims, qr, kp, vp, gc.hc, c.window, c.n_sink, o, gc.ws, popt))
     G = H_q // gc.H_kv
     loc = [h for h in range(H_q) if c.head_class[h // G] == 0]
-    assert torch.equal(a[:, loc], b[:, loc])
+    same(a[:, loc], b[:, loc], "local")
     # the decode step (kept sets too), top-p and static top-k, plain and with forced local rows
     for extra in (dict(), dict(topk=200), dict(force_local=True)):
         outs = []
@@ -109,7 +119,7 @@ def test_paged_decode_calls_match_contiguous(i):
     a = run(lambda o: ops.sparse_decode(gc.dims, qr, gc.k, gc.v, i0, c0, gc.hc, o, gc.ws))
     b = run(lambda o: ops.sparse_decode(gc.dims, qr, kp, vp, i0, c0, gc.hc, o, gc.ws, popt))
     ret = [h for h in range(H_q) if c.head_class[h // G] == 1]
-    assert torch.equal(a[:, ret], b[:, ret])
+    same(a[:, ret], b[:, ret], "sparse")
 
 
 def test_paged_prefill_matches_contiguous_and_oracle():
