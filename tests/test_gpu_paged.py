@@ -84,6 +84,8 @@ def test_paged_decode_calls_match_contiguous(i):
     exact = gc.k.dtype == torch.bfloat16
 
     def same(x, y, what):
+        if x.numel() == 0:
+            return
         if exact:
             assert torch.equal(x, y), what
         else:
