@@ -295,7 +295,7 @@ int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s, const After
     RTP_TRY(ln.run("hist", scan_kernel<Src>, grid, dim3(SCAN_THREADS), s.a, s.w));
     RTP_TRY(ln.run("collect", collect_kernel<Src>, grid, dim3(COL_THREADS), s.a, s.w));
     if (after_collect) RTP_TRY(after_collect());
-    RTP_TRY(ln.run("finalize", finalize_kernel, dim3(1u, (unsigned)(d->B * s.a.n_ret * s.a.G)),
+    RTP_TRY(ln.run("finalize", finalize_kernel<false>, dim3(1u, (unsigned)(d->B * s.a.n_ret * s.a.G)),
                    dim3(FIN_THREADS), s.a, s.w));
     return RTP_OK;
 }
@@ -314,7 +314,9 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sm
                 cudaSuccess ||
             cudaFuncSetAttribute(scan_tma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, TC_SMEM) !=
                 cudaSuccess ||
-            cudaFuncSetAttribute(collect_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, CL_SMEM) !=
+            cudaFuncSetAttribute(collect_mma_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, CL_SMEM) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(collect_mma_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, CL_SMEM) !=
                 cudaSuccess)
             return RTP_ERR_CUDA;
         attr_set[dev] = 1;
@@ -339,13 +341,18 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sm
     ln.pdl = true;
     int rc = s.a.topk > 0 ? ln.run_smem("hist", scan_tma_kernel<true>, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w)
                           : ln.run_smem("hist", scan_tma_kernel<false>, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w);
-    if (rc == RTP_OK) rc = ln.run_smem("collect", collect_mma_kernel, cl_grid, dim3(CL_THREADS), CL_SMEM, s.a, s.w);
+    const bool paged = s.a.kv.table != nullptr;
+    if (rc == RTP_OK)
+        rc = paged ? ln.run_smem("collect", collect_mma_kernel<true>, cl_grid, dim3(CL_THREADS), CL_SMEM, s.a, s.w)
+                   : ln.run_smem("collect", collect_mma_kernel<false>, cl_grid, dim3(CL_THREADS), CL_SMEM, s.a, s.w);
     if (rc == RTP_OK && after_collect) rc = after_collect();
     if (rc == RTP_OK) {
         // with the fused attention the CTAs of a head form a cluster
         const unsigned K = s.a.q_rope ? (unsigned)FIN_CLUSTER : 1u;
         ln.cluster_x = K > 1 ? K : 0u;
-        rc = ln.run("finalize", finalize_kernel, dim3(K, (unsigned)(d->B * s.a.n_ret * s.a.G)), dim3(FIN_THREADS),
+        const dim3 fgrid(K, (unsigned)(d->B * s.a.n_ret * s.a.G));
+        rc = paged ? ln.run("finalize", finalize_kernel<true>, fgrid, dim3(FIN_THREADS), s.a, s.w)
+                   : ln.run("finalize", finalize_kernel<false>, fgrid, dim3(FIN_THREADS),
                     s.a, s.w);
         ln.cluster_x = 0;
     }
@@ -447,6 +454,7 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
     a.q = q; a.k = k; a.v = v; a.lists = lists; a.counts = counts; a.out = out;
     a.first = first;
     a.spill = spill;
+    a.spill_any = reinterpret_cast<const uint32_t *>(ws + L.status) + 1;
     a.phase = phase;
     a.part = reinterpret_cast<float *>(ws + L.part_list);
     a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_list);
@@ -454,7 +462,7 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
     a.kv = kv ? *kv : make_kv(d, nullptr, a.status);
     const long long max_items = (long long)d->B * a.n_rq *
         std::min<long long>(LIST_MAX_SPLIT, (d->N_max + LCH - 1) / LCH);
-    const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(max_items, 2LL * num_sms()));
+    const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(max_items, (phase == LIST_SPILL ? 1LL : 2LL) * num_sms()));
     const size_t smem = list_smem_bytes(d->B * a.n_rq, d->B);
     const char *name = phase == LIST_FIRST ? "sparse_attn_first" : phase == LIST_SPILL ? "sparse_attn_spill"
                                                                                        : "sparse_attn";
@@ -938,6 +946,7 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
                 const bool can_spill = dims->N_max > FIN_SPILL;
                 s.a.spill_rows = can_spill ? FIN_SPILL : 0;
                 s.a.part_list = reinterpret_cast<float *>(w + L.part_list);
+                s.a.spill_any = reinterpret_cast<uint32_t *>(w + L.status) + 1;
                 rc = select_from_index(ln, dims, s, local_ctas);
                 if (rc == RTP_OK && can_spill) {
                     const bool pdl0 = ln.pdl;

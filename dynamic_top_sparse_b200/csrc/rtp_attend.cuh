@@ -284,6 +284,7 @@ struct ListArgs {
     // LIST_REST), or null
     const int32_t *first;
     const uint32_t *spill;       // [B*H_q] hand-over flags (LIST_SPILL)
+    const uint32_t *spill_any;   // nonzero when some head was handed over (LIST_SPILL)
     int phase;
     float *out;
     float *part;                 // [B*H_q][LIST_SLOTS][PSTRIDE]
@@ -320,6 +321,8 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
     __shared__ int s_last;
     pdl_wait();
     pdl_trigger();
+    // the hand-over pass has nothing to do unless finalize flagged a head
+    if (a.phase == LIST_SPILL && __ldcg(a.spill_any) == 0u) return;
 
     // items per head -> exclusive prefix, built by every CTA: thread t owns
     // heads [t * per, t * per + per), then a block-wide exclusive scan

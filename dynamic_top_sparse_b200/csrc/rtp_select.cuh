@@ -273,6 +273,7 @@ struct SelArgs {
     // list pass over all SMs.
     int spill_rows;
     float *part_list;                    // [B*H_q][LIST_SLOTS][PSTRIDE]
+    uint32_t *spill_any;                 // set when any head was handed over (the scan clears it)
 };
 
 // Record `r` of a cluster (the same shared variable in CTA rank r); the CTA's
@@ -330,15 +331,27 @@ __device__ __forceinline__ void prefetch_kv_l2(const __nv_bfloat16 *k_row, const
     asm volatile("prefetch.global.L2 [%0];" ::"l"(v_row + 64));
 }
 
+// PAGED: rows through the block table of a page pool (km.table), else the
+// contiguous (b, g) slab with 32-bit token offsets.
+template <bool PAGED>
 __device__ __forceinline__ void attend8(const __nv_bfloat16 *kc, const __nv_bfloat16 *vc, const KvMap &km, int b,
                                         int g, int id, const float (&qx)[4], WarpPart &p) {
     const int lane = threadIdx.x & 31;
     float kx[8][4], vx[8][4];
     bool ok[8];
-    const long long ro = id >= 0 ? kv_row(km, b, g, id) : -1LL;    // lanes 0-7: their token's row
+    long long ro = id;                                             // lanes 0-7: their token's row
+    if constexpr (PAGED) {
+        ro = id >= 0 ? kv_row(km, b, g, id) : -1LL;
+    } else {
+        const long long base = ((long long)b * km.H_kv + g) * km.N_max * D;
+        kc += base;
+        vc += base;
+    }
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
-        const long long r = __shfl_sync(0xffffffffu, ro, u);
+        long long r;
+        if constexpr (PAGED) r = __shfl_sync(0xffffffffu, ro, u);
+        else r = __shfl_sync(0xffffffffu, id, u);
         ok[u] = r >= 0;
         if (ok[u]) {
             Row<__nv_bfloat16>::load4(kc + r * D + lane * 4, kx[u]);
@@ -1029,6 +1042,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1) scan_tma_kernel(SelArgs a, SelW
         // stores come after the barriers of the prologue, which would wait
         // for them)
         if (blockIdx.x == 0) {
+            if (blockIdx.y == 0 && threadIdx.x == 0 && a.spill_any) *a.spill_any = 0u;
             for (int i = threadIdx.x; i < G * R; i += TC_WARPS * 32) w.qidx[bh0 * R + i] = qs[i];
             if (threadIdx.x < G) {
                 w.cand_cnt[(bh0 + threadIdx.x) * CNT_STRIDE] = 0u;
@@ -1330,6 +1344,7 @@ static_assert(CL_SLOTS >= CL_WARPS, "a round holds every warp's partial of any o
 // the pair's heads, and the attention partial slots
 constexpr int CL_SMEM = HP * CL_KCAP * 4 + HP * CCAP * 8 + HP * D * 4 + CL_SLOTS * PSTRIDE * 4;
 
+template <bool PAGED>
 __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, SelWs w) {
     extern __shared__ __align__(16) uint8_t csm[];
     int32_t *s_kbuf = reinterpret_cast<int32_t *>(csm);                                          // [HP][CL_KCAP]
@@ -1514,8 +1529,13 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
                         // finalize attends the candidates it keeps: their rows
                         // start toward L2 now (there are few of them)
                         if (a.q_rope) {
-                            const long long row = kv_row(a.kv, gk ? b1 : b0, gk ? g1 : g0, t);
-                            if (row >= 0) prefetch_kv_l2(a.k_cache + row * D, a.v_cache + row * D);
+                            if constexpr (PAGED) {
+                                const long long row = kv_row(a.kv, gk ? b1 : b0, gk ? g1 : g0, t);
+                                if (row >= 0) prefetch_kv_l2(a.k_cache + row * D, a.v_cache + row * D);
+                            } else {
+                                const size_t row = ((gk ? bg1 : bg0) * a.N_max + t) * D;
+                                prefetch_kv_l2(a.k_cache + row, a.v_cache + row);
+                            }
                         }
                     }
                 }
@@ -1599,8 +1619,8 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
             }
             const int r = (k - c0) * 8 + lane;
             const int id = lane < 8 && r < (int)s_kc[ph] ? s_kbuf[ph * CL_KCAP + r] : -1;
-            if (ph < GMAX) attend8(a.k_cache, a.v_cache, a.kv, b0, g0, id, qx, part);
-            else attend8(a.k_cache, a.v_cache, a.kv, b1, g1, id, qx, part);
+            if (ph < GMAX) attend8<PAGED>(a.k_cache, a.v_cache, a.kv, b0, g0, id, qx, part);
+            else attend8<PAGED>(a.k_cache, a.v_cache, a.kv, b1, g1, id, qx, part);
         }
         if (cur >= 0) part.store(s_slot + (cur_s0 + kfirst - cur_c0) * PSTRIDE);
         __syncthreads();
@@ -1641,6 +1661,7 @@ constexpr int FIN_SPILL = 2048;           // rows above which finalize hands a h
 // (staged in shared memory) or 2^62 / nc units per unit of mass, so sums
 // cannot wrap and do not depend on the order of the adds.  Rank 0 clears
 // the head's level-1 histogram for the next call, last.
+template <bool PAGED>
 __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs w) {
     __shared__ unsigned long long hfx[256];
     __shared__ uint32_t hfx32[256];
@@ -1910,7 +1931,10 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         if (tid == 0) {
             a.count_out[bh] = count;
             if (a.mass_out) a.mass_out[bh] = mass;
-            if (spill) a.ovf[bh] = (ovf || r.mode == MODE_KEEP_ALL) ? SPILL_ALL_ROWS : SPILL_FROM_FIRST;
+            if (spill) {
+                a.ovf[bh] = (ovf || r.mode == MODE_KEEP_ALL) ? SPILL_ALL_ROWS : SPILL_FROM_FIRST;
+                atomicExch(a.spill_any, 1u);
+            }
         }
         if (r.mode == MODE_KEEP_ALL) {
             for (int t = tid; t < r.N; t += blockDim.x) lst[t] = t;
@@ -1964,13 +1988,13 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             // the collect pass's rows, from its list
             for (int rb = worker * 8; rb < (int)base0; rb += workers * 8) {
                 const int id = lane < 8 && rb + lane < (int)base0 ? __ldcg(lst + rb + lane) : -1;
-                attend8(a.k_cache, a.v_cache, a.kv, b, g, id, qx_f, part);
+                attend8<PAGED>(a.k_cache, a.v_cache, a.kv, b, g, id, qx_f, part);
             }
         }
         if (r.mode == MODE_KEEP_ALL) {
             for (int rb = worker * 8; rb < count; rb += workers * 8) {
                 const int id = lane < 8 && rb + lane < count ? rb + lane : -1;
-                attend8(a.k_cache, a.v_cache, a.kv, b, g, id, qx_f, part);
+                attend8<PAGED>(a.k_cache, a.v_cache, a.kv, b, g, id, qx_f, part);
             }
         } else if (r.mode == MODE_NORMAL) {
             // boundary-bin candidates at or above theta: the compacted ids
@@ -1978,7 +2002,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
             if (fin_staged) {
                 const int nk = count - (int)base0;
                 for (int rb = worker * 8; rb < nk; rb += workers * 8)
-                    attend8(a.k_cache, a.v_cache, a.kv, b, g, lane < 8 && rb + lane < nk ? s_kid[rb + lane] : -1, qx_f, part);
+                    attend8<PAGED>(a.k_cache, a.v_cache, a.kv, b, g, lane < 8 && rb + lane < nk ? s_kid[rb + lane] : -1, qx_f, part);
             } else {
                 for (int cb = worker * 8; cb < (int)nc; cb += workers * 8) {
                     int id = -1;
@@ -1986,7 +2010,7 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
                         const unsigned long long v = __ldcg(cg + cb + lane);
                         if (v >= fin_theta) id = (int)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
                     }
-                    attend8(a.k_cache, a.v_cache, a.kv, b, g, id, qx_f, part);
+                    attend8<PAGED>(a.k_cache, a.v_cache, a.kv, b, g, id, qx_f, part);
                 }
             }
         }
