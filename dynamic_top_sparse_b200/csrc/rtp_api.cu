@@ -21,6 +21,8 @@ using namespace rtp;
 namespace {
 
 constexpr int RANGE_SPLIT_MAX = 256;
+// context above which the fused step adds the hand-over pass after finalize
+constexpr long long SPILL_MIN_CTX = 256 * 1024;
 // SMs given to the local heads while the selection runs beside them
 constexpr int LOCAL_SMS = 12;
 
@@ -941,9 +943,11 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
                 s.a.ovf = reinterpret_cast<uint32_t *>(w + L.ovf);
                 // heads that keep many rows beyond what the collect pass
                 // attended are finished by a list pass over every SM (a
-                // 4-CTA cluster per head would take long over them); it is
-                // needed only when a head can keep more than FIN_SPILL rows
-                const bool can_spill = dims->N_max > FIN_SPILL;
+                // 4-CTA cluster per head would take long over them).  The
+                // pass costs a launch in the chain (~2 us) even when no head
+                // needs it, so it is used from SPILL_MIN_CTX tokens on; below
+                // that a cluster attends at most SPILL_MIN_CTX rows per head.
+                const bool can_spill = dims->N_max > SPILL_MIN_CTX;
                 s.a.spill_rows = can_spill ? FIN_SPILL : 0;
                 s.a.part_list = reinterpret_cast<float *>(w + L.part_list);
                 s.a.spill_any = reinterpret_cast<uint32_t *>(w + L.status) + 1;

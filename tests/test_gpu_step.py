@@ -172,9 +172,10 @@ def test_step_large_index_logits(c_scale):
 def test_step_flat_logits_hand_over(p):
     """Every index key equal: all tokens share one logit, the boundary bin
     holds every token and the kept set is the first ceil(p N) tokens by
-    index -- thousands of boundary rows, more than finalize attends itself,
-    so the list pass over every SM finishes those heads."""
-    spec = synth.small_spec(B=2, H_q=16, H_kv=2, N=19999, head_class=(1, 0), seq_lens=[19999, 7001],
+    index -- tens of thousands of boundary rows at 300K tokens, more than
+    finalize attends itself, so the list pass over every SM finishes those
+    heads (the 7001-token sequence stays with finalize)."""
+    spec = synth.small_spec(B=2, H_q=16, H_kv=2, N=300001, head_class=(1, 0), seq_lens=[300001, 7001],
                             needles="none")
     c = synth.make_case(spec)
     c.kidx_cache[:, 0] = c.kidx_cache[:, 0, :1].clone()          # row 0's key everywhere
@@ -188,7 +189,9 @@ def test_step_flat_logits_hand_over(p):
             n = int(sc[b, h])
             assert n == math.ceil(float(np.float32(p)) * N), (b, h, n)      # p N is 0.1 - 0.9 off an integer
             assert sorted(gpu_set(si, sc, b, h).tolist()) == list(range(n))
-    _compare(gc, out, si, sc, sm, p, with_current=False)
+    # outputs of a sample of heads (each over up to 270K rows) and every local head
+    heads = [(0, 0), (0, 7), (1, 2), (1, 5)] + [(b, h) for b in range(2) for h in range(8, 16)]
+    _compare(gc, out, si, sc, sm, p, heads=heads, with_current=False)
 
 
 FORCE = [

@@ -123,6 +123,8 @@ STEP = [
     # k > N with more rows than finalize attends itself: the list pass takes them
     (dict(B=2, H_q=8, H_kv=1, N=6000, head_class=(1,), needles="none", seq_lens=[6000, 3000]), 10 ** 6),
     (dict(B=1, H_q=8, H_kv=1, N=20000, head_class=(1,), needles="none"), 9000),
+    # every token of a 262K-token sequence: the list pass over every SM takes them
+    (dict(B=1, H_q=8, H_kv=1, N=262200, head_class=(1,), needles="none"), 10 ** 6),
     (dict(B=2, H_q=4, H_kv=4, N=3000, head_class=(1, 0, 1, 0), kv_dtype="f32", idx_dtype="f32"), 300),
     (dict(B=2, H_q=16, H_kv=2, N=6000, head_class=(1, 0), kv_dtype="f32", idx_dtype="bf16"), 2048),
 ]
