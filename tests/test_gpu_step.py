@@ -187,7 +187,9 @@ def test_step_flat_logits_hand_over(p):
         N = int(c.seq_lens[b])
         for h in range(G):
             n = int(sc[b, h])
-            assert n == math.ceil(float(np.float32(p)) * N), (b, h, n)      # p N is 0.1 - 0.9 off an integer
+            # ceil(p N) tokens, give or take tokens within the 1e-5 mass window
+            # (the fixed-point sums round every equal term the same way)
+            assert abs(n - math.ceil(float(np.float32(p)) * N)) <= 1e-5 * N + 1, (b, h, n)
             assert sorted(gpu_set(si, sc, b, h).tolist()) == list(range(n))
     # outputs of a sample of heads (each over up to 270K rows) and every local head
     heads = [(0, 0), (0, 7), (1, 2), (1, 5)] + [(b, h) for b in range(2) for h in range(8, 16)]
