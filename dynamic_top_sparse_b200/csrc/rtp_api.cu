@@ -38,7 +38,7 @@ struct Layout {
     size_t end_range;       // local / dense
     size_t part_list;
     size_t end_list;        // sparse decode
-    size_t tilebin, lists, cands, part_sel, ovf;
+    size_t tilebin, lists, cands, part_sel, ovf, theta;
     size_t total;           // topp_select / decode_step
 };
 
@@ -74,6 +74,7 @@ Layout make_layout(const rtp_dims *d) {
     // and the collect grid twice as many
     L.part_sel = o; o = align_up(o + 2 * std::max((size_t)num_sms(), BHkv) * GMAX * PSTRIDE * 4, 256);
     L.ovf = o; o = align_up(o + BHq * 4, 256);
+    L.theta = o; o = align_up(o + BHq * 8, 256);
     L.total = o;
     return L;
 }
@@ -304,8 +305,12 @@ int launch_select(Launcher &ln, const rtp_dims *d, const SelPlan &s, const After
 
 // reserve_sms: SMs left free for work running beside the selection (the
 // local heads of a decode step), so that neither waits for the other.
+// which kernels of the TMA selection chain to launch (a context shard runs
+// them one at a time, with exchanges in between)
+enum SelPhases : int { SEL_SCAN = 1, SEL_COLLECT = 2, SEL_FINALIZE = 4, SEL_ALL = 7 };
+
 int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sms = 0,
-                      const AfterCollect &after_collect = {}) {
+                      const AfterCollect &after_collect = {}, int phases = SEL_ALL) {
     if (d->idx_dtype != RTP_BF16) return launch_select<SrcSimt<float>>(ln, d, s, after_collect);
     // bf16 index keys: the TMA-ring scan, one CTA per SM over all groups
     static int attr_set[64] = {0};
@@ -340,15 +345,17 @@ int select_from_index(Launcher &ln, const rtp_dims *d, SelPlan s, int reserve_sm
     // (programmatic dependent launch), so each one's launch overlaps the
     // previous kernel's tail
     const bool pdl0 = ln.pdl;
-    ln.pdl = true;
-    int rc = s.a.topk > 0 ? ln.run_smem("hist", scan_tma_kernel<true>, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w)
+    ln.pdl = phases == SEL_ALL;
+    int rc = RTP_OK;
+    if (phases & SEL_SCAN)
+        rc = s.a.topk > 0 ? ln.run_smem("hist", scan_tma_kernel<true>, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w)
                           : ln.run_smem("hist", scan_tma_kernel<false>, grid, dim3(TC_THREADS), TC_SMEM, s.a, s.w);
     const bool paged = s.a.kv.table != nullptr;
-    if (rc == RTP_OK)
+    if (rc == RTP_OK && (phases & SEL_COLLECT))
         rc = paged ? ln.run_smem("collect", collect_mma_kernel<true>, cl_grid, dim3(CL_THREADS), CL_SMEM, s.a, s.w)
                    : ln.run_smem("collect", collect_mma_kernel<false>, cl_grid, dim3(CL_THREADS), CL_SMEM, s.a, s.w);
     if (rc == RTP_OK && after_collect) rc = after_collect();
-    if (rc == RTP_OK) {
+    if (rc == RTP_OK && (phases & SEL_FINALIZE)) {
         // with the fused attention the CTAs of a head form a cluster
         const unsigned K = s.a.q_rope ? (unsigned)FIN_CLUSTER : 1u;
         ln.cluster_x = K > 1 ? K : 0u;
@@ -393,7 +400,8 @@ int side_stream(Side *&out, int slot = 0) {
 // ----------------------------------------------------------------- attention
 int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
                  const uint8_t *hc, int want_class, bool dense, int window, int n_sink, float *out,
-                 char *ws, const Layout &L, float attn_scale, int max_ctas = 0, const KvMap *kv = nullptr) {
+                 char *ws, const Layout &L, float attn_scale, int max_ctas = 0, const KvMap *kv = nullptr,
+                 const int32_t *glob_len = nullptr, const int32_t *id_off = nullptr, float *part_out = nullptr) {
     RangeArgs a{};
     a.B = d->B; a.H_q = d->H_q; a.H_kv = d->H_kv; a.G = d->H_q / d->H_kv;
     a.N_max = d->N_max; a.seq_lens = d->seq_lens;
@@ -421,6 +429,9 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
     a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_range);
     a.status = reinterpret_cast<uint32_t *>(ws + L.status);
     a.kv = kv ? *kv : make_kv(d, nullptr, a.status);
+    a.glob_len = glob_len;
+    a.id_off = id_off;
+    a.part_out = part_out;
     const dim3 grid((unsigned)a.n_split, (unsigned)(d->B * a.n_grp));
     const char *name = dense ? "dense_attn" : "local_attn";
     if (d->kv_dtype == RTP_BF16)
@@ -432,7 +443,8 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
 int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, const void *v,
                 const int32_t *lists, const int32_t *counts, const uint8_t *hc, float *out,
                 char *ws, const Layout &L, float attn_scale, int phase = LIST_ALL,
-                const int32_t *first = nullptr, const uint32_t *spill = nullptr, const KvMap *kv = nullptr) {
+                const int32_t *first = nullptr, const uint32_t *spill = nullptr, const KvMap *kv = nullptr,
+                const int32_t *id_off = nullptr, float *part_out = nullptr) {
     static int attr_set[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return RTP_ERR_CUDA;
@@ -462,6 +474,8 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
     a.arrive = reinterpret_cast<uint32_t *>(ws + L.arrive_list);
     a.status = reinterpret_cast<uint32_t *>(ws + L.status);
     a.kv = kv ? *kv : make_kv(d, nullptr, a.status);
+    a.id_off = id_off;
+    a.part_out = part_out;
     const long long max_items = (long long)d->B * a.n_rq *
         std::min<long long>(LIST_MAX_SPLIT, (d->N_max + LCH - 1) / LCH);
     const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(max_items, (phase == LIST_SPILL ? 1LL : 2LL) * num_sms()));
@@ -988,6 +1002,128 @@ int rtp_decode_step(const rtp_dims *dims, const rtp_opts *opts, const float *q, 
     }
     if (side && cudaStreamWaitEvent(main, side->join, 0) != cudaSuccess && rc == RTP_OK) rc = RTP_ERR_CUDA;
     return rc;
+}
+
+// ------------------------------------------------------------ context shards
+
+namespace {
+int check_shard(const rtp_dims *dims, const uint8_t *head_class, void *ws, size_t ws_bytes) {
+    RTP_TRY(check_dims(dims));
+    if (dims->kv_dtype != RTP_BF16 || dims->idx_dtype != RTP_BF16) return RTP_ERR_UNSUPPORTED;
+    RTP_TRY(check_head_class(dims, head_class));
+    return check_ws(dims, ws, ws_bytes, RTP_OP_DECODE_STEP);
+}
+}  // namespace
+
+int rtp_shard_scan(const rtp_dims *dims, const rtp_opts *opts, const float *q, const void *kidx_cache,
+                   const float *W_q_idx, const uint8_t *head_class, float p, void *ws, size_t ws_bytes,
+                   rtp_stream_t stream) {
+    RTP_TRY(check_shard(dims, head_class, ws, ws_bytes));
+    if (!q || !kidx_cache || !W_q_idx || std::isnan(p)) return RTP_ERR_INVALID_ARG;
+    if (p >= 1.0f) return RTP_OK;                    // every token kept: no threshold
+    if (!aligned16(q) || !aligned16(kidx_cache) || !aligned16(W_q_idx)) return RTP_ERR_INVALID_ARG;
+    const Layout L = make_layout(dims);
+    SelPlan s = make_sel(dims, head_class, (char *)ws, L);
+    if (s.a.n_ret == 0) return RTP_OK;
+    s.a.kidx = kidx_cache;
+    s.a.q = q;
+    s.a.Wq = W_q_idx;
+    s.a.idx_scale = scale_or_default(opts ? opts->idx_scale : 0.f);
+    Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
+    return select_from_index(ln, dims, s, 0, {}, SEL_SCAN);
+}
+
+int rtp_shard_hist(const rtp_dims *dims, void *ws, double **hist, int64_t *count) {
+    RTP_TRY(check_dims(dims));
+    if (!ws || !hist || !count) return RTP_ERR_INVALID_ARG;
+    const Layout L = make_layout(dims);
+    *hist = reinterpret_cast<double *>((char *)ws + L.hist);
+    *count = (int64_t)dims->B * dims->H_q * HSTRIDE;
+    return RTP_OK;
+}
+
+int rtp_shard_collect(const rtp_dims *dims, const rtp_opts *opts, const void *kidx_cache, const uint8_t *head_class,
+                      float p, const int32_t *shard_off, void *ws, size_t ws_bytes, rtp_stream_t stream) {
+    RTP_TRY(check_shard(dims, head_class, ws, ws_bytes));
+    if (std::isnan(p) || !kidx_cache || !aligned16(kidx_cache) || !shard_off || !aligned4(shard_off))
+        return RTP_ERR_INVALID_ARG;
+    const Layout L = make_layout(dims);
+    char *w = (char *)ws;
+    SelPlan s = make_sel(dims, head_class, w, L);
+    if (s.a.n_ret == 0 || p >= 1.0f) return RTP_OK;
+    s.a.kidx = kidx_cache;
+    s.a.p = p;
+    s.a.id_off = shard_off;
+    s.a.lists = opts && opts->sel_idx ? opts->sel_idx : reinterpret_cast<int32_t *>(w + L.lists);
+    s.a.count_out = opts && opts->sel_count ? opts->sel_count : reinterpret_cast<int32_t *>(w + L.counts);
+    Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
+    return select_from_index(ln, dims, s, 0, {}, SEL_COLLECT);
+}
+
+int rtp_shard_cands(const rtp_dims *dims, void *ws, uint64_t **cands, uint32_t **counts, int64_t *stride,
+                    int64_t *count_stride) {
+    RTP_TRY(check_dims(dims));
+    if (!ws || !cands || !counts || !stride || !count_stride) return RTP_ERR_INVALID_ARG;
+    const Layout L = make_layout(dims);
+    *cands = reinterpret_cast<uint64_t *>((char *)ws + L.cands);
+    *counts = reinterpret_cast<uint32_t *>((char *)ws + L.cand_cnt);
+    *stride = dims->N_max;
+    *count_stride = CNT_STRIDE;
+    return RTP_OK;
+}
+
+int rtp_shard_finish(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope, const void *k_cache,
+                     const void *v_cache, const void *kidx_cache, const uint8_t *head_class, float p, int32_t window,
+                     int32_t n_sink, const int32_t *shard_off, const int32_t *glob_len, const uint64_t *all_cands,
+                     const int32_t *all_counts, int64_t all_stride, float *part_out, void *ws, size_t ws_bytes,
+                     rtp_stream_t stream) {
+    RTP_TRY(check_shard(dims, head_class, ws, ws_bytes));
+    if (std::isnan(p) || window < 1 || n_sink < 0) return RTP_ERR_INVALID_ARG;
+    if (!q_rope || !k_cache || !v_cache || !kidx_cache || !shard_off || !glob_len || !part_out)
+        return RTP_ERR_INVALID_ARG;
+    if (!aligned16(q_rope) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(part_out) ||
+        !aligned4(shard_off) || !aligned4(glob_len))
+        return RTP_ERR_INVALID_ARG;
+    RTP_TRY(check_kv(dims, opts));
+    const Layout L = make_layout(dims);
+    char *w = (char *)ws;
+    const KvMap kv = make_kv(dims, opts, w + L.status);
+    SelPlan s = make_sel(dims, head_class, w, L);
+    const bool selecting = s.a.n_ret > 0 && p < 1.0f;
+    if (selecting && (!all_cands || !all_counts || all_stride < 1 || !aligned16(all_cands) || !aligned4(all_counts)))
+        return RTP_ERR_INVALID_ARG;
+    Launcher ln{(cudaStream_t)stream, opts ? opts->prof : nullptr};
+    const float asc = scale_or_default(opts ? opts->attn_scale : 0.f);
+    // local heads: their rows of the shard (sinks and window in global positions)
+    if (s.a.n_ret < dims->H_kv) {
+        RTP_TRY(launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_LOCAL, false, window, n_sink,
+                             nullptr, w, L, asc, 0, &kv, glob_len, shard_off, part_out));
+    }
+    if (s.a.n_ret == 0) return RTP_OK;
+    if (!selecting)   // every token kept: the shard's rows of the retrieval heads, densely
+        return launch_range(ln, dims, q_rope, k_cache, v_cache, head_class, RTP_HEAD_RETRIEVAL, true, 1, 0, nullptr,
+                            w, L, asc, 0, &kv, glob_len, shard_off, part_out);
+    s.a.kidx = kidx_cache;
+    s.a.p = p;
+    s.a.id_off = shard_off;
+    s.a.ext_cands = reinterpret_cast<const unsigned long long *>(all_cands);
+    s.a.ext_cnt = all_counts;
+    s.a.ext_stride = all_stride;
+    s.a.theta_out = reinterpret_cast<unsigned long long *>(w + L.theta);
+    s.a.lists = opts && opts->sel_idx ? opts->sel_idx : reinterpret_cast<int32_t *>(w + L.lists);
+    s.a.count_out = opts && opts->sel_count ? opts->sel_count : reinterpret_cast<int32_t *>(w + L.counts);
+    s.a.mass_out = opts ? opts->sel_mass : nullptr;
+    RTP_TRY(select_from_index(ln, dims, s, 0, {}, SEL_FINALIZE));
+    RTP_TRY(ln.run("shard_own", shard_own_kernel, dim3((unsigned)(dims->B * s.a.n_ret * s.a.G)), dim3(OWN_THREADS),
+                   s.a, s.w));
+    return launch_list(ln, dims, q_rope, k_cache, v_cache, s.a.lists, s.a.count_out, head_class, nullptr, w, L, asc,
+                       LIST_ALL, nullptr, nullptr, &kv, shard_off, part_out);
+}
+
+int rtp_merge_shards(const float *parts, int32_t P, int32_t n_heads, float *out, rtp_stream_t stream) {
+    if (!parts || !out || P < 1 || n_heads < 1 || !aligned16(parts) || !aligned16(out)) return RTP_ERR_INVALID_ARG;
+    merge_shards_kernel<<<(unsigned)n_heads, 32, 0, (cudaStream_t)stream>>>(parts, P, n_heads, out);
+    return cudaGetLastError() == cudaSuccess ? RTP_OK : RTP_ERR_CUDA;
 }
 
 int rtp_prof_init(rtp_prof *prof, int32_t capacity) {

@@ -31,8 +31,11 @@ constexpr int MAX_LIST_HEADS = 4096;
 // records; record h of a group at + h * PSTRIDE) for heads [0, nh) into
 // out[h * D + d].  Every thread owns 4 dims of one head and merges in one
 // pass with a running max, keeping 16 records' loads in flight.
+// raw != null: the merged records (m, l, unnormalised o) go to raw + h
+// PSTRIDE instead of the normalised outputs (a shard's partial of a
+// context-sharded step).
 __device__ __forceinline__ void merge_partials(const float *__restrict__ pb, int n, int rec, int nh,
-                                               float *__restrict__ out) {
+                                               float *__restrict__ out, float *__restrict__ raw = nullptr) {
     constexpr int U = 16;
     for (int i = threadIdx.x; i < nh * (D / 4); i += blockDim.x) {
         const int h = i / (D / 4), d4 = i % (D / 4);
@@ -69,6 +72,12 @@ __device__ __forceinline__ void merge_partials(const float *__restrict__ pb, int
             }
             M = Mb;
         }
+        if (raw) {
+            float *rr = raw + (size_t)h * PSTRIDE;
+            reinterpret_cast<float4 *>(rr + POFF)[d4] = o;
+            if (d4 == 0) { rr[0] = M; rr[1] = l; }
+            continue;
+        }
         const float inv = l > 0.0f ? 1.0f / l : 0.0f;
         reinterpret_cast<float4 *>(out + h * D)[d4] = make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
     }
@@ -93,7 +102,31 @@ struct RangeArgs {
     uint32_t *arrive;   // [B*H_kv]
     uint32_t *status;
     KvMap kv;           // row addressing of k / v
+    // context shard (null: the whole sequence): this shard holds global
+    // tokens [id_off[b], id_off[b] + seq_lens[b]) of a sequence of
+    // glob_len[b] tokens; sinks and window are taken in global positions and
+    // the merged partials go to part_out [B*H_q][PSTRIDE] unnormalised
+    const int32_t *glob_len;
+    const int32_t *id_off;
+    float *part_out;
 };
+
+// The row set of a range launch in the shard's own positions 0..N-1: rows
+// [0, s1) and [w0, N).  Dense: every row.  Sinks and window: the first
+// n_sink and the last `window` positions of the (global) sequence, as seen
+// from the shard's offset.
+__device__ __forceinline__ void shard_range(const RangeArgs &a, int b, int N, int &s1, int &w0) {
+    if (a.dense) { s1 = N; w0 = N; return; }
+    if (!a.glob_len) {
+        s1 = min(a.n_sink, N);
+        w0 = max(s1, N - a.window);
+        return;
+    }
+    const long long off = a.id_off[b], Ng = a.glob_len[b];
+    const long long sg = min((long long)a.n_sink, Ng), wg = max(sg, Ng - a.window);   // global [0, sg), [wg, Ng)
+    s1 = (int)max(0LL, min((long long)N, sg - off));
+    w0 = (int)max((long long)s1, min((long long)N, wg - off));
+}
 
 template <typename KT>
 __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
@@ -113,15 +146,20 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
     if (N < 1 || (long long)N > a.N_max) {
         if (blockIdx.x == 0) {
             if (tid == 0) set_status(a.status, RTP_ERR_DEVICE_ARG);
-            for (int i = tid; i < G * D; i += blockDim.x) a.out[bh0 * D + i] = 0.0f;
+            if (a.part_out) {
+                for (int i = tid; i < G * PSTRIDE; i += blockDim.x)
+                    a.part_out[bh0 * PSTRIDE + i] = i % PSTRIDE == 0 ? -INFINITY : 0.0f;
+            } else {
+                for (int i = tid; i < G * D; i += blockDim.x) a.out[bh0 * D + i] = 0.0f;
+            }
         }
         return;
     }
-    const int s1 = a.dense ? N : min(a.n_sink, N);
-    const int w0 = a.dense ? N : max(s1, N - a.window);
+    int s1, w0;
+    shard_range(a, b, N, s1, w0);
     const long long L = (long long)s1 + (N - w0);
     const long long seg = (L + a.n_split - 1) / a.n_split;
-    const int n_active = (int)((L + seg - 1) / seg);
+    const int n_active = L > 0 ? (int)((L + seg - 1) / seg) : 1;
     if ((int)blockIdx.x >= n_active) return;
     const long long lo = (long long)blockIdx.x * seg;
     const long long hi = min(L, lo + seg);
@@ -249,7 +287,8 @@ __global__ void __launch_bounds__(ATT_THREADS) range_attn_kernel(RangeArgs a) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    merge_partials(a.part + bg * a.slots * GMAX * PSTRIDE, n_active, GMAX * PSTRIDE, G, a.out + bh0 * D);
+    merge_partials(a.part + bg * a.slots * GMAX * PSTRIDE, n_active, GMAX * PSTRIDE, G, a.out + bh0 * D,
+                   a.part_out ? a.part_out + bh0 * PSTRIDE : nullptr);
     if (tid == 0) a.arrive[bg] = 0;
 }
 
@@ -285,6 +324,11 @@ struct ListArgs {
     const int32_t *first;
     const uint32_t *spill;       // [B*H_q] hand-over flags (LIST_SPILL)
     const uint32_t *spill_any;   // nonzero when some head was handed over (LIST_SPILL)
+    // context shard (null: whole sequences): list ids are global positions,
+    // this shard's rows are id - id_off[b]; per-head merged partials go to
+    // part_out [B*H_q][PSTRIDE] unnormalised (empty record for no rows)
+    const int32_t *id_off;
+    float *part_out;
     int phase;
     float *out;
     float *part;                 // [B*H_q][LIST_SLOTS][PSTRIDE]
@@ -406,6 +450,13 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
             if (pre[hi + 1] != pre[hi]) continue;
             const int b = hi / a.n_rq, h = a.ret_h[hi % a.n_rq];
             if (a.phase == LIST_SPILL && __ldcg(a.spill + (size_t)b * a.H_q + h) < SPILL_FROM_FIRST) continue;
+            if (a.part_out) {
+                // a shard that keeps no row of this head: an empty partial
+                float *r = a.part_out + ((size_t)b * a.H_q + h) * PSTRIDE;
+                *reinterpret_cast<float4 *>(r + POFF + 4 * lane) = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (lane == 0) { r[0] = -INFINITY; r[1] = 0.0f; }
+                continue;
+            }
             float *o = a.out + ((size_t)b * a.H_q + h) * D + lane * 4;
             o[0] = o[1] = o[2] = o[3] = 0.0f;
             if (lane == 0) set_status(a.status, RTP_ERR_DEVICE_ARG);
@@ -438,11 +489,12 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
         const KT *kc = reinterpret_cast<const KT *>(a.k);
         const KT *vc = reinterpret_cast<const KT *>(a.v);
         const int32_t *lst = a.lists + bh * a.N_max;
+        const int id0 = a.id_off ? a.id_off[b] : 0;
         float m = -INFINITY, l = 0.0f, o[4] = {0.f, 0.f, 0.f, 0.f};
         constexpr int U = 8;       // rows per warp per pass: all their K/V loads in flight
         for (int rb = r0 + warp * U; rb < r1; rb += (ATT_THREADS / 32) * U) {
             int myid = -1;
-            if (lane < U && rb + lane < r1) myid = __ldcg(lst + rb + lane);
+            if (lane < U && rb + lane < r1) myid = __ldcg(lst + rb + lane) - id0;
             // lanes 0-7: the cache row of their token (-1: none or invalid)
             const long long myrow = myid >= 0 && myid < N ? kv_row(a.kv, b, g, myid) : -1LL;
             float kx[U][4], vx[U][4];
@@ -495,7 +547,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
         float *hp = a.part + bh * (size_t)LIST_SLOTS * PSTRIDE;
         float *pp = hp + (size_t)slot * PSTRIDE;
         // a head attended by this one item only: normalise and write directly
-        const bool direct = a.phase != LIST_FIRST && nrec == 1;
+        const bool direct = a.phase != LIST_FIRST && nrec == 1 && !a.part_out;
         if (tid < D) {
             float M = -INFINITY;
             for (int w = 0; w < ATT_THREADS / 32; ++w) M = fmaxf(M, wm[w]);
@@ -524,11 +576,21 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
         __syncthreads();
         if (s_last) {
             __threadfence();
-            merge_partials(hp, nrec, PSTRIDE, 1, a.out + bh * D);
+            merge_partials(hp, nrec, PSTRIDE, 1, a.out + bh * D, a.part_out ? a.part_out + bh * PSTRIDE : nullptr);
             if (tid == 0) a.arrive[bh] = 0;
         }
         __syncthreads();
     }
+}
+
+// ---------------------------------------------------------------------------
+// Context shards: the P shards' partial records of each head (parts
+// [P][n_heads][PSTRIDE], m and l in log2 units) merged into the output.
+// grid = (n_heads), 32 threads.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(32) merge_shards_kernel(const float *parts, int P, int nh, float *out) {
+    const int h = blockIdx.x;
+    merge_partials(parts + (size_t)h * PSTRIDE, P, nh * PSTRIDE, 1, out + (size_t)h * D);
 }
 
 // ---------------------------------------------------------------------------

@@ -75,15 +75,20 @@ __global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a
     if (N < 1 || (long long)N > a.N_max) {
         if (blockIdx.x == 0) {
             if (tid == 0) set_status(a.status, RTP_ERR_DEVICE_ARG);
-            for (int i = tid; i < G * D; i += blockDim.x) a.out[bh0 * D + i] = 0.0f;
+            if (a.part_out) {
+                for (int i = tid; i < G * PSTRIDE; i += blockDim.x)
+                    a.part_out[bh0 * PSTRIDE + i] = i % PSTRIDE == 0 ? -INFINITY : 0.0f;
+            } else {
+                for (int i = tid; i < G * D; i += blockDim.x) a.out[bh0 * D + i] = 0.0f;
+            }
         }
         return;
     }
-    const int s1 = a.dense ? N : min(a.n_sink, N);
-    const int w0 = a.dense ? N : max(s1, N - a.window);
+    int s1, w0;
+    shard_range(a, b, N, s1, w0);
     const long long L = (long long)s1 + (N - w0);
     const long long seg = (L + a.n_split - 1) / a.n_split;
-    const int n_active = (int)((L + seg - 1) / seg);
+    const int n_active = L > 0 ? (int)((L + seg - 1) / seg) : 1;
     if ((int)blockIdx.x >= n_active) return;
     const long long lo = (long long)blockIdx.x * seg;
     const long long hi = min(L, lo + seg);
@@ -240,7 +245,8 @@ __global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    merge_partials(a.part + bg * a.slots * GMAX * PSTRIDE, n_active, GMAX * PSTRIDE, G, a.out + bh0 * D);
+    merge_partials(a.part + bg * a.slots * GMAX * PSTRIDE, n_active, GMAX * PSTRIDE, G, a.out + bh0 * D,
+                   a.part_out ? a.part_out + bh0 * PSTRIDE : nullptr);
     if (tid == 0) a.arrive[bg] = 0;
 }
 

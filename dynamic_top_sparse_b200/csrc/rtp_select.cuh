@@ -274,6 +274,17 @@ struct SelArgs {
     int spill_rows;
     float *part_list;                    // [B*H_q][LIST_SLOTS][PSTRIDE]
     uint32_t *spill_any;                 // set when any head was handed over (the scan clears it)
+    // Context shard (all null: whole sequences).  The shard holds global
+    // tokens [id_off[b], id_off[b] + seq_lens[b]); collect writes global ids
+    // (kept lists, candidate keys); finalize takes every shard's boundary
+    // candidates from ext_cands [B*H_q][ext_stride] with ext_cnt[bh] each,
+    // and writes each head's threshold key to theta_out instead of lists
+    // and counts (shard_own_kernel appends this shard's kept candidates).
+    const int32_t *id_off;
+    const unsigned long long *ext_cands;
+    const int32_t *ext_cnt;
+    long long ext_stride;
+    unsigned long long *theta_out;
 };
 
 // Record `r` of a cluster (the same shared variable in CTA rank r); the CTA's
@@ -1366,6 +1377,8 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
     const int b0 = y0 / a.n_ret, b1 = has1 ? y1 / a.n_ret : b0;
     const int g0 = a.ret_g[y0 % a.n_ret], g1 = has1 ? a.ret_g[y1 % a.n_ret] : g0;
     const size_t bg0 = (size_t)b0 * a.H_kv + g0, bg1 = (size_t)b1 * a.H_kv + g1;
+    // global position of this shard's token 0 in each group's sequence
+    const int off0 = a.id_off ? a.id_off[b0] : 0, off1 = a.id_off ? a.id_off[b1] : 0;
     const size_t bh00 = (size_t)b0 * a.H_q + (size_t)g0 * G, bh01 = (size_t)b1 * a.H_q + (size_t)g1 * G;
     // pair-head ph is valid when its group exists and its head is < G
     auto ph_ok = [&](int ph) { return (ph < GMAX || has1) && ph % GMAX < G; };
@@ -1514,11 +1527,12 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
                             s_kbuf[ph * CL_KCAP + p] = t;
                         } else {
                             const unsigned q = atomicAdd(&w.list_cnt[bh * CNT_STRIDE], 1u);
-                            a.lists[bh * a.N_max + q] = t;
+                            a.lists[bh * a.N_max + q] = t + (gk ? off1 : off0);
                         }
                     } else {
-                        const unsigned long long key = ((unsigned long long)logit_key(zv + 0.0f) << 32) |
-                                                       (unsigned long long)(0xffffffffu - (uint32_t)t);
+                        const unsigned long long key =
+                            ((unsigned long long)logit_key(zv + 0.0f) << 32) |
+                            (unsigned long long)(0xffffffffu - (uint32_t)(t + (gk ? off1 : off0)));
                         const unsigned p = atomicAdd(&s_cc[ph], 1u);
                         if (p < (unsigned)CCAP) {
                             s_cbuf[ph * CCAP + p] = key;
@@ -1561,7 +1575,8 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
         if (cx == 0 && lane == 0 && wok) w.res[wbh] = s_res[warp];
         kb = __shfl_sync(0xffffffffu, kb, 0);
         cb = __shfl_sync(0xffffffffu, cb, 0);
-        for (unsigned j = lane; j < nk; j += 32) a.lists[wbh * a.N_max + kb + j] = s_kbuf[warp * CL_KCAP + j];
+        const int offw = warp < GMAX ? off0 : off1;
+        for (unsigned j = lane; j < nk; j += 32) a.lists[wbh * a.N_max + kb + j] = s_kbuf[warp * CL_KCAP + j] + offw;
         for (unsigned j = lane; j < ncd; j += 32) w.cands[wbh * a.N_max + cb + j] = s_cbuf[warp * CCAP + j];
     };
     if (!a.q_rope) {
@@ -1700,13 +1715,13 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     pdl_trigger();
     // the head's resolve record and both counters in one round of loads
     const Resolve r = w.res[bh];
-    const unsigned nc_all = w.cand_cnt[bh * CNT_STRIDE];
+    const unsigned nc_all = a.ext_cnt ? (unsigned)a.ext_cnt[bh] : w.cand_cnt[bh * CNT_STRIDE];
     const unsigned base0 = w.list_cnt[bh * CNT_STRIDE];
     const unsigned ovf = a.q_rope ? a.ovf[bh] : 0u;
-    const unsigned long long *cg = w.cands + bh * a.N_max;
+    const unsigned long long *cg = a.ext_cands ? a.ext_cands + bh * a.ext_stride : w.cands + bh * a.N_max;
     // first candidate of each thread, loaded before the count is known (the
-    // buffer holds N_max entries, so the read is in bounds)
-    const unsigned long long c_first = tid < a.N_max ? __ldcg(cg + tid) : 0ull;
+    // buffer holds N_max -- or ext_stride -- entries, so the read is in bounds)
+    const unsigned long long c_first = tid < (a.ext_cands ? a.ext_stride : a.N_max) ? __ldcg(cg + tid) : 0ull;
     // fused attention: fold the collect CTAs' partials of this head while the
     // selection's own loads are in flight (discarded below after an overflow)
     WarpPart part;
@@ -1928,6 +1943,17 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
     bool spill = false;
     auto finish = [&]() {
         if (rank != 0) return;
+        if (a.theta_out) {
+            // context shard: the threshold key (every key at or above it is
+            // kept; 0 keeps all, ~0 none of the candidates) and the mass
+            if (tid == 0) {
+                a.theta_out[bh] = r.mode == MODE_KEEP_ALL ? 0ull
+                                  : (r.mode == MODE_NORMAL && nc > 0u) ? fin_theta : ~0ull;
+                if (a.mass_out) a.mass_out[bh] = mass;
+            }
+            for (int i = tid; i < HSTRIDE; i += blockDim.x) w.hist[bh * HSTRIDE + i] = 0.0;
+            return;
+        }
         if (tid == 0) {
             a.count_out[bh] = count;
             if (a.mass_out) a.mass_out[bh] = mass;
@@ -2066,6 +2092,49 @@ __global__ void __launch_bounds__(FIN_THREADS) finalize_kernel(SelArgs a, SelWs 
         }
     }
     finish();
+}
+
+// ---------------------------------------------------------------------------
+// Context shard: this shard's kept list of each retrieval head -- the ids
+// the collect pass kept (global, already in the list) plus the shard's own
+// boundary candidates at or above the head's threshold key (their global
+// ids), or every token of the shard for a keep-all head.  grid = (B * n_ret
+// * G), OWN_THREADS threads.
+// ---------------------------------------------------------------------------
+constexpr int OWN_THREADS = 256;
+__global__ void __launch_bounds__(OWN_THREADS) shard_own_kernel(SelArgs a, SelWs w) {
+    __shared__ unsigned s_n;
+    const int hb = blockIdx.x;
+    const int G = a.G;
+    const int b = hb / (a.n_ret * G);
+    const int gi = (hb / G) % a.n_ret;
+    const int h = a.ret_g[gi] * G + hb % G;
+    const size_t bh = (size_t)b * a.H_q + h;
+    const int N = a.seq_lens[b];
+    const int off = a.id_off[b];
+    int32_t *lst = a.lists + bh * a.N_max;
+    if (N < 1 || (long long)N > a.N_max) {
+        if (threadIdx.x == 0) a.count_out[bh] = 0;
+        return;
+    }
+    const Resolve r = w.res[bh];
+    if (r.mode == MODE_KEEP_ALL) {
+        for (int t = threadIdx.x; t < N; t += blockDim.x) lst[t] = off + t;
+        if (threadIdx.x == 0) a.count_out[bh] = N;
+        return;
+    }
+    const unsigned base0 = r.mode == MODE_NORMAL ? w.list_cnt[bh * CNT_STRIDE] : 0u;
+    const unsigned nc = r.mode == MODE_NORMAL ? w.cand_cnt[bh * CNT_STRIDE] : 0u;
+    const unsigned long long theta = a.theta_out[bh];
+    if (threadIdx.x == 0) s_n = 0u;
+    __syncthreads();
+    const unsigned long long *cg = w.cands + bh * a.N_max;
+    for (unsigned c = threadIdx.x; c < nc; c += blockDim.x) {
+        const unsigned long long v = cg[c];
+        if (v >= theta) lst[base0 + atomicAdd(&s_n, 1u)] = (int32_t)(0xffffffffu - (uint32_t)(v & 0xffffffffull));
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) a.count_out[bh] = (int)(base0 + s_n);
 }
 
 // ---------------------------------------------------------------------------

@@ -38,12 +38,14 @@ OP_LOCAL_DECODE = 4
 OP_DENSE_DECODE = 5
 OP_DECODE_STEP = 6
 OP_PREFILL = 7
+PART_STRIDE = 132          # floats per partial record: m, l, 2 unused, o[128]
 
 EXPORTS = ("rtp_workspace_size", "rtp_workspace_init", "rtp_check", "rtp_error_string",
            "rtp_version", "rtp_append_index_keys", "rtp_index_scores", "rtp_topp_select", "rtp_topk_select",
            "rtp_sparse_decode", "rtp_local_decode", "rtp_dense_decode", "rtp_decode_step",
            "rtp_prof_init", "rtp_prof_elapsed", "rtp_prof_destroy", "rtp_dense_decode_noalloc",
-           "rtp_selftest_wait_timeout", "rtp_prefill_attention")
+           "rtp_selftest_wait_timeout", "rtp_prefill_attention", "rtp_shard_scan", "rtp_shard_hist",
+           "rtp_shard_collect", "rtp_shard_cands", "rtp_shard_finish", "rtp_merge_shards")
 
 NOALLOC_SCRATCH_BYTES = 8 << 20
 NOALLOC_MAX_GROUPS = 1024
@@ -108,6 +110,19 @@ _SIGS = {
     "rtp_dense_decode_noalloc": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Opts), _P, _P, _P, _P, _P,
                                                 _P]),
     "rtp_selftest_wait_timeout": (ctypes.c_int, [_P, _P]),
+    "rtp_shard_scan": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Opts), _P, _P, _P, _P, ctypes.c_float,
+                                      _P, ctypes.c_size_t, _P]),
+    "rtp_shard_hist": (ctypes.c_int, [ctypes.POINTER(Dims), _P, ctypes.POINTER(ctypes.c_void_p),
+                                      ctypes.POINTER(ctypes.c_int64)]),
+    "rtp_shard_collect": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Opts), _P, _P, ctypes.c_float, _P,
+                                         _P, ctypes.c_size_t, _P]),
+    "rtp_shard_cands": (ctypes.c_int, [ctypes.POINTER(Dims), _P, ctypes.POINTER(ctypes.c_void_p),
+                                       ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_int64),
+                                       ctypes.POINTER(ctypes.c_int64)]),
+    "rtp_shard_finish": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Opts), _P, _P, _P, _P, _P,
+                                        ctypes.c_float, ctypes.c_int32, ctypes.c_int32, _P, _P, _P, _P,
+                                        ctypes.c_int64, _P, _P, ctypes.c_size_t, _P]),
+    "rtp_merge_shards": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P, _P]),
     "rtp_prefill_attention": (ctypes.c_int, [ctypes.POINTER(Dims), ctypes.POINTER(Opts), _P, ctypes.c_int32, _P,
                                              _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P, _P,
                                              ctypes.c_size_t, _P]),
@@ -318,6 +333,65 @@ def prefill_attention(dims: Dims, q, pos0, k_cache, v_cache, head_class, window:
                                     _ptr(pos0), _ptr(k_cache), _ptr(v_cache), _hc(head_class), int(window),
                                     int(n_sink), _ptr(out), ws.ptr, ws.nbytes, _stream()),
         "rtp_prefill_attention")
+
+
+# ------------------------------------------------- context-sharded decode step
+
+def shard_scan(dims: Dims, q, kidx_cache, W_q_idx, head_class, p: float, ws: Workspace, opts: Opts | None = None):
+    _ck(lib().rtp_shard_scan(ctypes.byref(dims), ctypes.byref(opts) if opts else None, _ptr(q), _ptr(kidx_cache),
+                             _ptr(W_q_idx), _hc(head_class), float(p), ws.ptr, ws.nbytes, _stream()),
+        "rtp_shard_scan")
+
+
+def _dev_view(ptr: int, count: int, dtype, like: torch.Tensor) -> torch.Tensor:
+    """A torch view of `count` elements of device memory at `ptr` inside the
+    workspace buffer `like` (no copy)."""
+    esize = torch.empty(0, dtype=dtype).element_size()
+    off = ptr - like.data_ptr()
+    if off < 0 or off % esize or off + count * esize > like.numel() * like.element_size():
+        raise ValueError("region outside the workspace")
+    return like.view(torch.uint8)[off:off + count * esize].view(dtype)
+
+
+def shard_hist(dims: Dims, ws: Workspace) -> torch.Tensor:
+    """The workspace's per-head level-1 histograms (fp64) that exchange 1
+    sums over the shards, as a view."""
+    p, n = ctypes.c_void_p(), ctypes.c_int64()
+    _ck(lib().rtp_shard_hist(ctypes.byref(dims), ws.ptr, ctypes.byref(p), ctypes.byref(n)), "rtp_shard_hist")
+    return _dev_view(p.value, n.value, torch.float64, ws.buf)
+
+
+def shard_collect(dims: Dims, kidx_cache, head_class, p: float, shard_off, ws: Workspace, opts: Opts | None = None):
+    _ck(lib().rtp_shard_collect(ctypes.byref(dims), ctypes.byref(opts) if opts else None, _ptr(kidx_cache),
+                                _hc(head_class), float(p), _ptr(shard_off), ws.ptr, ws.nbytes, _stream()),
+        "rtp_shard_collect")
+
+
+def shard_cands(dims: Dims, ws: Workspace):
+    """This shard's boundary candidates (views): keys [B*H_q, N_max] int64
+    (the bits of the 64-bit keys) and their counts [B*H_q] int32."""
+    c, n, st, cst = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_int64(), ctypes.c_int64()
+    _ck(lib().rtp_shard_cands(ctypes.byref(dims), ws.ptr, ctypes.byref(c), ctypes.byref(n), ctypes.byref(st),
+                              ctypes.byref(cst)), "rtp_shard_cands")
+    nh = dims.B * dims.H_q
+    keys = _dev_view(c.value, nh * st.value, torch.int64, ws.buf).view(nh, st.value)
+    cnts = _dev_view(n.value, nh * cst.value, torch.int32, ws.buf).view(nh, cst.value)[:, 0]
+    return keys, cnts
+
+
+def shard_finish(dims: Dims, q_rope, k_cache, v_cache, kidx_cache, head_class, p: float, window: int, n_sink: int,
+                 shard_off, glob_len, all_cands, all_counts, part_out, ws: Workspace, opts: Opts | None = None):
+    stride = all_cands.shape[1] if all_cands is not None else 0
+    _ck(lib().rtp_shard_finish(ctypes.byref(dims), ctypes.byref(opts) if opts else None, _ptr(q_rope),
+                               _ptr(k_cache), _ptr(v_cache), _ptr(kidx_cache), _hc(head_class), float(p), int(window),
+                               int(n_sink), _ptr(shard_off), _ptr(glob_len), _ptr(all_cands), _ptr(all_counts),
+                               int(stride), _ptr(part_out), ws.ptr, ws.nbytes, _stream()), "rtp_shard_finish")
+
+
+def merge_shards(parts, out):
+    """parts [P, B*H_q, 132] fp32 -> out [B*H_q, 128] (or [B, H_q, 128])."""
+    P, nh = parts.shape[0], parts.shape[1]
+    _ck(lib().rtp_merge_shards(_ptr(parts), int(P), int(nh), _ptr(out), _stream()), "rtp_merge_shards")
 
 
 def selftest_wait_timeout(dev_status):

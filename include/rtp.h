@@ -401,6 +401,67 @@ RTP_API int rtp_dense_decode_noalloc(const rtp_dims *dims, const rtp_opts *opts,
                                      const void *k_cache, const void *v_cache, float *out,
                                      int32_t *dev_status, rtp_stream_t stream);
 
+/*
+ * Context-sharded decode step (a multi-GPU layout beside the method: one
+ * long sequence split over P GPUs, each holding a contiguous range of its
+ * tokens).  The result is the step of the whole sequence -- the same kept
+ * sets and output as rtp_decode_step over all tokens -- reached with three
+ * exchanges that the caller makes between these calls (over NCCL or any
+ * transport; every shard runs the same calls in the same order):
+ *
+ *   1. rtp_shard_scan      index-key scan of this shard: per-head level-1
+ *                          mass histograms in the workspace;
+ *      exchange 1          sum the histograms of all shards in place
+ *                          (rtp_shard_hist gives their address and length,
+ *                          fp64);
+ *   2. rtp_shard_collect   the boundary bin of every head from the summed
+ *                          histograms; this shard's tokens above it (kept) and
+ *                          in it (boundary candidates, 64-bit keys: logit bits,
+ *                          then the inverted GLOBAL token id);
+ *      exchange 2          gather every shard's candidates of each head
+ *                          (rtp_shard_cands gives this shard's, count at
+ *                          stride count_stride) into all_cands [B*H_q][stride]
+ *                          with all_counts [B*H_q];
+ *   3. rtp_shard_finish    the exact threshold from all candidates, this
+ *                          shard's kept list (global ids; opts->sel_idx /
+ *                          sel_count if given) and the attention over its kept
+ *                          rows and, for local heads, its rows among the
+ *                          sinks and window of the global sequence: one
+ *                          partial record per head in part_out [B*H_q][132]
+ *                          fp32 (m and l in log2 units, then 2 unused, then
+ *                          the 128 unnormalised output dims);
+ *      exchange 3          gather every shard's part_out into parts
+ *                          [P][B*H_q][132];
+ *   4. rtp_merge_shards    merge the P records of each head into out
+ *                          [B*H_q][128] (the same on every shard).
+ *
+ * dims describe this shard: seq_lens[b] its tokens of sequence b (>= 1),
+ * N_max its capacity; shard_off[b] (device int32) the global position of
+ * its token 0, glob_len[b] (device int32) the sequence's global length.
+ * bf16 caches and index keys only (else RTP_ERR_UNSUPPORTED); top-p only
+ * (opts->topk and force_local are not used).  p >= 1 makes the scan and
+ * collect calls no-ops (the histograms are then not summed either) and the
+ * finish call attend the shard's rows densely.
+ * The workspace is rtp_workspace_size(dims, RTP_OP_DECODE_STEP) and must
+ * stay untouched between the calls of one step.  Argument errors as for
+ * rtp_decode_step.
+ */
+RTP_API int rtp_shard_scan(const rtp_dims *dims, const rtp_opts *opts, const float *q, const void *kidx_cache,
+                           const float *W_q_idx, const uint8_t *head_class, float p, void *ws, size_t ws_bytes,
+                           rtp_stream_t stream);
+RTP_API int rtp_shard_hist(const rtp_dims *dims, void *ws, double **hist, int64_t *count);
+RTP_API int rtp_shard_collect(const rtp_dims *dims, const rtp_opts *opts, const void *kidx_cache,
+                              const uint8_t *head_class, float p, const int32_t *shard_off, void *ws,
+                              size_t ws_bytes, rtp_stream_t stream);
+RTP_API int rtp_shard_cands(const rtp_dims *dims, void *ws, uint64_t **cands, uint32_t **counts, int64_t *stride,
+                            int64_t *count_stride);
+RTP_API int rtp_shard_finish(const rtp_dims *dims, const rtp_opts *opts, const float *q_rope, const void *k_cache,
+                             const void *v_cache, const void *kidx_cache, const uint8_t *head_class, float p,
+                             int32_t window, int32_t n_sink, const int32_t *shard_off, const int32_t *glob_len,
+                             const uint64_t *all_cands, const int32_t *all_counts, int64_t all_stride,
+                             float *part_out, void *ws, size_t ws_bytes, rtp_stream_t stream);
+RTP_API int rtp_merge_shards(const float *parts, int32_t P, int32_t n_heads, float *out, rtp_stream_t stream);
+
 /* Self-test of failure detection (no counterpart in the pages).  The
  * library's device-side waits -- the index scan's waits on its own bulk
  * copies -- are bounded: after 0.2 s a waiting kernel records
