@@ -139,7 +139,8 @@ def test_sharded_step_repeats_on_the_same_workspaces():
         outs.append(out)
     for s in shards:
         assert s.ws.check() == 0
-    within(outs[0].cpu().numpy(), outs[2].cpu().numpy(), 1e-6, "repeat")
+    # kept ids are listed in atomic order, which sets the fp32 summation order
+    within(outs[0].cpu().numpy(), outs[2].cpu().numpy(), 1e-5, "repeat")
 
 
 @pytest.mark.slow
