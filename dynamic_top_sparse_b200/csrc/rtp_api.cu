@@ -478,7 +478,7 @@ int launch_list(Launcher &ln, const rtp_dims *d, const float *q, const void *k, 
     a.part_out = part_out;
     const long long max_items = (long long)d->B * a.n_rq *
         std::min<long long>(LIST_MAX_SPLIT, (d->N_max + LCH - 1) / LCH);
-    const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(max_items, (phase == LIST_SPILL ? 1LL : 2LL) * num_sms()));
+    const unsigned grid = (unsigned)std::max(1LL, std::min<long long>(max_items, 2LL * num_sms()));
     const size_t smem = list_smem_bytes(d->B * a.n_rq, d->B);
     const char *name = phase == LIST_FIRST ? "sparse_attn_first" : phase == LIST_SPILL ? "sparse_attn_spill"
                                                                                        : "sparse_attn";

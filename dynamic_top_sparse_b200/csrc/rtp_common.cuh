@@ -158,7 +158,7 @@ __device__ __forceinline__ float warp_max(float v) {
 // List attention splits a head's kept rows into items of about LCH rows,
 // at most LIST_MAX_SPLIT per head.
 constexpr int LCH = 64;
-constexpr int LIST_MAX_SPLIT = 64;
+constexpr int LIST_MAX_SPLIT = 256;
 constexpr int LIST_SLOTS = 2 * LIST_MAX_SPLIT;   // partial record slots per head
 // Flags by which the fused step's finalize hands a head's remaining rows to
 // a list pass: the rows from the collect pass's count on, or every row.
