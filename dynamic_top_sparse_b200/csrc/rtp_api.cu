@@ -611,9 +611,10 @@ int rtp_append_index_keys(const rtp_dims *dims, const void *k_pre, int32_t T, co
     // the append waits on the device for the previous kernel of the stream,
     // so its launch overlaps that kernel's tail
     ln.pdl = true;
-    // about two CTAs per SM over all (b, g); runs of APP_TOK tokens
+    // about eight CTAs per SM over all (b, g), so that a long append (a
+    // prompt) keeps many keys in flight; runs of APP_TOK tokens
     const long long units = (long long)dims->B * dims->H_kv;
-    const long long per_bg = std::max(1LL, 2LL * num_sms() / units);
+    const long long per_bg = std::max(1LL, 8LL * num_sms() / units);
     long long tpc = std::max<long long>(APP_TOK, (T + per_bg - 1) / per_bg);
     tpc = (tpc + APP_TOK - 1) / APP_TOK * APP_TOK;
     const dim3 grid((unsigned)((T + tpc - 1) / tpc), (unsigned)units);

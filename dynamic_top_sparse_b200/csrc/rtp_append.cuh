@@ -15,7 +15,7 @@ namespace rtp {
 // reduction; longer appends give each CTA a run of `tpc` tokens, loading
 // APP_TOK of them at a time.
 constexpr int APP_THREADS = R * (D / 8);   // 256
-constexpr int APP_TOK = 4;
+constexpr int APP_TOK = 8;
 
 template <typename KT, typename IT>
 __global__ void __launch_bounds__(APP_THREADS)
