@@ -3,21 +3,29 @@
 // ("Full Attention Strikes Back", gist.science technical summary, Method
 // section 1), or every row (the dense comparison kernel).  bf16 caches.
 //
-// mma.sync m16n8k16 with the heads on M (8 used of 16, FlashAttention-2
-// style so that the softmax output of Q.K^T is already the A operand of
-// P.V):
-//   S[h, t]  = sum_d q[h, d] k[t, d]       A = q (3-term bf16 split, ~24-bit
-//                                          exact), B = K^T, 2 n-tiles of 8 rows
-//   O[h, d] += sum_t p[h, t] v[t, d]       A = p (2-term split), B = V,
-//                                          16 n-tiles of 8 dims
-// The k dimension of each product is permuted so that every thread reads
-// contiguous 16-byte pieces of K and V rows straight from HBM:
-//   Q.K^T, k-step kk: thread (gid, tig) supplies dims 32 tig + 4 kk + {0..3};
-//   P.V, n-tile j, column n: dim 16 n + j, so thread gid reads dims
-//   [16 gid, 16 gid + 16) of its four rows (tokens 2tig, 2tig+1, 2tig+8,
-//   2tig+9 of the 16-row tile) and pairs them with byte permutes.
-// Partials (m, l, o) per head are merged over warps, then over CTAs by the
-// last CTA to finish (same record layout as range_attn_kernel).
+// mma.sync m16n8k16 with the tokens on M and the heads on N, so that all 16
+// rows of every product do work (8 query heads fill N exactly):
+//   S^T[t, h] = sum_d k[t, d] q[h, d]      A = K (16 rows of the tile),
+//                                          B = q^T (3-term bf16 split, ~24-bit
+//                                          exact), 8 k-steps of 16 dims
+//   O^T[d, h] += sum_t v[t, d] p[h, t]     A = V^T (16 dims per m-tile, 8
+//                                          m-tiles), B = p^T (2-term split)
+// S^T leaves the first product in the accumulator layout (a thread holds
+// tokens gid, gid + 8 of heads 2 tig, 2 tig + 1); packed to bf16 pairs it is
+// the 8x8 fragment layout, and one movmatrix transpose per 8 tokens turns it
+// into the B operand of the second product.
+// The k and m indices are permuted so that every thread reads contiguous
+// 16-byte pieces of K and V rows straight from HBM:
+//   Q.K^T, k-step kk: thread (gid, tig) supplies dims 32 tig + 4 kk + {0..3}
+//   of rows gid and gid + 8;
+//   P.V, m-tile mt: rows gid, gid + 8 are dims 16 gid + 2 mt, 16 gid + 2 mt + 1,
+//   so thread gid reads dims [16 gid, 16 gid + 16) of its four tokens (2tig,
+//   2tig+1, 2tig+8, 2tig+9 of the 16-row tile) and pairs them with byte
+//   permutes.
+// Each warp keeps the next tile's K/V loads in flight while it computes the
+// current one (two register sets).  Partials (m, l, o) per head are merged
+// over warps, then over CTAs by the last CTA to finish (same record layout
+// as range_attn_kernel).
 #pragma once
 
 #include "rtp_attend.cuh"
@@ -28,19 +36,22 @@ constexpr int GQ_WARPS = 8;
 constexpr int GQ_THREADS = GQ_WARPS * 32;
 constexpr int GQ_TILE = 16;                 // rows per mma tile
 
-// D[rows 0-7] = A.B + C for an A whose rows 8-15 are zero: only the two
-// accumulators of rows gid are kept; rows 8-15 go to write-only temporaries
-// (no dependency between independent products).
-__device__ __forceinline__ void mma16816_top(float &d0, float &d1, uint32_t a0, uint32_t a2, uint32_t b0,
-                                             uint32_t b1) {
-    float j0, j1;
+// D = A.B + D (m16n8k16, bf16 inputs, fp32 accumulators)
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
     asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%10,%11,%12,%12};\n"
-        : "=f"(d0), "=f"(d1), "=f"(j0), "=f"(j1)
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(d0), "f"(d1), "f"(0.0f));
-    (void)j0;
-    (void)j1;
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};\n"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// transpose of an 8x8 matrix of 16-bit values held one pair per lane (lane
+// 4r + c holds row r, columns 2c and 2c + 1)
+__device__ __forceinline__ uint32_t movm_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
 }
 
 __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
@@ -93,8 +104,8 @@ __global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a
     const long long lo = (long long)blockIdx.x * seg;
     const long long hi = min(L, lo + seg);
 
-    // Q fragments: head gid (zero for gid >= G), dims 32 tig + 4 kk + {0..3}
-    uint32_t qa[3][8][2];
+    // q as the B operand: head gid (zero for gid >= G), dims 32 tig + 4 kk + {0..3}
+    uint32_t qb[3][8][2];
     {
         const float *qh = a.q + (bh0 + (gid < G ? gid : 0)) * D + 32 * tig;
 #pragma unroll
@@ -104,9 +115,9 @@ __global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a
             float h[4], m[4], l[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) split3(x[i], h[i], m[i], l[i]);
-            qa[0][kk][0] = bf16x2(h[0], h[1]); qa[0][kk][1] = bf16x2(h[2], h[3]);
-            qa[1][kk][0] = bf16x2(m[0], m[1]); qa[1][kk][1] = bf16x2(m[2], m[3]);
-            qa[2][kk][0] = bf16x2(l[0], l[1]); qa[2][kk][1] = bf16x2(l[2], l[3]);
+            qb[0][kk][0] = bf16x2(h[0], h[1]); qb[0][kk][1] = bf16x2(h[2], h[3]);
+            qb[1][kk][0] = bf16x2(m[0], m[1]); qb[1][kk][1] = bf16x2(m[2], m[3]);
+            qb[2][kk][0] = bf16x2(l[0], l[1]); qb[2][kk][1] = bf16x2(l[2], l[3]);
         }
     }
     const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(a.k);
@@ -121,22 +132,23 @@ __global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a
         return base + t;
     };
 
-    float m_run = -INFINITY, l_run = 0.0f;        // head gid (shared by the 4 lanes of gid)
-    float o[16][2];
+    // heads 2 tig + c, c = 0, 1 (shared by the 8 lanes of tig); l_run is this
+    // lane's part (its tokens), summed over the lanes at the end
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+    // m-tile mt: {O[2tig][16gid+2mt], O[2tig+1][16gid+2mt], O[2tig][16gid+2mt+1], O[2tig+1][16gid+2mt+1]}
+    float o[8][4];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = 0.0f;
+    for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.0f;
 
-    for (long long t0 = lo + (long long)warp * GQ_TILE; t0 < hi; t0 += GQ_WARPS * GQ_TILE) {
-        // K: rows t0 + gid (n-tile 0) and t0 + 8 + gid (n-tile 1), dims [32 tig, 32 tig + 32)
-        uint4 kr[2][4];
+    // K: rows t0 + gid (+ 8 n), dims [32 tig, 32 tig + 32); V: rows t0 + {2tig,
+    // 2tig+1, 2tig+8, 2tig+9}, dims [16 gid, 16 gid + 16)
+    auto load_tile = [&](long long t0, uint4 (&kr)[2][4], uint4 (&vr)[4][2]) {
 #pragma unroll
         for (int n = 0; n < 2; ++n) {
             const uint4 *p = reinterpret_cast<const uint4 *>(kb + row_of(t0 + 8 * n + gid) * D + 32 * tig);
 #pragma unroll
             for (int i = 0; i < 4; ++i) kr[n][i] = __ldg(p + i);
         }
-        // V: rows t0 + {2tig, 2tig+1, 2tig+8, 2tig+9}, dims [16 gid, 16 gid + 16)
-        uint4 vr[4][2];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
             const int tr = 2 * tig + (r & 1) + 8 * (r >> 1);
@@ -144,81 +156,103 @@ __global__ void __launch_bounds__(GQ_THREADS, 1) gqa_mma_attn_kernel(RangeArgs a
             vr[r][0] = __ldg(p);
             vr[r][1] = __ldg(p + 1);
         }
-        // S = Q K^T (log2 units), n-tile n covers rows t0 + 8n .. t0 + 8n + 7;
-        // one accumulator chain per (n-tile, term), summed low to high
-        float sc[2][2];
+    };
+    auto compute_tile = [&](long long t0, const uint4 (&kr)[2][4], const uint4 (&vr)[4][2]) {
+        // S^T (log2 units): one accumulator chain per term, summed low to high
+        float acc[3][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-        for (int n = 0; n < 2; ++n) {
-            float acc[3][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+        for (int kk = 0; kk < 8; ++kk) {
+            // dims 32 tig + 4 kk + {0,1} and {2,3}: words 2kk, 2kk+1 of the slice
+            const uint4 &k0 = kr[0][kk >> 1], &k1 = kr[1][kk >> 1];
+            const uint32_t a0 = (kk & 1) ? k0.z : k0.x, a2 = (kk & 1) ? k0.w : k0.y;
+            const uint32_t a1 = (kk & 1) ? k1.z : k1.x, a3 = (kk & 1) ? k1.w : k1.y;
 #pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                // dims 32 tig + 4 kk + {0,1} and {2,3}: words 2kk, 2kk+1 of the slice
-                const uint4 &k4 = kr[n][kk >> 1];
-                const uint32_t b0 = (kk & 1) ? k4.z : k4.x;
-                const uint32_t b1 = (kk & 1) ? k4.w : k4.y;
-#pragma unroll
-                for (int term = 0; term < 3; ++term)
-                    mma16816_top(acc[term][0], acc[term][1], qa[term][kk][0], qa[term][kk][1], b0, b1);
-            }
-            sc[n][0] = (acc[2][0] + acc[1][0]) + acc[0][0];
-            sc[n][1] = (acc[2][1] + acc[1][1]) + acc[0][1];
+            for (int term = 0; term < 3; ++term) mma16816(acc[term], a0, a1, a2, a3, qb[term][kk][0], qb[term][kk][1]);
         }
-        // mask rows past the end of this CTA's range
+        // s[0], s[1]: token t0 + gid, heads 2tig, 2tig+1; s[2], s[3]: token t0 + gid + 8
+        float s[4];
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
+        for (int i = 0; i < 4; ++i) s[i] = (acc[2][i] + acc[1][i]) + acc[0][i];
+        if (t0 + gid >= hi) s[0] = s[1] = -INFINITY;
+        if (t0 + 8 + gid >= hi) s[2] = s[3] = -INFINITY;
+        // online softmax per head; token t0 < hi, so every head's tile max is finite
+        float alpha[2], mnew[2];
 #pragma unroll
-            for (int c = 0; c < 2; ++c)
-                if (t0 + 8 * n + 2 * tig + c >= hi) sc[n][c] = -INFINITY;
-        // online softmax for head gid (4 lanes share it)
-        float tmax = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 1));
-        tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 2));
-        const float m_new = fmaxf(m_run, tmax);
-        const float alpha = m_new == -INFINITY ? 1.0f : exp2f(m_run - m_new);
-        float p[2][2];
+        for (int c = 0; c < 2; ++c) {
+            float tmax = fmaxf(s[c], s[2 + c]);
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+            mnew[c] = fmaxf(m_run[c], tmax);
+            alpha[c] = exp2f(m_run[c] - mnew[c]);
+            m_run[c] = mnew[c];
+        }
+        float p[4];
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
+        for (int i = 0; i < 4; ++i) p[i] = exp2f(s[i] - mnew[i & 1]);
 #pragma unroll
-            for (int c = 0; c < 2; ++c) p[n][c] = m_new == -INFINITY ? 0.0f : exp2f(sc[n][c] - m_new);
-        l_run = l_run * alpha + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
-        m_run = m_new;
+        for (int c = 0; c < 2; ++c) l_run[c] = l_run[c] * alpha[c] + (p[c] + p[2 + c]);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) { o[j][0] *= alpha; o[j][1] *= alpha; }
-        // P as A operand: a0 = tokens (2tig, 2tig+1), a2 = tokens (2tig+8, 2tig+9)
-        float ph[2][2], pl[2][2];
+        for (int mt = 0; mt < 8; ++mt) {
+            o[mt][0] *= alpha[0]; o[mt][1] *= alpha[1];
+            o[mt][2] *= alpha[0]; o[mt][3] *= alpha[1];
+        }
+        // p^T as the B operand: the bf16 pairs (tokens gid / gid + 8, heads
+        // 2tig, 2tig+1) transposed to (tokens 2tig, 2tig+1 / 2tig+8, 2tig+9, head gid)
+        float ph[4], pl[4];
 #pragma unroll
-        for (int n = 0; n < 2; ++n)
+        for (int i = 0; i < 4; ++i) {
+            ph[i] = __bfloat162float(__float2bfloat16_rn(p[i]));
+            pl[i] = p[i] - ph[i];
+        }
+        const uint32_t b0h = movm_trans(bf16x2(ph[0], ph[1])), b1h = movm_trans(bf16x2(ph[2], ph[3]));
+        const uint32_t b0l = movm_trans(bf16x2(pl[0], pl[1])), b1l = movm_trans(bf16x2(pl[2], pl[3]));
+        // O^T += V^T P^T: m-tile mt takes word mt (elements 2mt, 2mt+1) of each token's slice
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                ph[n][c] = __bfloat162float(__float2bfloat16_rn(p[n][c]));
-                pl[n][c] = p[n][c] - ph[n][c];
-            }
-        const uint32_t pa0h = bf16x2(ph[0][0], ph[0][1]), pa2h = bf16x2(ph[1][0], ph[1][1]);
-        const uint32_t pa0l = bf16x2(pl[0][0], pl[0][1]), pa2l = bf16x2(pl[1][0], pl[1][1]);
-        // O += P V: n-tile j, column gid <-> dim 16 gid + j
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            const int wi = j >> 1;                       // word index within the 16-dim slice
-            const uint32_t sel = (j & 1) ? 0x7632u : 0x5410u;
-            const uint32_t w_r0 = (&vr[0][wi >> 2].x)[wi & 3];
-            const uint32_t w_r1 = (&vr[1][wi >> 2].x)[wi & 3];
-            const uint32_t w_r2 = (&vr[2][wi >> 2].x)[wi & 3];
-            const uint32_t w_r3 = (&vr[3][wi >> 2].x)[wi & 3];
-            const uint32_t b0 = __byte_perm(w_r0, w_r1, sel);
-            const uint32_t b1 = __byte_perm(w_r2, w_r3, sel);
-            mma16816_top(o[j][0], o[j][1], pa0l, pa2l, b0, b1);
-            mma16816_top(o[j][0], o[j][1], pa0h, pa2h, b0, b1);
+        for (int mt = 0; mt < 8; ++mt) {
+            const uint32_t w_r0 = (&vr[0][mt >> 2].x)[mt & 3];
+            const uint32_t w_r1 = (&vr[1][mt >> 2].x)[mt & 3];
+            const uint32_t w_r2 = (&vr[2][mt >> 2].x)[mt & 3];
+            const uint32_t w_r3 = (&vr[3][mt >> 2].x)[mt & 3];
+            const uint32_t a0 = __byte_perm(w_r0, w_r1, 0x5410u), a1 = __byte_perm(w_r0, w_r1, 0x7632u);
+            const uint32_t a2 = __byte_perm(w_r2, w_r3, 0x5410u), a3 = __byte_perm(w_r2, w_r3, 0x7632u);
+            mma16816(o[mt], a0, a1, a2, a3, b0l, b1l);
+            mma16816(o[mt], a0, a1, a2, a3, b0h, b1h);
+        }
+    };
+
+    // two register sets: the next tile's loads go out before this tile's math
+    {
+        uint4 kA[2][4], vA[4][2], kB[2][4], vB[4][2];
+        const long long step = (long long)GQ_WARPS * GQ_TILE;
+        long long t0 = lo + (long long)warp * GQ_TILE;
+        if (t0 < hi) load_tile(t0, kA, vA);
+        while (t0 < hi) {
+            const long long t1 = t0 + step;
+            if (t1 < hi) load_tile(t1, kB, vB);
+            compute_tile(t0, kA, vA);
+            if (t1 >= hi) break;
+            const long long t2 = t1 + step;
+            if (t2 < hi) load_tile(t2, kA, vA);
+            compute_tile(t1, kB, vB);
+            t0 = t2;
         }
     }
-    // warp partials: l summed over the 4 lanes of head gid; o[j][c] is dim
-    // 16 (2 tig + c) + j of head gid
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-    if (gid < GMAX && tig == 0) { s_m[warp][gid] = m_run; s_l[warp][gid] = l_run; }
+    // warp partials: l summed over the 8 lanes of each tig
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        s_o[warp][gid][32 * tig + j] = o[j][0];
-        s_o[warp][gid][32 * tig + 16 + j] = o[j][1];
+    for (int c = 0; c < 2; ++c) {
+        l_run[c] += __shfl_xor_sync(0xffffffffu, l_run[c], 4);
+        l_run[c] += __shfl_xor_sync(0xffffffffu, l_run[c], 8);
+        l_run[c] += __shfl_xor_sync(0xffffffffu, l_run[c], 16);
+    }
+    if (gid == 0) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) { s_m[warp][2 * tig + c] = m_run[c]; s_l[warp][2 * tig + c] = l_run[c]; }
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+        *reinterpret_cast<float2 *>(&s_o[warp][2 * tig][16 * gid + 2 * mt]) = make_float2(o[mt][0], o[mt][2]);
+        *reinterpret_cast<float2 *>(&s_o[warp][2 * tig + 1][16 * gid + 2 * mt]) = make_float2(o[mt][1], o[mt][3]);
     }
     __syncthreads();
     float *pp = a.part + (bg * a.slots + blockIdx.x) * GMAX * PSTRIDE;

@@ -1236,7 +1236,6 @@ __global__ void __launch_bounds__(COL_THREADS, 2) collect_kernel(SelArgs a, SelW
     init_src(src, a, b, g, qs);
     const int t_lo = (int)((long long)blockIdx.x * a.chunk);
     const int t_hi = (int)min((long long)N, (long long)t_lo + a.chunk);
-    const unsigned lt = (1u << lane) - 1u;
     const uint16_t *tbin = w.tilebin + ((size_t)b * a.H_kv + g) * a.ntile * GMAX;
     int bst[GMAX];
 #pragma unroll
@@ -1451,7 +1450,7 @@ __global__ void __launch_bounds__(CL_THREADS, 1) collect_mma_kernel(SelArgs a, S
     SrcMma src0, src1;
     src0.init(rows0, a.N_max, qs[0], G);
     src1.init(rows1, a.N_max, qs[1], G);
-    const int gid = lane >> 2, tig = lane & 3;
+    const int tig = lane & 3;
     // thresholds of the lane's two head slots (heads 2 tig, 2 tig + 1) in
     // either group: kept z > khi, candidate clo <= z <= khi
     const float khi00 = s_khi[2 * tig], khi01 = s_khi[2 * tig + 1];
