@@ -252,7 +252,7 @@ struct SelPlan {
 // GPU (one wave), each on a contiguous, tile-aligned token range.
 void plan_chunks(SelArgs &a, long long N_max) {
     const long long groups = (long long)a.B * std::max(a.n_ret, 1);
-    long long ctas = (2LL * num_sms() + groups - 1) / groups;
+    long long ctas = std::max(1LL, 2LL * num_sms() / groups);
     const long long tiles = (N_max + TILE - 1) / TILE;
     ctas = std::max(1LL, std::min({ctas, tiles, (long long)SCAN_CTAS_MAX}));
     // at most MAX_CTA_TOKENS tokens per CTA (its 64-bit wide-bin sums cannot wrap)
@@ -416,7 +416,9 @@ int launch_range(Launcher &ln, const rtp_dims *d, const float *q, const void *k,
     const int rows_min = 2 * GQ_WARPS * GQ_TILE;
     const int per_sm = 1;
     const long long chunks = (Lmax + rows_min - 1) / rows_min;
-    long long want = ((long long)per_sm * num_sms() + (long long)d->B * a.n_grp - 1) / ((long long)d->B * a.n_grp);
+    // whole waves: a CTA count just above the SM count would leave a second
+    // wave of a few CTAs running alone
+    long long want = std::max(1LL, (long long)per_sm * num_sms() / ((long long)d->B * a.n_grp));
     if (max_ctas > 0) want = std::max(1LL, (long long)max_ctas / ((long long)d->B * a.n_grp));
     a.n_split = (int)std::max(1LL, std::min(want, std::min(chunks, (long long)RANGE_SPLIT_MAX)));
     // Slots are indexed by (b, g) at a fixed stride, not by this launch's
@@ -825,7 +827,7 @@ int rtp_dense_decode_noalloc(const rtp_dims *dims, const rtp_opts *opts, const f
     const long long rec = (long long)GMAX * PSTRIDE * 4;            // bytes per split per group
     const long long cap = ((long long)RTP_NOALLOC_SCRATCH_BYTES - (long long)NOALLOC_PART_OFF) / (groups * rec);
     const long long chunks = (dims->N_max + 255) / 256;
-    const long long want = (2LL * num_sms() + groups - 1) / groups;
+    const long long want = std::max(1LL, (long long)num_sms() / groups);   // one CTA per SM, one wave
     a.n_split = (int)std::max(1LL, std::min({want, chunks, cap, (long long)RANGE_SPLIT_MAX}));
     a.slots = a.n_split;
     a.scale_log2 = scale_or_default(opts ? opts->attn_scale : 0.f) * L2E;
