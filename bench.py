@@ -436,16 +436,65 @@ def e2e_measure(bn, p, graphs, steps, world):
     """End to end through the C ABI from pinned host memory: every step
     copies its q, q_rope and new key from the host, runs the C-ABI calls
     (rtp_append_index_keys + rtp_decode_step per layer) and copies the
-    output back.  Three forms: a host wait after every step; double-buffered
-    host buffers with one wait per `depth` steps (a decode loop that does
-    not block on each step); and the per-step-wait form with the calls
-    replayed from a CUDA graph."""
+    output back.  The headline form keeps each replica's step inputs in one
+    device buffer (one pinned host buffer per double-buffer slot), so a step
+    moves them with one copy, issues the calls through `ops.Prepared` (their
+    arguments marshalled once) and waits on the host once per `depth` steps.
+    Also measured: the same with the binding's per-call marshalling and one
+    copy per tensor; a host wait after every step; and the per-step-wait
+    form with the calls replayed from a CUDA graph."""
     n_rep = len(bn.reps)
     L0 = bn.reps[0]
+    has_rope = L0[0].q_rope is not None
+    spec = bn.spec
 
     def pinned_like(t):
         return torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
 
+    # packed step inputs of each replica: (layer, q / q_rope / k_new) pieces at
+    # 256-byte offsets of one buffer
+    def pieces(R):
+        out = []
+        for L in R:
+            out.append(L.q)
+            if has_rope:
+                out.append(L.q_rope)
+            out.append(L.k_new)
+        return out
+
+    def layout(ts):
+        offs, o = [], 0
+        for t in ts:
+            offs.append(o)
+            o += (t.numel() * t.element_size() + 255) // 256 * 256
+        return offs, o
+
+    offs, total = layout(pieces(L0))
+    packed, prepared = [], []
+    for R in bn.reps:
+        dev = torch.empty(total, dtype=torch.uint8, device=bn.dev)
+        views = []
+        for t, o in zip(pieces(R), offs):
+            v = dev[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+            v.copy_(t)
+            views.append(v)
+        calls, it = [], iter(views)
+        for L in R:
+            q = next(it)
+            qr = next(it) if has_rope else None
+            kn = next(it)
+            calls.append(ops.prepare_append_index_keys(L.dims, kn, L.Wk, L.pos, L.hc, L.kidx, bn.ws))
+            calls.append(ops.prepare_decode_step(L.dims, q, qr, L.k, L.v, L.kidx, L.Wq, L.hc, p, spec.window,
+                                                 spec.n_sink, bn.out, bn.ws))
+        packed.append((dev, views))
+        prepared.append(calls)
+    hpk = []
+    for _ in range(2):
+        h = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+        h.copy_(packed[0][0].cpu())
+        hpk.append(h)
+    hout = [pinned_like(bn.out) for _ in range(2)]
+    # the per-call form's host buffers (one per tensor)
     bufs = []
     for _ in range(2):
         hq = [pinned_like(L.q) for L in L0]
@@ -455,15 +504,20 @@ def e2e_measure(bn, p, graphs, steps, world):
             hq[i].copy_(L.q)
             hqr[i].copy_(L.q_rope if L.q_rope is not None else L.q)
             hk[i].copy_(L.k_new)
-        bufs.append((hq, hqr, hk, pinned_like(bn.out)))
-    has_rope = L0[0].q_rope is not None
-    hq, hqr, hk, hout = bufs[0]
-    h2d = sum(t.numel() * t.element_size() for t in hq + hk) + (
-        sum(t.numel() * t.element_size() for t in hqr) if has_rope else 0)
-    d2h = hout.numel() * hout.element_size()
+        bufs.append((hq, hqr, hk))
+    h2d = sum(t.numel() * t.element_size() for t in pieces(L0))
+    d2h = bn.out.numel() * bn.out.element_size()
 
-    def one(i, use_graph, wait):
-        hq, hqr, hk, hout = bufs[i % 2]
+    def one_prepared(i, wait):
+        packed[i % n_rep][0].copy_(hpk[i % 2], non_blocking=True)
+        for c in prepared[i % n_rep]:
+            c()
+        hout[i % 2].copy_(bn.out, non_blocking=True)
+        if wait:
+            torch.cuda.current_stream().synchronize()
+
+    def one_per_call(i, use_graph, wait):
+        hq, hqr, hk = bufs[i % 2]
         R = bn.reps[i % n_rep]
         for j, L in enumerate(R):
             L.q.copy_(hq[j], non_blocking=True)
@@ -474,36 +528,41 @@ def e2e_measure(bn, p, graphs, steps, world):
             graphs[i % n_rep].replay()
         else:
             bn.step(R, p)
-        hout.copy_(bn.out, non_blocking=True)
+        hout[i % 2].copy_(bn.out, non_blocking=True)
         if wait:
             torch.cuda.current_stream().synchronize()
 
-    def run(use_graph, depth):
+    def run(one, depth):
         for i in range(3):
-            one(i, use_graph, True)
+            one(i, True)
         barrier(world)
         x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         x0.record()
         for i in range(steps):
-            one(i, use_graph, (i + 1) % depth == 0)
+            one(i, (i + 1) % depth == 0)
         x1.record()
         torch.cuda.synchronize()
         return world * steps / (allreduce_max(x0.elapsed_time(x1), world, bn.dev) / 1e3)
 
     depth = 64
-    pipelined = run(False, depth)
-    per_step = run(False, 1)
-    graph_step = run(True, 1)
+    pipelined = run(one_prepared, depth)
+    per_call = run(lambda i, w: one_per_call(i, False, w), depth)
+    per_step = run(one_prepared, 1)
+    graph_step = run(lambda i, w: one_per_call(i, True, w), 1)
     return {"value": pipelined, "unit": "steps/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps,
-            "note": f"per step: pinned host q/q_rope/k_new -> device, the C-ABI calls "
-                    f"(rtp_append_index_keys + rtp_decode_step per layer), out -> pinned host; "
-                    f"double-buffered host buffers, one host wait per {depth} steps",
+            "note": f"per step: the step's q/q_rope/k_new of every layer, packed in one pinned host buffer "
+                    f"(double-buffered), -> device in one copy; the C-ABI calls (rtp_append_index_keys + "
+                    f"rtp_decode_step per layer) through ops.Prepared; out -> pinned host; one host wait "
+                    f"per {depth} steps",
+            "per_call_value": per_call,
+            "per_call_note": "the same with the binding's per-call argument marshalling and one host-to-device "
+                             "copy per tensor",
             "sync_value": per_step,
-            "sync_note": "the same with a host wait after every step",
+            "sync_note": "the headline form with a host wait after every step",
             "graph_value": graph_step,
-            "graph_note": "the per-step-wait form with the step's C-ABI calls captured once in a "
-                          "CUDA graph and replayed"}
+            "graph_note": "one copy per tensor, the step's C-ABI calls captured once in a CUDA graph and "
+                          "replayed, a host wait after every step"}
 
 
 # static top-k budget measured beside the headline's top-p (tokens per head)

@@ -316,6 +316,51 @@ def dense_decode(dims: Dims, q_rope, k_cache, v_cache, out, ws: Workspace, opts:
         "rtp_dense_decode")
 
 
+class Prepared:
+    """One C-ABI call with every argument marshalled once (pointers, sizes,
+    head classes, stream): calling the object re-issues the same call, so the
+    tensors it names may change contents between calls but not storage.  For
+    decode loops in which converting the arguments on every call would cost
+    more host time than the GPU spends on the step."""
+
+    __slots__ = ("_fn", "_args", "_name", "_keep")
+
+    def __init__(self, name: str, args, keep=()):
+        self._fn = getattr(lib(), name)
+        self._args = tuple(args)
+        self._name = name
+        self._keep = keep           # objects the marshalled pointers refer to
+
+    def __call__(self):
+        code = self._fn(*self._args)
+        if code != RTP_OK:
+            raise RtpError(code, self._name)
+
+
+def _vp(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(_ptr(t))
+
+
+def prepare_append_index_keys(dims: Dims, k_pre, W_k_idx, pos, head_class, kidx_cache,
+                              ws: Workspace) -> Prepared:
+    """append_index_keys with its arguments marshalled once, on the current stream."""
+    hc = _hc(head_class) if head_class is not None else None
+    return Prepared("rtp_append_index_keys",
+                    (ctypes.byref(dims), _vp(k_pre), k_pre.shape[2], _vp(W_k_idx), _vp(pos), hc,
+                     _vp(kidx_cache), ctypes.c_void_p(ws.ptr), ws.nbytes, _stream()), keep=(dims, hc, ws))
+
+
+def prepare_decode_step(dims: Dims, q, q_rope, k_cache, v_cache, kidx_cache, W_q_idx, head_class, p: float,
+                        window: int, n_sink: int, out, ws: Workspace, opts: Opts | None = None) -> Prepared:
+    """decode_step with its arguments marshalled once, on the current stream."""
+    hc = _hc(head_class)
+    return Prepared("rtp_decode_step",
+                    (ctypes.byref(dims), ctypes.byref(opts) if opts else None, _vp(q),
+                     _vp(q_rope) if q_rope is not None else None, _vp(k_cache), _vp(v_cache),
+                     _vp(kidx_cache), _vp(W_q_idx), hc, float(p), int(window), int(n_sink), _vp(out),
+                     ctypes.c_void_p(ws.ptr), ws.nbytes, _stream()), keep=(dims, opts, hc, ws))
+
+
 def decode_step(dims: Dims, q, q_rope, k_cache, v_cache, kidx_cache, W_q_idx, head_class, p: float,
                 window: int, n_sink: int, out, ws: Workspace, opts: Opts | None = None):
     _ck(lib().rtp_decode_step(ctypes.byref(dims), ctypes.byref(opts) if opts else None, _ptr(q),

@@ -181,6 +181,16 @@ def test_other_calls_reject_bad_arguments(L):
     assert L.rtp_selftest_wait_timeout(FAKE + 2, None) == ops.RTP_ERR_INVALID_ARG     # misaligned
 
 
+def test_prepared_call_raises_the_library_error(L):
+    """ops.Prepared re-issues one call and raises what the library returns
+    (a null dims pointer is rejected before anything touches the GPU)."""
+    from dynamic_top_sparse_b200 import ops
+    call = ops.Prepared("rtp_decode_step", (None,) * 9 + (0.9, 0, 0) + (None, None, 0, None))
+    with pytest.raises(ops.RtpError) as e:
+        call()
+    assert e.value.code == ops.RTP_ERR_INVALID_ARG and "rtp_decode_step" in str(e.value)
+
+
 def test_binding_fails_loudly_without_the_library(monkeypatch, tmp_path):
     """No CPU fallback: with the library missing every call raises."""
     from dynamic_top_sparse_b200 import ops

@@ -88,6 +88,41 @@ def test_step_small(k):
     _compare(gc, out, si, sc, sm, p)
 
 
+def test_prepared_calls_match_the_binding():
+    """ops.Prepared re-issues the same C-ABI calls with arguments marshalled
+    once: new inputs written into the same tensors give the per-call
+    binding's results (kept sets and counts exactly, outputs within the
+    atomic-order rounding of the fused step), and those pass the oracle."""
+    spec = synth.small_spec(B=2, H_q=16, H_kv=2, N=6000, head_class=(1, 0), seq_lens=[6000, 2500],
+                            name="prepared")
+    gc = GpuCase(synth.make_case(spec))
+    dev = gc.q.device
+    p = 0.9
+    si = torch.full((gc.B, gc.H_q, gc.N_max), -1, dtype=torch.int32, device=dev)
+    sc = torch.zeros((gc.B, gc.H_q), dtype=torch.int32, device=dev)
+    sm = torch.zeros((gc.B, gc.H_q), dtype=torch.float32, device=dev)
+    opts = ops.make_opts(sel_idx=si, sel_count=sc, sel_mass=sm)
+    pos = (gc.seq - 1).to(torch.int32)
+    out_p = torch.full((gc.B, gc.H_q, 128), float("nan"), device=dev)
+    app = ops.prepare_append_index_keys(gc.dims, gc.k_new, gc.Wk, pos, gc.hc, gc.kidx, gc.ws)
+    stp = ops.prepare_decode_step(gc.dims, gc.q, gc.q_rope, gc.k, gc.v, gc.kidx, gc.Wq, gc.hc, p,
+                                  gc.c.window, gc.c.n_sink, out_p, gc.ws, opts)
+    q0 = gc.q.clone()
+    for scale in (0.5, 1.0):                  # new query contents, same storage; the oracle's last
+        gc.q.copy_(q0 * scale)
+        app()
+        stp()
+        assert gc.ws.check() == 0
+        sets = lambda i_, c_: [sorted(gpu_set(i_, c_, b, h).tolist()) for b in range(gc.B) for h in range(gc.H_q)]
+        sel_p = sets(si, sc)
+        cnt_p = sc.clone()
+        out, si2, sc2, sm2 = gc.step(p)
+        assert torch.equal(cnt_p, sc2)
+        assert sel_p == sets(si2, sc2)
+        within(out_p.cpu().numpy(), out.cpu().numpy(), 1e-5, f"prepared vs per-call (q x {scale})")
+    _compare(gc, out_p, si, sc, sm, p)
+
+
 def test_step_p_one_equals_dense():
     spec = synth.small_spec(B=2, H_q=16, H_kv=2, N=7000, head_class=(1, 1), seq_lens=[7000, 3000])
     gc = GpuCase(synth.make_case(spec))
