@@ -439,10 +439,13 @@ def e2e_measure(bn, p, graphs, steps, world):
     output back.  The headline form keeps each replica's step inputs in one
     device buffer (one pinned host buffer per double-buffer slot), so a step
     moves them with one copy, issues the calls through `ops.Prepared` (their
-    arguments marshalled once) and waits on the host once per `depth` steps.
-    Also measured: the same with the binding's per-call marshalling and one
-    copy per tensor; a host wait after every step; and the per-step-wait
-    form with the calls replayed from a CUDA graph."""
+    arguments marshalled once) into an output buffer of the replica's own,
+    runs the two copies on copy streams ordered by events (a step's copies
+    overlap its neighbours' kernels) and waits on the host once per `depth`
+    steps.  Also measured: the same with the copies in the compute stream;
+    the binding's per-call marshalling with one copy per tensor; a host wait
+    after every step; and the per-step-wait form with the calls replayed
+    from a CUDA graph."""
     n_rep = len(bn.reps)
     L0 = bn.reps[0]
     has_rope = L0[0].q_rope is not None
@@ -470,7 +473,7 @@ def e2e_measure(bn, p, graphs, steps, world):
         return offs, o
 
     offs, total = layout(pieces(L0))
-    packed, prepared = [], []
+    packed, prepared, prepared_own, outs = [], [], [], []
     for R in bn.reps:
         dev = torch.empty(total, dtype=torch.uint8, device=bn.dev)
         views = []
@@ -478,16 +481,23 @@ def e2e_measure(bn, p, graphs, steps, world):
             v = dev[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
             v.copy_(t)
             views.append(v)
-        calls, it = [], iter(views)
+        own = torch.empty_like(bn.out)
+        calls, calls_own, it = [], [], iter(views)
         for L in R:
             q = next(it)
             qr = next(it) if has_rope else None
             kn = next(it)
-            calls.append(ops.prepare_append_index_keys(L.dims, kn, L.Wk, L.pos, L.hc, L.kidx, bn.ws))
+            a = ops.prepare_append_index_keys(L.dims, kn, L.Wk, L.pos, L.hc, L.kidx, bn.ws)
+            calls.append(a)
             calls.append(ops.prepare_decode_step(L.dims, q, qr, L.k, L.v, L.kidx, L.Wq, L.hc, p, spec.window,
                                                  spec.n_sink, bn.out, bn.ws))
+            calls_own.append(a)
+            calls_own.append(ops.prepare_decode_step(L.dims, q, qr, L.k, L.v, L.kidx, L.Wq, L.hc, p,
+                                                     spec.window, spec.n_sink, own, bn.ws))
         packed.append((dev, views))
         prepared.append(calls)
+        prepared_own.append(calls_own)
+        outs.append(own)
     hpk = []
     for _ in range(2):
         h = torch.empty(total, dtype=torch.uint8, pin_memory=True)
@@ -516,6 +526,30 @@ def e2e_measure(bn, p, graphs, steps, world):
         if wait:
             torch.cuda.current_stream().synchronize()
 
+    main = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(n_rep)]
+    ev_done = [torch.cuda.Event() for _ in range(n_rep)]
+    ev_out = [torch.cuda.Event() for _ in range(n_rep)]
+
+    def one_overlapped(i, wait):
+        r = i % n_rep
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_done[r])          # the replica's previous step has read its inputs
+            packed[r][0].copy_(hpk[i % 2], non_blocking=True)
+            ev_in[r].record(s_in)
+        main.wait_event(ev_in[r])
+        main.wait_event(ev_out[r])               # its previous output has been copied out
+        for c in prepared_own[r]:
+            c()
+        ev_done[r].record(main)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_done[r])
+            hout[i % 2].copy_(outs[r], non_blocking=True)
+            ev_out[r].record(s_out)
+        if wait:
+            torch.cuda.synchronize()
+
     def one_per_call(i, use_graph, wait):
         hq, hqr, hk = bufs[i % 2]
         R = bn.reps[i % n_rep]
@@ -538,23 +572,29 @@ def e2e_measure(bn, p, graphs, steps, world):
         barrier(world)
         x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         x0.record()
+        s_in.wait_stream(main)                   # the first input copy is inside the timed region
         for i in range(steps):
             one(i, (i + 1) % depth == 0)
+        main.wait_stream(s_out)                  # the last output copy is inside the timed region
         x1.record()
         torch.cuda.synchronize()
         return world * steps / (allreduce_max(x0.elapsed_time(x1), world, bn.dev) / 1e3)
 
     depth = 64
+    overlapped = run(one_overlapped, depth)
     pipelined = run(one_prepared, depth)
     per_call = run(lambda i, w: one_per_call(i, False, w), depth)
     per_step = run(one_prepared, 1)
     graph_step = run(lambda i, w: one_per_call(i, True, w), 1)
-    return {"value": pipelined, "unit": "steps/s", "h2d_bytes_per_step": int(h2d),
+    return {"value": overlapped, "unit": "steps/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "steps": steps,
             "note": f"per step: the step's q/q_rope/k_new of every layer, packed in one pinned host buffer "
-                    f"(double-buffered), -> device in one copy; the C-ABI calls (rtp_append_index_keys + "
-                    f"rtp_decode_step per layer) through ops.Prepared; out -> pinned host; one host wait "
-                    f"per {depth} steps",
+                    f"(double-buffered), -> device in one copy on a copy stream; the C-ABI calls "
+                    f"(rtp_append_index_keys + rtp_decode_step per layer) through ops.Prepared into the "
+                    f"replica's output buffer; out -> pinned host on a second copy stream; streams ordered "
+                    f"by events; one host wait per {depth} steps",
+            "inorder_value": pipelined,
+            "inorder_note": "the same with both copies in the compute stream and one output buffer",
             "per_call_value": per_call,
             "per_call_note": "the same with the binding's per-call argument marshalling and one host-to-device "
                              "copy per tensor",
