@@ -17,6 +17,8 @@
 // finish, found with an arrival counter.
 #pragma once
 
+#include <type_traits>
+
 #include "rtp_common.cuh"
 
 namespace rtp {
@@ -483,13 +485,118 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
         const int r0 = s_row0[hix] + sub * per_item;
         const int r1 = s_row0[hix] + min(rows, sub * per_item + per_item);
 
-        const float4 q4 = *reinterpret_cast<const float4 *>(a.q + bh * D + lane * 4);
-        const float qx[4] = {q4.x * a.scale_log2, q4.y * a.scale_log2, q4.z * a.scale_log2,
-                             q4.w * a.scale_log2};
         const KT *kc = reinterpret_cast<const KT *>(a.k);
         const KT *vc = reinterpret_cast<const KT *>(a.v);
         const int32_t *lst = a.lists + bh * a.N_max;
         const int id0 = a.id_off ? a.id_off[b] : 0;
+        if constexpr (std::is_same<KT, __nv_bfloat16>::value) {
+            // bf16 rows: a half-warp per row (lane l holds dims 8 (l % 16) ..
+            // + 7, one 16-byte load per row and tensor), 16 rows per warp per
+            // pass with all their loads in flight; the next pass's row ids
+            // are loaded while this pass computes.  Each half keeps its own
+            // running (m, l, o), merged with the other half's at the end.
+            const int half = lane >> 4, hl = lane & 15;
+            float qx[8];
+            {
+                const float4 qa = *reinterpret_cast<const float4 *>(a.q + bh * D + hl * 8);
+                const float4 qb = *reinterpret_cast<const float4 *>(a.q + bh * D + hl * 8 + 4);
+                qx[0] = qa.x * a.scale_log2; qx[1] = qa.y * a.scale_log2; qx[2] = qa.z * a.scale_log2;
+                qx[3] = qa.w * a.scale_log2; qx[4] = qb.x * a.scale_log2; qx[5] = qb.y * a.scale_log2;
+                qx[6] = qb.z * a.scale_log2; qx[7] = qb.w * a.scale_log2;
+            }
+            float m = -INFINITY, l = 0.0f, o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = 0.0f;
+            constexpr int U2 = 16;                  // rows per warp per pass
+            constexpr int STEP = (ATT_THREADS / 32) * U2;
+            const uint4 *kc4 = reinterpret_cast<const uint4 *>(kc);
+            const uint4 *vc4 = reinterpret_cast<const uint4 *>(vc);
+            int rb = r0 + warp * U2;
+            int nid = -1;                           // lanes 0-15: the ids of the pass at rb
+            if (lane < U2 && rb + lane < r1) nid = __ldcg(lst + rb + lane) - id0;
+            for (; rb < r1; rb += STEP) {
+                const int myid = nid;
+                nid = -1;
+                if (lane < U2 && rb + STEP + lane < r1) nid = __ldcg(lst + rb + STEP + lane) - id0;
+                const long long myrow = myid >= 0 && myid < N ? kv_row(a.kv, b, g, myid) : -1LL;
+                // row u of this half: pass row 2 u + half
+                uint4 kw[U2 / 2], vw[U2 / 2];
+                bool ok[U2 / 2];
+#pragma unroll
+                for (int u = 0; u < U2 / 2; ++u) {
+                    const int j = 2 * u + half;
+                    const long long r = __shfl_sync(0xffffffffu, myrow, j);
+                    ok[u] = rb + j < r1 && r >= 0;
+                    if (ok[u]) {
+                        kw[u] = __ldcg(kc4 + (r * D) / 8 + hl);
+                        vw[u] = __ldcg(vc4 + (r * D) / 8 + hl);
+                    } else {
+                        kw[u] = vw[u] = make_uint4(0u, 0u, 0u, 0u);
+                    }
+                    if (rb + j < r1 && !ok[u] && hl == 0) set_status(a.status, RTP_ERR_DEVICE_ARG);
+                }
+                float sc[U2 / 2];
+                float mb = -INFINITY;
+#pragma unroll
+                for (int u = 0; u < U2 / 2; ++u) {
+                    const uint32_t w4[4] = {kw[u].x, kw[u].y, kw[u].z, kw[u].w};
+                    float s = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        s = fmaf(qx[2 * i], bf16_lo(w4[i]), s);
+                        s = fmaf(qx[2 * i + 1], bf16_hi(w4[i]), s);
+                    }
+#pragma unroll
+                    for (int off = 8; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+                    sc[u] = ok[u] ? s : -INFINITY;
+                    mb = fmaxf(mb, sc[u]);
+                }
+                // (a half with no row yet skips the update; no shuffle inside,
+                // so the halves may differ here)
+                const float mn = fmaxf(m, mb);
+                if (mn != -INFINITY) {
+                    const float al = exp2f(m - mn);
+                    l *= al;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) o[i] *= al;
+#pragma unroll
+                    for (int u = 0; u < U2 / 2; ++u) {
+                        const float pw = exp2f(sc[u] - mn);
+                        l += pw;
+                        const uint32_t w4[4] = {vw[u].x, vw[u].y, vw[u].z, vw[u].w};
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            o[2 * i] = fmaf(pw, bf16_lo(w4[i]), o[2 * i]);
+                            o[2 * i + 1] = fmaf(pw, bf16_hi(w4[i]), o[2 * i + 1]);
+                        }
+                    }
+                    m = mn;
+                }
+            }
+            // the two halves' partials into lanes 0-15 (dims 8 hl .. 8 hl + 7)
+            {
+                const float m2 = __shfl_xor_sync(0xffffffffu, m, 16);
+                const float l2 = __shfl_xor_sync(0xffffffffu, l, 16);
+                const float M = fmaxf(m, m2);
+                const float w1 = m == -INFINITY ? 0.0f : exp2f(m - M);
+                const float w2 = m2 == -INFINITY ? 0.0f : exp2f(m2 - M);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float o2 = __shfl_xor_sync(0xffffffffu, o[i], 16);
+                    o[i] = o[i] * w1 + o2 * w2;
+                }
+                l = l * w1 + l2 * w2;
+                m = M;
+            }
+            if (lane == 0) { wm[warp] = m; wl[warp] = l; }
+            if (half == 0) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) wo[warp][hl * 8 + i] = o[i];
+            }
+        } else {
+        const float4 q4 = *reinterpret_cast<const float4 *>(a.q + bh * D + lane * 4);
+        const float qx[4] = {q4.x * a.scale_log2, q4.y * a.scale_log2, q4.z * a.scale_log2,
+                             q4.w * a.scale_log2};
         float m = -INFINITY, l = 0.0f, o[4] = {0.f, 0.f, 0.f, 0.f};
         constexpr int U = 8;       // rows per warp per pass: all their K/V loads in flight
         for (int rb = r0 + warp * U; rb < r1; rb += (ATT_THREADS / 32) * U) {
@@ -543,6 +650,7 @@ __global__ void __launch_bounds__(ATT_THREADS, 2) list_attn_kernel(ListArgs a) {
         if (lane == 0) { wm[warp] = m; wl[warp] = l; }
 #pragma unroll
         for (int i = 0; i < 4; ++i) wo[warp][lane * 4 + i] = o[i];
+        }
         __syncthreads();
         float *hp = a.part + bh * (size_t)LIST_SLOTS * PSTRIDE;
         float *pp = hp + (size_t)slot * PSTRIDE;
