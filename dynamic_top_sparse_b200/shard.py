@@ -88,13 +88,12 @@ def phase_finish(s: Shard, p: float, window: int, n_sink: int, all_keys, all_cou
 def run_local_shards(shards: list, p: float, window: int, n_sink: int, out: torch.Tensor) -> list:
     """All shards of a step in one process on one device, in lockstep; the
     exchanges are tensor operations.  Returns each shard's partials."""
-    hists = [phase_scan(s, p) for s in shards]
-    if p < 1.0:
+    all_keys = all_counts = None
+    if p < 1.0:          # p >= 1 keeps every token: no threshold, no exchanges before the partials
+        hists = [phase_scan(s, p) for s in shards]
         total = torch.stack(hists).sum(0)
         for h in hists:
             h.copy_(total)
-    all_keys = all_counts = None
-    if p < 1.0:
         cands = [phase_collect(s, p) for s in shards]
         all_keys, all_counts = gather_candidates([c[0] for c in cands], [c[1] for c in cands])
     parts = [phase_finish(s, p, window, n_sink, all_keys, all_counts) for s in shards]
