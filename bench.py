@@ -648,6 +648,91 @@ def prefill_pairs(pos0: int, T: int, window: int, n_sink: int, local: bool) -> i
     return sum(local_pairs(P + 1, window, n_sink) for P in range(pos0, pos0 + T))
 
 
+def measure_sharded(args, world, dev, Ps=(2, 4)):
+    """The context-sharded step on the 1M-token workload, its P shards run
+    one after another on this one GPU (the exchanges as tensor operations):
+    each phase's device time per shard (CUDA events, L2 flushed before each
+    repetition) and the bytes each exchange moves.  On P GPUs the shards'
+    phases would run side by side with NCCL exchanges between them; that
+    time is not measured here (every run of this bench has its own GPU)."""
+    from dynamic_top_sparse_b200 import shard as rshard
+    spec = synth.spec_for("ctx1m")
+    p = 0.9
+    c = synth.make_case(spec, device="cuda", seed=rank_seed(0, 0), layer=0)
+    L = Layer(c)
+    ops.append_index_keys(L.dims, L.k_new, L.Wk, L.pos, L.hc, L.kidx, ops.Workspace(L.dims))
+    N = int(c.seq_lens[0])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    whole = torch.empty((1, spec.H_q, spec.d), device=dev)
+    ws = ops.Workspace(L.dims)
+    ops.decode_step(L.dims, L.q, L.q_rope, L.k, L.v, L.kidx, L.Wq, L.hc, p, spec.window, spec.n_sink, whole, ws)
+    res = {"workload": "1M ctx, B1, 32q/4kv, bf16, all retrieval, ranked needles, p=0.9, split into P "
+                       "contiguous token ranges", "p": p, "points": {}}
+    for P in Ps:
+        bounds = [round(i * N / P) for i in range(P + 1)]
+        shards, seqs = [], []          # dims hold the device address of seq_lens: keep them alive
+        for i in range(P):
+            lo, n = bounds[i], bounds[i + 1] - bounds[i]
+            seqs.append(torch.tensor([n], dtype=torch.int32, device=dev))
+            dims = ops.make_dims(1, spec.H_q, spec.H_kv, n, seqs[-1], ops.RTP_BF16, ops.RTP_BF16)
+            shards.append(rshard.Shard(dims, L.q, L.q_rope, L.k[:, :, lo:lo + n].contiguous(),
+                                       L.v[:, :, lo:lo + n].contiguous(), L.kidx[:, :, lo:lo + n].contiguous(),
+                                       L.Wq, L.hc, torch.tensor([lo], dtype=torch.int32, device=dev),
+                                       c.seq_lens.clone(), ops.Workspace(dims)))
+        out = torch.empty_like(whole)
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        times = {"scan": [], "collect": [], "finish": []}
+        ncand = 0
+        for rep in range(4):
+            flush.fill_(rep)
+            marks = {k: [] for k in times}
+            hists = []
+            for sh in shards:
+                e0, e1 = ev(), ev()
+                e0.record(); hists.append(rshard.phase_scan(sh, p)); e1.record()
+                marks["scan"].append((e0, e1))
+            total = torch.stack(hists).sum(0)
+            for h in hists:
+                h.copy_(total)
+            cands = []
+            for sh in shards:
+                e0, e1 = ev(), ev()
+                e0.record(); cands.append(rshard.phase_collect(sh, p)); e1.record()
+                marks["collect"].append((e0, e1))
+            all_keys, all_counts = rshard.gather_candidates([k for k, _ in cands], [n for _, n in cands])
+            parts = []
+            for sh in shards:
+                e0, e1 = ev(), ev()
+                e0.record()
+                parts.append(rshard.phase_finish(sh, p, spec.window, spec.n_sink, all_keys, all_counts))
+                e1.record()
+                marks["finish"].append((e0, e1))
+            ops.merge_shards(torch.stack(parts).contiguous(), out)
+            torch.cuda.synchronize()
+            if rep > 0:                                   # the first repetition warms up
+                for k in times:
+                    times[k].append([a.elapsed_time(b) for a, b in marks[k]])
+            ncand = int(all_counts.sum())
+        for sh in shards:
+            st = sh.ws.check()
+            if st:
+                raise RuntimeError(f"sharded step: device status {st}: {ops.error_string(st)}")
+        per = {k: [float(np.median([r[i] for r in v])) for i in range(P)] for k, v in times.items()}
+        nh = spec.H_q
+        res["points"][str(P)] = {
+            "P": P,
+            "ms_per_shard": per,
+            "ms_sum_of_phase_maxima": sum(max(v) for v in per.values()),
+            "exchange_bytes": {"histograms_allreduce": nh * 640 * 8,
+                               "candidates_allgather": ncand * 8 + P * nh * 4,
+                               "partials_allgather": P * nh * ops.PART_STRIDE * 4},
+            "max_abs_diff_vs_whole_step": float((out - whole).abs().max()),
+        }
+        del shards, seqs
+    res["whole_step_ms_note"] = "the unsharded 1M step at p = 0.9 is the ctx1m point of `workloads`"
+    return res
+
+
 def measure_prefill(args, world, dev):
     """Prefill of a whole 64K-token prompt in the 64K workload's shape (32 q /
     4 KV heads, KV0 retrieval, window 4096 + 4 sinks): the prompt's index
@@ -760,6 +845,7 @@ def run_ours(args, rank, world, dev):
             sweep[key] = measure_workload(key, ps, args, rank, world, dev, hbm_peak)
 
     prefill = None if args.no_prefill else measure_prefill(args, world, dev)
+    sharded = None if args.no_sharded or world > 1 else measure_sharded(args, world, dev)
 
     sc = pt["scan"]
     res = {
@@ -795,6 +881,7 @@ def run_ours(args, rank, world, dev):
         "topk": topk_pt,
         "workloads": sweep,
         "prefill": prefill,
+        "sharded": sharded,
         "pages_context": {"decode_speedup_1M_H20": 2.01, "prefill_speedup_1M_H20": 9.36},
     }
     if rank == 0 and world == 1 and not args.no_cpu:
@@ -891,6 +978,7 @@ def main():
                     help="measure only --workload (no other workloads in the same run)")
     ap.add_argument("--sweep-steps", type=int, default=400)
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-sharded", action="store_true")
     ap.add_argument("--prefill-steps", type=int, default=5)
     args = ap.parse_args()
     if args.warmup < 3:

@@ -187,9 +187,13 @@ def _hc(head_class) -> ctypes.Array:
 
 
 def make_dims(B, H_q, H_kv, N_max, seq_lens: torch.Tensor, kv_dtype, idx_dtype, d=128, r=16) -> Dims:
+    """The dims struct of a call; it holds the device address of seq_lens and
+    keeps the tensor alive with it (a freed tensor's memory would be reused)."""
     if seq_lens.dtype != torch.int32:
         raise ValueError("seq_lens must be int32")
-    return Dims(B, H_q, H_kv, d, r, kv_dtype, idx_dtype, 0, N_max, _ptr(seq_lens))
+    dm = Dims(B, H_q, H_kv, d, r, kv_dtype, idx_dtype, 0, N_max, _ptr(seq_lens))
+    dm._seq_lens = seq_lens
+    return dm
 
 
 def dims_for(k_cache: torch.Tensor, kidx_cache: torch.Tensor | None, H_q: int,
