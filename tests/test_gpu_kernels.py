@@ -210,6 +210,33 @@ def test_sparse_decode(kvdt):
     assert np.all(o[:, 4:] == 7.0)    # local heads untouched
 
 
+@pytest.mark.parametrize("kvdt", ["bf16", "f32"])
+def test_sparse_decode_list_sizes(kvdt):
+    """List lengths around the list kernel's row groups (bf16: a half-warp
+    per row, 16 rows per warp and pass, so one half may have no row; f32: 8
+    rows per warp and pass) and its per-head slices of 64 rows."""
+    counts = [1, 2, 15, 16, 17, 33, 1023, 4999]
+    spec = synth.small_spec(B=1, H_q=8, H_kv=1, N=5000, head_class=(1,), kv_dtype=kvdt, name=f"lists_{kvdt}")
+    c = synth.make_case(spec)
+    gc = GpuCase(c)
+    g = np.random.default_rng(3)
+    idx = torch.full((1, 8, gc.N_max), -1, dtype=torch.int32)
+    cnt = torch.tensor([counts], dtype=torch.int32)
+    sets = []
+    for h, n in enumerate(counts):
+        ids = g.choice(5000, size=n, replace=False).astype(np.int32)
+        sets.append(ids)
+        idx[0, h, :n] = torch.from_numpy(ids)
+    out = torch.full((1, 8, 128), float("nan"), device="cuda")
+    ops.sparse_decode(gc.dims, gc.q_rope, gc.k, gc.v, idx.cuda(), cnt.cuda(), gc.hc, out, gc.ws)
+    assert gc.ws.check() == 0
+    o = out.cpu().numpy()
+    K, V, qr = np64(c.k_cache), np64(c.v_cache), np64(c.q_rope)
+    for h, ids in enumerate(sets):
+        ref = oracle.attend(qr[0, h], K[0, 0], V[0, 0], ids, 1 / math.sqrt(128))
+        within(o[0, h], ref, OUT_TOL_SAME_SET, f"h={h} n={len(ids)}")
+
+
 # ------------------------------------------------------------------ a7 / dense
 
 @pytest.mark.parametrize("kvdt", ["bf16", "f32"])
